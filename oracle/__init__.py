@@ -1,0 +1,262 @@
+"""CPU oracle for the quantized Mamba-2 recurrent-state update.
+
+TEST INFRASTRUCTURE ONLY.  The tests, the package smoke check and the
+benchmark's CPU-baseline leg may import this package; the library and its
+Python binding never do.  It wraps ``ssq_oracle.c`` (plain scalar C, built
+with ``-ffp-contract=off``) through ctypes and works on a *logical* state:
+integer codes, per-row step and zero point, and fp32 values for fp rows.  It
+knows nothing of the library's pool byte layout.
+
+Every function states the passage of the pages it follows in ``ssq_oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssq_oracle.c")
+_LIB = os.path.join(_HERE, "liboref.so")
+
+F32, BF16, I8_SYM, I8_ASYM, I4_SYM, I4_ASYM = range(6)
+FORMATS = {"f32": F32, "bf16": BF16, "i8s": I8_SYM, "i8a": I8_ASYM,
+           "i4s": I4_SYM, "i4a": I4_ASYM}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboref.so`` (gcc, scalar, no FMA
+    contraction).  Rebuilds when the source is newer than the library."""
+    hdr = os.path.join(_HERE, "ssq_oracle.h")
+    stale = (not os.path.exists(_LIB)
+             or os.path.getmtime(_LIB) < max(os.path.getmtime(_SRC),
+                                             os.path.getmtime(hdr)))
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([
+            "gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11",
+            "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int), ("nheads", ctypes.c_int),
+                ("headdim", ctypes.c_int), ("d_state", ctypes.c_int),
+                ("ngroups", ctypes.c_int),
+                ("head_mask", ctypes.POINTER(ctypes.c_uint8))]
+
+
+class _State(ctypes.Structure):
+    _fields_ = [("q", ctypes.POINTER(ctypes.c_int32)),
+                ("delta", ctypes.POINTER(ctypes.c_float)),
+                ("zero", ctypes.POINTER(ctypes.c_float)),
+                ("val", ctypes.POINTER(ctypes.c_float))]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        # SSQ_ORACLE_LIB points the tests' mutation check at a deliberately
+        # broken build of the oracle; normally the library is built here.
+        path = os.environ.get("SSQ_ORACLE_LIB") or build()
+        _lib = ctypes.CDLL(path)
+        _lib.oref_lambda.restype = ctypes.c_float
+        _lib.oref_lambda.argtypes = [ctypes.c_float, ctypes.c_float]
+        _lib.oref_bf16_round.restype = ctypes.c_float
+        _lib.oref_bf16_round.argtypes = [ctypes.c_float]
+    return _lib
+
+
+def _p(a, ct):
+    return a.ctypes.data_as(ctypes.POINTER(ct))
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+@dataclass
+class Cfg:
+    """Shape and format of one layer's state: nheads x headdim rows of
+    d_state entries, ngroups B/C groups, optional per-head quantize mask."""
+    fmt: int
+    nheads: int
+    headdim: int
+    d_state: int
+    ngroups: int = 1
+    head_mask: np.ndarray | None = None
+
+    def c(self):
+        cfg = _Cfg(self.fmt, self.nheads, self.headdim, self.d_state,
+                   self.ngroups, None)
+        if self.head_mask is not None:
+            self._mask = np.ascontiguousarray(self.head_mask, dtype=np.uint8)
+            cfg.head_mask = _p(self._mask, ctypes.c_uint8)
+        return cfg
+
+    @property
+    def rows(self):
+        return self.nheads * self.headdim
+
+    def row_is_quant(self, h):
+        if self.fmt in (F32, BF16):
+            return False
+        return self.head_mask is None or bool(self.head_mask[h])
+
+
+class State:
+    """Logical state of ``count`` (layer, request) pairs."""
+
+    def __init__(self, cfg: Cfg, count: int = 1):
+        R, N = cfg.rows, cfg.d_state
+        self.cfg = cfg
+        self.count = count
+        self.q = np.zeros((count, R, N), np.int32)
+        self.delta = np.zeros((count, R), np.float32)
+        self.zero = np.zeros((count, R), np.float32)
+        self.val = np.zeros((count, R, N), np.float32)
+
+    def c(self, i):
+        return _State(_p(self.q[i], ctypes.c_int32),
+                      _p(self.delta[i], ctypes.c_float),
+                      _p(self.zero[i], ctypes.c_float),
+                      _p(self.val[i], ctypes.c_float))
+
+    def copy(self):
+        s = State(self.cfg, self.count)
+        s.q[...] = self.q
+        s.delta[...] = self.delta
+        s.zero[...] = self.zero
+        s.val[...] = self.val
+        return s
+
+
+def lam(dt, A):
+    return float(lib().oref_lambda(float(dt), float(A)))
+
+
+def bf16_round(v):
+    v = _f32(v)
+    out = np.empty_like(v)
+    f = lib().oref_bf16_round
+    for i, x in enumerate(v.reshape(-1)):
+        out.reshape(-1)[i] = f(float(x))
+    return out
+
+
+def quantize_row(fmt, v):
+    """Refit and round one row.  Returns (codes, delta, zero, pre) where pre
+    is the pre-rounding value fl(v*inv) of each entry."""
+    v = _f32(v)
+    N = v.shape[0]
+    q = np.zeros(N, np.int32)
+    pre = np.zeros(N, np.float32)
+    d = ctypes.c_float()
+    z = ctypes.c_float()
+    lib().oref_quantize_row_dbg(fmt, N, _p(v, ctypes.c_float),
+                                _p(q, ctypes.c_int32), ctypes.byref(d),
+                                ctypes.byref(z), _p(pre, ctypes.c_float))
+    return q, np.float32(d.value), np.float32(z.value), pre
+
+
+def dequantize_row(fmt, q, delta, zero):
+    q = np.ascontiguousarray(q, dtype=np.int32)
+    out = np.zeros(q.shape[0], np.float32)
+    lib().oref_dequantize_row(fmt, q.shape[0], _p(q, ctypes.c_int32),
+                              ctypes.c_float(delta), ctypes.c_float(zero),
+                              _p(out, ctypes.c_float))
+    return out
+
+
+def state_from_f32(cfg: Cfg, S):
+    """S[count][H][P][N] (or [H][P][N]) fp32 -> logical State."""
+    S = _f32(S)
+    if S.ndim == 3:
+        S = S[None]
+    st = State(cfg, S.shape[0])
+    c = cfg.c()
+    for i in range(S.shape[0]):
+        Si = np.ascontiguousarray(S[i])
+        lib().oref_state_from_f32(ctypes.byref(c), _p(Si, ctypes.c_float),
+                                  ctypes.byref(st.c(i)))
+    return st
+
+
+def state_to_f32(st: State):
+    cfg = st.cfg
+    out = np.zeros((st.count, cfg.nheads, cfg.headdim, cfg.d_state),
+                   np.float32)
+    c = cfg.c()
+    for i in range(st.count):
+        lib().oref_state_to_f32(ctypes.byref(c), ctypes.byref(st.c(i)),
+                                _p(out[i], ctypes.c_float))
+    return out
+
+
+def step(cfg: Cfg, st: State, i, x, B, C, dt, A, D, want_pre=False):
+    """One decode step of state pair i.  x[H][P], B/C[G][N], dt/A/D[H].
+    Returns y[H][P] (and pre[H*P][N] when want_pre)."""
+    x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))
+    y = np.zeros((cfg.nheads, cfg.headdim), np.float32)
+    pre = np.zeros((cfg.rows, cfg.d_state), np.float32) if want_pre else None
+    c = cfg.c()
+    lib().oref_step(ctypes.byref(c), ctypes.byref(st.c(i)),
+                    _p(x, ctypes.c_float), _p(B, ctypes.c_float),
+                    _p(C, ctypes.c_float), _p(dt, ctypes.c_float),
+                    _p(A, ctypes.c_float), _p(D, ctypes.c_float),
+                    _p(y, ctypes.c_float),
+                    _p(pre, ctypes.c_float) if want_pre else None)
+    return (y, pre) if want_pre else y
+
+
+def scan(cfg: Cfg, st: State, i, x, B, C, dt, A, D):
+    """T steps on state pair i.  x[T][H][P], B/C[T][G][N], dt[T][H]."""
+    x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))
+    T = x.shape[0]
+    y = np.zeros((T, cfg.nheads, cfg.headdim), np.float32)
+    c = cfg.c()
+    lib().oref_scan(ctypes.byref(c), ctypes.byref(st.c(i)), T,
+                    _p(x, ctypes.c_float), _p(B, ctypes.c_float),
+                    _p(C, ctypes.c_float), _p(dt, ctypes.c_float),
+                    _p(A, ctypes.c_float), _p(D, ctypes.c_float),
+                    _p(y, ctypes.c_float))
+    return y
+
+
+def scan_f64(cfg: Cfg, S0, x, B, C, dt, A, D):
+    """Unquantized fp64 trajectory from S0[H][P][N]; returns (S_T, y[T])."""
+    x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))
+    S = np.ascontiguousarray(S0, dtype=np.float64).copy()
+    T = x.shape[0]
+    y = np.zeros((T, cfg.nheads, cfg.headdim), np.float64)
+    c = cfg.c()
+    lib().oref_scan_f64(ctypes.byref(c), _p(S, ctypes.c_double), T,
+                        _p(x, ctypes.c_float), _p(B, ctypes.c_float),
+                        _p(C, ctypes.c_float), _p(dt, ctypes.c_float),
+                        _p(A, ctypes.c_float), _p(D, ctypes.c_float),
+                        _p(y, ctypes.c_double))
+    return S, y
+
+
+def decode_batch(cfg: Cfg, st: State, nl, batch, x, B, C, dt, A, D):
+    """One decode step for nl layers x batch requests; st holds nl*batch
+    pairs ordered [l][b].  x[nl][batch][H][P], B/C[nl][batch][G][N],
+    dt[nl][batch][H], A/D[nl][H].  Returns y[nl][batch][H][P]."""
+    assert st.count == nl * batch
+    x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))
+    y = np.zeros((nl, batch, cfg.nheads, cfg.headdim), np.float32)
+    arr = (_State * st.count)(*[st.c(i) for i in range(st.count)])
+    c = cfg.c()
+    lib().oref_decode_batch(ctypes.byref(c), nl, batch, arr,
+                            _p(x, ctypes.c_float), _p(B, ctypes.c_float),
+                            _p(C, ctypes.c_float), _p(dt, ctypes.c_float),
+                            _p(A, ctypes.c_float), _p(D, ctypes.c_float),
+                            _p(y, ctypes.c_float))
+    return y

@@ -1,0 +1,358 @@
+/*
+ * ssq_oracle.c -- plain, slow CPU oracle for the quantized Mamba-2
+ * recurrent-state update.
+ *
+ * TEST INFRASTRUCTURE ONLY: used by the tests, the smoke check and the
+ * benchmark's CPU-baseline leg, never by the product path.  Scalar loops, no
+ * blocking, no vectorisation, no reordering beyond what the definitions
+ * state.  Build with -O2 -ffp-contract=off so that every fp32 operation below
+ * is one correctly rounded IEEE operation in the order written.
+ *
+ * Citations use the page title and section; see ssq_oracle.h for the list
+ * of sources and of the readings taken where the pages are silent.
+ *
+ * Parity pins (tests/test_oracle_*.py): the recurrence against its unrolled
+ * closed form; the quantizer against brute-force code enumeration, the
+ * |deq - v| <= Delta/2 bound, the grid-endpoint and dyadic-exactness
+ * invariants, idempotence and scale equivariance; the readout against its
+ * closed form at T=1.  The fp64 trajectory is pinned by the same closed
+ * form.  Multi-step drift is reported, not pinned.
+ */
+#include "ssq_oracle.h"
+
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+int oref_bits(int fmt)
+{
+    switch (fmt) {
+    case OREF_I8_SYM: case OREF_I8_ASYM: return 8;
+    case OREF_I4_SYM: case OREF_I4_ASYM: return 4;
+    case OREF_BF16: return 16;
+    default: return 32;
+    }
+}
+
+int oref_is_quant(int fmt) { return fmt >= OREF_I8_SYM && fmt <= OREF_I4_ASYM; }
+int oref_is_sym(int fmt) { return fmt == OREF_I8_SYM || fmt == OREF_I4_SYM; }
+
+/* ssm-state-quantization README, Setup: heads outside the chosen lambda band
+ * are not rounded ("mid band only" vs "all heads").  A head is quantized when
+ * the format is an integer format and its mask entry is non-zero. */
+int oref_row_is_quant(const oref_cfg* c, int h)
+{
+    if (!oref_is_quant(c->fmt)) return 0;
+    if (c->head_mask == NULL) return 1;
+    return c->head_mask[h] != 0;
+}
+
+/* ssm-state-quantization README, Setup: lambda = exp(dt * A).  dt*A is one
+ * fp32 product; the exponential is taken in double and rounded once to
+ * fp32. */
+float oref_lambda(float dt, float A)
+{
+    float dA = dt * A;
+    double e = exp((double)dA);
+    return (float)e;
+}
+
+/* Round an fp32 value to the nearest bf16 value, ties to even, and return it
+ * widened back to fp32 (bf16 keeps the top 16 bits of the fp32 pattern). */
+float oref_bf16_round(float v)
+{
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u) { /* inf / nan: truncate */
+        u &= 0xffff0000u;
+    } else {
+        uint32_t lsb = (u >> 16) & 1u;
+        u = u + 0x7fffu + lsb;
+        u &= 0xffff0000u;
+    }
+    float r;
+    memcpy(&r, &u, 4);
+    return r;
+}
+
+/* Largest code magnitude: qs = 2^(b-1)-1 on the symmetric grid, qa = 2^b-1 on
+ * the asymmetric grid (ssm-state-quantization README, Setup). */
+static float qmax_of(int fmt)
+{
+    int b = oref_bits(fmt);
+    if (oref_is_sym(fmt)) return (float)((1 << (b - 1)) - 1);
+    return (float)((1 << b) - 1);
+}
+
+/* Refit and round one row (ssm-state-quantization README, Setup: per-row
+ * scale refit every step, symmetric or asymmetric grid; Findings 1: nearest
+ * rounding).  'pre' (optional) receives the pre-rounding value fl(v*inv) of
+ * each entry, used by the tests to find entries on a rounding boundary. */
+void oref_quantize_row_dbg(int fmt, int N, const float* v, int32_t* q,
+                           float* delta_out, float* zero_out, float* pre)
+{
+    const float qm = qmax_of(fmt);
+    const int sym = oref_is_sym(fmt);
+    float delta, inv, z = 0.0f, lo = 0.0f;
+
+    if (sym) {
+        /* amax over the row; step amax / qs. */
+        float amax = 0.0f;
+        for (int n = 0; n < N; ++n) {
+            float a = fabsf(v[n]);
+            if (a > amax) amax = a;
+        }
+        delta = amax / qm;
+    } else {
+        /* [min, max] over the row; step (max - min) / qa. */
+        float hi = v[0];
+        lo = v[0];
+        for (int n = 1; n < N; ++n) {
+            if (v[n] < lo) lo = v[n];
+            if (v[n] > hi) hi = v[n];
+        }
+        float range = hi - lo;
+        delta = range / qm;
+        /* Constant row: any positive step reproduces it; |lo| makes the
+         * reconstruction exact (z = -/+1, code 0). */
+        if (delta == 0.0f) delta = fabsf(lo);
+    }
+    /* A step below the smallest normal fp32 flushes the row to zero. */
+    if (delta < FLT_MIN) delta = 0.0f;
+    inv = (delta == 0.0f) ? 0.0f : 1.0f / delta;
+    if (!sym) {
+        /* Integer zero point: the code of lo is rint(lo*inv) + z = 0.
+         * Adding +0 stores a negative zero as +0. */
+        z = rintf(-lo * inv) + 0.0f;
+    }
+
+    for (int n = 0; n < N; ++n) {
+        float p = v[n] * inv;          /* one fp32 product */
+        float r = rintf(p);            /* nearest, ties to even */
+        if (pre) pre[n] = p;
+        float c;
+        if (sym) {
+            c = r;
+            if (c > qm) c = qm;
+            if (c < -qm) c = -qm;
+        } else {
+            c = r + z;                 /* exact: both are integers of equal
+                                          sign or within a factor 2 */
+            if (c > qm) c = qm;
+        }
+        q[n] = (int32_t)c;
+    }
+    *delta_out = delta;
+    *zero_out = z;
+}
+
+void oref_quantize_row(int fmt, int N, const float* v, int32_t* q,
+                       float* delta, float* zero)
+{
+    oref_quantize_row_dbg(fmt, N, v, q, delta, zero, NULL);
+}
+
+/* Dequantize a row: s = (q - z) * Delta on the asymmetric grid, q * Delta on
+ * the symmetric grid.  q - z is exact in fp32 for the code and zero-point
+ * ranges that occur; the product is one rounding. */
+void oref_dequantize_row(int fmt, int N, const int32_t* q, float delta,
+                         float zero, float* out)
+{
+    for (int n = 0; n < N; ++n) {
+        if (oref_is_sym(fmt)) {
+            out[n] = (float)q[n] * delta;
+        } else {
+            float d = (float)q[n] - zero;
+            out[n] = d * delta;
+        }
+    }
+}
+
+/* Fill a logical state from an fp32 tensor S[H][P][N]: quantized rows go
+ * through the row quantizer, fp rows are stored (bf16-rounded for bf16). */
+void oref_state_from_f32(const oref_cfg* c, const float* S, oref_state* st)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state;
+    for (int h = 0; h < H; ++h) {
+        for (int p = 0; p < P; ++p) {
+            const int r = h * P + p;
+            const float* v = S + (size_t)r * N;
+            if (oref_row_is_quant(c, h)) {
+                oref_quantize_row(c->fmt, N, v, st->q + (size_t)r * N,
+                                  st->delta + r, st->zero + r);
+            } else {
+                for (int n = 0; n < N; ++n) {
+                    float s = v[n];
+                    if (c->fmt == OREF_BF16) s = oref_bf16_round(s);
+                    st->val[(size_t)r * N + n] = s;
+                }
+            }
+        }
+    }
+}
+
+/* Read a logical state back as fp32 S[H][P][N]. */
+void oref_state_to_f32(const oref_cfg* c, const oref_state* st, float* S)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state;
+    for (int h = 0; h < H; ++h) {
+        for (int p = 0; p < P; ++p) {
+            const int r = h * P + p;
+            if (oref_row_is_quant(c, h)) {
+                oref_dequantize_row(c->fmt, N, st->q + (size_t)r * N,
+                                    st->delta[r], st->zero[r],
+                                    S + (size_t)r * N);
+            } else {
+                memcpy(S + (size_t)r * N, st->val + (size_t)r * N,
+                       sizeof(float) * (size_t)N);
+            }
+        }
+    }
+}
+
+/* One decode step of one (layer, request).
+ *
+ * For every head h and row p:
+ *   1. decode the stored row;
+ *   2. lambda = exp(dt_h*A_h); dtx = dt_h*x_p; w_n = dtx*B_{g,n};
+ *      s'_n = fma(lambda, s_n, w_n)          (the Mamba-2 recurrence
+ *      S = exp(dt*A)*S + dt*B(x)x of "ssm-state-quantization", Setup, with
+ *      the FP32 update of "Mamba state quantization for inference");
+ *   3-5. refit, round and store the row (quantized heads), or store s'
+ *      (fp heads; bf16-rounded for the bf16 format);
+ *   6. y_p = sum_n C_{g,n} * stored_n + D_h*x_p, accumulated in double and
+ *      read from the newly stored state ("ssm-state-quantization", Setup:
+ *      the output is read from the quantized state).
+ * x[H][P], B/C[G][N], dt/A/D[H], y[H][P].  'pre' (optional, [H*P*N])
+ * receives fl(s'*inv) for quantized rows. */
+void oref_step(const oref_cfg* c, oref_state* st, const float* x,
+               const float* B, const float* C, const float* dt,
+               const float* A, const float* D, float* y, float* pre)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state, G = c->ngroups;
+    const int heads_per_group = H / G;
+    float* s = (float*)malloc(sizeof(float) * (size_t)N);
+    float* sn = (float*)malloc(sizeof(float) * (size_t)N);
+    float* stored = (float*)malloc(sizeof(float) * (size_t)N);
+
+    for (int h = 0; h < H; ++h) {
+        const int g = h / heads_per_group;
+        const float lam = oref_lambda(dt[h], A[h]);
+        const float* Bg = B + (size_t)g * N;
+        const float* Cg = C + (size_t)g * N;
+        const int quant = oref_row_is_quant(c, h);
+        for (int p = 0; p < P; ++p) {
+            const int r = h * P + p;
+            /* 1. decode */
+            if (quant) {
+                oref_dequantize_row(c->fmt, N, st->q + (size_t)r * N,
+                                    st->delta[r], st->zero[r], s);
+            } else {
+                memcpy(s, st->val + (size_t)r * N, sizeof(float) * (size_t)N);
+            }
+            /* 2. decay and input */
+            const float dtx = dt[h] * x[r];
+            for (int n = 0; n < N; ++n) {
+                float w = dtx * Bg[n];
+                sn[n] = fmaf(lam, s[n], w);
+            }
+            /* 3-5. refit, round, store */
+            if (quant) {
+                int32_t* qr = st->q + (size_t)r * N;
+                oref_quantize_row_dbg(c->fmt, N, sn, qr, st->delta + r,
+                                      st->zero + r,
+                                      pre ? pre + (size_t)r * N : NULL);
+                oref_dequantize_row(c->fmt, N, qr, st->delta[r], st->zero[r],
+                                    stored);
+            } else {
+                for (int n = 0; n < N; ++n) {
+                    float v = sn[n];
+                    if (c->fmt == OREF_BF16) v = oref_bf16_round(v);
+                    st->val[(size_t)r * N + n] = v;
+                    stored[n] = v;
+                }
+            }
+            /* 6. readout from the stored state */
+            double acc = 0.0;
+            for (int n = 0; n < N; ++n)
+                acc += (double)Cg[n] * (double)stored[n];
+            acc += (double)D[h] * (double)x[r];
+            y[r] = (float)acc;
+        }
+    }
+    free(s);
+    free(sn);
+    free(stored);
+}
+
+/* Per-token scan ("ssm-state-quantization", Setup: a sequential scan that
+ * rounds the state at every step): T applications of the decode step, token
+ * t+1 reading the state stored at token t.
+ * x[T][H][P], B/C[T][G][N], dt[T][H], A/D[H], y[T][H][P]. */
+void oref_scan(const oref_cfg* c, oref_state* st, int T, const float* x,
+               const float* B, const float* C, const float* dt,
+               const float* A, const float* D, float* y)
+{
+    const size_t HP = (size_t)c->nheads * c->headdim;
+    const size_t GN = (size_t)c->ngroups * c->d_state;
+    for (int t = 0; t < T; ++t) {
+        oref_step(c, st, x + t * HP, B + t * GN, C + t * GN,
+                  dt + (size_t)t * c->nheads, A, D, y + t * HP, NULL);
+    }
+}
+
+/* Unquantized trajectory in double, used only to report drift: the exact
+ * recurrence S_t = A_t S_(t-1) + W_t of "Mamba state quantization for
+ * inference" (no residual R_t), with lambda = exp(dt*A) and W = dt*B(x)x,
+ * every operation in double.  S[H][P][N] in/out. */
+void oref_scan_f64(const oref_cfg* c, double* S, int T, const float* x,
+                   const float* B, const float* C, const float* dt,
+                   const float* A, const float* D, double* y)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state, G = c->ngroups;
+    const int hpg = H / G;
+    const size_t HP = (size_t)H * P;
+    const size_t GN = (size_t)G * N;
+    for (int t = 0; t < T; ++t) {
+        for (int h = 0; h < H; ++h) {
+            const int g = h / hpg;
+            const double dtd = (double)dt[(size_t)t * H + h];
+            const double lam = exp(dtd * (double)A[h]);
+            const float* Bg = B + t * GN + (size_t)g * N;
+            const float* Cg = C + t * GN + (size_t)g * N;
+            for (int p = 0; p < P; ++p) {
+                const size_t r = (size_t)h * P + p;
+                const double xv = (double)x[t * HP + r];
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    double* sv = S + r * N + n;
+                    *sv = lam * (*sv) + dtd * xv * (double)Bg[n];
+                    acc += (double)Cg[n] * (*sv);
+                }
+                y[t * HP + r] = acc + (double)D[h] * xv;
+            }
+        }
+    }
+}
+
+/* One decode step over nl layers and a batch of requests: the same step for
+ * every (layer, request) pair.  states[l*batch + b];
+ * x/y[nl][batch][H][P], B/C[nl][batch][G][N], dt[nl][batch][H], A/D[nl][H]. */
+void oref_decode_batch(const oref_cfg* c, int nl, int batch,
+                       oref_state* states, const float* x, const float* B,
+                       const float* C, const float* dt, const float* A,
+                       const float* D, float* y)
+{
+    const size_t HP = (size_t)c->nheads * c->headdim;
+    const size_t GN = (size_t)c->ngroups * c->d_state;
+    const size_t H = (size_t)c->nheads;
+    for (int l = 0; l < nl; ++l) {
+        for (int b = 0; b < batch; ++b) {
+            const size_t lb = (size_t)l * batch + b;
+            oref_step(c, &states[lb], x + lb * HP, B + lb * GN, C + lb * GN,
+                      dt + lb * H, A + l * H, D + l * H, y + lb * HP, NULL);
+        }
+    }
+}

@@ -1,0 +1,60 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case plants one mistake in a copy of the oracle's C source (on the CPU,
+in a temporary directory), builds it, and runs the pin suite against that
+build: the suite must fail.  The mistakes are the ones a transcription of the
+pages could plausibly make: a dropped or misplaced term of the recurrence, a
+wrong sign, an off-by-one grid, a transposed group index, the wrong rounding
+rule or the wrong read point of the output.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "ssq_oracle.c")
+
+MUTATIONS = {
+    "z_sign": ("z = rintf(-lo * inv) + 0.0f;", "z = rintf(lo * inv) + 0.0f;"),
+    "asym_levels_2b": ("return (float)((1 << b) - 1);", "return (float)(1 << b);"),
+    "sym_levels_2b1": ("return (float)((1 << (b - 1)) - 1);",
+                       "return (float)(1 << (b - 1));"),
+    "no_dt_on_input": ("const float dtx = dt[h] * x[r];", "const float dtx = x[r];"),
+    "decay_not_exp": ("double e = exp((double)dA);", "double e = 1.0 + (double)dA;"),
+    "group_map": ("const int g = h / heads_per_group;",
+                  "const int g = h % G;"),
+    "round_half_away": ("float r = rintf(p);", "float r = roundf(p);"),
+    "y_before_rounding": ("acc += (double)Cg[n] * (double)stored[n];",
+                          "acc += (double)Cg[n] * (double)sn[n];"),
+    "no_skip_term": ("acc += (double)D[h] * (double)x[r];", "acc += 0.0;"),
+    "no_clamp": ("if (c > qm) c = qm;\n        }", "}"),
+    "truncate": ("float r = rintf(p);", "float r = truncf(p);"),
+    "deq_drop_zero": ("float d = (float)q[n] - zero;", "float d = (float)q[n];"),
+    "swap_B_C": ("float w = dtx * Bg[n];", "float w = dtx * Cg[n];"),
+    "constant_row_step": ("if (delta == 0.0f) delta = fabsf(lo);",
+                          "if (delta == 0.0f) delta = 1.0f;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(name):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor missing: {name}"
+    mutated = src.replace(old, new, 1)
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "ssq_oracle.c")
+        open(c, "w").write(mutated)
+        subprocess.check_call(["cp", os.path.join(ROOT, "oracle", "ssq_oracle.h"), d])
+        so = os.path.join(d, "liboref_mut.so")
+        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-std=c11",
+                               "-shared", "-fPIC", "-o", so, c, "-lm"])
+        env = dict(os.environ, SSQ_ORACLE_LIB=so)
+        r = subprocess.run(
+            [sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+             os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"
