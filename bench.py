@@ -1,0 +1,542 @@
+#!/usr/bin/env python
+"""Benchmark of libssq's quantized state update on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+A step is one pass of the decode hot path -- read the packed state, decode,
+recurrence, refit, requantize, write back, readout -- over one batch of
+synthetic input.  The default workload is the Mamba-2 130M-shaped decode
+step: 24 layers x batch 256 in one launch, 24 heads x 64 x 128 per layer,
+int8 asymmetric state, N(0, 1) initial state.  Other workloads (--workload)
+are the 8B-shaped decode, the serving-scale format sweep and the 370M-shaped
+per-token scan.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
+device synchronize, timed with CUDA events on the launching stream; the max
+over ranks is taken.  The state pool (gigabytes) is far larger than the
+126 MB L2, so the state is read from HBM every step; no L2 flush is needed.
+Multi-GPU runs are independent replicas (weak scaling, no collective on the
+data path).  --impl reference times the CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_recurrent_state_mamba_b200 import workloads as W  # noqa: E402
+
+METRIC = "quantized state-update HBM GB/s (% of B200 peak) and request-steps/s/layer"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# Workloads and their algorithmic bytes
+# ---------------------------------------------------------------------------
+
+def workload(name):
+    table = {
+        "decode_130m": lambda: W.decode_130m("i8a"),
+        "decode_130m_f32": lambda: W.decode_130m("f32"),
+        "decode_8b_b1_i8a": lambda: W.decode_8b("i8a", 1),
+        "decode_8b_b16_i8a": lambda: W.decode_8b("i8a", 16),
+        "decode_8b_b64_i8a": lambda: W.decode_8b("i8a", 64),
+        "decode_8b_b256_i8a": lambda: W.decode_8b("i8a", 256),
+        "decode_8b_b64_i8s": lambda: W.decode_8b("i8s", 64),
+        "decode_8b_b256_i8s": lambda: W.decode_8b("i8s", 256),
+        "decode_8b_b64_f32": lambda: W.decode_8b("f32", 64),
+        "decode_8b_b256_f32": lambda: W.decode_8b("f32", 256),
+        "sweep_f32": lambda: W.sweep_serving("f32"),
+        "sweep_bf16": lambda: W.sweep_serving("bf16"),
+        "sweep_i8a": lambda: W.sweep_serving("i8a"),
+        "sweep_i4a": lambda: W.sweep_serving("i4a"),
+        "scan_370m_all": lambda: W.scan_370m("all"),
+        "scan_370m_mid": lambda: W.scan_370m("mid"),
+    }
+    if name not in table:
+        raise SystemExit(f"unknown workload {name}; choose from {sorted(table)}")
+    return table[name]()
+
+
+def row_state_bytes(fmt, N):
+    """Bytes one stored row occupies (codes + metadata, or fp values)."""
+    return {"f32": 4 * N, "bf16": 2 * N, "i8s": N + 4, "i8a": N + 8,
+            "i4s": N // 2 + 4, "i4a": N // 2 + 8}[fmt]
+
+
+def decode_bytes(wl):
+    """Algorithmic bytes of one decode step: every stored row read and written
+    once (codes + metadata), x / B / C / dt read and y written once.  A and D
+    (per layer and head) are left out."""
+    rows = wl.nl * wl.batch * wl.nheads * wl.headdim
+    mask = wl.head_mask
+    if mask is not None and wl.fmt not in ("f32", "bf16"):
+        qfrac = float(np.mean(np.asarray(mask) != 0))
+    else:
+        qfrac = 1.0
+    state = rows * (qfrac * row_state_bytes(wl.fmt, wl.d_state)
+                    + (1 - qfrac) * row_state_bytes("f32", wl.d_state))
+    io = rows * 4 * 2 + wl.nl * wl.batch * (2 * wl.ngroups * wl.d_state + wl.nheads) * 4
+    return int(round(2 * state + io))
+
+
+def scan_bytes(wl):
+    """Algorithmic bytes of one scan call: inputs x / B / C / dt read and y
+    written once per token, the state read and written once."""
+    per_tok = wl.batch * (2 * wl.nheads * wl.headdim + 2 * wl.ngroups * wl.d_state
+                          + wl.nheads) * 4
+    rows = wl.batch * wl.nheads * wl.headdim
+    return int(per_tok * wl.T + 2 * rows * row_state_bytes(wl.fmt, wl.d_state))
+
+
+def elem_steps(wl):
+    if isinstance(wl, W.Scan):
+        return wl.batch * wl.T * wl.nheads * wl.headdim * wl.d_state
+    return wl.nl * wl.batch * wl.nheads * wl.headdim * wl.d_state
+
+
+# ---------------------------------------------------------------------------
+# Measured peaks, clocks, ncu traffic
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    pkg = os.path.join(ROOT, "quantized_recurrent_state_mamba_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(pkg, "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    with open(os.path.join(ROOT, "include", "ssq.h"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload_name):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary for this workload, if it was captured on the current kernel
+    sources (else None)."""
+    src = kernel_source_hash()
+    for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        kv = {}
+        with open(p) as f:
+            for line in f:
+                line = line.strip()
+                if line.startswith("- ") and ":" in line:
+                    k, v = line[2:].split(":", 1)
+                    kv[k.strip()] = v.strip().strip("`")
+        if kv.get("bench_workload") == workload_name and kv.get("source_hash") == src:
+            try:
+                return float(kv["dram_bytes_per_launch"])
+            except (KeyError, ValueError):
+                return None
+    return None
+
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event reasons through NVML in a
+    background thread (every ~5 ms) and keeps the samples taken inside a
+    marked window."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.window = None
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                uuid = None
+            h = None
+            if uuid:
+                u = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(u)
+                except Exception:
+                    h = None
+            if h is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+                idx = int(vis.split(",")[device_index]) if vis else device_index
+                h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that clocks were not sampled
+            self.err = str(e)
+
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": "NVML unavailable: " + getattr(self, "err", "")}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "samples inside the timed region"
+        if not inside:
+            # the region is shorter than the sampling period: take the
+            # samples nearest to it
+            near = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))
+            inside = near[:3]
+            note = "timed region shorter than the sampling period; nearest samples"
+        reasons = set()
+        for _, _, rs in inside:
+            for bit, name in self.REASONS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in inside) if inside else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(inside), "note": note}
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------------------
+# The CPU oracle leg (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_decode_sample(wl, budget_s):
+    """Time the CPU oracle on the first pairs of the decode workload until
+    about budget_s seconds of work; returns (seconds, bytes, pairs)."""
+    import oracle as O
+    fmt = O.FORMATS[wl.fmt]
+    H, P, N, G = wl.nheads, wl.headdim, wl.d_state, wl.ngroups
+    ocfg = O.Cfg(fmt, H, P, N, G, wl.head_mask)
+    inp = wl.inputs()
+    per_pair = decode_bytes(wl) / (wl.nl * wl.batch)
+    # calibrate on one pair
+    st = O.state_from_f32(ocfg, wl.state_pair(0, 0).reshape(1, H, P, N))
+    t = time.perf_counter()
+    O.step(ocfg, st, 0, inp["x"][0, 0], inp["B"][0, 0], inp["C"][0, 0], inp["dt"][0, 0],
+           inp["A"][0], inp["D"][0])
+    one = max(time.perf_counter() - t, 1e-6)
+    npairs = int(max(1, min(wl.nl * wl.batch, budget_s / one)))
+    pairs = [(i // wl.batch, i % wl.batch) for i in range(npairs)]
+    S0 = np.stack([wl.state_pair(l, b).reshape(H, P, N) for (l, b) in pairs])
+    st = O.state_from_f32(ocfg, S0)
+    t = time.perf_counter()
+    for i, (l, b) in enumerate(pairs):
+        O.step(ocfg, st, i, inp["x"][l, b], inp["B"][l, b], inp["C"][l, b], inp["dt"][l, b],
+               inp["A"][l], inp["D"][l])
+    sec = time.perf_counter() - t
+    return sec, per_pair * npairs, npairs
+
+
+def oracle_scan_sample(wl, budget_s):
+    import oracle as O
+    H, P, N = wl.nheads, wl.headdim, wl.d_state
+    inp = wl.inputs()
+    ocfg = O.Cfg(O.FORMATS[wl.fmt], H, P, N, wl.ngroups, wl.head_mask)
+    t = time.perf_counter()
+    st = O.State(ocfg, 1)
+    T1 = min(wl.T, 8)
+    O.scan(ocfg, st, 0, inp["x"][0, :T1], inp["B"][0, :T1], inp["C"][0, :T1],
+           inp["dt"][0, :T1], inp["A"], inp["D"])
+    per_tok = max((time.perf_counter() - t) / T1, 1e-6)
+    ntok = int(max(1, min(wl.T * wl.batch, budget_s / per_tok)))
+    st = O.State(ocfg, 1)
+    b, done = 0, 0
+    t = time.perf_counter()
+    while done < ntok:
+        n = min(wl.T, ntok - done)
+        O.scan(ocfg, st, 0, inp["x"][b, :n], inp["B"][b, :n], inp["C"][b, :n],
+               inp["dt"][b, :n], inp["A"], inp["D"])
+        done += n
+        b = (b + 1) % wl.batch
+    sec = time.perf_counter() - t
+    frac = ntok / (wl.T * wl.batch)
+    return sec, scan_bytes(wl) * frac, ntok
+
+
+def cpu_leg(wl, budget_s):
+    if isinstance(wl, W.Scan):
+        sec, nbytes, n = oracle_scan_sample(wl, budget_s)
+        sample = f"{n} request-tokens of the scan (request 0 onward), single thread"
+        rsps = n / sec
+    else:
+        sec, nbytes, n = oracle_decode_sample(wl, budget_s)
+        sample = (f"{n} of {wl.nl * wl.batch} (layer, request) pairs of one decode step "
+                  f"(layer-major from pair 0), single thread")
+        rsps = n / sec
+    return {"value": nbytes / sec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": sample, "seconds": round(sec, 3),
+            "request_steps_per_s_per_layer": rsps}
+
+
+def run_reference(args, wl, name):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    steps, warm = args.steps, args.warmup
+    budget = max(0.5, 120.0 / max(1, steps + warm))
+    for _ in range(warm):
+        cpu_leg(wl, budget)
+    vals, secs = [], 0.0
+    for _ in range(steps):
+        r = cpu_leg(wl, budget)
+        vals.append(r["value"])
+        secs += r["seconds"]
+    value = statistics.mean(vals)
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+           "n_gpus": world, "steps": steps, "warmup": warm,
+           "ms_per_step": 1000 * secs / max(1, steps), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+           "config": {"workload": wl.name, "bench_workload": name},
+           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                            "sample": r["sample"] + " per step"},
+           "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, wl, name):
+    import torch
+    import torch.distributed as dist
+    from quantized_recurrent_state_mamba_b200 import ssq
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    is_scan = isinstance(wl, W.Scan)
+    fmt = wl.fmt
+    H, P, N, G = wl.nheads, wl.headdim, wl.d_state, wl.ngroups
+    n_layers = 1 if is_scan else wl.nl
+    cfg = ssq.Config(n_layers=n_layers, n_slots=wl.batch, nheads=H, headdim=P, d_state=N,
+                     ngroups=G, fmt=fmt, head_mask=wl.head_mask)
+    pool = ssq.alloc_pool(cfg, dev)
+    inp = wl.inputs()
+    d = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in inp.items()}
+
+    # initial state
+    if not is_scan and wl.init != "zero":
+        for l in range(wl.nl):
+            S = np.empty((wl.batch, wl.rows, N), np.float32)
+            for b in range(wl.batch):
+                S[b] = wl.state_pair(l, b)
+            ssq.ssq_quantize_rows(cfg, pool, None, wl.batch, l, 1,
+                                  torch.from_numpy(S).to(dev))
+        torch.cuda.synchronize()
+
+    if is_scan:
+        y = torch.empty((wl.batch, wl.T, H, P), device=dev)
+        nbytes = scan_bytes(wl)
+
+        def step():
+            ssq.ssq_scan(cfg, pool, None, wl.batch, 0, wl.T, d["x"], d["B"], d["C"], d["dt"],
+                         d["A"], d["D"], y)
+        units = wl.batch * wl.T          # request-tokens
+    else:
+        y = torch.empty((wl.nl, wl.batch, H, P), device=dev)
+        nbytes = decode_bytes(wl)
+
+        def step():
+            ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, d["x"], d["B"], d["C"],
+                                d["dt"], d["A"], d["D"], y)
+        units = wl.batch * wl.nl         # request-layer steps
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ssq.ssq_pool_error(cfg, pool) != 0:
+        raise SystemExit("device error word set during warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.05)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(K):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    barrier()
+    sampler.stop()
+    region_ms = ev[0][0].elapsed_time(ev[-1][1])
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    kern_ms = statistics.mean(launch_ms)
+    if world > 1:
+        tt = torch.tensor([region_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        region_ms = float(tt.item())
+    value = nbytes * K * world / (region_ms / 1e3) / 1e9
+    ms_per_step = region_ms / K
+
+    # end to end: pinned host inputs in, y out, through the public API
+    h = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory()
+         for k in ("x", "B", "C", "dt")}
+    y_host = torch.empty(y.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * 4 for t in h.values())
+    d2h = y.numel() * 4
+
+    def e2e_step():
+        for k2 in ("x", "B", "C", "dt"):
+            d[k2].copy_(h[k2], non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = nbytes * K * world / (e2e_ms / 1e3) / 1e9
+    err = ssq.ssq_pool_error(cfg, pool)
+
+    peak, peak_kind = measured_peaks()
+    achieved = nbytes / (kern_ms / 1e3) / 1e9
+    traffic = ncu_traffic(name)
+    clocks = sampler.summary(t0, t1)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "bench_workload": name, "format": fmt,
+                   "layers_per_launch": n_layers, "batch_per_gpu": wl.batch,
+                   "nheads": H, "headdim": P, "d_state": N, "ngroups": G,
+                   "T": getattr(wl, "T", 1),
+                   "algorithmic_bytes_per_step": nbytes,
+                   "l2": "state pool and per-step traffic far above the 126 MB L2; no flush",
+                   "parallelism": f"replicas x{world}"},
+        "request_steps_per_s_per_layer": round(units * K * world / (region_ms / 1e3), 1),
+        "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+        "pct_of_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "peak_source": peak_kind,
+                     "kernel_ms_per_launch": round(kern_ms, 5)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5)},
+        "gpu_launches": K,
+        "clocks": clocks,
+        "device_error_word": err,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_leg(wl, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_130m")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    wl = workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl, args.workload)
+    return run_ours(args, wl, args.workload)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,246 @@
+/*
+ * ssq.h -- libssq: the Mamba-2 recurrent-state update with the per-request
+ * state stored in low-bit form, on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources are page title + section):
+ *
+ *   "ssm-state-quantization" README, Setup:
+ *     - each head decays its state by lambda = exp(dt*A) per step;
+ *     - the quantizer keeps one scale per row of the state (per head and
+ *       head_dim, over the d_state entries) and refits it every step;
+ *     - symmetric grid [-amax, amax] with step amax/(2^(b-1)-1), or
+ *       asymmetric grid [min, max] with an integer zero point and step
+ *       (max-min)/(2^b-1);
+ *     - the output is read from the quantized state;
+ *     - heads are grouped into decay bands (lambda <= 0.9, 0.9 < lambda <=
+ *       0.99, lambda > 0.99) and a band can be rounded on its own.
+ *   "ssm-state-quantization" README, Findings 1: nearest rounding (RTN).
+ *   "Mamba state quantization for inference":
+ *     - "Recurrent state is fixed per request, not free": every token reads
+ *       the state matrix, applies the recurrence and writes it back; one
+ *       state per live request;
+ *     - "Mixed precision spends bits on persistent channels": one fused
+ *       kernel reconstructs the low-precision tier, runs the recurrence in
+ *       FP32, derives new quantization parameters and writes the packed state
+ *       back; tiers sit in contiguous regions so no per-token gather is
+ *       needed;
+ *     - "Mamba state quantization needs phase-aware benchmarks": prefill
+ *       computes in FP32 and writes its final state into the packed cache.
+ *   "SSDi8: Accurate and Efficient 8-bit Quantization for State Space
+ *   Duality", 4 Methodology, State quantization: per-(H,P) state scales,
+ *   nothing along N.
+ *
+ * One step for one (layer, request, head h, row p), entries n < d_state:
+ *     s_n   = decode(stored row)                 (q - z)*Delta, q*Delta, fp
+ *     lam   = (float) exp((double)(dt_h * A_h))
+ *     s'_n  = fma(lam, s_n, (dt_h * x_p) * B_{g(h),n})        all fp32
+ *     refit Delta (and z) from s', round s'_n*inv to nearest (ties to even)
+ *     y_p   = sum_n C_{g(h),n} * decode(new row)_n + D_h * x_p
+ * with g(h) = h / (nheads/ngroups).  Quantized codes are bit-identical to a
+ * plain scalar evaluation of these formulas in that order; y is fp32 with
+ * fp32 accumulation.  A head whose mask entry is 0 keeps an fp32 row.
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions for every entry point
+ *   - Device pointers are CUDA device (or managed) memory owned by the caller;
+ *     the library never allocates, frees or synchronises except where an
+ *     entry point says so.  Every launch is asynchronous on `stream`.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and nothing is written; the call returns SSQ_ERR_INVALID_ARG,
+ *     SSQ_ERR_UNSUPPORTED or SSQ_ERR_ALIGNMENT.  A failed launch returns
+ *     SSQ_ERR_CUDA.  ssq_last_error_detail() gives a one-line reason.
+ *   - Values that live on the device (slot indices, state contents) are
+ *     checked by the kernels: a bad value sets a bit in the pool's error word
+ *     (SSQ_DEVERR_*), the affected request is skipped, and no kernel traps.
+ *     Read the word with ssq_pool_error().
+ *   - Results are deterministic: no atomics on any output.
+ *   - Two calls that write the same slot and layer must not overlap on the
+ *     GPU; one call must not name a slot twice in slot_idx.
+ * ---------------------------------------------------------------------------
+ */
+#ifndef SSQ_H
+#define SSQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols of libssq (the library is built with hidden default
+ * visibility). */
+#if defined(__GNUC__)
+#define SSQ_API __attribute__((visibility("default")))
+#else
+#define SSQ_API
+#endif
+
+#define SSQ_MAX_HEADS 512
+#define SSQ_POOL_HEADER_BYTES 256
+#define SSQ_POOL_ALIGN 256
+
+typedef enum {
+    SSQ_OK = 0,
+    SSQ_ERR_INVALID_ARG = 1, /* null pointer, bad size or index          */
+    SSQ_ERR_UNSUPPORTED = 2, /* shape or format this build does not cover */
+    SSQ_ERR_ALIGNMENT = 3,   /* pointer not aligned as documented        */
+    SSQ_ERR_CUDA = 4         /* a CUDA call or launch failed              */
+} ssq_status;
+
+/* State storage formats.  b = 8 or 4 bits per code; "sym" uses the
+ * symmetric grid, "asym" the asymmetric grid with an integer zero point. */
+typedef enum {
+    SSQ_F32 = 0,     /* fp32 state, no rounding                        */
+    SSQ_BF16 = 1,    /* bf16 state, fp32 -> bf16 round to nearest even  */
+    SSQ_I8_SYM = 2,  /* int8 two's complement codes in [-127, 127]     */
+    SSQ_I8_ASYM = 3, /* uint8 codes in [0, 255]                        */
+    SSQ_I4_SYM = 4,  /* 4-bit two's complement codes in [-7, 7]         */
+    SSQ_I4_ASYM = 5  /* 4-bit codes in [0, 15]                          */
+} ssq_format;
+
+/* Bits of the pool's device error word (SSQ_DEVERR_*). */
+#define SSQ_DEVERR_SLOT 0x1u      /* slot index outside [0, n_slots)      */
+#define SSQ_DEVERR_NONFINITE 0x2u /* a row's updated values were not finite */
+
+/* Shape of one state pool.  Every request slot holds the state of n_layers
+ * layers; each layer holds nheads x headdim rows of d_state entries.
+ *   nheads      1 .. SSQ_MAX_HEADS
+ *   headdim     >= 1
+ *   d_state     16, 32, 64, 128 or 256
+ *   ngroups     >= 1 and divides nheads; B and C are shared by the
+ *               nheads/ngroups consecutive heads of a group
+ *   head_mask   HOST array of nheads bytes, or NULL.  For the integer
+ *               formats, heads with mask 0 keep an fp32 row and are never
+ *               rounded ("ssm-state-quantization", Setup: rounding one decay
+ *               band only).  Ignored for SSQ_F32 and SSQ_BF16.  Read during
+ *               each call; the library keeps no pointer to it. */
+typedef struct {
+    int n_layers;
+    int n_slots;
+    int nheads;
+    int headdim;
+    int d_state;
+    int ngroups;
+    ssq_format fmt;
+    const uint8_t* head_mask;
+} ssq_config;
+
+/* Byte layout of a pool (all offsets in bytes).
+ *
+ *   pool = [header: SSQ_POOL_HEADER_BYTES][slot 0][slot 1] ... [slot n-1]
+ *   slot s starts at header_bytes + s*slot_bytes.  Inside a slot:
+ *     codes  at codes_off: [n_layers][n_quant_heads][headdim][row_code_bytes]
+ *     meta   at meta_off:  [n_layers][n_quant_heads][headdim][row_meta_bytes]
+ *     fp     at fp_off:    [n_layers][n_fp_heads][headdim][d_state] elements
+ *                          of fp_elem_bytes (fp32, or bf16 for SSQ_BF16)
+ *   Heads are stored in region order: the quantized heads first in increasing
+ *   head index, then the fp heads (head_perm of ssq_pool_layout).  So a
+ *   masked band is one contiguous region and no kernel gathers per token
+ *   ("Mamba state quantization for inference", mixed-precision layout).
+ *   Codes of a row: 8-bit formats store entry n in byte n; 4-bit formats store
+ *   entries 2k and 2k+1 in the low and high nibble of byte k.  Sym codes are
+ *   two's complement (int8 / 4-bit).  Meta of a row: asym {float Delta,
+ *   float z} (8 bytes), sym {float Delta} (4 bytes).
+ *   Header: uint32 error word (SSQ_DEVERR_* bits) at byte 0; the rest is
+ *   reserved.  Every region and slot starts on a SSQ_POOL_ALIGN boundary.
+ *   An all-zero pool is a valid all-zero state in every format. */
+typedef struct {
+    size_t pool_bytes;
+    size_t header_bytes;
+    size_t slot_bytes;
+    size_t codes_off, meta_off, fp_off;
+    size_t codes_layer_bytes, meta_layer_bytes, fp_layer_bytes;
+    size_t row_code_bytes, row_meta_bytes, fp_elem_bytes;
+    int n_quant_heads, n_fp_heads;
+} ssq_layout;
+
+/* Compute the pool layout for cfg.  head_perm (HOST, nheads int32, may be
+ * NULL) receives the natural head index stored at each region position.
+ * Host only; no CUDA call. */
+SSQ_API ssq_status ssq_pool_layout(const ssq_config* cfg, ssq_layout* out,
+                           int32_t* head_perm);
+
+/* Set a whole pool to the all-zero state and clear its error word
+ * (cudaMemsetAsync of layout.pool_bytes bytes).  pool: device, aligned to
+ * SSQ_POOL_ALIGN. */
+SSQ_API ssq_status ssq_pool_init(const ssq_config* cfg, void* pool,
+                         cudaStream_t stream);
+
+/* Read the pool's error word into *flags (HOST) and clear it.  This call
+ * synchronises `stream`. */
+SSQ_API ssq_status ssq_pool_error(const ssq_config* cfg, void* pool,
+                          uint32_t* flags, cudaStream_t stream);
+
+/* Write fp32 states into pool slots through the row quantizer: the prefill
+ * hand-off of "Mamba state quantization for inference" ("phase-aware
+ * benchmarks": an FP32 chunk-final state written into the packed cache), and
+ * pool initialisation.
+ *   S         device fp32 [nl][batch][nheads][headdim][d_state], natural head
+ *             order, 16-byte aligned
+ *   slot_idx  device int32 [batch]: pool slot of request b; NULL = slot b
+ *   layers    layer0 .. layer0+nl-1 of each slot are written */
+SSQ_API ssq_status ssq_quantize_rows(const ssq_config* cfg, void* pool,
+                             const int32_t* slot_idx, int batch, int layer0,
+                             int nl, const float* S, cudaStream_t stream);
+
+/* Read pool slots back as fp32 (checkpointing, tests): the inverse layout of
+ * ssq_quantize_rows, each row decoded as (q - z)*Delta, q*Delta or the fp
+ * value.  S_out: device fp32 [nl][batch][nheads][headdim][d_state]. */
+SSQ_API ssq_status ssq_dequantize_rows(const ssq_config* cfg, const void* pool,
+                               const int32_t* slot_idx, int batch,
+                               int layer0, int nl, float* S_out,
+                               cudaStream_t stream);
+
+/* One decode token for a batch of live requests over nl layers, in one
+ * launch: the fused read -> recurrence -> refit -> requantize -> write-back
+ * -> readout of "Mamba state quantization for inference" (mixed-precision
+ * section) with the quantizer of "ssm-state-quantization", Setup.  The nl
+ * layer updates are independent (a model calls nl = 1 per layer because
+ * layer l+1's input depends on layer l's output).
+ *   slot_idx  device int32 [batch] or NULL (slot b)
+ *   x         device fp32 [nl][batch][nheads][headdim]      (16-B aligned)
+ *   B, C      device fp32 [nl][batch][ngroups][d_state]     (16-B aligned)
+ *   dt        device fp32 [nl][batch][nheads], already positive (softplus
+ *             and bias applied by the caller)
+ *   A, D      device fp32 [nl][nheads]
+ *   y         device fp32 [nl][batch][nheads][headdim]      (16-B aligned)
+ * The state of layers layer0 .. layer0+nl-1 of each named slot is updated
+ * in place.  y of a request whose slot index is out of range is not
+ * written. */
+SSQ_API ssq_status ssq_decode_step(const ssq_config* cfg, void* pool,
+                           const int32_t* slot_idx, int batch, int layer0,
+                           int nl, const float* x, const float* B,
+                           const float* C, const float* dt, const float* A,
+                           const float* D, float* y, cudaStream_t stream);
+
+/* T tokens of one layer with the state rounded at every token and held on
+ * chip between tokens ("ssm-state-quantization", Setup: a sequential
+ * per-token scan in place of the chunked scan, so the state can be rounded
+ * at every step).  Equal, bit for bit in the stored codes and meta, to T
+ * calls of ssq_decode_step with nl = 1.
+ *   x   device fp32 [batch][T][nheads][headdim]     (16-B aligned)
+ *   B,C device fp32 [batch][T][ngroups][d_state]    (16-B aligned)
+ *   dt  device fp32 [batch][T][nheads]
+ *   A,D device fp32 [nheads]
+ *   y   device fp32 [batch][T][nheads][headdim]     (16-B aligned)
+ * Only the final state is written to the pool. */
+SSQ_API ssq_status ssq_scan(const ssq_config* cfg, void* pool,
+                    const int32_t* slot_idx, int batch, int layer, int T,
+                    const float* x, const float* B, const float* C,
+                    const float* dt, const float* A, const float* D,
+                    float* y, cudaStream_t stream);
+
+/* Static string for a status code. */
+SSQ_API const char* ssq_status_string(ssq_status s);
+
+/* One-line reason for the last non-OK status returned on this host thread
+ * (static thread-local storage; valid until the next call). */
+SSQ_API const char* ssq_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSQ_H */

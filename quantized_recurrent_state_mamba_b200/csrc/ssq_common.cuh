@@ -1,0 +1,435 @@
+// ssq_common.cuh -- device building blocks shared by the libssq kernels.
+//
+// The row engine below implements one step of the quantized recurrent-state
+// update for one state row (head h, head_dim index p, d_state entries), as
+// specified by "ssm-state-quantization" README, Setup (lambda = exp(dt*A);
+// one scale per (head, head_dim) row over the d_state entries, refit every
+// step; symmetric grid [-amax, amax], step amax/(2^(b-1)-1); asymmetric grid
+// [min, max], integer zero point, step (max-min)/(2^b-1); output read from
+// the quantized state) and Findings 1 (nearest rounding), with the FP32
+// update of "Mamba state quantization for inference" (mixed-precision
+// section).  Every fp32 operation that decides a stored value is a single
+// correctly rounded IEEE operation in a fixed order (the library is built
+// with -fmad=false; FMAs are explicit), so codes and metadata are identical
+// to a plain scalar evaluation of the same formulas.
+//
+// Thread mapping: a row of N entries is owned by LPR = N/E consecutive lanes
+// of a warp, each holding E consecutive entries in registers.  Row-wide
+// min/max and the C.S readout are warp-shuffle butterflies inside the group.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssq.h"
+
+namespace ssq {
+
+constexpr int kThreads = 256;
+
+// x + 1.5*2^23 rounds x (|x| < 2^22) to the nearest integer, ties to even,
+// and leaves that integer in the low mantissa bits of the sum.
+constexpr float kMagic = 12582912.0f;
+constexpr float kTwo23 = 8388608.0f;
+// Below 2^22 in magnitude the magic-number paths are exact.
+constexpr float kFastLimit = 4194304.0f;
+
+// ---------------------------------------------------------------------------
+// Format traits
+// ---------------------------------------------------------------------------
+template <int FMT>
+struct Fmt {
+    static constexpr bool quant = (FMT >= SSQ_I8_SYM);
+    static constexpr bool sym = (FMT == SSQ_I8_SYM || FMT == SSQ_I4_SYM);
+    static constexpr int bits =
+        (FMT == SSQ_I8_SYM || FMT == SSQ_I8_ASYM) ? 8
+        : (FMT == SSQ_I4_SYM || FMT == SSQ_I4_ASYM) ? 4
+        : (FMT == SSQ_BF16) ? 16 : 32;
+    // qs = 2^(b-1)-1 (sym) or qa = 2^b-1 (asym)
+    static constexpr float qmax =
+        quant ? (sym ? float((1 << (bits - 1)) - 1) : float((1 << bits) - 1))
+              : 0.0f;
+    // Sym codes are stored two's complement; flipping the sign bit of each
+    // code gives q + 2^(b-1) as an unsigned field.
+    static constexpr float bias = sym ? float(1 << (bits - 1)) : 0.0f;
+    static constexpr int meta_bytes = quant ? (sym ? 4 : 8) : 0;
+};
+
+template <int N>
+struct Shape {
+    static constexpr int E = (N >= 32) ? 32 : N;  // entries per lane
+    static constexpr int LPR = N / E;             // lanes per row
+    static constexpr int RPW = 32 / LPR;          // rows per warp
+    static_assert(N == 16 || N == 32 || N == 64 || N == 128 || N == 256,
+                  "d_state must be 16, 32, 64, 128 or 256");
+};
+
+// ---------------------------------------------------------------------------
+// Small helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float fmin3(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+template <int LPR>
+__device__ __forceinline__ float grp_min(float v)
+{
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1)
+        v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+template <int LPR>
+__device__ __forceinline__ float grp_max(float v)
+{
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+template <int LPR>
+__device__ __forceinline__ float grp_sum(float v)
+{
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1)
+        v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// lambda = exp(dt*A): the fp32 product, exponentiated in double and rounded
+// once to fp32 ("ssm-state-quantization", Setup).
+__device__ __forceinline__ float decay(float dt, float A)
+{
+    return (float)exp((double)__fmul_rn(dt, A));
+}
+
+// Vector loads / stores of a lane's contiguous chunk.
+template <int BYTES>
+struct Chunk {
+    static_assert(BYTES % 4 == 0, "chunk must be whole words");
+    uint32_t w[BYTES / 4];
+};
+
+template <int BYTES>
+__device__ __forceinline__ void load_chunk(Chunk<BYTES>& c, const void* p)
+{
+    if constexpr (BYTES % 16 == 0) {
+#pragma unroll
+        for (int i = 0; i < BYTES / 16; ++i) {
+            uint4 v = __ldcs(reinterpret_cast<const uint4*>(p) + i);
+            c.w[4 * i + 0] = v.x; c.w[4 * i + 1] = v.y;
+            c.w[4 * i + 2] = v.z; c.w[4 * i + 3] = v.w;
+        }
+    } else if constexpr (BYTES == 8) {
+        uint2 v = __ldcs(reinterpret_cast<const uint2*>(p));
+        c.w[0] = v.x; c.w[1] = v.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < BYTES / 4; ++i)
+            c.w[i] = __ldcs(reinterpret_cast<const uint32_t*>(p) + i);
+    }
+}
+
+template <int BYTES>
+__device__ __forceinline__ void store_chunk(void* p, const Chunk<BYTES>& c)
+{
+    if constexpr (BYTES % 16 == 0) {
+#pragma unroll
+        for (int i = 0; i < BYTES / 16; ++i)
+            __stcs(reinterpret_cast<uint4*>(p) + i,
+                   make_uint4(c.w[4 * i], c.w[4 * i + 1], c.w[4 * i + 2],
+                              c.w[4 * i + 3]));
+    } else if constexpr (BYTES == 8) {
+        __stcs(reinterpret_cast<uint2*>(p), make_uint2(c.w[0], c.w[1]));
+    } else {
+#pragma unroll
+        for (int i = 0; i < BYTES / 4; ++i)
+            __stcs(reinterpret_cast<uint32_t*>(p) + i, c.w[i]);
+    }
+}
+
+// E consecutive fp32 values from (cached) global memory, 16-byte vectors.
+template <int E>
+__device__ __forceinline__ void load_f32(float (&v)[E], const float* p)
+{
+    static_assert(E % 4 == 0, "");
+#pragma unroll
+    for (int i = 0; i < E / 4; ++i) {
+        float4 t = __ldg(reinterpret_cast<const float4*>(p) + i);
+        v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Code (un)packing.
+//
+// Entry n of a row: 8-bit formats keep it in byte n; 4-bit formats keep
+// entries 2k and 2k+1 in the low and high nibble of byte k.  Sym codes are
+// two's complement.  Within a lane's chunk word i holds entries 4i..4i+3
+// (8-bit) or 8i..8i+7 (4-bit).
+// ---------------------------------------------------------------------------
+
+// f[n] = 2^23 + u_n where u_n is the unsigned code field (sym: q + 2^(b-1)).
+template <int FMT, int E>
+__device__ __forceinline__ void unpack_biased(const Chunk<E * Fmt<FMT>::bits / 8>& c,
+                                              float (&f)[E])
+{
+    constexpr bool sym = Fmt<FMT>::sym;
+    constexpr uint32_t kExp = 0x4B000000u;  // bits of 2^23
+    if constexpr (Fmt<FMT>::bits == 8) {
+#pragma unroll
+        for (int i = 0; i < E / 4; ++i) {
+            const uint32_t v = sym ? (c.w[i] ^ 0x80808080u) : c.w[i];
+            f[4 * i + 0] = __uint_as_float(__byte_perm(v, kExp, 0x7540));
+            f[4 * i + 1] = __uint_as_float(__byte_perm(v, kExp, 0x7541));
+            f[4 * i + 2] = __uint_as_float(__byte_perm(v, kExp, 0x7542));
+            f[4 * i + 3] = __uint_as_float(__byte_perm(v, kExp, 0x7543));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < E / 8; ++i) {
+            const uint32_t v = sym ? (c.w[i] ^ 0x88888888u) : c.w[i];
+            const uint32_t lo = v & 0x0F0F0F0Fu;          // entries 8i+0,2,4,6
+            const uint32_t hi = (v >> 4) & 0x0F0F0F0Fu;   // entries 8i+1,3,5,7
+            f[8 * i + 0] = __uint_as_float(__byte_perm(lo, kExp, 0x7540));
+            f[8 * i + 1] = __uint_as_float(__byte_perm(hi, kExp, 0x7540));
+            f[8 * i + 2] = __uint_as_float(__byte_perm(lo, kExp, 0x7541));
+            f[8 * i + 3] = __uint_as_float(__byte_perm(hi, kExp, 0x7541));
+            f[8 * i + 4] = __uint_as_float(__byte_perm(lo, kExp, 0x7542));
+            f[8 * i + 5] = __uint_as_float(__byte_perm(hi, kExp, 0x7542));
+            f[8 * i + 6] = __uint_as_float(__byte_perm(lo, kExp, 0x7543));
+            f[8 * i + 7] = __uint_as_float(__byte_perm(hi, kExp, 0x7543));
+        }
+    }
+}
+
+// Integer codes (sign-extended for sym), for the exact slow path.
+template <int FMT, int E>
+__device__ __forceinline__ void unpack_int(const Chunk<E * Fmt<FMT>::bits / 8>& c,
+                                           int (&q)[E])
+{
+    if constexpr (Fmt<FMT>::bits == 8) {
+#pragma unroll
+        for (int n = 0; n < E; ++n) {
+            const uint32_t b = (c.w[n / 4] >> (8 * (n % 4))) & 0xFFu;
+            q[n] = Fmt<FMT>::sym ? (int)(int8_t)b : (int)b;
+        }
+    } else {
+#pragma unroll
+        for (int n = 0; n < E; ++n) {
+            const uint32_t b = (c.w[n / 8] >> (4 * (n % 8))) & 0xFu;
+            q[n] = Fmt<FMT>::sym ? (int)((b ^ 8u) - 8u) : (int)b;
+        }
+    }
+}
+
+// Pack code carriers (the code sits in the low 8 or 4 bits of each carrier)
+// into the row's byte layout.
+template <int FMT, int E>
+__device__ __forceinline__ void pack_codes(const uint32_t (&k)[E],
+                                           Chunk<E * Fmt<FMT>::bits / 8>& c)
+{
+    if constexpr (Fmt<FMT>::bits == 8) {
+#pragma unroll
+        for (int i = 0; i < E / 4; ++i) {
+            const uint32_t a = __byte_perm(k[4 * i + 0], k[4 * i + 1], 0x0040);
+            const uint32_t b = __byte_perm(k[4 * i + 2], k[4 * i + 3], 0x0040);
+            c.w[i] = __byte_perm(a, b, 0x5410);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < E / 8; ++i) {
+            const uint32_t e01 = __byte_perm(k[8 * i + 0], k[8 * i + 2], 0x0040);
+            const uint32_t e23 = __byte_perm(k[8 * i + 4], k[8 * i + 6], 0x0040);
+            const uint32_t o01 = __byte_perm(k[8 * i + 1], k[8 * i + 3], 0x0040);
+            const uint32_t o23 = __byte_perm(k[8 * i + 5], k[8 * i + 7], 0x0040);
+            const uint32_t ev = __byte_perm(e01, e23, 0x5410);
+            const uint32_t od = __byte_perm(o01, o23, 0x5410);
+            c.w[i] = (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Row decode: s_n = (q_n - z)*Delta (asym) or q_n*Delta (sym).
+// ---------------------------------------------------------------------------
+template <int FMT, int E>
+__device__ __forceinline__ void decode_row(const Chunk<E * Fmt<FMT>::bits / 8>& c,
+                                           float delta, float z, float (&s)[E])
+{
+    using F = Fmt<FMT>;
+    if (F::sym || fabsf(z) < kFastLimit) {
+        // (2^23 + u) - (2^23 + z + bias) = q - z exactly; one rounding in
+        // the product, as in the scalar formula.
+        float f[E];
+        unpack_biased<FMT, E>(c, f);
+        const float c0 = __fadd_rn(kTwo23, __fadd_rn(z, F::bias));
+        const float2 nc02 = make_float2(-c0, -c0);
+        const float2 d2 = make_float2(delta, delta);
+#pragma unroll
+        for (int n = 0; n < E; n += 2) {
+            float2 v = __fadd2_rn(make_float2(f[n], f[n + 1]), nc02);
+            v = __fmul2_rn(v, d2);
+            s[n] = v.x; s[n + 1] = v.y;
+        }
+    } else {
+        int q[E];
+        unpack_int<FMT, E>(c, q);
+#pragma unroll
+        for (int n = 0; n < E; ++n)
+            s[n] = __fmul_rn(__fsub_rn((float)q[n], z), delta);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Row refit + round.
+//
+// Given the updated row s' (E entries per lane, LPR lanes per row), compute
+// Delta, inv = 1/Delta and z, round every entry, and produce
+//   r[n]  = q_n - z as fp32 (what the stored row decodes to, before * Delta)
+//   k[n]  = a carrier whose low bits are the stored code.
+// Reading of the pages' silent points: ties to even on fl(s'*inv); z =
+// rint(-lo*inv) unclamped (negative zero stored as +0); a constant row takes
+// Delta = |lo|; Delta below FLT_MIN flushes the row to zero; asym codes
+// clamp at qa (the minimum maps to 0 by construction); the sym clamp never
+// binds because |fl(amax*inv)| rounds to qs.
+// ---------------------------------------------------------------------------
+struct RowParams {
+    float delta, inv, z;
+    bool fast;    // magic-number rounding is exact for this row
+    bool clamp;   // some entry rounds above qa (asym)
+    bool finite;
+};
+
+template <int FMT, int E, int LPR>
+__device__ __forceinline__ RowParams refit_row(const float (&s)[E])
+{
+    using F = Fmt<FMT>;
+    float lo = s[0], hi = s[0];
+#pragma unroll
+    for (int n = 1; n + 1 < E; n += 2) {
+        lo = fmin3(lo, s[n], s[n + 1]);
+        hi = fmax3(hi, s[n], s[n + 1]);
+    }
+    if constexpr (E % 2 == 0) {
+        lo = fminf(lo, s[E - 1]);
+        hi = fmaxf(hi, s[E - 1]);
+    }
+    lo = grp_min<LPR>(lo);
+    hi = grp_max<LPR>(hi);
+
+    RowParams rp;
+    rp.finite = isfinite(lo) && isfinite(hi);
+    float delta;
+    if constexpr (F::sym) {
+        const float amax = fmaxf(-lo, hi);
+        delta = __fdiv_rn(amax, F::qmax);
+    } else {
+        delta = __fdiv_rn(__fsub_rn(hi, lo), F::qmax);
+        if (delta == 0.0f) delta = fabsf(lo);
+    }
+    if (delta < 1.17549435e-38f) delta = 0.0f;  // FLT_MIN
+    const float inv = (delta == 0.0f) ? 0.0f : __frcp_rn(delta);
+    float z = 0.0f;
+    if constexpr (!F::sym) z = __fadd_rn(rintf(__fmul_rn(-lo, inv)), 0.0f);
+    const float plo = __fmul_rn(lo, inv), phi = __fmul_rn(hi, inv);
+    rp.delta = delta;
+    rp.inv = inv;
+    rp.z = z;
+    rp.fast = fmaxf(fabsf(plo), fabsf(phi)) < kFastLimit && fabsf(z) < kFastLimit;
+    rp.clamp = (!F::sym) && (__fadd_rn(rintf(phi), z) > F::qmax);
+    return rp;
+}
+
+template <int FMT, int E>
+__device__ __forceinline__ void round_row(const RowParams& rp, const float (&s)[E],
+                                          float (&r)[E], uint32_t (&k)[E])
+{
+    using F = Fmt<FMT>;
+    if (rp.fast && !rp.clamp) {
+        const float2 inv2 = make_float2(rp.inv, rp.inv);
+        const float2 m2 = make_float2(kMagic, kMagic);
+        const float2 nm2 = make_float2(-kMagic, -kMagic);
+        const float2 z2 = make_float2(rp.z, rp.z);
+#pragma unroll
+        for (int n = 0; n < E; n += 2) {
+            float2 p = __fmul2_rn(make_float2(s[n], s[n + 1]), inv2);
+            float2 t = __fadd2_rn(p, m2);            // 1.5*2^23 + rint(p)
+            float2 rr = __fadd2_rn(t, nm2);          // rint(p), exact
+            r[n] = rr.x; r[n + 1] = rr.y;
+            if constexpr (F::sym) {
+                k[n] = __float_as_uint(t.x);         // low bits: rint(p) two's complement
+                k[n + 1] = __float_as_uint(t.y);
+            } else {
+                float2 u = __fadd2_rn(t, z2);        // 1.5*2^23 + q, exact
+                k[n] = __float_as_uint(u.x);
+                k[n + 1] = __float_as_uint(u.y);
+            }
+        }
+    } else {
+        // The scalar formulas verbatim.
+#pragma unroll
+        for (int n = 0; n < E; ++n) {
+            const float rr = rintf(__fmul_rn(s[n], rp.inv));
+            float c;
+            if constexpr (F::sym) {
+                c = fminf(fmaxf(rr, -F::qmax), F::qmax);
+                r[n] = c;
+            } else {
+                c = fminf(__fadd_rn(rr, rp.z), F::qmax);
+                r[n] = __fsub_rn(c, rp.z);
+            }
+            k[n] = (uint32_t)(int)c;
+        }
+    }
+}
+
+// The stored row as fp32: fl(r_n * Delta).
+template <int E>
+__device__ __forceinline__ void scale_row(float delta, const float (&r)[E], float (&s)[E])
+{
+    const float2 d2 = make_float2(delta, delta);
+#pragma unroll
+    for (int n = 0; n < E; n += 2) {
+        float2 v = __fmul2_rn(make_float2(r[n], r[n + 1]), d2);
+        s[n] = v.x; s[n + 1] = v.y;
+    }
+}
+
+// s'_n = fma(lambda, s_n, fl(dtx * B_n)).
+template <int E>
+__device__ __forceinline__ void update_row(float lam, float dtx, const float (&Bv)[E],
+                                           float (&s)[E])
+{
+    const float2 l2 = make_float2(lam, lam);
+    const float2 x2 = make_float2(dtx, dtx);
+#pragma unroll
+    for (int n = 0; n < E; n += 2) {
+        float2 w = __fmul2_rn(x2, make_float2(Bv[n], Bv[n + 1]));
+        float2 v = __ffma2_rn(l2, make_float2(s[n], s[n + 1]), w);
+        s[n] = v.x; s[n + 1] = v.y;
+    }
+}
+
+// sum_n C_n * v_n over the lane's entries (fp32, paired accumulators).
+template <int E>
+__device__ __forceinline__ float dot_row(const float (&Cv)[E], const float (&v)[E])
+{
+    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int n = 0; n < E; n += 2)
+        acc = __ffma2_rn(make_float2(Cv[n], Cv[n + 1]), make_float2(v[n], v[n + 1]), acc);
+    return __fadd_rn(acc.x, acc.y);
+}
+
+}  // namespace ssq

@@ -1,0 +1,69 @@
+// ssq_params.h -- launch parameters shared by the host API and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssq.h"
+
+namespace ssq {
+
+// Everything a kernel needs to address one pool and one call's tensors.
+// Passed by value as a __grid_constant__ kernel parameter (< 4 KB).
+struct PoolView {
+    uint8_t* pool;             // base of the pool (header at offset 0)
+    long long header_bytes, slot_bytes;
+    long long codes_off, meta_off, fp_off;
+    long long codes_layer_bytes, meta_layer_bytes, fp_layer_bytes;
+    int n_slots, n_layers;
+    int H, P, N, G, hpg;       // heads, head_dim, d_state, groups, heads/group
+    int Hq, Hf;                // heads in the quantized / fp region
+    uint16_t perm[SSQ_MAX_HEADS];  // region position -> natural head index
+};
+
+struct CallView {
+    const int32_t* slot_idx;   // [batch] or null (identity)
+    int batch, layer0, nl;
+    int rows_per_tile;         // rows of one region handled per tile
+    int qtiles, ftiles;        // tiles per (layer, request) in each region
+    long long total_tiles;
+    int T;                     // tokens (scan only)
+    const float* x;
+    const float* B;
+    const float* C;
+    const float* dt;
+    const float* A;
+    const float* D;
+    float* y;
+    const float* S_in;         // quantize_rows input
+    float* S_out;              // dequantize_rows output
+};
+
+// Host-side launchers (one per kernel family); each returns the CUDA error of
+// its launch.  The decode and rows kernels run a grid-stride loop over tiles
+// on a grid sized to the device's resident capacity.
+cudaError_t launch_decode(const PoolView& pv, const CallView& cv, int fmt,
+                          cudaStream_t stream);
+cudaError_t launch_quantize(const PoolView& pv, const CallView& cv, int fmt,
+                            cudaStream_t stream);
+cudaError_t launch_dequantize(const PoolView& pv, const CallView& cv, int fmt,
+                              cudaStream_t stream);
+cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt,
+                        cudaStream_t stream);
+
+// Rows of one region each scan CTA owns.
+int scan_rows_per_cta(int d_state);
+
+// Grid for a grid-stride kernel: resident blocks on the current device,
+// capped by the number of tiles.
+int grid_for(const void* kernel, int threads, long long tiles);
+
+// Rows handled per tile for a given d_state (256 threads, LPR lanes per row).
+inline int rows_per_tile(int d_state)
+{
+    const int E = d_state >= 32 ? 32 : d_state;
+    const int lpr = d_state / E;
+    return 256 / lpr;
+}
+
+}  // namespace ssq

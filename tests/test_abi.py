@@ -1,0 +1,183 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol
+include/ssq.h declares, computes the documented pool layout, and rejects bad
+arguments before touching the GPU.  No compute call is made."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssq.h")
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module")
+def ssq():
+    from quantized_recurrent_state_mamba_b200 import build
+    build.build()
+    from quantized_recurrent_state_mamba_b200 import ssq as m
+    return m
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"SSQ_API\s+[\w\s\*]+?\b(ssq_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(ssq):
+    syms = declared_symbols()
+    assert len(syms) == 9, syms
+    lib = ctypes.CDLL(ssq.LIB_PATH)
+    for s in syms:
+        assert hasattr(lib, s), f"libssq.so does not export {s}"
+
+
+def test_status_strings(ssq):
+    assert ssq.ssq_status_string(0) == "SSQ_OK"
+    assert ssq.ssq_status_string(4) == "SSQ_ERR_CUDA"
+
+
+def _layout(ssq, **kw):
+    return ssq.ssq_pool_layout(ssq.Config(**kw))
+
+
+def expected_slot_bytes(fmt, L, H, P, N, mask=None):
+    """Bytes per slot from the header's description, computed here."""
+    quant = fmt in ("i8s", "i8a", "i4s", "i4a")
+    hq = (sum(1 for m in mask if m) if mask is not None else H) if quant else 0
+    hf = H - hq
+    b = {"i8s": 8, "i8a": 8, "i4s": 4, "i4a": 4}.get(fmt, 0)
+    meta = {"i8s": 4, "i4s": 4, "i8a": 8, "i4a": 8}.get(fmt, 0)
+    eb = 2 if fmt == "bf16" else 4
+    up = lambda v: (v + 255) // 256 * 256
+    codes = L * hq * P * N * b // 8
+    metab = L * hq * P * meta
+    fp = L * hf * P * N * eb
+    return up(up(up(codes) + metab) + fp) if True else None
+
+
+@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8s", "i8a", "i4s", "i4a"])
+@pytest.mark.parametrize("shape", [(24, 24, 64, 128, 1), (1, 128, 64, 128, 8),
+                                   (30, 32, 128, 128, 1), (1, 2, 8, 16, 1), (3, 5, 7, 32, 5)])
+def test_layout_matches_documentation(ssq, fmt, shape):
+    L, H, P, N, G = shape
+    d, perm = _layout(ssq, n_layers=L, n_slots=3, nheads=H, headdim=P, d_state=N,
+                      ngroups=G, fmt=fmt)
+    assert d["header_bytes"] == 256
+    assert d["slot_bytes"] == expected_slot_bytes(fmt, L, H, P, N)
+    assert d["pool_bytes"] == 256 + 3 * d["slot_bytes"]
+    for k in ("codes_off", "meta_off", "fp_off", "slot_bytes"):
+        assert d[k] % 256 == 0
+    # regions do not overlap
+    assert d["codes_off"] + L * d["codes_layer_bytes"] <= d["meta_off"]
+    assert d["meta_off"] + L * d["meta_layer_bytes"] <= d["fp_off"]
+    assert d["fp_off"] + L * d["fp_layer_bytes"] <= d["slot_bytes"]
+    assert perm == list(range(H))
+
+
+def test_mask_regions(ssq):
+    mask = [0, 1, 1, 0, 1]
+    d, perm = _layout(ssq, n_layers=2, n_slots=1, nheads=5, headdim=4, d_state=16,
+                      fmt="i4a", head_mask=mask)
+    assert d["n_quant_heads"] == 3 and d["n_fp_heads"] == 2
+    assert perm == [1, 2, 4, 0, 3]
+    assert d["slot_bytes"] == expected_slot_bytes("i4a", 2, 5, 4, 16, mask)
+    # the mask is ignored by the fp formats
+    d2, perm2 = _layout(ssq, n_layers=2, n_slots=1, nheads=5, headdim=4, d_state=16,
+                        fmt="f32", head_mask=mask)
+    assert d2["n_quant_heads"] == 0 and perm2 == list(range(5))
+
+
+def _golden_pool_sizes():
+    vals = {}
+    for line in open(os.path.join(GOLDEN, "state_pool_sizes.txt")):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            k, v = line.split("=")
+            vals[k.strip()] = float(v)
+    return vals
+
+
+def test_fp32_pool_matches_page_figure(ssq):
+    """The serving-scale fp32 pool (30 layers, 32 heads x 128 x 128, batch
+    256) is the 15 GB, ~60 MB per request that "Mamba state quantization for
+    inference" reports ("Recurrent state is fixed per request, not free")."""
+    g = _golden_pool_sizes()
+    d, _ = _layout(ssq, n_layers=30, n_slots=256, nheads=32, headdim=128, d_state=128,
+                   fmt="f32")
+    per_req = d["slot_bytes"]
+    total = d["pool_bytes"] - d["header_bytes"]
+    assert abs(total / 2 ** 30 - g["pool_gib_batch256"]) / g["pool_gib_batch256"] < 0.01
+    assert abs(per_req / 1e6 - g["mb_per_request"]) / g["mb_per_request"] < 0.06
+    # proportional estimates the page gives at batch 32 and 96
+    assert abs(32 * per_req / 1e9 - g["gb_batch32"]) / g["gb_batch32"] < 0.12
+    assert abs(96 * per_req / 1e9 - g["gb_batch96"]) / g["gb_batch96"] < 0.12
+    # bits per value of the quantized formats, metadata included
+    for fmt, bpv in (("i8a", 8.5), ("i8s", 8.25), ("i4a", 4.5), ("i4s", 4.25), ("bf16", 16)):
+        dq, _ = _layout(ssq, n_layers=30, n_slots=1, nheads=32, headdim=128, d_state=128,
+                        fmt=fmt)
+        assert abs(dq["slot_bytes"] * 8 / (30 * 32 * 128 * 128) - bpv) < 1e-3
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d_state=48), 2), (dict(d_state=0), 2), (dict(nheads=0), 2),
+    (dict(nheads=513), 2), (dict(ngroups=3), 1), (dict(n_layers=0), 1),
+    (dict(n_slots=0), 1), (dict(headdim=0), 1), (dict(fmt=9), 1)])
+def test_layout_rejects_bad_configs(ssq, kw, status):
+    base = dict(n_layers=2, n_slots=4, nheads=8, headdim=16, d_state=64, ngroups=2, fmt="i8a")
+    base.update(kw)
+    with pytest.raises(ssq.SsqError) as e:
+        ssq.ssq_pool_layout(ssq.Config(**base))
+    assert e.value.status == status
+
+
+def test_entry_points_validate_before_launch(ssq):
+    """Bad pointers, sizes and ranges are rejected on the host: the calls
+    return an argument status without any CUDA call (no GPU here)."""
+    lib = ssq.raw()
+    cfg = ssq.Config(n_layers=2, n_slots=4, nheads=4, headdim=8, d_state=32, fmt="i8a")
+    P = ctypes.c_void_p
+    good = 0x10000000
+    args = dict(pool=good, slots=None, batch=2, layer0=0, nl=1, x=good, B=good, C=good,
+                dt=good, A=good, D=good, y=good)
+
+    def call(**over):
+        a = dict(args, **over)
+        return lib.ssq_decode_step(cfg.ref, P(a["pool"]), P(a["slots"]), a["batch"],
+                                   a["layer0"], a["nl"], P(a["x"]), P(a["B"]), P(a["C"]),
+                                   P(a["dt"]), P(a["A"]), P(a["D"]), P(a["y"]), None)
+
+    assert call(pool=good + 16) == ssq.SSQ_ERR_ALIGNMENT
+    assert call(pool=0) == ssq.SSQ_ERR_INVALID_ARG
+    assert call(x=good + 4) == ssq.SSQ_ERR_ALIGNMENT
+    assert call(y=0) == ssq.SSQ_ERR_INVALID_ARG
+    assert call(dt=good + 2) == ssq.SSQ_ERR_ALIGNMENT
+    assert call(batch=-1) == ssq.SSQ_ERR_INVALID_ARG
+    assert call(batch=5) == ssq.SSQ_ERR_INVALID_ARG        # > n_slots, identity slots
+    assert call(layer0=1, nl=2) == ssq.SSQ_ERR_INVALID_ARG
+    assert call(nl=0) == ssq.SSQ_ERR_INVALID_ARG
+    assert call(slots=good + 2) == ssq.SSQ_ERR_ALIGNMENT
+    assert "aligned" in ssq.ssq_last_error_detail()
+    # an empty batch is a no-op that succeeds without a launch
+    assert call(batch=0) == ssq.SSQ_OK
+    r = lib.ssq_scan(cfg.ref, P(good), None, 2, 0, -1, P(good), P(good), P(good), P(good),
+                     P(good), P(good), P(good), None)
+    assert r == ssq.SSQ_ERR_INVALID_ARG
+    r = lib.ssq_scan(cfg.ref, P(good), None, 2, 2, 4, P(good), P(good), P(good), P(good),
+                     P(good), P(good), P(good), None)
+    assert r == ssq.SSQ_ERR_INVALID_ARG                      # layer out of range
+    r = lib.ssq_quantize_rows(cfg.ref, P(good), None, 2, 0, 1, P(good + 8), None)
+    assert r == ssq.SSQ_ERR_ALIGNMENT
+
+
+def test_no_cpu_fallback_in_product(ssq):
+    """The product modules neither import nor name the oracle."""
+    pkg = os.path.join(ROOT, "quantized_recurrent_state_mamba_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f
+                assert "oref_" not in src, f
