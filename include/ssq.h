@@ -104,6 +104,7 @@ typedef enum {
 /* Bits of the pool's device error word (SSQ_DEVERR_*). */
 #define SSQ_DEVERR_SLOT 0x1u      /* slot index outside [0, n_slots)      */
 #define SSQ_DEVERR_NONFINITE 0x2u /* a row's updated values were not finite */
+#define SSQ_DEVERR_TIMEOUT 0x4u   /* a pipeline wait gave up (about 1 s)    */
 
 /* Shape of one state pool.  Every request slot holds the state of n_layers
  * layers; each layer holds nheads x headdim rows of d_state entries.
@@ -131,11 +132,14 @@ typedef struct {
 /* Byte layout of a pool (all offsets in bytes).
  *
  *   pool = [header: SSQ_POOL_HEADER_BYTES][slot 0][slot 1] ... [slot n-1]
- *   slot s starts at header_bytes + s*slot_bytes.  Inside a slot:
- *     codes  at codes_off: [n_layers][n_quant_heads][headdim][row_code_bytes]
- *     meta   at meta_off:  [n_layers][n_quant_heads][headdim][row_meta_bytes]
- *     fp     at fp_off:    [n_layers][n_fp_heads][headdim][d_state] elements
- *                          of fp_elem_bytes (fp32, or bf16 for SSQ_BF16)
+ *   slot s starts at header_bytes + s*slot_bytes.  Inside a slot, layer l's
+ *   block of each region starts at region_off + l*region_layer_bytes:
+ *     codes  at codes_off: [n_quant_heads][headdim][row_code_bytes]
+ *     meta   at meta_off:  [n_quant_heads][headdim][row_meta_bytes]
+ *     fp     at fp_off:    [n_fp_heads][headdim][d_state] elements of
+ *                          fp_elem_bytes (fp32, or bf16 for SSQ_BF16)
+ *   and the *_layer_bytes strides are those sizes rounded up to
+ *   SSQ_POOL_ALIGN.
  *   Heads are stored in region order: the quantized heads first in increasing
  *   head index, then the fp heads (head_perm of ssq_pool_layout).  So a
  *   masked band is one contiguous region and no kernel gathers per token

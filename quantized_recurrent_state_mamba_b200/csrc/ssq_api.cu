@@ -82,9 +82,11 @@ ssq_status layout_of(const ssq_config* cfg, ssq_layout* L, int32_t* perm)
     L->row_code_bytes = q ? Nz * bits_of(cfg->fmt) / 8 : 0;
     L->row_meta_bytes = q ? (is_sym(cfg->fmt) ? 4 : 8) : 0;
     L->fp_elem_bytes = cfg->fmt == SSQ_BF16 ? 2 : 4;
-    L->codes_layer_bytes = (size_t)hq * P * L->row_code_bytes;
-    L->meta_layer_bytes = (size_t)hq * P * L->row_meta_bytes;
-    L->fp_layer_bytes = (size_t)hf * P * Nz * L->fp_elem_bytes;
+    // each layer's block starts on a SSQ_POOL_ALIGN boundary (bulk copies
+    // need 16-byte aligned sources)
+    L->codes_layer_bytes = round_up((size_t)hq * P * L->row_code_bytes, SSQ_POOL_ALIGN);
+    L->meta_layer_bytes = round_up((size_t)hq * P * L->row_meta_bytes, SSQ_POOL_ALIGN);
+    L->fp_layer_bytes = round_up((size_t)hf * P * Nz * L->fp_elem_bytes, SSQ_POOL_ALIGN);
     L->codes_off = 0;
     L->meta_off = round_up(L->codes_off + Ly * L->codes_layer_bytes, SSQ_POOL_ALIGN);
     L->fp_off = round_up(L->meta_off + Ly * L->meta_layer_bytes, SSQ_POOL_ALIGN);
@@ -124,6 +126,7 @@ ssq_status make_pool_view(const ssq_config* cfg, void* pool, ssq::PoolView* pv,
     pv->hpg = cfg->nheads / cfg->ngroups;
     pv->Hq = L->n_quant_heads;
     pv->Hf = L->n_fp_heads;
+    pv->neg_zero = -0.0f;
     for (int i = 0; i < cfg->nheads; ++i) pv->perm[i] = (uint16_t)perm[i];
     return SSQ_OK;
 }

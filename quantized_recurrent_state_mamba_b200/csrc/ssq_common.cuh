@@ -66,6 +66,40 @@ struct Shape {
 };
 
 // ---------------------------------------------------------------------------
+// Packed fp32 pairs (f32x2, sm_100a).  Written as PTX with an explicit
+// round-to-nearest modifier: an instruction with an explicit rounding mode is
+// never contracted with a neighbour into a fused multiply-add, so a product
+// followed by an add stays two roundings, as the scalar definition has it.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned long long pk(float2 a)
+{
+    return ((unsigned long long)__float_as_uint(a.y) << 32) | __float_as_uint(a.x);
+}
+__device__ __forceinline__ float2 upk(unsigned long long v)
+{
+    return make_float2(__uint_as_float((unsigned)(v & 0xffffffffull)),
+                       __uint_as_float((unsigned)(v >> 32)));
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)));
+    return upk(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b)
+{
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)));
+    return upk(d);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)), "l"(pk(c)));
+    return upk(d);
+}
+
+// ---------------------------------------------------------------------------
 // Small helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float fmin3(float a, float b, float c)
@@ -278,8 +312,8 @@ __device__ __forceinline__ void decode_row(const Chunk<E * Fmt<FMT>::bits / 8>& 
         const float2 d2 = make_float2(delta, delta);
 #pragma unroll
         for (int n = 0; n < E; n += 2) {
-            float2 v = __fadd2_rn(make_float2(f[n], f[n + 1]), nc02);
-            v = __fmul2_rn(v, d2);
+            float2 v = add2(make_float2(f[n], f[n + 1]), nc02);
+            v = mul2(v, d2);
             s[n] = v.x; s[n + 1] = v.y;
         }
     } else {
@@ -351,27 +385,35 @@ __device__ __forceinline__ RowParams refit_row(const float (&s)[E])
     return rp;
 }
 
+// `nz` is -0.0f read from kernel parameters.  The product fl(s*inv) is
+// formed as fma(s, inv, nz): an FMA result is never fused again, so the magic
+// add that follows sees the rounded product.  (A packed multiply followed by
+// a packed add can be contracted into one FMA by the toolchain even with
+// explicit rounding modifiers, which would round the exact product instead.)
+// Adding -0 is exact for every product, and the compiler cannot fold away a
+// zero it cannot see.
 template <int FMT, int E>
 __device__ __forceinline__ void round_row(const RowParams& rp, const float (&s)[E],
-                                          float (&r)[E], uint32_t (&k)[E])
+                                          float (&r)[E], uint32_t (&k)[E], float nz)
 {
     using F = Fmt<FMT>;
     if (rp.fast && !rp.clamp) {
+        const float2 nz2 = make_float2(nz, nz);
         const float2 inv2 = make_float2(rp.inv, rp.inv);
         const float2 m2 = make_float2(kMagic, kMagic);
         const float2 nm2 = make_float2(-kMagic, -kMagic);
         const float2 z2 = make_float2(rp.z, rp.z);
 #pragma unroll
         for (int n = 0; n < E; n += 2) {
-            float2 p = __fmul2_rn(make_float2(s[n], s[n + 1]), inv2);
-            float2 t = __fadd2_rn(p, m2);            // 1.5*2^23 + rint(p)
-            float2 rr = __fadd2_rn(t, nm2);          // rint(p), exact
+            float2 p = fma2(make_float2(s[n], s[n + 1]), inv2, nz2);
+            float2 t = add2(p, m2);            // 1.5*2^23 + rint(p)
+            float2 rr = add2(t, nm2);          // rint(p), exact
             r[n] = rr.x; r[n + 1] = rr.y;
             if constexpr (F::sym) {
                 k[n] = __float_as_uint(t.x);         // low bits: rint(p) two's complement
                 k[n + 1] = __float_as_uint(t.y);
             } else {
-                float2 u = __fadd2_rn(t, z2);        // 1.5*2^23 + q, exact
+                float2 u = add2(t, z2);        // 1.5*2^23 + q, exact
                 k[n] = __float_as_uint(u.x);
                 k[n + 1] = __float_as_uint(u.y);
             }
@@ -401,7 +443,7 @@ __device__ __forceinline__ void scale_row(float delta, const float (&r)[E], floa
     const float2 d2 = make_float2(delta, delta);
 #pragma unroll
     for (int n = 0; n < E; n += 2) {
-        float2 v = __fmul2_rn(make_float2(r[n], r[n + 1]), d2);
+        float2 v = mul2(make_float2(r[n], r[n + 1]), d2);
         s[n] = v.x; s[n + 1] = v.y;
     }
 }
@@ -415,8 +457,8 @@ __device__ __forceinline__ void update_row(float lam, float dtx, const float (&B
     const float2 x2 = make_float2(dtx, dtx);
 #pragma unroll
     for (int n = 0; n < E; n += 2) {
-        float2 w = __fmul2_rn(x2, make_float2(Bv[n], Bv[n + 1]));
-        float2 v = __ffma2_rn(l2, make_float2(s[n], s[n + 1]), w);
+        float2 w = mul2(x2, make_float2(Bv[n], Bv[n + 1]));
+        float2 v = fma2(l2, make_float2(s[n], s[n + 1]), w);
         s[n] = v.x; s[n + 1] = v.y;
     }
 }
@@ -428,7 +470,7 @@ __device__ __forceinline__ float dot_row(const float (&Cv)[E], const float (&v)[
     float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int n = 0; n < E; n += 2)
-        acc = __ffma2_rn(make_float2(Cv[n], Cv[n + 1]), make_float2(v[n], v[n + 1]), acc);
+        acc = fma2(make_float2(Cv[n], Cv[n + 1]), make_float2(v[n], v[n + 1]), acc);
     return __fadd_rn(acc.x, acc.y);
 }
 

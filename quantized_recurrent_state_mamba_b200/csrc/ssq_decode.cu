@@ -137,7 +137,7 @@ decode_kernel(const __grid_constant__ PoolView pv,
                 const RowParams rp = refit_row<FMT, E, LPR>(s);
                 float rq[E];
                 uint32_t k[E];
-                round_row<FMT, E>(rp, s, rq, k);
+                round_row<FMT, E>(rp, s, rq, k, pv.neg_zero);
                 pack_codes<FMT, E>(k, c);
                 float Cv[E];
                 load_f32<E>(Cv, Cp);

@@ -18,6 +18,7 @@ struct PoolView {
     int n_slots, n_layers;
     int H, P, N, G, hpg;       // heads, head_dim, d_state, groups, heads/group
     int Hq, Hf;                // heads in the quantized / fp region
+    float neg_zero;            // -0.0f, opaque to the compiler (see round_row)
     uint16_t perm[SSQ_MAX_HEADS];  // region position -> natural head index
 };
 

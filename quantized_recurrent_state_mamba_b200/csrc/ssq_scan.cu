@@ -247,7 +247,7 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
                     rp = refit_row<FMT, E, LPR>(s);
                     finite_all = finite_all && rp.finite;
                     float rq[E];
-                    round_row<FMT, E>(rp, s, rq, kfin);
+                    round_row<FMT, E>(rp, s, rq, kfin, pv.neg_zero);
                     scale_row<E>(rp.delta, rq, s);
                 }
             } else if constexpr (kBf16) {

@@ -29,6 +29,7 @@ FORMATS = {"f32": SSQ_F32, "bf16": SSQ_BF16, "i8s": SSQ_I8_SYM, "i8a": SSQ_I8_AS
            "i4s": SSQ_I4_SYM, "i4a": SSQ_I4_ASYM}
 SSQ_DEVERR_SLOT = 0x1
 SSQ_DEVERR_NONFINITE = 0x2
+SSQ_DEVERR_TIMEOUT = 0x4
 SSQ_MAX_HEADS = 512
 SSQ_POOL_HEADER_BYTES = 256
 

@@ -52,10 +52,10 @@ def expected_slot_bytes(fmt, L, H, P, N, mask=None):
     meta = {"i8s": 4, "i4s": 4, "i8a": 8, "i4a": 8}.get(fmt, 0)
     eb = 2 if fmt == "bf16" else 4
     up = lambda v: (v + 255) // 256 * 256
-    codes = L * hq * P * N * b // 8
-    metab = L * hq * P * meta
-    fp = L * hf * P * N * eb
-    return up(up(up(codes) + metab) + fp) if True else None
+    codes = L * up(hq * P * N * b // 8)
+    metab = L * up(hq * P * meta)
+    fp = L * up(hf * P * N * eb)
+    return up(up(up(codes) + metab) + fp)
 
 
 @pytest.mark.parametrize("fmt", ["f32", "bf16", "i8s", "i8a", "i4s", "i4a"])
