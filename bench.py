@@ -447,28 +447,58 @@ def run_ours(args, wl, name):
     value = nbytes * K * world / (region_ms / 1e3) / 1e9
     ms_per_step = region_ms / K
 
-    # end to end: pinned host inputs in, y out, through the public API
-    h = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory()
-         for k in ("x", "B", "C", "dt")}
-    y_host = torch.empty(y.shape, dtype=torch.float32).pin_memory()
+    # End to end through the public API: every step copies that step's inputs
+    # from pinned host memory and reads its result y back.  Copies in, the
+    # kernel and the copy out run on three streams with double-buffered
+    # device inputs and outputs, so step i's copies overlap steps i-1 and
+    # i+1's work, as a serving loop would run them.
+    keys = ("x", "B", "C", "dt")
+    h = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory() for k in keys}
+    din = [{k: torch.empty_like(d[k]) for k in keys} for _ in range(2)]
+    yb = [torch.empty_like(y) for _ in range(2)]
+    yh = [torch.empty(y.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    s_in, s_c, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_c = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
     h2d = sum(t.numel() * 4 for t in h.values())
     d2h = y.numel() * 4
 
-    def e2e_step():
-        for k2 in ("x", "B", "C", "dt"):
-            d[k2].copy_(h[k2], non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
+    def e2e_step(i):
+        kk = i & 1
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_c[kk])
+            for k2 in keys:
+                din[kk][k2].copy_(h[k2], non_blocking=True)
+            ev_in[kk].record(s_in)
+        s_c.wait_event(ev_in[kk])
+        if i >= 2:
+            s_c.wait_event(ev_out[kk])
+        t = din[kk]
+        if is_scan:
+            ssq.ssq_scan(cfg, pool, None, wl.batch, 0, wl.T, t["x"], t["B"], t["C"], t["dt"],
+                         d["A"], d["D"], yb[kk], stream=s_c)
+        else:
+            ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, t["x"], t["B"], t["C"],
+                                t["dt"], d["A"], d["D"], yb[kk], stream=s_c)
+        ev_c[kk].record(s_c)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_c[kk])
+            yh[kk].copy_(yb[kk], non_blocking=True)
+            ev_out[kk].record(s_out)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    for i in range(max(3, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    s_c.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(K):
+        e2e_step(i)
+    e1.record(s_out)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
@@ -477,6 +507,7 @@ def run_ours(args, wl, name):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e2e_ms = float(tt.item())
     e2e_value = nbytes * K * world / (e2e_ms / 1e3) / 1e9
+    e2e_launches = K
     err = ssq.ssq_pool_error(cfg, pool)
 
     peak, peak_kind = measured_peaks()
@@ -504,7 +535,9 @@ def run_ours(args, wl, name):
                      "traffic": traffic, "peak_source": peak_kind,
                      "kernel_ms_per_launch": round(kern_ms, 5)},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5)},
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5),
+                "note": "pinned host inputs in and y out every step; copies overlap "
+                        "neighbouring steps' kernels (three streams, double buffers)"},
         "gpu_launches": K,
         "clocks": clocks,
         "device_error_word": err,

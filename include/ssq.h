@@ -109,7 +109,7 @@ typedef enum {
 /* Shape of one state pool.  Every request slot holds the state of n_layers
  * layers; each layer holds nheads x headdim rows of d_state entries.
  *   nheads      1 .. SSQ_MAX_HEADS
- *   headdim     >= 1
+ *   headdim     1 .. 2048
  *   d_state     16, 32, 64, 128 or 256
  *   ngroups     >= 1 and divides nheads; B and C are shared by the
  *               nheads/ngroups consecutive heads of a group

@@ -54,6 +54,8 @@ ssq_status layout_of(const ssq_config* cfg, ssq_layout* L, int32_t* perm)
     if (cfg->nheads < 1 || cfg->nheads > SSQ_MAX_HEADS)
         return fail(SSQ_ERR_UNSUPPORTED, "nheads %d outside [1, %d]", cfg->nheads, SSQ_MAX_HEADS);
     if (cfg->headdim < 1) return fail(SSQ_ERR_INVALID_ARG, "headdim %d < 1", cfg->headdim);
+    if (cfg->headdim > 2048)
+        return fail(SSQ_ERR_UNSUPPORTED, "headdim %d > 2048", cfg->headdim);
     const int N = cfg->d_state;
     if (N != 16 && N != 32 && N != 64 && N != 128 && N != 256)
         return fail(SSQ_ERR_UNSUPPORTED, "d_state %d not in {16,32,64,128,256}", N);
@@ -127,6 +129,8 @@ ssq_status make_pool_view(const ssq_config* cfg, void* pool, ssq::PoolView* pv,
     pv->Hq = L->n_quant_heads;
     pv->Hf = L->n_fp_heads;
     pv->neg_zero = -0.0f;
+    pv->mP = ssq::fdiv_magic(pv->P);
+    pv->mHpg = ssq::fdiv_magic(pv->hpg);
     for (int i = 0; i < cfg->nheads; ++i) pv->perm[i] = (uint16_t)perm[i];
     return SSQ_OK;
 }
@@ -314,7 +318,10 @@ ssq_status ssq_decode_step(const ssq_config* cfg, void* pool, const int32_t* slo
     cv.A = A;
     cv.D = D;
     cv.y = y;
-    fill_tiles(pv, &cv, ssq::rows_per_tile(cfg->d_state));
+    if (!ssq::decode_fits(cfg->d_state, cfg->nheads, cfg->ngroups))
+        return fail(SSQ_ERR_UNSUPPORTED, "ngroups*d_state %d too large for the decode kernel",
+                    cfg->ngroups * cfg->d_state);
+    fill_tiles(pv, &cv, ssq::decode_rows_per_tile(cfg->d_state));
     cudaError_t e = ssq::launch_decode(pv, cv, (int)cfg->fmt, stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return SSQ_OK;

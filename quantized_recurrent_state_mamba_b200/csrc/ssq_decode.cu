@@ -9,11 +9,19 @@
 // parameters, and writes the packed state back"), with the quantizer of
 // "ssm-state-quantization" README, Setup.
 //
-// Work decomposition: a tile is up to rows_per_tile consecutive rows of one
-// region (quantized or fp) of one (layer, request); tiles are distributed
-// over a grid-stride loop.  A row is owned by LPR lanes (E entries each).
-// The decay lambda of each head in a tile is computed once (exp in double)
-// and shared through shared memory.
+// Structure (persistent, warp-specialised, two CTAs per SM):
+//   - work is a sequence of tiles (up to RPT rows of one region of one
+//     (layer, request)); each CTA owns a contiguous range of that sequence;
+//   - a producer warp streams each tile's packed rows and metadata from HBM
+//     into a ring of shared-memory stages with bulk asynchronous copies
+//     (cp.async.bulk, completion counted in bytes on an mbarrier) and the
+//     tile's x values with cp.async; once per (layer, request, region)
+//     "unit" it stages B, C, dt, A, D into one of two unit buffers;
+//   - 8 consumer warps compute from shared memory and store the new rows,
+//     metadata and y straight to global memory;
+//   - every wait is bounded: a wait that runs out sets SSQ_DEVERR_TIMEOUT in
+//     the pool's error word and the CTA winds down (the producer first waits
+//     for its own copies in flight).
 #include "ssq_common.cuh"
 #include "ssq_params.h"
 
@@ -21,126 +29,417 @@ namespace ssq {
 
 namespace {
 
-template <int N>
-struct TileHeads {
-    static constexpr int RPT = kThreads / Shape<N>::LPR;
-    static constexpr int kMax = RPT + 2;
-};
+constexpr int kCWarps = 7;  // + 1 producer: 8-warp CTAs, two per SM
+constexpr int kCThreads = kCWarps * 32;
+constexpr int kDThreads = kCThreads + 32;
+constexpr int kMaxStages = 8;
+constexpr long long kWaitLimit = 2000000000LL;  // clock cycles, about one second
 
-// Per-tile bookkeeping, identical in every thread of the block.
-struct Tile {
-    int l, b, slot;
-    bool quant;      // quantized region
-    int rbase;       // first region row of the tile
-    int nrows;       // rows in the region (Hq*P or Hf*P)
-    int hr0;         // first region head touched by the tile
-};
-
-__device__ __forceinline__ Tile make_tile(const PoolView& pv, const CallView& cv,
-                                          long long t)
+// ---- PTX wrappers -------------------------------------------------------
+__device__ __forceinline__ unsigned saddr(const void* p)
 {
-    Tile tl;
-    const int per_lb = cv.qtiles + cv.ftiles;
-    const long long lb = t / per_lb;
-    const int k = (int)(t - lb * per_lb);
-    tl.l = (int)(lb / cv.batch);
-    tl.b = (int)(lb - (long long)tl.l * cv.batch);
-    tl.quant = k < cv.qtiles;
-    const int kk = tl.quant ? k : k - cv.qtiles;
-    tl.rbase = kk * cv.rows_per_tile;
-    tl.nrows = (tl.quant ? pv.Hq : pv.Hf) * pv.P;
-    tl.hr0 = tl.rbase / pv.P;
-    tl.slot = cv.slot_idx ? __ldg(cv.slot_idx + tl.b) : tl.b;
-    return tl;
+    return (unsigned)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, unsigned bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(saddr(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, unsigned parity)
+{
+    unsigned ok;
+    asm volatile("{\n .reg .pred p;\n"
+                 " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+                 " selp.u32 %0, 1, 0, p;\n}\n"
+                 : "=r"(ok) : "r"(saddr(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Wait for the phase of the given parity to complete; false after about a
+// second without progress.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, unsigned parity)
+{
+    if (mbar_try(b, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try(b, parity))
+        if (clock64() - t0 > kWaitLimit) return false;
+    return true;
+}
+// Bulk copy global -> shared; completion counted in bytes on `bar`.
+// Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(saddr(dst)), "l"(src), "r"(bytes), "r"(saddr(bar)) : "memory");
+}
+__device__ __forceinline__ void cpa4(void* dst, const void* src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(saddr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa16(void* dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr(dst)), "l"(src) : "memory");
+}
+// The mbarrier's current phase also waits for this thread's earlier cp.async.
+__device__ __forceinline__ void cpa_arrive(uint64_t* b)
+{
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(saddr(b)) : "memory");
+}
+
+__host__ __device__ inline int r16(int v) { return (v + 15) & ~15; }
+
+// ---- tile sequence -----------------------------------------------------
+// Tiles are ordered (layer, request, region, row block).  A CTA walks a
+// contiguous range of them with counters (one division at the start).
+struct TileWalk {
+    long long lb;   // layer * batch + request
+    int l, b, k;    // k: tile within (layer, request)
+    bool quant;
+    int rbase, n;   // first region row, rows in this tile
+    long long key;  // unit key: (lb, region)
+
+    __device__ __forceinline__ void fill(const PoolView& pv, const CallView& cv)
+    {
+        quant = k < cv.qtiles;
+        rbase = (quant ? k : k - cv.qtiles) * cv.rows_per_tile;
+        const int nrows = (quant ? pv.Hq : pv.Hf) * pv.P;
+        n = min(cv.rows_per_tile, nrows - rbase);
+        key = lb * 2 + (quant ? 0 : 1);
+    }
+    __device__ __forceinline__ void start(const PoolView& pv, const CallView& cv, long long t)
+    {
+        const int per_lb = cv.qtiles + cv.ftiles;
+        lb = t / per_lb;
+        k = (int)(t - lb * per_lb);
+        l = (int)(lb / cv.batch);
+        b = (int)(lb - (long long)l * cv.batch);
+        fill(pv, cv);
+    }
+    __device__ __forceinline__ void next(const PoolView& pv, const CallView& cv)
+    {
+        if (++k == cv.qtiles + cv.ftiles) {
+            k = 0;
+            ++lb;
+            if (++b == cv.batch) {
+                b = 0;
+                ++l;
+            }
+        }
+        fill(pv, cv);
+    }
+};
+
+// ---- shared-memory geometry (host and device agree on it) --------------
+struct DecodeGeom {
+    int S;            // stages
+    int RPT;          // rows per tile
+    int x_bytes;      // x area of a stage
+    int qcodes_bytes; // codes area of a quantized tile
+    int pay_bytes;    // payload area of a stage
+    int stage_bytes;
+    int ub_B, ub_C, ub_dt, ub_A, ub_D, unit_bytes;  // unit buffer layout
+    int Hpad;         // floats per lambda array
+    int off_units, off_lam, off_stages, smem_bytes;
+};
+
+__host__ __device__ inline DecodeGeom decode_geom(int S, int RPT, int RB, int MB, int fpEB,
+                                                  bool has_fp, int N, int H, int G)
+{
+    DecodeGeom g;
+    g.S = S;
+    g.RPT = RPT;
+    g.x_bytes = r16(RPT * 4);
+    g.qcodes_bytes = r16(RPT * RB);
+    const int qpay = g.qcodes_bytes + r16(RPT * MB);
+    const int fpay = has_fp ? RPT * N * fpEB : 0;
+    g.pay_bytes = qpay > fpay ? qpay : fpay;
+    g.stage_bytes = g.x_bytes + g.pay_bytes;
+    g.Hpad = (H + 3) & ~3;
+    g.ub_B = 16;  // 16-byte header: slot, bad flag
+    g.ub_C = g.ub_B + G * N * 4;
+    g.ub_dt = g.ub_C + G * N * 4;
+    g.ub_A = g.ub_dt + g.Hpad * 4;
+    g.ub_D = g.ub_A + g.Hpad * 4;
+    g.unit_bytes = r16(g.ub_D + g.Hpad * 4);
+    const int bars = r16((2 * kMaxStages + 4) * 8);
+    g.off_units = bars;
+    g.off_lam = g.off_units + 2 * g.unit_bytes;
+    g.off_stages = r16(g.off_lam + kCWarps * 2 * g.Hpad * 4);
+    g.smem_bytes = g.off_stages + S * g.stage_bytes;
+    return g;
 }
 
 template <int FMT, int N>
-__global__ void __launch_bounds__(kThreads)
-decode_kernel(const __grid_constant__ PoolView pv,
-              const __grid_constant__ CallView cv)
+__global__ void __launch_bounds__(kDThreads, 2)
+decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv,
+              const __grid_constant__ DecodeGeom geo)
 {
-    using S = Shape<N>;
+    using Sh = Shape<N>;
     using F = Fmt<FMT>;
-    constexpr int E = S::E, LPR = S::LPR;
-    constexpr int CB = F::quant ? E * F::bits / 8 : 4;  // code bytes per lane
+    constexpr int E = Sh::E, LPR = Sh::LPR;
     constexpr bool kBf16 = (FMT == SSQ_BF16);
+    constexpr int RB = F::quant ? N * F::bits / 8 : 0;      // code bytes per row
+    constexpr int CB = F::quant ? E * F::bits / 8 : 16;     // code bytes per lane
+    constexpr int MB = F::meta_bytes;
+    constexpr int FEB = kBf16 ? 2 : 4;                       // fp element bytes
+    constexpr int CPL = E / 4;                               // B/C 16-byte chunks per lane
 
-    __shared__ float s_lam[TileHeads<N>::kMax];
-    __shared__ float s_dt[TileHeads<N>::kMax];
-
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    uint64_t* ufull = empty + kMaxStages;
+    uint64_t* uempty = ufull + 2;
     uint32_t* err = reinterpret_cast<uint32_t*>(pv.pool);
-    const int tid = threadIdx.x;
-    const int grow = tid / LPR;     // row within the tile
-    const int j = tid % LPR;        // lane within the row group
-    const int P = pv.P, H = pv.H, G = pv.G;
 
-    for (long long t = blockIdx.x; t < cv.total_tiles; t += gridDim.x) {
-        const Tile tl = make_tile(pv, cv, t);
-        if (tl.slot < 0 || tl.slot >= pv.n_slots) {
-            if (tid == 0) atomicOr(err, SSQ_DEVERR_SLOT);
-            continue;  // block-uniform
+    const int S = geo.S;
+    const int H = pv.H, P = pv.P, G = pv.G;
+    const long long total = cv.total_tiles;
+    const long long t0 = total * blockIdx.x / gridDim.x;
+    const long long t1 = total * (blockIdx.x + 1) / gridDim.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kCWarps);
         }
-        const long long lb = (long long)tl.l * cv.batch + tl.b;
-        const int layer = cv.layer0 + tl.l;
-        const int regbase = tl.quant ? 0 : pv.Hq;
-
-        // lambda and dt of every head this tile touches
-        const int hr_last = min((tl.rbase + cv.rows_per_tile - 1) / P,
-                                tl.nrows / P - 1);
-        if (tid <= hr_last - tl.hr0) {
-            const int h = pv.perm[regbase + tl.hr0 + tid];
-            const float dtv = __ldg(cv.dt + lb * H + h);
-            const float Av = __ldg(cv.A + (long long)tl.l * H + h);
-            s_dt[tid] = dtv;
-            s_lam[tid] = decay(dtv, Av);
+        for (int u = 0; u < 2; ++u) {
+            mbar_init(&ufull[u], 1);
+            mbar_init(&uempty[u], kCWarps);
         }
-        __syncthreads();
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
 
-        const int r = tl.rbase + grow;
-        const bool active = r < tl.nrows;
-        const int rr = active ? r : tl.rbase;     // inactive rows shadow a real one
-        const int hrl = rr / P;
+    uint8_t* const units = smem + geo.off_units;
+    uint8_t* const stages = smem + geo.off_stages;
+
+    if (warp == kCWarps) {
+        // ================= producer warp =================
+        int k = 0, uk = -1;
+        long long prev = -1;
+        bool bad = false, ok = true;
+        int slot = 0;
+        TileWalk ti;
+        ti.start(pv, cv, t0);
+        for (long long t = t0; t < t1; ++t, ti.next(pv, cv)) {
+            const int regbase = ti.quant ? 0 : pv.Hq;
+            if (ti.key != prev) {
+                prev = ti.key;
+                ++uk;
+                const int u = uk & 1;
+                if (!mbar_wait(&uempty[u], ((uk >> 1) & 1) ^ 1)) { ok = false; break; }
+                slot = cv.slot_idx ? __ldg(cv.slot_idx + ti.b) : ti.b;
+                bad = slot < 0 || slot >= pv.n_slots;
+                uint8_t* ub = units + u * geo.unit_bytes;
+                if (lane == 0) {
+                    reinterpret_cast<int*>(ub)[0] = slot;
+                    reinterpret_cast<int*>(ub)[1] = bad ? 1 : 0;
+                    if (bad) atomicOr(err, SSQ_DEVERR_SLOT);
+                }
+                if (!bad) {
+                    // B and C in 16-byte chunks; in quantized units chunk i
+                    // of lane j goes to slot (i + j) mod CPL of that lane, so
+                    // the lanes of a row read distinct banks
+                    float* dB = reinterpret_cast<float*>(ub + geo.ub_B);
+                    float* dC = reinterpret_cast<float*>(ub + geo.ub_C);
+                    const float* sB = cv.B + ti.lb * G * N;
+                    const float* sC = cv.C + ti.lb * G * N;
+                    for (int m = lane; m < G * N / 4; m += 32) {
+                        int pos = m;
+                        if (ti.quant) {
+                            const int gi = m / (N / 4), mm = m - gi * (N / 4);
+                            const int jj = mm / CPL, ii = mm - jj * CPL;
+                            pos = gi * (N / 4) + jj * CPL + ((ii + jj) & (CPL - 1));
+                        }
+                        cpa16(dB + 4 * pos, sB + 4 * m);
+                        cpa16(dC + 4 * pos, sC + 4 * m);
+                    }
+                    float* ddt = reinterpret_cast<float*>(ub + geo.ub_dt);
+                    float* dA = reinterpret_cast<float*>(ub + geo.ub_A);
+                    float* dD = reinterpret_cast<float*>(ub + geo.ub_D);
+                    for (int h = lane; h < H; h += 32) {
+                        cpa4(ddt + h, cv.dt + ti.lb * H + h);
+                        cpa4(dA + h, cv.A + (long long)ti.l * H + h);
+                        cpa4(dD + h, cv.D + (long long)ti.l * H + h);
+                    }
+                }
+                cpa_arrive(&ufull[u]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ufull[u]);
+            }
+            if (bad) continue;
+            const int s = k % S;
+            if (!mbar_wait(&empty[s], ((k / S) & 1) ^ 1)) { ok = false; break; }
+            uint8_t* st = stages + s * geo.stage_bytes;
+            float* sx = reinterpret_cast<float*>(st);
+            for (int i = lane; i < ti.n; i += 32) {
+                const int rr = ti.rbase + i;
+                const int hr = fdiv(rr, pv.mP);
+                const int hh = pv.perm[regbase + hr];
+                cpa4(sx + i, cv.x + (ti.lb * H + hh) * P + (rr - hr * P));
+            }
+            cpa_arrive(&full[s]);
+            __syncwarp();
+            if (lane == 0) {
+                const int layer = cv.layer0 + ti.l;
+                const uint8_t* sb = pv.pool + pv.header_bytes + (long long)slot * pv.slot_bytes;
+                uint8_t* pay = st + geo.x_bytes;
+                if (F::quant && ti.quant) {
+                    const uint8_t* csrc = sb + pv.codes_off + (long long)layer * pv.codes_layer_bytes
+                                          + (long long)ti.rbase * RB;
+                    const uint8_t* msrc = sb + pv.meta_off + (long long)layer * pv.meta_layer_bytes
+                                          + (long long)ti.rbase * MB;
+                    const unsigned cb = (unsigned)r16(ti.n * RB), mb = (unsigned)r16(ti.n * MB);
+                    mbar_arrive_tx(&full[s], cb + mb);
+                    bulk_g2s(pay, csrc, cb, &full[s]);
+                    bulk_g2s(pay + geo.qcodes_bytes, msrc, mb, &full[s]);
+                } else {
+                    const uint8_t* fsrc = sb + pv.fp_off + (long long)layer * pv.fp_layer_bytes
+                                          + (long long)ti.rbase * N * FEB;
+                    const unsigned fb = (unsigned)(ti.n * N * FEB);
+                    mbar_arrive_tx(&full[s], fb);
+                    bulk_g2s(pay, fsrc, fb, &full[s]);
+                }
+            }
+            ++k;
+        }
+        if (!ok && lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
+        // No copy may still be writing shared memory when the CTA exits.
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if (lane == 0) {
+            for (int jj = (k > S ? k - S : 0); jj < k; ++jj)
+                mbar_wait(&full[jj % S], (jj / S) & 1);
+        }
+        return;
+    }
+
+    // ================= consumer warps =================
+    const int ct = threadIdx.x;
+    const int grow = ct / LPR;
+    const int j = ct % LPR;
+    int k = 0, uk = -1;
+    long long prev = -1;
+    bool bad = false;
+    int slot = 0;
+    const uint8_t* ub = units;
+    float* lam = nullptr;
+
+    TileWalk ti;
+    ti.start(pv, cv, t0);
+    for (long long t = t0; t < t1; ++t, ti.next(pv, cv)) {
+        if (ti.key != prev) {
+            if (uk >= 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&uempty[uk & 1]);
+            }
+            prev = ti.key;
+            ++uk;
+            const int u = uk & 1;
+            if (!mbar_wait(&ufull[u], (uk >> 1) & 1)) {
+                if (lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
+                break;
+            }
+            ub = units + u * geo.unit_bytes;
+            slot = reinterpret_cast<const int*>(ub)[0];
+            bad = reinterpret_cast<const int*>(ub)[1] != 0;
+            lam = reinterpret_cast<float*>(smem + geo.off_lam) + (warp * 2 + u) * geo.Hpad;
+            if (!bad) {
+                const float* udt = reinterpret_cast<const float*>(ub + geo.ub_dt);
+                const float* uA = reinterpret_cast<const float*>(ub + geo.ub_A);
+                for (int h = lane; h < H; h += 32) lam[h] = decay(udt[h], uA[h]);
+                __syncwarp();
+            }
+        }
+        if (bad) continue;
+        const int s = k % S;
+        if (!mbar_wait(&full[s], (k / S) & 1)) {
+            if (lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
+            break;
+        }
+        const uint8_t* st = stages + s * geo.stage_bytes;
+        const float* sx = reinterpret_cast<const float*>(st);
+        const uint8_t* pay = st + geo.x_bytes;
+        const int regbase = ti.quant ? 0 : pv.Hq;
+        const bool active = grow < ti.n;
+        const int rl = active ? grow : 0;          // inactive rows shadow row 0
+        const int rr = ti.rbase + rl;
+        const int hrl = fdiv(rr, pv.mP);
         const int p = rr - hrl * P;
         const int h = pv.perm[regbase + hrl];
-        const int g = h / pv.hpg;
-        const float lam = s_lam[hrl - tl.hr0];
-        const float dtv = s_dt[hrl - tl.hr0];
-        const float xv = __ldg(cv.x + lb * H * P + (long long)h * P + p);
-        const float Dv = __ldg(cv.D + (long long)tl.l * H + h);
+        const int g = fdiv(h, pv.mHpg);
+        const float xv = sx[rl];
+        const float lamv = lam[h];
+        const float dtv = reinterpret_cast<const float*>(ub + geo.ub_dt)[h];
+        const float Dv = reinterpret_cast<const float*>(ub + geo.ub_D)[h];
         const float dtx = __fmul_rn(dtv, xv);
-        const float* Bp = cv.B + (lb * G + g) * N + j * E;
-        const float* Cp = cv.C + (lb * G + g) * N + j * E;
-        uint8_t* slot_base = pv.pool + pv.header_bytes + (long long)tl.slot * pv.slot_bytes;
+        const float* gB = reinterpret_cast<const float*>(ub + geo.ub_B) + g * N;
+        const float* gC = reinterpret_cast<const float*>(ub + geo.ub_C) + g * N;
+        const int layer = cv.layer0 + ti.l;
+        uint8_t* sb = pv.pool + pv.header_bytes + (long long)slot * pv.slot_bytes;
+        float ysum = 0.0f;
+        bool done = false;
 
-        float Bv[E], s[E];
-        load_f32<E>(Bv, Bp);
-
-        float ysum;
         if constexpr (F::quant) {
-            if (tl.quant) {
-                uint8_t* crow = slot_base + pv.codes_off + (long long)layer * pv.codes_layer_bytes
-                                + (long long)rr * (N * F::bits / 8) + j * CB;
-                uint8_t* mrow = slot_base + pv.meta_off + (long long)layer * pv.meta_layer_bytes
-                                + (long long)rr * F::meta_bytes;
+            if (ti.quant) {
+                done = true;
                 Chunk<CB> c;
-                load_chunk<CB>(c, crow);
-                float delta0, z0 = 0.0f;
-                if constexpr (F::sym) {
-                    delta0 = __ldcs(reinterpret_cast<const float*>(mrow));
+                const uint8_t* cs = pay + rl * RB + j * CB;
+                if constexpr (CB % 16 == 0) {
+#pragma unroll
+                    for (int i = 0; i < CB / 16; ++i) {
+                        const uint4 v = reinterpret_cast<const uint4*>(cs)[i];
+                        c.w[4 * i] = v.x; c.w[4 * i + 1] = v.y; c.w[4 * i + 2] = v.z; c.w[4 * i + 3] = v.w;
+                    }
                 } else {
-                    const float2 m = __ldcs(reinterpret_cast<const float2*>(mrow));
+#pragma unroll
+                    for (int i = 0; i < CB / 8; ++i) {
+                        const uint2 v = reinterpret_cast<const uint2*>(cs)[i];
+                        c.w[2 * i] = v.x; c.w[2 * i + 1] = v.y;
+                    }
+                }
+                float delta0, z0 = 0.0f;
+                const uint8_t* ms = pay + geo.qcodes_bytes + rl * MB;
+                if constexpr (F::sym) {
+                    delta0 = *reinterpret_cast<const float*>(ms);
+                } else {
+                    const float2 m = *reinterpret_cast<const float2*>(ms);
                     delta0 = m.x;
                     z0 = m.y;
                 }
+                float s[E];
                 decode_row<FMT, E>(c, delta0, z0, s);
-                update_row<E>(lam, dtx, Bv, s);
+                {
+                    float Bv[E];
+#pragma unroll
+                    for (int i = 0; i < CPL; ++i) {
+                        const int pos = j * CPL + ((i + j) & (CPL - 1));
+                        const float4 v = reinterpret_cast<const float4*>(gB)[pos];
+                        Bv[4 * i] = v.x; Bv[4 * i + 1] = v.y; Bv[4 * i + 2] = v.z; Bv[4 * i + 3] = v.w;
+                    }
+                    update_row<E>(lamv, dtx, Bv, s);
+                }
                 const RowParams rp = refit_row<FMT, E, LPR>(s);
                 float rq[E];
-                uint32_t k[E];
-                round_row<FMT, E>(rp, s, rq, k, pv.neg_zero);
-                pack_codes<FMT, E>(k, c);
+                {
+                    uint32_t kk[E];
+                    round_row<FMT, E>(rp, s, rq, kk, pv.neg_zero);
+                    pack_codes<FMT, E>(kk, c);
+                }
                 float Cv[E];
-                load_f32<E>(Cv, Cp);
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) {
+                    const int pos = j * CPL + ((i + j) & (CPL - 1));
+                    const float4 v = reinterpret_cast<const float4*>(gC)[pos];
+                    Cv[4 * i] = v.x; Cv[4 * i + 1] = v.y; Cv[4 * i + 2] = v.z; Cv[4 * i + 3] = v.w;
+                }
                 if (rp.fast && !rp.clamp) {
                     // y = Delta * sum_n C_n (q_n - z): the stored row read back
                     ysum = __fmul_rn(rp.delta, grp_sum<LPR>(dot_row<E>(Cv, rq)));
@@ -150,8 +449,12 @@ decode_kernel(const __grid_constant__ PoolView pv,
                     ysum = grp_sum<LPR>(dot_row<E>(Cv, sv));
                 }
                 if (active) {
+                    uint8_t* crow = sb + pv.codes_off + (long long)layer * pv.codes_layer_bytes
+                                    + (long long)rr * RB + j * CB;
                     store_chunk<CB>(crow, c);
                     if (j == 0) {
+                        uint8_t* mrow = sb + pv.meta_off + (long long)layer * pv.meta_layer_bytes
+                                        + (long long)rr * MB;
                         if constexpr (F::sym) {
                             __stcs(reinterpret_cast<float*>(mrow), rp.delta);
                         } else {
@@ -162,57 +465,113 @@ decode_kernel(const __grid_constant__ PoolView pv,
                 }
             }
         }
-        if (!F::quant || !tl.quant) {
-            // fp row: fp32 state (bf16 for the bf16 format)
-            constexpr int EB = kBf16 ? 2 : 4;
-            uint8_t* frow = slot_base + pv.fp_off + (long long)layer * pv.fp_layer_bytes
-                            + ((long long)rr * N + j * E) * EB;
+        if (!done) {
+            // fp row (fp32, or bf16 for the bf16 format).  Lane j owns the
+            // 16-byte storage chunks LPR*c + j of its row, so the lanes of a
+            // row touch consecutive chunks (no bank conflicts on B and C).
+            constexpr int EPC = 16 / FEB;           // elements per chunk
+            constexpr int NCH = E / EPC;            // chunks per lane
+            const uint8_t* fs = pay + (long long)rl * N * FEB;
+            float s[E];
+            uint32_t w[E * FEB / 4];
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                const uint4 v = reinterpret_cast<const uint4*>(fs)[LPR * c + j];
+                w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+            }
             if constexpr (kBf16) {
-                Chunk<E * 2> c;
-                load_chunk<E * 2>(c, frow);
 #pragma unroll
                 for (int n = 0; n < E; ++n)
-                    s[n] = __uint_as_float((c.w[n / 2] >> (16 * (n % 2))) << 16);
-                update_row<E>(lam, dtx, Bv, s);
+                    s[n] = __uint_as_float((w[n / 2] >> (16 * (n % 2))) << 16);
+            } else {
+#pragma unroll
+                for (int n = 0; n < E; ++n) s[n] = __uint_as_float(w[n]);
+            }
+            float Bv[E], Cv[E];
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+#pragma unroll
+                for (int q = 0; q < EPC / 4; ++q) {
+                    const int ch = (LPR * c + j) * (EPC / 4) + q;
+                    const float4 vb = reinterpret_cast<const float4*>(gB)[ch];
+                    const float4 vc = reinterpret_cast<const float4*>(gC)[ch];
+                    const int o = c * EPC + 4 * q;
+                    Bv[o] = vb.x; Bv[o + 1] = vb.y; Bv[o + 2] = vb.z; Bv[o + 3] = vb.w;
+                    Cv[o] = vc.x; Cv[o + 1] = vc.y; Cv[o + 2] = vc.z; Cv[o + 3] = vc.w;
+                }
+            }
+            update_row<E>(lamv, dtx, Bv, s);
+            if constexpr (kBf16) {
 #pragma unroll
                 for (int n = 0; n < E; n += 2) {
                     const __nv_bfloat16 a = __float2bfloat16_rn(s[n]);
                     const __nv_bfloat16 b2 = __float2bfloat16_rn(s[n + 1]);
-                    c.w[n / 2] = (uint32_t)__bfloat16_as_ushort(a)
-                                 | ((uint32_t)__bfloat16_as_ushort(b2) << 16);
+                    w[n / 2] = (uint32_t)__bfloat16_as_ushort(a)
+                               | ((uint32_t)__bfloat16_as_ushort(b2) << 16);
                     s[n] = __bfloat162float(a);
                     s[n + 1] = __bfloat162float(b2);
                 }
-                if (active) store_chunk<E * 2>(frow, c);
             } else {
-                Chunk<E * 4> c;
-                load_chunk<E * 4>(c, frow);
 #pragma unroll
-                for (int n = 0; n < E; ++n) s[n] = __uint_as_float(c.w[n]);
-                update_row<E>(lam, dtx, Bv, s);
-#pragma unroll
-                for (int n = 0; n < E; ++n) c.w[n] = __float_as_uint(s[n]);
-                if (active) store_chunk<E * 4>(frow, c);
+                for (int n = 0; n < E; ++n) w[n] = __float_as_uint(s[n]);
             }
-            float Cv[E];
-            load_f32<E>(Cv, Cp);
             ysum = grp_sum<LPR>(dot_row<E>(Cv, s));
+            if (active) {
+                uint8_t* frow = sb + pv.fp_off + (long long)layer * pv.fp_layer_bytes
+                                + (long long)rr * N * FEB;
+#pragma unroll
+                for (int c = 0; c < NCH; ++c)
+                    __stcs(reinterpret_cast<uint4*>(frow) + (LPR * c + j),
+                           make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]));
+            }
         }
         if (active && j == 0) {
             const float yv = __fadd_rn(ysum, __fmul_rn(Dv, xv));
-            __stcs(cv.y + lb * H * P + (long long)h * P + p, yv);
+            __stcs(cv.y + (ti.lb * H + h) * P + p, yv);
         }
-        __syncthreads();  // s_lam / s_dt are rewritten by the next tile
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        ++k;
     }
 }
 
 template <int FMT, int N>
 cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
 {
+    using F = Fmt<FMT>;
+    constexpr int E = Shape<N>::E;
+    constexpr int LPR = N / E;
+    constexpr int RPT = kCThreads / LPR;
+    constexpr int RB = F::quant ? N * F::bits / 8 : 0;
+    const bool has_fp = pv.Hf > 0;
+    const int fpEB = FMT == SSQ_BF16 ? 2 : 4;
+    // stages: as many as fit a budget that leaves room for two CTAs per SM
+    const int budget = 110 * 1024;
+    DecodeGeom g = decode_geom(2, RPT, RB, F::meta_bytes, fpEB, has_fp, N, pv.H, pv.G);
+    int S = (budget - g.off_stages) / g.stage_bytes;
+    if (S > kMaxStages) S = kMaxStages;
+    if (S < 2) S = 2;
+    g = decode_geom(S, RPT, RB, F::meta_bytes, fpEB, has_fp, N, pv.H, pv.G);
+    if (g.smem_bytes > 227 * 1024) return cudaErrorInvalidConfiguration;
     auto kern = decode_kernel<FMT, N>;
-    const int grid = grid_for((const void*)kern, kThreads, cv.total_tiles);
-    if (grid <= 0) return cudaErrorInvalidConfiguration;
-    kern<<<grid, kThreads, 0, st>>>(pv, cv);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         g.smem_bytes);
+    if (e != cudaSuccess) return e;
+    // ask for the largest shared-memory carveout so two CTAs fit per SM
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, occ = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kDThreads,
+                                                           g.smem_bytes)) != cudaSuccess)
+        return e;
+    if (occ < 1) return cudaErrorInvalidConfiguration;
+    long long grid = (long long)sms * occ;
+    if (grid > cv.total_tiles) grid = cv.total_tiles;
+    kern<<<(int)grid, kDThreads, g.smem_bytes, st>>>(pv, cv, g);
     return cudaGetLastError();
 }
 
@@ -230,6 +589,22 @@ cudaError_t launch_fmt(const PoolView& pv, const CallView& cv, cudaStream_t st)
 }
 
 }  // namespace
+
+int decode_rows_per_tile(int d_state)
+{
+    const int E = d_state >= 32 ? 32 : d_state;
+    return kCThreads / (d_state / E);
+}
+
+bool decode_fits(int d_state, int nheads, int ngroups)
+{
+    // B and C of every group plus the lambda arrays must leave room for two
+    // pipeline stages within one CTA's shared memory
+    const int E = d_state >= 32 ? 32 : d_state;
+    const int rpt = kCThreads / (d_state / E);
+    const DecodeGeom g = decode_geom(2, rpt, d_state, 8, 4, true, d_state, nheads, ngroups);
+    return g.smem_bytes <= 227 * 1024;
+}
 
 cudaError_t launch_decode(const PoolView& pv, const CallView& cv, int fmt,
                           cudaStream_t st)

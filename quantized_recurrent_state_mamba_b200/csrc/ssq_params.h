@@ -19,6 +19,9 @@ struct PoolView {
     int H, P, N, G, hpg;       // heads, head_dim, d_state, groups, heads/group
     int Hq, Hf;                // heads in the quantized / fp region
     float neg_zero;            // -0.0f, opaque to the compiler (see round_row)
+    // n / P and h / hpg as (n * m) >> 32 with m = floor(2^32 / d) + 1: exact
+    // for n < 2^32 / d (row and head indices are far below that)
+    unsigned long long mP, mHpg;
     uint16_t perm[SSQ_MAX_HEADS];  // region position -> natural head index
 };
 
@@ -52,12 +55,25 @@ cudaError_t launch_dequantize(const PoolView& pv, const CallView& cv, int fmt,
 cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt,
                         cudaStream_t stream);
 
-// Rows of one region each scan CTA owns.
+// Rows of one region each scan CTA owns; rows per decode tile.
 int scan_rows_per_cta(int d_state);
+int decode_rows_per_tile(int d_state);
+// Whether the decode kernel's per-unit shared memory (B and C of every group,
+// per-head arrays) fits one CTA.
+bool decode_fits(int d_state, int nheads, int ngroups);
 
 // Grid for a grid-stride kernel: resident blocks on the current device,
 // capped by the number of tiles.
 int grid_for(const void* kernel, int threads, long long tiles);
+
+__host__ __device__ inline int fdiv(int n, unsigned long long m)
+{
+    return (int)(((unsigned long long)(unsigned)n * m) >> 32);
+}
+inline unsigned long long fdiv_magic(int d)
+{
+    return (1ull << 32) / (unsigned long long)d + 1ull;
+}
 
 // Rows handled per tile for a given d_state (256 threads, LPR lanes per row).
 inline int rows_per_tile(int d_state)
