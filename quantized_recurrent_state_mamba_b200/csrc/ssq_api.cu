@@ -318,10 +318,10 @@ ssq_status ssq_decode_step(const ssq_config* cfg, void* pool, const int32_t* slo
     cv.A = A;
     cv.D = D;
     cv.y = y;
-    if (!ssq::decode_fits(cfg->d_state, cfg->nheads, cfg->ngroups))
+    if (!ssq::decode_fits((int)cfg->fmt, cfg->d_state, cfg->nheads, cfg->ngroups))
         return fail(SSQ_ERR_UNSUPPORTED, "ngroups*d_state %d too large for the decode kernel",
                     cfg->ngroups * cfg->d_state);
-    fill_tiles(pv, &cv, ssq::decode_rows_per_tile(cfg->d_state));
+    fill_tiles(pv, &cv, ssq::decode_rows_per_tile((int)cfg->fmt, cfg->d_state));
     cudaError_t e = ssq::launch_decode(pv, cv, (int)cfg->fmt, stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return SSQ_OK;

@@ -66,38 +66,12 @@ struct Shape {
 };
 
 // ---------------------------------------------------------------------------
-// Packed fp32 pairs (f32x2, sm_100a).  Written as PTX with an explicit
-// round-to-nearest modifier: an instruction with an explicit rounding mode is
-// never contracted with a neighbour into a fused multiply-add, so a product
-// followed by an add stays two roundings, as the scalar definition has it.
+// Packed fp32 pairs (f32x2, sm_100a): one instruction for two lanes of work,
+// each component rounded like the scalar operation.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ unsigned long long pk(float2 a)
-{
-    return ((unsigned long long)__float_as_uint(a.y) << 32) | __float_as_uint(a.x);
-}
-__device__ __forceinline__ float2 upk(unsigned long long v)
-{
-    return make_float2(__uint_as_float((unsigned)(v & 0xffffffffull)),
-                       __uint_as_float((unsigned)(v >> 32)));
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b)
-{
-    unsigned long long d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)));
-    return upk(d);
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b)
-{
-    unsigned long long d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)));
-    return upk(d);
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
-{
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)), "l"(pk(c)));
-    return upk(d);
-}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 // ---------------------------------------------------------------------------
 // Small helpers
@@ -295,6 +269,87 @@ __device__ __forceinline__ void pack_codes(const uint32_t (&k)[E],
 }
 
 // ---------------------------------------------------------------------------
+// 16-entry pieces of a lane's codes (4 words of 8-bit codes, 2 words of
+// 4-bit codes), for kernels that stream a row through registers.
+// ---------------------------------------------------------------------------
+template <int FMT>
+struct Piece {
+    static constexpr int words = 16 * Fmt<FMT>::bits / 32;  // 4 or 2
+};
+
+// f[n] = 2^23 + u_n for the 16 entries held in w[0 .. words).
+template <int FMT>
+__device__ __forceinline__ void unpack16_biased(const uint32_t* w, float (&f)[16])
+{
+    constexpr bool sym = Fmt<FMT>::sym;
+    constexpr uint32_t kExp = 0x4B000000u;
+    if constexpr (Fmt<FMT>::bits == 8) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t v = sym ? (w[i] ^ 0x80808080u) : w[i];
+            f[4 * i + 0] = __uint_as_float(__byte_perm(v, kExp, 0x7540));
+            f[4 * i + 1] = __uint_as_float(__byte_perm(v, kExp, 0x7541));
+            f[4 * i + 2] = __uint_as_float(__byte_perm(v, kExp, 0x7542));
+            f[4 * i + 3] = __uint_as_float(__byte_perm(v, kExp, 0x7543));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t v = sym ? (w[i] ^ 0x88888888u) : w[i];
+            const uint32_t lo = v & 0x0F0F0F0Fu;
+            const uint32_t hi = (v >> 4) & 0x0F0F0F0Fu;
+            f[8 * i + 0] = __uint_as_float(__byte_perm(lo, kExp, 0x7540));
+            f[8 * i + 1] = __uint_as_float(__byte_perm(hi, kExp, 0x7540));
+            f[8 * i + 2] = __uint_as_float(__byte_perm(lo, kExp, 0x7541));
+            f[8 * i + 3] = __uint_as_float(__byte_perm(hi, kExp, 0x7541));
+            f[8 * i + 4] = __uint_as_float(__byte_perm(lo, kExp, 0x7542));
+            f[8 * i + 5] = __uint_as_float(__byte_perm(hi, kExp, 0x7542));
+            f[8 * i + 6] = __uint_as_float(__byte_perm(lo, kExp, 0x7543));
+            f[8 * i + 7] = __uint_as_float(__byte_perm(hi, kExp, 0x7543));
+        }
+    }
+}
+
+template <int FMT>
+__device__ __forceinline__ void unpack16_int(const uint32_t* w, int (&q)[16])
+{
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        if constexpr (Fmt<FMT>::bits == 8) {
+            const uint32_t b = (w[n / 4] >> (8 * (n % 4))) & 0xFFu;
+            q[n] = Fmt<FMT>::sym ? (int)(int8_t)b : (int)b;
+        } else {
+            const uint32_t b = (w[n / 8] >> (4 * (n % 8))) & 0xFu;
+            q[n] = Fmt<FMT>::sym ? (int)((b ^ 8u) - 8u) : (int)b;
+        }
+    }
+}
+
+template <int FMT>
+__device__ __forceinline__ void pack16(const uint32_t (&k)[16], uint32_t* w)
+{
+    if constexpr (Fmt<FMT>::bits == 8) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t a = __byte_perm(k[4 * i + 0], k[4 * i + 1], 0x0040);
+            const uint32_t b = __byte_perm(k[4 * i + 2], k[4 * i + 3], 0x0040);
+            w[i] = __byte_perm(a, b, 0x5410);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t e01 = __byte_perm(k[8 * i + 0], k[8 * i + 2], 0x0040);
+            const uint32_t e23 = __byte_perm(k[8 * i + 4], k[8 * i + 6], 0x0040);
+            const uint32_t o01 = __byte_perm(k[8 * i + 1], k[8 * i + 3], 0x0040);
+            const uint32_t o23 = __byte_perm(k[8 * i + 5], k[8 * i + 7], 0x0040);
+            const uint32_t ev = __byte_perm(e01, e23, 0x5410);
+            const uint32_t od = __byte_perm(o01, o23, 0x5410);
+            w[i] = (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Row decode: s_n = (q_n - z)*Delta (asym) or q_n*Delta (sym).
 // ---------------------------------------------------------------------------
 template <int FMT, int E>
@@ -302,7 +357,9 @@ __device__ __forceinline__ void decode_row(const Chunk<E * Fmt<FMT>::bits / 8>& 
                                            float delta, float z, float (&s)[E])
 {
     using F = Fmt<FMT>;
-    if (F::sym || fabsf(z) < kFastLimit) {
+    // Warp-uniform choice (every lane of the warp calls this): the exact
+    // scalar path serves the whole warp when any of its rows needs it.
+    if (F::sym || __all_sync(0xffffffffu, fabsf(z) < kFastLimit)) {
         // (2^23 + u) - (2^23 + z + bias) = q - z exactly; one rounding in
         // the product, as in the scalar formula.
         float f[E];
@@ -338,6 +395,23 @@ __device__ __forceinline__ void decode_row(const Chunk<E * Fmt<FMT>::bits / 8>& 
 // clamp at qa (the minimum maps to 0 by construction); the sym clamp never
 // binds because |fl(amax*inv)| rounds to qs.
 // ---------------------------------------------------------------------------
+// a / qmax, correctly rounded, for every non-negative finite a: the product
+// by the rounded reciprocal corrected once with two FMAs (Brisebarre,
+// Muller, Raina, "Accelerating correctly rounded floating-point division
+// when the divisor is known in advance", IEEE Trans. Computers 2004).  For
+// qmax in {255, 15, 127, 7} the identity was checked against IEEE division on
+// every non-negative finite fp32 value; tests/test_host_math.py re-checks a
+// large sample of it on each run.
+template <int FMT>
+__device__ __forceinline__ float div_qmax(float a)
+{
+    constexpr float d = Fmt<FMT>::qmax;
+    constexpr float r = 1.0f / Fmt<FMT>::qmax;
+    const float q0 = __fmul_rn(a, r);
+    const float rem = __fmaf_rn(-q0, d, a);
+    return __fmaf_rn(rem, r, q0);
+}
+
 struct RowParams {
     float delta, inv, z;
     bool fast;    // magic-number rounding is exact for this row
@@ -345,20 +419,12 @@ struct RowParams {
     bool finite;
 };
 
-template <int FMT, int E, int LPR>
-__device__ __forceinline__ RowParams refit_row(const float (&s)[E])
+// Refit from the lane's partial min and max of the updated row: reduce them
+// over the row's LPR lanes, then derive Delta, inv and z.
+template <int FMT, int LPR>
+__device__ __forceinline__ RowParams refit_from_minmax(float lo, float hi)
 {
     using F = Fmt<FMT>;
-    float lo = s[0], hi = s[0];
-#pragma unroll
-    for (int n = 1; n + 1 < E; n += 2) {
-        lo = fmin3(lo, s[n], s[n + 1]);
-        hi = fmax3(hi, s[n], s[n + 1]);
-    }
-    if constexpr (E % 2 == 0) {
-        lo = fminf(lo, s[E - 1]);
-        hi = fmaxf(hi, s[E - 1]);
-    }
     lo = grp_min<LPR>(lo);
     hi = grp_max<LPR>(hi);
 
@@ -367,9 +433,9 @@ __device__ __forceinline__ RowParams refit_row(const float (&s)[E])
     float delta;
     if constexpr (F::sym) {
         const float amax = fmaxf(-lo, hi);
-        delta = __fdiv_rn(amax, F::qmax);
+        delta = div_qmax<FMT>(amax);
     } else {
-        delta = __fdiv_rn(__fsub_rn(hi, lo), F::qmax);
+        delta = div_qmax<FMT>(__fsub_rn(hi, lo));
         if (delta == 0.0f) delta = fabsf(lo);
     }
     if (delta < 1.17549435e-38f) delta = 0.0f;  // FLT_MIN
@@ -385,19 +451,88 @@ __device__ __forceinline__ RowParams refit_row(const float (&s)[E])
     return rp;
 }
 
-// `nz` is -0.0f read from kernel parameters.  The product fl(s*inv) is
-// formed as fma(s, inv, nz): an FMA result is never fused again, so the magic
-// add that follows sees the rounded product.  (A packed multiply followed by
-// a packed add can be contracted into one FMA by the toolchain even with
-// explicit rounding modifiers, which would round the exact product instead.)
-// Adding -0 is exact for every product, and the compiler cannot fold away a
-// zero it cannot see.
+// Lane-local min / max of n values, folded into (lo, hi).
+template <int M>
+__device__ __forceinline__ void minmax_acc(const float* v, float& lo, float& hi)
+{
+#pragma unroll
+    for (int n = 0; n + 1 < M; n += 2) {
+        lo = fmin3(lo, v[n], v[n + 1]);
+        hi = fmax3(hi, v[n], v[n + 1]);
+    }
+    if constexpr (M % 2 == 1) {
+        lo = fminf(lo, v[M - 1]);
+        hi = fmaxf(hi, v[M - 1]);
+    }
+}
+
+template <int FMT, int E, int LPR>
+__device__ __forceinline__ RowParams refit_row(const float (&s)[E])
+{
+    float lo = s[0], hi = s[0];
+    minmax_acc<E - 1>(s + 1, lo, hi);
+    return refit_from_minmax<FMT, LPR>(lo, hi);
+}
+
+// Fast rounding of 16 entries (valid when the warp's rows all passed the
+// fast test): r = rint(fl(s*inv)) exactly, k carries the stored code.
+template <int FMT>
+__device__ __forceinline__ void round16_fast(const RowParams& rp, const float* s, float* r,
+                                             uint32_t (&k)[16], float nz)
+{
+    using F = Fmt<FMT>;
+    const float2 nz2 = make_float2(nz, nz);
+    const float2 inv2 = make_float2(rp.inv, rp.inv);
+    const float2 m2 = make_float2(kMagic, kMagic);
+    const float2 nm2 = make_float2(-kMagic, -kMagic);
+    const float2 z2 = make_float2(rp.z, rp.z);
+#pragma unroll
+    for (int n = 0; n < 16; n += 2) {
+        float2 p = fma2(make_float2(s[n], s[n + 1]), inv2, nz2);
+        float2 t = add2(p, m2);
+        float2 rr = add2(t, nm2);
+        r[n] = rr.x; r[n + 1] = rr.y;
+        if constexpr (F::sym) {
+            k[n] = __float_as_uint(t.x);
+            k[n + 1] = __float_as_uint(t.y);
+        } else {
+            float2 u = add2(t, z2);
+            k[n] = __float_as_uint(u.x);
+            k[n + 1] = __float_as_uint(u.y);
+        }
+    }
+}
+
+// Exact scalar rounding of 16 entries (the definition verbatim).
+template <int FMT>
+__device__ __forceinline__ void round16_slow(const RowParams& rp, const float* s, float* r,
+                                             uint32_t (&k)[16])
+{
+    using F = Fmt<FMT>;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        const float rr = rintf(__fmul_rn(s[n], rp.inv));
+        float c;
+        if constexpr (F::sym) {
+            c = fminf(fmaxf(rr, -F::qmax), F::qmax);
+            r[n] = c;
+        } else {
+            c = fminf(__fadd_rn(rr, rp.z), F::qmax);
+            r[n] = __fsub_rn(c, rp.z);
+        }
+        k[n] = (uint32_t)(int)c;
+    }
+}
+
+// Returns true when the magic-number path ran (then r holds exact q - z);
+// the choice is warp-uniform and every lane of the warp must call this.
 template <int FMT, int E>
-__device__ __forceinline__ void round_row(const RowParams& rp, const float (&s)[E],
+__device__ __forceinline__ bool round_row(const RowParams& rp, const float (&s)[E],
                                           float (&r)[E], uint32_t (&k)[E], float nz)
 {
     using F = Fmt<FMT>;
-    if (rp.fast && !rp.clamp) {
+    const bool fast = __all_sync(0xffffffffu, rp.fast && !rp.clamp);
+    if (fast) {
         const float2 nz2 = make_float2(nz, nz);
         const float2 inv2 = make_float2(rp.inv, rp.inv);
         const float2 m2 = make_float2(kMagic, kMagic);
@@ -434,6 +569,7 @@ __device__ __forceinline__ void round_row(const RowParams& rp, const float (&s)[
             k[n] = (uint32_t)(int)c;
         }
     }
+    return fast;
 }
 
 // The stored row as fp32: fl(r_n * Delta).

@@ -176,14 +176,22 @@ __host__ __device__ inline DecodeGeom decode_geom(int S, int RPT, int RB, int MB
     return g;
 }
 
+// Lane shape of the decode kernel: quantized rows give each lane 64 entries
+// (two lanes per 128-entry row), which halves the per-row and per-tile
+// bookkeeping per entry; fp rows keep 32 entries per lane.
+template <int FMT, int N>
+struct DShape {
+    static constexpr int E = Fmt<FMT>::quant ? (N >= 64 ? 64 : N) : (N >= 32 ? 32 : N);
+    static constexpr int LPR = N / E;
+};
+
 template <int FMT, int N>
 __global__ void __launch_bounds__(kDThreads, 2)
 decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv,
               const __grid_constant__ DecodeGeom geo)
 {
-    using Sh = Shape<N>;
     using F = Fmt<FMT>;
-    constexpr int E = Sh::E, LPR = Sh::LPR;
+    constexpr int E = DShape<FMT, N>::E, LPR = DShape<FMT, N>::LPR;
     constexpr bool kBf16 = (FMT == SSQ_BF16);
     constexpr int RB = F::quant ? N * F::bits / 8 : 0;      // code bytes per row
     constexpr int CB = F::quant ? E * F::bits / 8 : 16;     // code bytes per lane
@@ -223,10 +231,13 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
 
     if (warp == kCWarps) {
         // ================= producer warp =================
-        int k = 0, uk = -1;
+        int si = 0, sph = 0, k = 0, uk = -1;
         long long prev = -1;
         bool bad = false, ok = true;
-        int slot = 0;
+        const uint8_t* codes_u = nullptr;
+        const uint8_t* meta_u = nullptr;
+        const uint8_t* fp_u = nullptr;
+        const float* x_u = nullptr;
         TileWalk ti;
         ti.start(pv, cv, t0);
         for (long long t = t0; t < t1; ++t, ti.next(pv, cv)) {
@@ -236,7 +247,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 ++uk;
                 const int u = uk & 1;
                 if (!mbar_wait(&uempty[u], ((uk >> 1) & 1) ^ 1)) { ok = false; break; }
-                slot = cv.slot_idx ? __ldg(cv.slot_idx + ti.b) : ti.b;
+                const int slot = cv.slot_idx ? __ldg(cv.slot_idx + ti.b) : ti.b;
                 bad = slot < 0 || slot >= pv.n_slots;
                 uint8_t* ub = units + u * geo.unit_bytes;
                 if (lane == 0) {
@@ -245,9 +256,17 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     if (bad) atomicOr(err, SSQ_DEVERR_SLOT);
                 }
                 if (!bad) {
-                    // B and C in 16-byte chunks; in quantized units chunk i
-                    // of lane j goes to slot (i + j) mod CPL of that lane, so
-                    // the lanes of a row read distinct banks
+                    const int layer = cv.layer0 + ti.l;
+                    const uint8_t* sb = pv.pool + pv.header_bytes + (long long)slot * pv.slot_bytes;
+                    codes_u = sb + pv.codes_off + (long long)layer * pv.codes_layer_bytes;
+                    meta_u = sb + pv.meta_off + (long long)layer * pv.meta_layer_bytes;
+                    fp_u = sb + pv.fp_off + (long long)layer * pv.fp_layer_bytes;
+                    x_u = cv.x + ti.lb * H * P;
+                    // B and C in 16-byte chunks.  In quantized units lane j
+                    // of a row owns chunks j*CPL .. j*CPL+CPL-1; chunk i of
+                    // lane j is stored at i*LPR + j, so at each step the
+                    // lanes of a row read consecutive chunks (distinct banks)
+                    // at compile-time offsets from a per-lane base.
                     float* dB = reinterpret_cast<float*>(ub + geo.ub_B);
                     float* dC = reinterpret_cast<float*>(ub + geo.ub_C);
                     const float* sB = cv.B + ti.lb * G * N;
@@ -257,7 +276,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         if (ti.quant) {
                             const int gi = m / (N / 4), mm = m - gi * (N / 4);
                             const int jj = mm / CPL, ii = mm - jj * CPL;
-                            pos = gi * (N / 4) + jj * CPL + ((ii + jj) & (CPL - 1));
+                            pos = gi * (N / 4) + ii * LPR + jj;
                         }
                         cpa16(dB + 4 * pos, sB + 4 * m);
                         cpa16(dC + 4 * pos, sC + 4 * m);
@@ -276,40 +295,33 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 if (lane == 0) mbar_arrive(&ufull[u]);
             }
             if (bad) continue;
-            const int s = k % S;
-            if (!mbar_wait(&empty[s], ((k / S) & 1) ^ 1)) { ok = false; break; }
-            uint8_t* st = stages + s * geo.stage_bytes;
+            if (!mbar_wait(&empty[si], sph ^ 1)) { ok = false; break; }
+            uint8_t* st = stages + si * geo.stage_bytes;
             float* sx = reinterpret_cast<float*>(st);
             for (int i = lane; i < ti.n; i += 32) {
                 const int rr = ti.rbase + i;
                 const int hr = fdiv(rr, pv.mP);
                 const int hh = pv.perm[regbase + hr];
-                cpa4(sx + i, cv.x + (ti.lb * H + hh) * P + (rr - hr * P));
+                cpa4(sx + i, x_u + hh * P + (rr - hr * P));
             }
-            cpa_arrive(&full[s]);
+            cpa_arrive(&full[si]);
             __syncwarp();
             if (lane == 0) {
-                const int layer = cv.layer0 + ti.l;
-                const uint8_t* sb = pv.pool + pv.header_bytes + (long long)slot * pv.slot_bytes;
                 uint8_t* pay = st + geo.x_bytes;
                 if (F::quant && ti.quant) {
-                    const uint8_t* csrc = sb + pv.codes_off + (long long)layer * pv.codes_layer_bytes
-                                          + (long long)ti.rbase * RB;
-                    const uint8_t* msrc = sb + pv.meta_off + (long long)layer * pv.meta_layer_bytes
-                                          + (long long)ti.rbase * MB;
                     const unsigned cb = (unsigned)r16(ti.n * RB), mb = (unsigned)r16(ti.n * MB);
-                    mbar_arrive_tx(&full[s], cb + mb);
-                    bulk_g2s(pay, csrc, cb, &full[s]);
-                    bulk_g2s(pay + geo.qcodes_bytes, msrc, mb, &full[s]);
+                    mbar_arrive_tx(&full[si], cb + mb);
+                    bulk_g2s(pay, codes_u + (long long)ti.rbase * RB, cb, &full[si]);
+                    bulk_g2s(pay + geo.qcodes_bytes, meta_u + (long long)ti.rbase * MB, mb,
+                             &full[si]);
                 } else {
-                    const uint8_t* fsrc = sb + pv.fp_off + (long long)layer * pv.fp_layer_bytes
-                                          + (long long)ti.rbase * N * FEB;
                     const unsigned fb = (unsigned)(ti.n * N * FEB);
-                    mbar_arrive_tx(&full[s], fb);
-                    bulk_g2s(pay, fsrc, fb, &full[s]);
+                    mbar_arrive_tx(&full[si], fb);
+                    bulk_g2s(pay, fp_u + (long long)ti.rbase * N * FEB, fb, &full[si]);
                 }
             }
             ++k;
+            if (++si == S) { si = 0; sph ^= 1; }
         }
         if (!ok && lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
         // No copy may still be writing shared memory when the CTA exits.
@@ -325,12 +337,15 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     const int ct = threadIdx.x;
     const int grow = ct / LPR;
     const int j = ct % LPR;
-    int k = 0, uk = -1;
+    int si = 0, sph = 0, uk = -1;
     long long prev = -1;
     bool bad = false;
-    int slot = 0;
     const uint8_t* ub = units;
     float* lam = nullptr;
+    uint8_t* codes_u = nullptr;
+    uint8_t* meta_u = nullptr;
+    uint8_t* fp_u = nullptr;
+    float* y_u = nullptr;
 
     TileWalk ti;
     ti.start(pv, cv, t0);
@@ -348,10 +363,16 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 break;
             }
             ub = units + u * geo.unit_bytes;
-            slot = reinterpret_cast<const int*>(ub)[0];
+            const int slot = reinterpret_cast<const int*>(ub)[0];
             bad = reinterpret_cast<const int*>(ub)[1] != 0;
             lam = reinterpret_cast<float*>(smem + geo.off_lam) + (warp * 2 + u) * geo.Hpad;
             if (!bad) {
+                const int layer = cv.layer0 + ti.l;
+                uint8_t* sb = pv.pool + pv.header_bytes + (long long)slot * pv.slot_bytes;
+                codes_u = sb + pv.codes_off + (long long)layer * pv.codes_layer_bytes;
+                meta_u = sb + pv.meta_off + (long long)layer * pv.meta_layer_bytes;
+                fp_u = sb + pv.fp_off + (long long)layer * pv.fp_layer_bytes;
+                y_u = cv.y + ti.lb * H * P;
                 const float* udt = reinterpret_cast<const float*>(ub + geo.ub_dt);
                 const float* uA = reinterpret_cast<const float*>(ub + geo.ub_A);
                 for (int h = lane; h < H; h += 32) lam[h] = decay(udt[h], uA[h]);
@@ -359,12 +380,11 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             }
         }
         if (bad) continue;
-        const int s = k % S;
-        if (!mbar_wait(&full[s], (k / S) & 1)) {
+        if (!mbar_wait(&full[si], sph)) {
             if (lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
             break;
         }
-        const uint8_t* st = stages + s * geo.stage_bytes;
+        const uint8_t* st = stages + si * geo.stage_bytes;
         const float* sx = reinterpret_cast<const float*>(st);
         const uint8_t* pay = st + geo.x_bytes;
         const int regbase = ti.quant ? 0 : pv.Hq;
@@ -382,79 +402,126 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         const float dtx = __fmul_rn(dtv, xv);
         const float* gB = reinterpret_cast<const float*>(ub + geo.ub_B) + g * N;
         const float* gC = reinterpret_cast<const float*>(ub + geo.ub_C) + g * N;
-        const int layer = cv.layer0 + ti.l;
-        uint8_t* sb = pv.pool + pv.header_bytes + (long long)slot * pv.slot_bytes;
         float ysum = 0.0f;
         bool done = false;
 
         if constexpr (F::quant) {
             if (ti.quant) {
                 done = true;
-                Chunk<CB> c;
-                const uint8_t* cs = pay + rl * RB + j * CB;
-                if constexpr (CB % 16 == 0) {
+                constexpr int PW = Piece<FMT>::words;        // words per 16 entries
+                constexpr int NP = E / 16;                   // 16-entry pieces per lane
+                uint32_t cw[CB / 4];
+                {
+                    const uint8_t* cs = pay + rl * RB + j * CB;
+                    if constexpr (CB % 16 == 0) {
 #pragma unroll
-                    for (int i = 0; i < CB / 16; ++i) {
-                        const uint4 v = reinterpret_cast<const uint4*>(cs)[i];
-                        c.w[4 * i] = v.x; c.w[4 * i + 1] = v.y; c.w[4 * i + 2] = v.z; c.w[4 * i + 3] = v.w;
-                    }
-                } else {
+                        for (int i = 0; i < CB / 16; ++i) {
+                            const uint4 v = reinterpret_cast<const uint4*>(cs)[i];
+                            cw[4 * i] = v.x; cw[4 * i + 1] = v.y; cw[4 * i + 2] = v.z; cw[4 * i + 3] = v.w;
+                        }
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < CB / 8; ++i) {
-                        const uint2 v = reinterpret_cast<const uint2*>(cs)[i];
-                        c.w[2 * i] = v.x; c.w[2 * i + 1] = v.y;
+                        for (int i = 0; i < CB / 8; ++i) {
+                            const uint2 v = reinterpret_cast<const uint2*>(cs)[i];
+                            cw[2 * i] = v.x; cw[2 * i + 1] = v.y;
+                        }
                     }
                 }
                 float delta0, z0 = 0.0f;
-                const uint8_t* ms = pay + geo.qcodes_bytes + rl * MB;
-                if constexpr (F::sym) {
-                    delta0 = *reinterpret_cast<const float*>(ms);
-                } else {
-                    const float2 m = *reinterpret_cast<const float2*>(ms);
-                    delta0 = m.x;
-                    z0 = m.y;
-                }
-                float s[E];
-                decode_row<FMT, E>(c, delta0, z0, s);
                 {
-                    float Bv[E];
+                    const uint8_t* ms = pay + geo.qcodes_bytes + rl * MB;
+                    if constexpr (F::sym) {
+                        delta0 = *reinterpret_cast<const float*>(ms);
+                    } else {
+                        const float2 m = *reinterpret_cast<const float2*>(ms);
+                        delta0 = m.x;
+                        z0 = m.y;
+                    }
+                }
+                // decode + update, 16 entries at a time, tracking min / max
+                float s[E];
+                float lo = __int_as_float(0x7f800000), hi = -__int_as_float(0x7f800000);
+                const bool dfast = F::sym || __all_sync(0xffffffffu, fabsf(z0) < kFastLimit);
+                const float c0 = __fadd_rn(kTwo23, __fadd_rn(z0, F::bias));
+                const float4* b4 = reinterpret_cast<const float4*>(gB) + j;
 #pragma unroll
-                    for (int i = 0; i < CPL; ++i) {
-                        const int pos = j * CPL + ((i + j) & (CPL - 1));
-                        const float4 v = reinterpret_cast<const float4*>(gB)[pos];
+                for (int pc = 0; pc < NP; ++pc) {
+                    float* sp = s + 16 * pc;
+                    if (dfast) {
+                        float f[16];
+                        unpack16_biased<FMT>(cw + PW * pc, f);
+                        const float2 nc02 = make_float2(-c0, -c0);
+                        const float2 d2 = make_float2(delta0, delta0);
+#pragma unroll
+                        for (int n = 0; n < 16; n += 2) {
+                            float2 v = mul2(add2(make_float2(f[n], f[n + 1]), nc02), d2);
+                            sp[n] = v.x; sp[n + 1] = v.y;
+                        }
+                    } else {
+                        int q[16];
+                        unpack16_int<FMT>(cw + PW * pc, q);
+#pragma unroll
+                        for (int n = 0; n < 16; ++n)
+                            sp[n] = __fmul_rn(__fsub_rn((float)q[n], z0), delta0);
+                    }
+                    float Bv[16];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float4 v = b4[(4 * pc + i) * LPR];
                         Bv[4 * i] = v.x; Bv[4 * i + 1] = v.y; Bv[4 * i + 2] = v.z; Bv[4 * i + 3] = v.w;
                     }
-                    update_row<E>(lamv, dtx, Bv, s);
-                }
-                const RowParams rp = refit_row<FMT, E, LPR>(s);
-                float rq[E];
-                {
-                    uint32_t kk[E];
-                    round_row<FMT, E>(rp, s, rq, kk, pv.neg_zero);
-                    pack_codes<FMT, E>(kk, c);
-                }
-                float Cv[E];
+                    const float2 l2 = make_float2(lamv, lamv);
+                    const float2 x2 = make_float2(dtx, dtx);
 #pragma unroll
-                for (int i = 0; i < CPL; ++i) {
-                    const int pos = j * CPL + ((i + j) & (CPL - 1));
-                    const float4 v = reinterpret_cast<const float4*>(gC)[pos];
-                    Cv[4 * i] = v.x; Cv[4 * i + 1] = v.y; Cv[4 * i + 2] = v.z; Cv[4 * i + 3] = v.w;
+                    for (int n = 0; n < 16; n += 2) {
+                        const float2 w = mul2(x2, make_float2(Bv[n], Bv[n + 1]));
+                        const float2 v = fma2(l2, make_float2(sp[n], sp[n + 1]), w);
+                        sp[n] = v.x; sp[n + 1] = v.y;
+                    }
+                    minmax_acc<16>(sp, lo, hi);
                 }
-                if (rp.fast && !rp.clamp) {
-                    // y = Delta * sum_n C_n (q_n - z): the stored row read back
-                    ysum = __fmul_rn(rp.delta, grp_sum<LPR>(dot_row<E>(Cv, rq)));
-                } else {
-                    float sv[E];
-                    scale_row<E>(rp.delta, rq, sv);
-                    ysum = grp_sum<LPR>(dot_row<E>(Cv, sv));
+                const RowParams rp = refit_from_minmax<FMT, LPR>(lo, hi);
+                const bool fast = __all_sync(0xffffffffu, rp.fast && !rp.clamp);
+                // round, pack and read back, 16 entries at a time
+                const float4* c4 = reinterpret_cast<const float4*>(gC) + j;
+                float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int pc = 0; pc < NP; ++pc) {
+                    float r[16];
+                    uint32_t kk[16];
+                    if (fast) {
+                        round16_fast<FMT>(rp, s + 16 * pc, r, kk, pv.neg_zero);
+                    } else {
+                        round16_slow<FMT>(rp, s + 16 * pc, r, kk);
+#pragma unroll
+                        for (int n = 0; n < 16; ++n) r[n] = __fmul_rn(r[n], rp.delta);
+                    }
+                    pack16<FMT>(kk, cw + PW * pc);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float4 v = c4[(4 * pc + i) * LPR];
+                        acc = fma2(make_float2(v.x, v.y), make_float2(r[4 * i], r[4 * i + 1]), acc);
+                        acc = fma2(make_float2(v.z, v.w), make_float2(r[4 * i + 2], r[4 * i + 3]), acc);
+                    }
                 }
+                // fast: acc = sum C (q - z), scaled by Delta once; slow: acc
+                // already sums C * fl((q - z) * Delta)
+                const float part = __fadd_rn(acc.x, acc.y);
+                ysum = fast ? __fmul_rn(rp.delta, grp_sum<LPR>(part)) : grp_sum<LPR>(part);
                 if (active) {
-                    uint8_t* crow = sb + pv.codes_off + (long long)layer * pv.codes_layer_bytes
-                                    + (long long)rr * RB + j * CB;
-                    store_chunk<CB>(crow, c);
+                    uint8_t* crow = codes_u + (long long)rr * RB + j * CB;
+                    if constexpr (CB % 16 == 0) {
+#pragma unroll
+                        for (int i = 0; i < CB / 16; ++i)
+                            __stcs(reinterpret_cast<uint4*>(crow) + i,
+                                   make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < CB / 8; ++i)
+                            __stcs(reinterpret_cast<uint2*>(crow) + i, make_uint2(cw[2 * i], cw[2 * i + 1]));
+                    }
                     if (j == 0) {
-                        uint8_t* mrow = sb + pv.meta_off + (long long)layer * pv.meta_layer_bytes
-                                        + (long long)rr * MB;
+                        uint8_t* mrow = meta_u + (long long)rr * MB;
                         if constexpr (F::sym) {
                             __stcs(reinterpret_cast<float*>(mrow), rp.delta);
                         } else {
@@ -466,72 +533,68 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             }
         }
         if (!done) {
-            // fp row (fp32, or bf16 for the bf16 format).  Lane j owns the
-            // 16-byte storage chunks LPR*c + j of its row, so the lanes of a
-            // row touch consecutive chunks (no bank conflicts on B and C).
+            // fp row (fp32, or bf16 for the bf16 format), streamed one 16-byte
+            // storage chunk at a time.  Lane j owns chunks LPR*c + j, so the
+            // lanes of a row touch consecutive chunks.
             constexpr int EPC = 16 / FEB;           // elements per chunk
             constexpr int NCH = E / EPC;            // chunks per lane
             const uint8_t* fs = pay + (long long)rl * N * FEB;
-            float s[E];
-            uint32_t w[E * FEB / 4];
+            uint8_t* frow = fp_u + (long long)rr * N * FEB;
+            const float2 l2 = make_float2(lamv, lamv);
+            const float2 x2 = make_float2(dtx, dtx);
+            float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
-                const uint4 v = reinterpret_cast<const uint4*>(fs)[LPR * c + j];
-                w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
-            }
-            if constexpr (kBf16) {
+                const int m = LPR * c + j;
+                const uint4 v = reinterpret_cast<const uint4*>(fs)[m];
+                uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                float sv[EPC];
+                if constexpr (kBf16) {
 #pragma unroll
-                for (int n = 0; n < E; ++n)
-                    s[n] = __uint_as_float((w[n / 2] >> (16 * (n % 2))) << 16);
-            } else {
+                    for (int n = 0; n < EPC; ++n)
+                        sv[n] = __uint_as_float((w[n / 2] >> (16 * (n % 2))) << 16);
+                } else {
 #pragma unroll
-                for (int n = 0; n < E; ++n) s[n] = __uint_as_float(w[n]);
-            }
-            float Bv[E], Cv[E];
-#pragma unroll
-            for (int c = 0; c < NCH; ++c) {
+                    for (int n = 0; n < EPC; ++n) sv[n] = __uint_as_float(w[n]);
+                }
 #pragma unroll
                 for (int q = 0; q < EPC / 4; ++q) {
-                    const int ch = (LPR * c + j) * (EPC / 4) + q;
-                    const float4 vb = reinterpret_cast<const float4*>(gB)[ch];
-                    const float4 vc = reinterpret_cast<const float4*>(gC)[ch];
-                    const int o = c * EPC + 4 * q;
-                    Bv[o] = vb.x; Bv[o + 1] = vb.y; Bv[o + 2] = vb.z; Bv[o + 3] = vb.w;
-                    Cv[o] = vc.x; Cv[o + 1] = vc.y; Cv[o + 2] = vc.z; Cv[o + 3] = vc.w;
+                    const float4 vb = reinterpret_cast<const float4*>(gB)[m * (EPC / 4) + q];
+                    const float4 vc = reinterpret_cast<const float4*>(gC)[m * (EPC / 4) + q];
+                    float2 a = fma2(l2, make_float2(sv[4 * q], sv[4 * q + 1]),
+                                    mul2(x2, make_float2(vb.x, vb.y)));
+                    float2 b = fma2(l2, make_float2(sv[4 * q + 2], sv[4 * q + 3]),
+                                    mul2(x2, make_float2(vb.z, vb.w)));
+                    if constexpr (kBf16) {
+                        a = make_float2(__bfloat162float(__float2bfloat16_rn(a.x)),
+                                        __bfloat162float(__float2bfloat16_rn(a.y)));
+                        b = make_float2(__bfloat162float(__float2bfloat16_rn(b.x)),
+                                        __bfloat162float(__float2bfloat16_rn(b.y)));
+                    }
+                    sv[4 * q] = a.x; sv[4 * q + 1] = a.y; sv[4 * q + 2] = b.x; sv[4 * q + 3] = b.y;
+                    acc = fma2(make_float2(vc.x, vc.y), a, acc);
+                    acc = fma2(make_float2(vc.z, vc.w), b, acc);
                 }
-            }
-            update_row<E>(lamv, dtx, Bv, s);
-            if constexpr (kBf16) {
+                if constexpr (kBf16) {
 #pragma unroll
-                for (int n = 0; n < E; n += 2) {
-                    const __nv_bfloat16 a = __float2bfloat16_rn(s[n]);
-                    const __nv_bfloat16 b2 = __float2bfloat16_rn(s[n + 1]);
-                    w[n / 2] = (uint32_t)__bfloat16_as_ushort(a)
-                               | ((uint32_t)__bfloat16_as_ushort(b2) << 16);
-                    s[n] = __bfloat162float(a);
-                    s[n + 1] = __bfloat162float(b2);
+                    for (int n = 0; n < EPC; n += 2)
+                        w[n / 2] = (__float_as_uint(sv[n]) >> 16) | (__float_as_uint(sv[n + 1]) & 0xffff0000u);
+                } else {
+#pragma unroll
+                    for (int n = 0; n < EPC; ++n) w[n] = __float_as_uint(sv[n]);
                 }
-            } else {
-#pragma unroll
-                for (int n = 0; n < E; ++n) w[n] = __float_as_uint(s[n]);
+                if (active)
+                    __stcs(reinterpret_cast<uint4*>(frow) + m, make_uint4(w[0], w[1], w[2], w[3]));
             }
-            ysum = grp_sum<LPR>(dot_row<E>(Cv, s));
-            if (active) {
-                uint8_t* frow = sb + pv.fp_off + (long long)layer * pv.fp_layer_bytes
-                                + (long long)rr * N * FEB;
-#pragma unroll
-                for (int c = 0; c < NCH; ++c)
-                    __stcs(reinterpret_cast<uint4*>(frow) + (LPR * c + j),
-                           make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]));
-            }
+            ysum = grp_sum<LPR>(__fadd_rn(acc.x, acc.y));
         }
         if (active && j == 0) {
             const float yv = __fadd_rn(ysum, __fmul_rn(Dv, xv));
-            __stcs(cv.y + (ti.lb * H + h) * P + p, yv);
+            __stcs(y_u + h * P + p, yv);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        ++k;
+        if (lane == 0) mbar_arrive(&empty[si]);
+        if (++si == S) { si = 0; sph ^= 1; }
     }
 }
 
@@ -539,8 +602,7 @@ template <int FMT, int N>
 cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
 {
     using F = Fmt<FMT>;
-    constexpr int E = Shape<N>::E;
-    constexpr int LPR = N / E;
+    constexpr int LPR = DShape<FMT, N>::LPR;
     constexpr int RPT = kCThreads / LPR;
     constexpr int RB = F::quant ? N * F::bits / 8 : 0;
     const bool has_fp = pv.Hf > 0;
@@ -590,18 +652,18 @@ cudaError_t launch_fmt(const PoolView& pv, const CallView& cv, cudaStream_t st)
 
 }  // namespace
 
-int decode_rows_per_tile(int d_state)
+int decode_rows_per_tile(int fmt, int d_state)
 {
-    const int E = d_state >= 32 ? 32 : d_state;
+    const bool quant = fmt >= SSQ_I8_SYM;
+    const int E = quant ? (d_state >= 64 ? 64 : d_state) : (d_state >= 32 ? 32 : d_state);
     return kCThreads / (d_state / E);
 }
 
-bool decode_fits(int d_state, int nheads, int ngroups)
+bool decode_fits(int fmt, int d_state, int nheads, int ngroups)
 {
     // B and C of every group plus the lambda arrays must leave room for two
     // pipeline stages within one CTA's shared memory
-    const int E = d_state >= 32 ? 32 : d_state;
-    const int rpt = kCThreads / (d_state / E);
+    const int rpt = decode_rows_per_tile(fmt, d_state);
     const DecodeGeom g = decode_geom(2, rpt, d_state, 8, 4, true, d_state, nheads, ngroups);
     return g.smem_bytes <= 227 * 1024;
 }

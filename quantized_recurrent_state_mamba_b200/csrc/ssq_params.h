@@ -57,10 +57,10 @@ cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt,
 
 // Rows of one region each scan CTA owns; rows per decode tile.
 int scan_rows_per_cta(int d_state);
-int decode_rows_per_tile(int d_state);
+int decode_rows_per_tile(int fmt, int d_state);
 // Whether the decode kernel's per-unit shared memory (B and C of every group,
 // per-head arrays) fits one CTA.
-bool decode_fits(int d_state, int nheads, int ngroups);
+bool decode_fits(int fmt, int d_state, int nheads, int ngroups);
 
 // Grid for a grid-stride kernel: resident blocks on the current device,
 // capped by the number of tiles.

@@ -211,6 +211,8 @@ def decode_8b(fmt="i8a", batch=64):
 
 
 def sweep_serving(fmt="i8a", batch=256, nl=30):
+    # The serving-scale pool starts from the zero state (the workload names
+    # no initial state); a few steps of input make it non-zero.
     return Decode(f"serving sweep L{nl} b{batch} H32 P128 N128 {fmt}",
                   seed=4, nl=nl, batch=batch, nheads=32, headdim=128,
-                  d_state=128, ngroups=1, fmt=fmt)
+                  d_state=128, ngroups=1, fmt=fmt, init="zero")

@@ -75,8 +75,9 @@ def compare_states(ocfg, got, ref, pre=None, where=""):
                 assert np.array_equal(got.zero[i, rows].view(np.uint32),
                                       ref.zero[i, rows].view(np.uint32)), \
                     f"{where} zero point differs (pair {i}, head {h})"
-                assert np.all(ulp_diff(got.delta[i, rows], ref.delta[i, rows]) <= 2), \
-                    f"{where} step differs by > 2 ulp (pair {i}, head {h})"
+                ud = ulp_diff(got.delta[i, rows], ref.delta[i, rows])
+                assert np.all(ud <= 2), f"{where} step differs by > 2 ulp (pair {i}, head {h})"
+                stats["delta_ulp_max"] = max(stats.get("delta_ulp_max", 0), int(ud.max()))
                 gq, rq = got.q[i, rows], ref.q[i, rows]
                 diff = gq != rq
                 stats["entries"] += gq.size

@@ -98,6 +98,7 @@ def test_quantize_rows_bit_exact(fmt, N):
     got = download(codec, pool, pairs, ocfg)
     stats = compare_states(ocfg, got, ref, None, f"quantize {fmt} N{N}")
     assert stats["code_mismatch"] == 0
+    assert stats.get("delta_ulp_max", 0) == 0        # the step is bit-exact too
     # untouched layer 0 and slots stay zero
     buf = pool.cpu().numpy()
     q0, d0, z0, v0 = codec.read(buf, 1, 0)
