@@ -440,7 +440,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 }
                 // decode + update, 16 entries at a time, tracking min / max
                 float s[E];
-                float lo = __int_as_float(0x7f800000), hi = -__int_as_float(0x7f800000);
+                float plo[NP], phi[NP];                      // per-piece min / max
                 const bool dfast = F::sym || __all_sync(0xffffffffu, fabsf(z0) < kFastLimit);
                 const float c0 = __fadd_rn(kTwo23, __fadd_rn(z0, F::bias));
                 const float4* b4 = reinterpret_cast<const float4*>(gB) + j;
@@ -478,15 +478,23 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         const float2 v = fma2(l2, make_float2(sp[n], sp[n + 1]), w);
                         sp[n] = v.x; sp[n + 1] = v.y;
                     }
-                    minmax_acc<16>(sp, lo, hi);
+                    minmax16(sp, plo[pc], phi[pc]);
+                }
+                float lo = plo[0], hi = phi[0];
+#pragma unroll
+                for (int pc = 1; pc < NP; ++pc) {
+                    lo = fminf(lo, plo[pc]);
+                    hi = fmaxf(hi, phi[pc]);
                 }
                 const RowParams rp = refit_from_minmax<FMT, LPR>(lo, hi);
                 const bool fast = __all_sync(0xffffffffu, rp.fast && !rp.clamp);
                 // round, pack and read back, 16 entries at a time
                 const float4* c4 = reinterpret_cast<const float4*>(gC) + j;
-                float2 acc = make_float2(0.0f, 0.0f);
+                float2 accp[NP];                             // one accumulator per piece
 #pragma unroll
                 for (int pc = 0; pc < NP; ++pc) {
+                    float2& acc = accp[pc];
+                    acc = make_float2(0.0f, 0.0f);
                     float r[16];
                     uint32_t kk[16];
                     if (fast) {
@@ -506,6 +514,9 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 }
                 // fast: acc = sum C (q - z), scaled by Delta once; slow: acc
                 // already sums C * fl((q - z) * Delta)
+                float2 acc = accp[0];
+#pragma unroll
+                for (int pc = 1; pc < NP; ++pc) acc = add2(acc, accp[pc]);
                 const float part = __fadd_rn(acc.x, acc.y);
                 ysum = fast ? __fmul_rn(rp.delta, grp_sum<LPR>(part)) : grp_sum<LPR>(part);
                 if (active) {
@@ -542,7 +553,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             uint8_t* frow = fp_u + (long long)rr * N * FEB;
             const float2 l2 = make_float2(lamv, lamv);
             const float2 x2 = make_float2(dtx, dtx);
-            float2 acc = make_float2(0.0f, 0.0f);
+            float2 acc = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
                 const int m = LPR * c + j;
@@ -573,7 +584,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     }
                     sv[4 * q] = a.x; sv[4 * q + 1] = a.y; sv[4 * q + 2] = b.x; sv[4 * q + 3] = b.y;
                     acc = fma2(make_float2(vc.x, vc.y), a, acc);
-                    acc = fma2(make_float2(vc.z, vc.w), b, acc);
+                    acc1 = fma2(make_float2(vc.z, vc.w), b, acc1);
                 }
                 if constexpr (kBf16) {
 #pragma unroll
@@ -586,6 +597,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 if (active)
                     __stcs(reinterpret_cast<uint4*>(frow) + m, make_uint4(w[0], w[1], w[2], w[3]));
             }
+            acc = add2(acc, acc1);
             ysum = grp_sum<LPR>(__fadd_rn(acc.x, acc.y));
         }
         if (active && j == 0) {

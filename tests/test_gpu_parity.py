@@ -383,3 +383,36 @@ def test_scan_equals_repeated_decode(fmt):
     torch.cuda.synchronize()
     assert torch.equal(pool_a, pool_b)
     assert torch.allclose(y_a, y_b, rtol=1e-4, atol=1e-4)
+
+
+@pytest.mark.parametrize("fmt", ["i8a", "i4s"])
+def test_decode_many_one_tile_units(fmt):
+    """Thousands of (layer, request, region) units of one tile each (3 heads x
+    5 rows, one head kept fp32): the decode kernel's consumer warps take every
+    7th tile, so each warp jumps over several units between its tiles."""
+    ssq = require_gpu()
+    H, P, N, G, batch, nl = 3, 5, 128, 1, 256, 16
+    mask = [1, 0, 1]
+    cfg, L, codec, ocfg = make_cfg(ssq, fmt, nl, batch, H, P, N, G, mask)
+    rng = np.random.default_rng(55)
+    S0 = rng.standard_normal((nl * batch, H, P, N)).astype(np.float32)
+    st = O.state_from_f32(ocfg, S0)
+    pairs = [(b, l) for l in range(nl) for b in range(batch)]
+    pool = upload(ssq, cfg, L, codec, st, pairs)
+    inp = W.Decode("units", 61, nl, batch, H, P, N, G, fmt).inputs()
+    y = torch.empty((nl, batch, H, P), device="cuda")
+    ssq.ssq_decode_step(cfg, pool, None, batch, 0, nl, cuda(inp["x"]), cuda(inp["B"]),
+                        cuda(inp["C"]), cuda(inp["dt"]), cuda(inp["A"]), cuda(inp["D"]), y)
+    y_ref = np.zeros((nl * batch, H, P), np.float32)
+    pre = np.zeros((nl * batch, H * P, N), np.float32)
+    for i in range(nl * batch):
+        l, b = divmod(i, batch)
+        y_ref[i], pre[i] = O.step(ocfg, st, i, inp["x"][l, b], inp["B"][l, b], inp["C"][l, b],
+                                  inp["dt"][l, b], inp["A"][l], inp["D"][l], want_pre=True)
+    got = download(codec, pool, pairs, ocfg)
+    compare_states(ocfg, got, st, pre, f"units {fmt}")
+    Dpair = np.repeat(inp["D"][:, None, :], batch, axis=1).reshape(nl * batch, H)
+    scale = y_scale(ocfg, st, inp["C"].reshape(nl * batch, G, N), Dpair,
+                    inp["x"].reshape(nl * batch, H, P))
+    check_y(y.cpu().numpy().reshape(nl * batch, H, P), y_ref, scale, f"units {fmt}")
+    assert ssq.ssq_pool_error(cfg, pool) == 0
