@@ -359,8 +359,18 @@ ssq_status ssq_scan(const ssq_config* cfg, void* pool, const int32_t* slot_idx, 
     cv.A = A;
     cv.D = D;
     cv.y = y;
-    fill_tiles(pv, &cv, ssq::scan_rows_per_cta(cfg->d_state));
-    cudaError_t e = ssq::launch_scan(pv, cv, (int)cfg->fmt, stream);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    const ssq::ScanPlan sp = ssq::scan_plan(cfg->d_state, cfg->headdim,
+                                            (long long)batch * cfg->nheads, sms);
+    cv.tiles_per_head = sp.tiles_per_head;
+    cv.scan_chunk = sp.chunk;
+    cv.qtiles = pv.Hq * sp.tiles_per_head;
+    cv.ftiles = pv.Hf * sp.tiles_per_head;
+    cv.total_tiles = (long long)batch * (cv.qtiles + cv.ftiles);
+    e = ssq::launch_scan(pv, cv, (int)cfg->fmt, sp, stream);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     return SSQ_OK;
 }

@@ -32,6 +32,8 @@ struct CallView {
     int qtiles, ftiles;        // tiles per (layer, request) in each region
     long long total_tiles;
     int T;                     // tokens (scan only)
+    int tiles_per_head;        // scan: CTAs per head
+    int scan_chunk;            // scan: tokens staged per shared-memory buffer
     const float* x;
     const float* B;
     const float* C;
@@ -52,11 +54,17 @@ cudaError_t launch_quantize(const PoolView& pv, const CallView& cv, int fmt,
                             cudaStream_t stream);
 cudaError_t launch_dequantize(const PoolView& pv, const CallView& cv, int fmt,
                               cudaStream_t stream);
-cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt,
+// How the scan splits its rows: entries per lane, warps per CTA, rows per
+// CTA, CTAs per head, tokens per staged chunk, dynamic shared memory.
+struct ScanPlan {
+    int E, warps, rows, tiles_per_head, chunk;
+    size_t smem_bytes;
+};
+ScanPlan scan_plan(int d_state, int headdim, long long batch_heads, int sms);
+cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt, const ScanPlan& sp,
                         cudaStream_t stream);
 
-// Rows of one region each scan CTA owns; rows per decode tile.
-int scan_rows_per_cta(int d_state);
+// Rows per decode tile.
 int decode_rows_per_tile(int fmt, int d_state);
 // Whether the decode kernel's per-unit shared memory (B and C of every group,
 // per-head arrays) fits one CTA.

@@ -2,22 +2,29 @@
 //
 // "ssm-state-quantization" README, Setup: a sequential per-token scan
 // replaces the chunked library scan so that the state can be rounded at
-// every step.  Here each CTA owns a fixed tile of rows of one request for
-// all T tokens; the state stays in registers between tokens as the value the
-// stored codes decode to (fl((q - z) * Delta)), so T tokens of the scan equal
-// T decode steps bit for bit.  Only the final codes and metadata are written
-// back.  The per-token inputs (x, dt, B, C) of a chunk of K tokens are staged
-// into shared memory with cp.async one chunk ahead of the compute; lambda for
-// each (token, head) is computed once per CTA.
+// every step.  The state of a row lives in registers for all T tokens as the
+// value its stored codes decode to, fl((q - z) * Delta), so T tokens of the
+// scan equal T decode steps bit for bit; only the final codes and metadata
+// go back to the pool.
+//
+// Work split: a CTA of W warps owns W * RPW consecutive head_dim rows of ONE
+// head of one request, so lambda, dt, B and C are uniform across the CTA.
+// A row of N entries is held by LPR = N / E lanes, E consecutive entries
+// each.  The per-token inputs of K tokens (B and C of the head's group, x of
+// the CTA's rows, dt) are staged into shared memory with cp.async one chunk
+// ahead of the compute; B and C go in chunk-interleaved order (16-byte chunk
+// i of lane j at position i * LPR + j), so the lanes of a warp read
+// consecutive 16-byte words.  lambda = exp(dt * A) is computed once per
+// token per CTA.  The token loop streams each lane's entries in pieces of 16:
+// update and min / max, refit, then round, rescale and read out.
 #include "ssq_common.cuh"
 #include "ssq_params.h"
+
+#include <type_traits>
 
 namespace ssq {
 
 namespace {
-
-constexpr int kScanThreads = 64;
-constexpr int kChunk = 8;  // tokens staged per shared-memory buffer
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
 {
@@ -38,127 +45,157 @@ __device__ __forceinline__ void cp_async_wait_all()
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 }
 
-struct ScanGeom {
-    int rpc;    // rows per CTA
-    int nh;     // max heads a tile touches (B/C are staged per touched head)
+// Geometry of one scan instantiation.
+template <int N, int E>
+struct SGeom {
+    static constexpr int LPR = N / E;                 // lanes per row
+    static constexpr int RPW = 32 / LPR;              // rows per warp
+    static constexpr int NP = E / 16;                 // 16-entry pieces per lane
+    static_assert(E % 16 == 0 && N % E == 0 && LPR <= 32, "bad scan shape");
 };
 
-__host__ __device__ inline ScanGeom scan_geom(int N, int P, int H)
+// Floats of one staging buffer: B, C [K][N]; x [K][rows]; dt, lambda [K].
+__host__ __device__ inline int scan_buf_floats(int N, int K, int rows)
 {
-    ScanGeom g;
-    const int E = N >= 32 ? 32 : N;
-    g.rpc = kScanThreads / (N / E);
-    // tiles start at multiples of rpc: when rpc divides P a tile lies in one
-    // head, otherwise it spans at most floor((rpc-1)/P) + 2 heads
-    g.nh = (P % g.rpc == 0) ? 1 : min(H, (g.rpc - 1) / P + 2);
-    return g;
+    const int f = 2 * K * N + K * rows + 2 * K;
+    return (f + 3) / 4 * 4;   // keep the next buffer 16-byte aligned
 }
 
-// Floats per shared-memory buffer: B and C [kChunk][nh][N], x [kChunk][rpc],
-// dt and lambda [kChunk][nh].  A multiple of 8 floats, so both buffers stay
-// 16-byte aligned.
-__host__ __device__ inline int scan_buf_floats(const ScanGeom& g, int N)
+// Entries a lane owns for a given d_state: 64 when the batch gives enough
+// rows to fill the machine, else 32 (more warps, more latency hiding).
+__host__ __device__ inline int scan_entries(int N, bool wide)
 {
-    return 2 * kChunk * g.nh * N + kChunk * g.rpc + 2 * kChunk * g.nh;
+    if (N < 64) return N;
+    return wide ? 64 : 32;
 }
 
-template <int FMT, int N>
-__global__ void __launch_bounds__(kScanThreads)
+// Round 16 entries of a row on the fast path: s <- fl(rint(fl(s*inv)) *
+// Delta); with CODES also the carriers of the stored codes.
+template <int FMT, bool CODES>
+__device__ __forceinline__ void round_piece_fast(const RowParams& rp, float* s,
+                                                 uint32_t (&k)[16], float nz)
+{
+    using F = Fmt<FMT>;
+    const float2 nz2 = make_float2(nz, nz);
+    const float2 inv2 = make_float2(rp.inv, rp.inv);
+    const float2 d2 = make_float2(rp.delta, rp.delta);
+    const float2 m2 = make_float2(kMagic, kMagic);
+    const float2 nm2 = make_float2(-kMagic, -kMagic);
+    const float2 z2 = make_float2(rp.z, rp.z);
+#pragma unroll
+    for (int n = 0; n < 16; n += 2) {
+        const float2 p = fma2(make_float2(s[n], s[n + 1]), inv2, nz2);
+        const float2 t = add2(p, m2);          // 1.5*2^23 + rint(p)
+        const float2 r = add2(t, nm2);         // rint(p) = q - z, exact
+        const float2 v = mul2(r, d2);
+        s[n] = v.x; s[n + 1] = v.y;
+        if constexpr (CODES) {
+            if constexpr (F::sym) {
+                k[n] = __float_as_uint(t.x);
+                k[n + 1] = __float_as_uint(t.y);
+            } else {
+                const float2 u = add2(t, z2);  // 1.5*2^23 + q, exact
+                k[n] = __float_as_uint(u.x);
+                k[n + 1] = __float_as_uint(u.y);
+            }
+        }
+    }
+}
+
+// The scalar formulas verbatim, for rows the fast path does not cover.
+template <int FMT>
+__device__ __forceinline__ void round_piece_slow(const RowParams& rp, float* s,
+                                                 uint32_t (&k)[16])
+{
+    using F = Fmt<FMT>;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        const float rr = rintf(__fmul_rn(s[n], rp.inv));
+        float c, r;
+        if constexpr (F::sym) {
+            c = fminf(fmaxf(rr, -F::qmax), F::qmax);
+            r = c;
+        } else {
+            c = fminf(__fadd_rn(rr, rp.z), F::qmax);
+            r = __fsub_rn(c, rp.z);
+        }
+        s[n] = __fmul_rn(r, rp.delta);
+        k[n] = (uint32_t)(int)c;
+    }
+}
+
+template <int FMT, int N, int E>
+__global__ void __launch_bounds__(64)
 scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv)
 {
-    using S = Shape<N>;
     using F = Fmt<FMT>;
-    constexpr int E = S::E, LPR = S::LPR;
-    constexpr int CB = F::quant ? E * F::bits / 8 : 4;
+    using SG = SGeom<N, E>;
+    constexpr int LPR = SG::LPR, RPW = SG::RPW, NP = SG::NP;
+    constexpr int CB = F::quant ? E * F::bits / 8 : 4;   // code bytes per lane
+    constexpr int PW = Piece<FMT>::words;
     constexpr bool kBf16 = (FMT == SSQ_BF16);
     extern __shared__ __align__(16) float smem[];
 
     const int P = pv.P, H = pv.H, G = pv.G, T = cv.T;
-    const ScanGeom geo = scan_geom(N, P, H);
-    const int bufsz = scan_buf_floats(geo, N);
+    const int K = cv.scan_chunk;                         // tokens per staged chunk
+    const int nthreads = blockDim.x;
+    const int rows = (nthreads / 32) * RPW;             // rows per CTA
+    const int bufsz = scan_buf_floats(N, K, rows);
     uint32_t* err = reinterpret_cast<uint32_t*>(pv.pool);
 
-    // tile -> (request, region, first row)
+    // CTA -> (request, region, head, first row)
     const int per_b = cv.qtiles + cv.ftiles;
     const int b = blockIdx.x / per_b;
     const int k = blockIdx.x - b * per_b;
     const bool quant = k < cv.qtiles;
-    const int rbase = (quant ? k : k - cv.qtiles) * geo.rpc;
-    const int nrows = (quant ? pv.Hq : pv.Hf) * P;
+    const int kk = quant ? k : k - cv.qtiles;
+    const int tph = cv.tiles_per_head;
+    const int hrl = kk / tph;
+    const int p0 = (kk - hrl * tph) * rows;
     const int regbase = quant ? 0 : pv.Hq;
+    const int h = pv.perm[regbase + hrl];
+    const int g = h / pv.hpg;
     const int slot = cv.slot_idx ? __ldg(cv.slot_idx + b) : b;
     if (slot < 0 || slot >= pv.n_slots) {
         if (threadIdx.x == 0) atomicOr(err, SSQ_DEVERR_SLOT);
         return;  // block-uniform, before any barrier
     }
-    const int rlast = min(rbase + geo.rpc, nrows) - 1;
-    const int hr0 = rbase / P;
-    const int nh = rlast / P - hr0 + 1;   // <= geo.nh
 
     const int tid = threadIdx.x;
-    const int grow = tid / LPR;
-    const int j = tid % LPR;
-    const int r = rbase + grow;
-    const bool active = r < nrows;
-    const int rr = active ? r : rbase;
-    const int hrl = rr / P;
-    const int p = rr - hrl * P;
-    const int h = pv.perm[regbase + hrl];
-    const int hl = hrl - hr0;
+    const int lane = tid & 31;
+    const int rowc = (tid >> 5) * RPW + lane / LPR;      // row within the CTA
+    const int j = lane % LPR;
+    const bool active = p0 + rowc < P;
+    const int rowe = active ? rowc : 0;                  // inactive rows shadow row p0
+    const int p = p0 + rowe;
+    const int rr = hrl * P + p;                          // row within its region
     const float Av = __ldg(cv.A + h);
     const float Dv = __ldg(cv.D + h);
+    const long long bT = (long long)b * T;
 
-    // Stage the inputs of tokens [t0, t0 + kChunk) into buffer `bi`.
+    // Stage tokens [t0, t0 + nt) into buffer `bi`.
     auto stage = [&](int t0, int bi) {
-        float* base = smem + bi * bufsz;
-        float* sB = base;
-        float* sC = sB + kChunk * geo.nh * N;
-        float* sx = sC + kChunk * geo.nh * N;
-        float* sdt = sx + kChunk * geo.rpc;
-        const int nt = min(kChunk, T - t0);
-        const int nvec = nt * nh * (N / 4);
-        for (int i = tid; i < nvec; i += kScanThreads) {
-            const int tt = i / (nh * (N / 4));
-            const int rem = i - tt * nh * (N / 4);
-            const int hh = rem / (N / 4);
-            const int v = rem - hh * (N / 4);
-            const int gg = pv.perm[regbase + hr0 + hh] / pv.hpg;
-            const long long src = (((long long)b * T + t0 + tt) * G + gg) * N + 4 * v;
-            const int dst = (tt * geo.nh + hh) * N + 4 * v;
+        float* sB = smem + bi * bufsz;
+        float* sC = sB + K * N;
+        float* sx = sC + K * N;
+        float* sdt = sx + K * rows;
+        const int nt = min(K, T - t0);
+        constexpr int NC = N / 4;            // 16-byte chunks per row
+        constexpr int CPL = E / 4;           // chunks per lane
+        for (int i = tid; i < nt * NC; i += nthreads) {
+            const int tt = i / NC, c = i % NC;
+            const int dst = tt * N + ((c % CPL) * LPR + c / CPL) * 4;
+            const long long src = ((bT + t0 + tt) * G + g) * N + 4 * c;
             cp_async16(sB + dst, cv.B + src);
             cp_async16(sC + dst, cv.C + src);
         }
-        const int nx = nt * geo.rpc;
-        for (int i = tid; i < nx; i += kScanThreads) {
-            const int tt = i / geo.rpc;
-            const int row = rbase + (i - tt * geo.rpc);
-            if (row < nrows) {
-                const int hh = pv.perm[regbase + row / P];
-                const int pp = row % P;
-                cp_async4(sx + i, cv.x + (((long long)b * T + t0 + tt) * H + hh) * P + pp);
-            }
+        for (int i = tid; i < nt * rows; i += nthreads) {
+            const int tt = i / rows, r = i - tt * rows;
+            const int pr = p0 + (p0 + r < P ? r : 0);
+            cp_async4(sx + i, cv.x + ((bT + t0 + tt) * H + h) * P + pr);
         }
-        const int nd = nt * nh;
-        for (int i = tid; i < nd; i += kScanThreads) {
-            const int tt = i / nh;
-            const int hh = pv.perm[regbase + hr0 + (i - tt * nh)];
-            cp_async4(sdt + tt * geo.nh + (i - tt * nh),
-                      cv.dt + ((long long)b * T + t0 + tt) * H + hh);
-        }
+        if (tid < nt) cp_async4(sdt + tid, cv.dt + (bT + t0 + tid) * H + h);
         cp_async_commit();
-    };
-    // lambda of every (token, head) of a staged buffer
-    auto decays = [&](int t0, int bi) {
-        float* base = smem + bi * bufsz;
-        float* sdt = base + 2 * kChunk * geo.nh * N + kChunk * geo.rpc;
-        float* slam = sdt + kChunk * geo.nh;
-        const int nt = min(kChunk, T - t0);
-        for (int i = tid; i < nt * nh; i += kScanThreads) {
-            const int tt = i / nh;
-            const int hh2 = i - tt * nh;
-            const int hn = pv.perm[regbase + hr0 + hh2];
-            slam[tt * geo.nh + hh2] = decay(sdt[tt * geo.nh + hh2], __ldg(cv.A + hn));
-        }
     };
 
     uint8_t* slot_base = pv.pool + pv.header_bytes + (long long)slot * pv.slot_bytes;
@@ -168,28 +205,28 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
     uint8_t* frow = nullptr;
     constexpr int EB = kBf16 ? 2 : 4;
 
-    // Initial state, decoded once.
+    // The initial state, decoded once.
     float s[E];
     bool qrow = false;
     if constexpr (F::quant) qrow = quant;
     if constexpr (F::quant) {
-      if (qrow) {
-        crow = slot_base + pv.codes_off + (long long)layer * pv.codes_layer_bytes
-               + (long long)rr * (N * F::bits / 8) + j * CB;
-        mrow = slot_base + pv.meta_off + (long long)layer * pv.meta_layer_bytes
-               + (long long)rr * F::meta_bytes;
-        Chunk<CB> c;
-        load_chunk<CB>(c, crow);
-        float delta0, z0 = 0.0f;
-        if constexpr (F::sym) {
-            delta0 = *reinterpret_cast<const float*>(mrow);
-        } else {
-            const float2 m = *reinterpret_cast<const float2*>(mrow);
-            delta0 = m.x;
-            z0 = m.y;
+        if (qrow) {
+            crow = slot_base + pv.codes_off + (long long)layer * pv.codes_layer_bytes
+                   + (long long)rr * (N * F::bits / 8) + j * CB;
+            mrow = slot_base + pv.meta_off + (long long)layer * pv.meta_layer_bytes
+                   + (long long)rr * F::meta_bytes;
+            Chunk<CB> c;
+            load_chunk<CB>(c, crow);
+            float delta0, z0 = 0.0f;
+            if constexpr (F::sym) {
+                delta0 = *reinterpret_cast<const float*>(mrow);
+            } else {
+                const float2 m = *reinterpret_cast<const float2*>(mrow);
+                delta0 = m.x;
+                z0 = m.y;
+            }
+            decode_row<FMT, E>(c, delta0, z0, s);
         }
-        decode_row<FMT, E>(c, delta0, z0, s);
-      }
     }
     if (!qrow) {
         frow = slot_base + pv.fp_off + (long long)layer * pv.fp_layer_bytes
@@ -208,77 +245,158 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
         }
     }
 
-    stage(0, 0);
-    cp_async_wait_all();
-    __syncthreads();
-    decays(0, 0);
-    __syncthreads();
-
     RowParams rp{};
-    uint32_t kfin[E];
+    uint32_t cw[F::quant ? CB / 4 : 1];
     bool finite_all = true;
-    const int nchunks = (T + kChunk - 1) / kChunk;
+    const long long HP = (long long)H * P;
+    float* const yrow = cv.y + (bT * H + h) * P + p;   // y of this row at token 0
+    const bool ylane = active && j == 0;
+    const int nchunks = (T + K - 1) / K;
+    stage(0, 0);
     for (int c = 0; c < nchunks; ++c) {
         const int bi = c & 1;
-        const int t0 = c * kChunk;
-        if (c + 1 < nchunks) stage(t0 + kChunk, bi ^ 1);
-        const float* base = smem + bi * bufsz;
-        const float* sB = base;
-        const float* sC = sB + kChunk * geo.nh * N;
-        const float* sx = sC + kChunk * geo.nh * N;
-        const float* sdt = sx + kChunk * geo.rpc;
-        const float* slam = sdt + kChunk * geo.nh;
-        const int nt = min(kChunk, T - t0);
-        for (int tt = 0; tt < nt; ++tt) {
-            const float lam = slam[tt * geo.nh + hl];
-            const float xv = sx[tt * geo.rpc + (active ? grow : 0)];
-            const float dtx = __fmul_rn(sdt[tt * geo.nh + hl], xv);
-            float Bv[E], Cv[E];
-            const float* bp = sB + (tt * geo.nh + hl) * N + j * E;
-            const float* cp = sC + (tt * geo.nh + hl) * N + j * E;
+        const int t0 = c * K;
+        const int nt = min(K, T - t0);
+        cp_async_wait_all();
+        __syncthreads();   // chunk c visible to all; everyone is done with chunk c-1
+        if (c + 1 < nchunks) stage(t0 + K, bi ^ 1);
+        const float* sB = smem + bi * bufsz;
+        const float* sC = sB + K * N;
+        const float* sx = sC + K * N;
+        float* sdt = const_cast<float*>(sx + K * rows);
+        float* slam = sdt + K;
+        if (tid < nt) slam[tid] = decay(sdt[tid], Av);
+        __syncthreads();
+
+        float* const yc = yrow + (long long)t0 * HP;
+        // update + min / max of one token's B over the lane's entries
+        auto update_q = [&](int tt, float& lo, float& hi) {
+            const float xv = sx[tt * rows + rowe];
+            const float dtx = __fmul_rn(sdt[tt], xv);
+            const float2 l2 = make_float2(slam[tt], slam[tt]);
+            const float2 x2 = make_float2(dtx, dtx);
+            const float4* b4 = reinterpret_cast<const float4*>(sB + tt * N) + j;
+            float plo[NP], phi[NP];
 #pragma unroll
-            for (int i = 0; i < E / 4; ++i) {
-                const float4 vb = reinterpret_cast<const float4*>(bp)[i];
-                Bv[4 * i] = vb.x; Bv[4 * i + 1] = vb.y; Bv[4 * i + 2] = vb.z; Bv[4 * i + 3] = vb.w;
-            }
-            update_row<E>(lam, dtx, Bv, s);
-            if constexpr (F::quant) {
-                if (qrow) {
-                    rp = refit_row<FMT, E, LPR>(s);
-                    finite_all = finite_all && rp.finite;
-                    float rq[E];
-                    round_row<FMT, E>(rp, s, rq, kfin, pv.neg_zero);
-                    scale_row<E>(rp.delta, rq, s);
+            for (int pc = 0; pc < NP; ++pc) {
+                float* sp = s + 16 * pc;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 v = b4[(4 * pc + i) * LPR];
+                    const float2 w0 = mul2(x2, make_float2(v.x, v.y));
+                    const float2 w1 = mul2(x2, make_float2(v.z, v.w));
+                    const float2 u0 = fma2(l2, make_float2(sp[4 * i], sp[4 * i + 1]), w0);
+                    const float2 u1 = fma2(l2, make_float2(sp[4 * i + 2], sp[4 * i + 3]), w1);
+                    sp[4 * i] = u0.x; sp[4 * i + 1] = u0.y;
+                    sp[4 * i + 2] = u1.x; sp[4 * i + 3] = u1.y;
                 }
-            } else if constexpr (kBf16) {
-#pragma unroll
-                for (int n = 0; n < E; ++n)
-                    s[n] = __bfloat162float(__float2bfloat16_rn(s[n]));
+                minmax16(sp, plo[pc], phi[pc]);
             }
+            lo = plo[0];
+            hi = phi[0];
 #pragma unroll
-            for (int i = 0; i < E / 4; ++i) {
-                const float4 vc = reinterpret_cast<const float4*>(cp)[i];
-                Cv[4 * i] = vc.x; Cv[4 * i + 1] = vc.y; Cv[4 * i + 2] = vc.z; Cv[4 * i + 3] = vc.w;
+            for (int pc = 1; pc < NP; ++pc) {
+                lo = fminf(lo, plo[pc]);
+                hi = fmaxf(hi, phi[pc]);
             }
-            const float ysum = grp_sum<LPR>(dot_row<E>(Cv, s));
-            if (active && j == 0) {
-                const float yv = __fadd_rn(ysum, __fmul_rn(Dv, xv));
-                __stcs(cv.y + (((long long)b * T + t0 + tt) * H + h) * P + p, yv);
+            return xv;
+        };
+        // C . s over the lane's entries
+        auto readout = [&](int tt) {
+            const float4* c4 = reinterpret_cast<const float4*>(sC + tt * N) + j;
+            float2 accp[NP];
+#pragma unroll
+            for (int pc = 0; pc < NP; ++pc) {
+                const float* sp = s + 16 * pc;
+                float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 v = c4[(4 * pc + i) * LPR];
+                    acc = fma2(make_float2(v.x, v.y), make_float2(sp[4 * i], sp[4 * i + 1]), acc);
+                    acc = fma2(make_float2(v.z, v.w), make_float2(sp[4 * i + 2], sp[4 * i + 3]), acc);
+                }
+                accp[pc] = acc;
+            }
+            float2 acc = accp[0];
+#pragma unroll
+            for (int pc = 1; pc < NP; ++pc) acc = add2(acc, accp[pc]);
+            return grp_sum<LPR>(__fadd_rn(acc.x, acc.y));
+        };
+        auto emit_y = [&](int tt, float ysum, float xv) {
+            if (ylane) __stcs(yc + (long long)tt * HP, __fadd_rn(ysum, __fmul_rn(Dv, xv)));
+        };
+        // one token of a quantized row; CODES: also pack the stored codes
+        auto qtoken = [&](auto codes_tag, int tt) {
+            constexpr bool CODES = decltype(codes_tag)::value;
+            float lo, hi;
+            const float xv = update_q(tt, lo, hi);
+            rp = refit_from_minmax<FMT, LPR>(lo, hi);
+            finite_all = finite_all && rp.finite;
+            uint32_t kc[16];
+            if (__all_sync(0xffffffffu, rp.fast && !rp.clamp)) {
+#pragma unroll
+                for (int pc = 0; pc < NP; ++pc) {
+                    round_piece_fast<FMT, CODES>(rp, s + 16 * pc, kc, pv.neg_zero);
+                    if constexpr (CODES) pack16<FMT>(kc, cw + PW * pc);
+                }
+            } else {
+#pragma unroll
+                for (int pc = 0; pc < NP; ++pc) {
+                    round_piece_slow<FMT>(rp, s + 16 * pc, kc);
+                    if constexpr (CODES) pack16<FMT>(kc, cw + PW * pc);
+                }
+            }
+            emit_y(tt, readout(tt), xv);
+        };
+        // one token of an fp row (fp32 update, rounded to bf16 for bf16)
+        auto ftoken = [&](int tt) {
+            const float xv = sx[tt * rows + rowe];
+            const float dtx = __fmul_rn(sdt[tt], xv);
+            const float2 l2 = make_float2(slam[tt], slam[tt]);
+            const float2 x2 = make_float2(dtx, dtx);
+            const float4* b4 = reinterpret_cast<const float4*>(sB + tt * N) + j;
+#pragma unroll
+            for (int pc = 0; pc < NP; ++pc) {
+                float* sp = s + 16 * pc;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 v = b4[(4 * pc + i) * LPR];
+                    const float2 w0 = mul2(x2, make_float2(v.x, v.y));
+                    const float2 w1 = mul2(x2, make_float2(v.z, v.w));
+                    float2 u0 = fma2(l2, make_float2(sp[4 * i], sp[4 * i + 1]), w0);
+                    float2 u1 = fma2(l2, make_float2(sp[4 * i + 2], sp[4 * i + 3]), w1);
+                    if constexpr (kBf16) {
+                        u0 = __bfloat1622float2(__float22bfloat162_rn(u0));
+                        u1 = __bfloat1622float2(__float22bfloat162_rn(u1));
+                    }
+                    sp[4 * i] = u0.x; sp[4 * i + 1] = u0.y;
+                    sp[4 * i + 2] = u1.x; sp[4 * i + 3] = u1.y;
+                }
+            }
+            emit_y(tt, readout(tt), xv);
+        };
+
+        bool qdone = false;
+        if constexpr (F::quant) {
+            if (qrow) {
+                qdone = true;
+                // the final token also packs the codes that go back to the pool
+                const int nmain = (t0 + nt == T) ? nt - 1 : nt;
+                for (int tt = 0; tt < nmain; ++tt) qtoken(std::false_type{}, tt);
+                if (nmain < nt) qtoken(std::true_type{}, nmain);
             }
         }
-        if (c + 1 < nchunks) {
-            cp_async_wait_all();
-            __syncthreads();               // staged data visible; old buffer free
-            decays(t0 + kChunk, bi ^ 1);
-            __syncthreads();
-        }
+        if (!qdone)
+            for (int tt = 0; tt < nt; ++tt) ftoken(tt);
     }
 
-    // Final state back to the pool.
-    if (active && qrow) {
+    // The final state back to the pool.
+    if (!active) return;
+    if (qrow) {
         if constexpr (F::quant) {
             Chunk<CB> c;
-            pack_codes<FMT, E>(kfin, c);
+#pragma unroll
+            for (int i = 0; i < CB / 4; ++i) c.w[i] = cw[i];
             store_chunk<CB>(crow, c);
             if (j == 0) {
                 if constexpr (F::sym) {
@@ -289,7 +407,7 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
                 if (!finite_all) atomicOr(err, SSQ_DEVERR_NONFINITE);
             }
         }
-    } else if (active) {
+    } else {
         if constexpr (kBf16) {
             Chunk<E * 2> c;
 #pragma unroll
@@ -306,57 +424,83 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
     }
 }
 
-template <int FMT, int N>
-cudaError_t launch_scan_n(const PoolView& pv, const CallView& cv, int grid,
-                          cudaStream_t st)
+template <int FMT, int N, int E>
+cudaError_t launch_scan_ne(const PoolView& pv, const CallView& cv, int warps, int grid,
+                           cudaStream_t st)
 {
-    const ScanGeom g = scan_geom(N, pv.P, pv.H);
-    const size_t smem = 2 * (size_t)scan_buf_floats(g, N) * sizeof(float);
-    auto kern = scan_kernel<FMT, N>;
+    using SG = SGeom<N, E>;
+    const size_t smem =
+        2 * (size_t)scan_buf_floats(N, cv.scan_chunk, warps * SG::RPW) * sizeof(float);
+    auto kern = scan_kernel<FMT, N, E>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
     }
-    kern<<<grid, kScanThreads, smem, st>>>(pv, cv);
+    kern<<<grid, 32 * warps, smem, st>>>(pv, cv);
     return cudaGetLastError();
 }
 
 template <int FMT>
-cudaError_t launch_scan_fmt(const PoolView& pv, const CallView& cv, int grid,
-                            cudaStream_t st)
+cudaError_t launch_scan_fmt(const PoolView& pv, const CallView& cv, int E, int warps,
+                            int grid, cudaStream_t st)
 {
     switch (pv.N) {
-    case 16: return launch_scan_n<FMT, 16>(pv, cv, grid, st);
-    case 32: return launch_scan_n<FMT, 32>(pv, cv, grid, st);
-    case 64: return launch_scan_n<FMT, 64>(pv, cv, grid, st);
-    case 128: return launch_scan_n<FMT, 128>(pv, cv, grid, st);
-    case 256: return launch_scan_n<FMT, 256>(pv, cv, grid, st);
+    case 16: return launch_scan_ne<FMT, 16, 16>(pv, cv, warps, grid, st);
+    case 32: return launch_scan_ne<FMT, 32, 32>(pv, cv, warps, grid, st);
+    case 64:
+        return E == 64 ? launch_scan_ne<FMT, 64, 64>(pv, cv, warps, grid, st)
+                       : launch_scan_ne<FMT, 64, 32>(pv, cv, warps, grid, st);
+    case 128:
+        return E == 64 ? launch_scan_ne<FMT, 128, 64>(pv, cv, warps, grid, st)
+                       : launch_scan_ne<FMT, 128, 32>(pv, cv, warps, grid, st);
+    case 256:
+        return E == 64 ? launch_scan_ne<FMT, 256, 64>(pv, cv, warps, grid, st)
+                       : launch_scan_ne<FMT, 256, 32>(pv, cv, warps, grid, st);
     default: return cudaErrorInvalidValue;
     }
 }
 
 }  // namespace
 
-int scan_rows_per_cta(int d_state)
+ScanPlan scan_plan(int d_state, int headdim, long long batch_heads, int sms)
 {
-    const int E = d_state >= 32 ? 32 : d_state;
-    return kScanThreads / (d_state / E);
+    // Wide rows (64 entries per lane) unless that leaves fewer than three
+    // warps per SM sub-partition.
+    const int N = d_state;
+    const int rpw64 = 32 / (N / scan_entries(N, true));
+    const long long warps64 = batch_heads * ((headdim + rpw64 - 1) / rpw64);
+    const bool wide = (N < 64) || warps64 >= 3LL * 4 * sms;
+    ScanPlan sp;
+    sp.E = scan_entries(N, wide);
+    const int rpw = 32 / (N / sp.E);
+    // Two warps per CTA (one when the head has rows for only one): small
+    // CTAs spread evenly over the SMs, and two warps halve the staging.
+    const int wneed = (headdim + rpw - 1) / rpw;
+    sp.warps = wneed < 2 ? 1 : 2;
+    sp.rows = sp.warps * rpw;
+    sp.tiles_per_head = (headdim + sp.rows - 1) / sp.rows;
+    // Tokens per staged chunk: two buffers of B and C of K tokens stay near
+    // 16 KB per CTA.
+    sp.chunk = N <= 128 ? 8 : 4;
+    sp.smem_bytes = 2 * (size_t)scan_buf_floats(N, sp.chunk, sp.rows) * sizeof(float);
+    return sp;
 }
 
-cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt,
+cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt, const ScanPlan& sp,
                         cudaStream_t st)
 {
     const long long grid = (long long)cv.batch * (cv.qtiles + cv.ftiles);
     if (grid <= 0) return cudaSuccess;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const int g = (int)grid, E = sp.E, w = sp.warps;
     switch (fmt) {
-    case SSQ_F32: return launch_scan_fmt<SSQ_F32>(pv, cv, (int)grid, st);
-    case SSQ_BF16: return launch_scan_fmt<SSQ_BF16>(pv, cv, (int)grid, st);
-    case SSQ_I8_SYM: return launch_scan_fmt<SSQ_I8_SYM>(pv, cv, (int)grid, st);
-    case SSQ_I8_ASYM: return launch_scan_fmt<SSQ_I8_ASYM>(pv, cv, (int)grid, st);
-    case SSQ_I4_SYM: return launch_scan_fmt<SSQ_I4_SYM>(pv, cv, (int)grid, st);
-    case SSQ_I4_ASYM: return launch_scan_fmt<SSQ_I4_ASYM>(pv, cv, (int)grid, st);
+    case SSQ_F32: return launch_scan_fmt<SSQ_F32>(pv, cv, E, w, g, st);
+    case SSQ_BF16: return launch_scan_fmt<SSQ_BF16>(pv, cv, E, w, g, st);
+    case SSQ_I8_SYM: return launch_scan_fmt<SSQ_I8_SYM>(pv, cv, E, w, g, st);
+    case SSQ_I8_ASYM: return launch_scan_fmt<SSQ_I8_ASYM>(pv, cv, E, w, g, st);
+    case SSQ_I4_SYM: return launch_scan_fmt<SSQ_I4_SYM>(pv, cv, E, w, g, st);
+    case SSQ_I4_ASYM: return launch_scan_fmt<SSQ_I4_ASYM>(pv, cv, E, w, g, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -356,6 +356,27 @@ def test_scan_groups_and_ragged_tiles(fmt):
     run_scan(fmt, H=6, P=12, N=64, G=3, batch=3, T=19, seed=8)
 
 
+def _wide_scan_batch(H, P, N):
+    """Requests that make the scan give each lane 64 entries of a row: at
+    least three warps per SM sub-partition at 32 / (N / 64) rows per warp."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rpw = 32 // (N // 64)
+    per_request = H * -(-P // rpw)
+    return -(-3 * 4 * sms // per_request)
+
+
+@pytest.mark.parametrize("fmt,H,N", [("i8a", 32, 128), ("i4s", 32, 128), ("bf16", 32, 128),
+                                     ("i8s", 16, 256), ("i4a", 32, 64), ("f32", 16, 256)])
+def test_scan_wide_rows(fmt, H, N):
+    """Batches large enough for 64 entries per lane (one lane per row at
+    d_state 64, four at 256), over several staged chunks."""
+    ssq = require_gpu()
+    del ssq
+    P = 64
+    batch = _wide_scan_batch(H, P, N)
+    run_scan(fmt, H=H, P=P, N=N, G=2, batch=batch, T=11, seed=12)
+
+
 @pytest.mark.parametrize("fmt", ["i8a", "i4a", "i8s", "f32"])
 def test_scan_equals_repeated_decode(fmt):
     """T tokens of the scan leave exactly the codes and metadata that T decode
