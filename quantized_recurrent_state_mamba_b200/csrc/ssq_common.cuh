@@ -517,6 +517,43 @@ __device__ __forceinline__ void round16_fast(const RowParams& rp, const float* s
     }
 }
 
+// Fast rounding of 16 entries for the decode step: r = q - z (asym) or q
+// (sym) exactly, k carries the stored code.  With CLAMP the asymmetric code
+// is capped at qa first (min(rint(p) + z, qa): the top code of a row whose
+// largest entry rounds one step past the grid).  mz2 holds -(1.5*2^23 + z),
+// nm2 -1.5*2^23; both sums are exact because every operand is an integer
+// below 2^24 in magnitude.
+template <int FMT, bool CLAMP>
+__device__ __forceinline__ void round16_carry(float2 inv2, float2 z2, float2 mz2, float* s,
+                                              float* r, uint32_t (&k)[16], float nz)
+{
+    using F = Fmt<FMT>;
+    const float2 nz2 = make_float2(nz, nz);
+    const float2 m2 = make_float2(kMagic, kMagic);
+    constexpr float kTop = kMagic + F::qmax;   // carrier of code qa
+#pragma unroll
+    for (int n = 0; n < 16; n += 2) {
+        const float2 p = fma2(make_float2(s[n], s[n + 1]), inv2, nz2);
+        const float2 t = add2(p, m2);                  // 1.5*2^23 + rint(p)
+        if constexpr (F::sym) {
+            const float2 rr = add2(t, mz2);            // rint(p), exact
+            r[n] = rr.x; r[n + 1] = rr.y;
+            k[n] = __float_as_uint(t.x);
+            k[n + 1] = __float_as_uint(t.y);
+        } else {
+            float2 u = add2(t, z2);                    // 1.5*2^23 + q
+            if constexpr (CLAMP) {
+                u.x = fminf(u.x, kTop);
+                u.y = fminf(u.y, kTop);
+            }
+            const float2 rr = add2(u, mz2);            // q - z, exact
+            r[n] = rr.x; r[n + 1] = rr.y;
+            k[n] = __float_as_uint(u.x);
+            k[n + 1] = __float_as_uint(u.y);
+        }
+    }
+}
+
 // Exact scalar rounding of 16 entries (the definition verbatim).
 template <int FMT>
 __device__ __forceinline__ void round16_slow(const RowParams& rp, const float* s, float* r,

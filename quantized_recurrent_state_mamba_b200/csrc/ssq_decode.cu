@@ -9,27 +9,39 @@
 // parameters, and writes the packed state back"), with the quantizer of
 // "ssm-state-quantization" README, Setup.
 //
-// Structure (persistent, warp-specialised, two CTAs per SM):
+// Structure (persistent, warp-specialised, one CTA of 12 warps per SM):
 //   - work is a sequence of tiles (up to RPT rows of one region of one
 //     (layer, request)); each CTA owns a contiguous range of that sequence;
 //   - a producer warp streams each tile's packed rows and metadata from HBM
 //     into a ring of shared-memory stages with bulk asynchronous copies
 //     (cp.async.bulk, completion counted in bytes on an mbarrier) and the
-//     tile's x values with cp.async; once per (layer, request, region)
-//     "unit" it stages B, C, dt, A, D into one of two unit buffers;
-//   - 8 consumer warps compute from shared memory and store the new rows,
-//     metadata and y straight to global memory;
-//   - every wait is bounded: a wait that runs out sets SSQ_DEVERR_TIMEOUT in
-//     the pool's error word and the CTA winds down (the producer first waits
-//     for its own copies in flight).
+//     tile's x values with cp.async.  Once per (layer, request, region)
+//     "unit" it stages B and C and builds a head table (lambda, dt, D, the
+//     y offset and the B/C group of every head of the region), so a
+//     consumer row finds everything it needs with two shared loads;
+//   - 11 consumer warps compute from shared memory and store the new rows,
+//     metadata and y straight to global memory.  A row of a quantized head
+//     is held by LPR lanes with E = 64 entries each, streamed 16 at a time;
+//   - B and C are staged with lane j's 16-byte chunks interleaved, so the
+//     lanes of a row read distinct banks;
+//   - waits sleep between tries of the mbarrier, and every wait is
+//     bounded: one that runs out sets SSQ_DEVERR_TIMEOUT in the pool's error
+//     word and the CTA winds down (the producer first waits for its own
+//     copies in flight).
 #include "ssq_common.cuh"
 #include "ssq_params.h"
+
+#include <type_traits>
 
 namespace ssq {
 
 namespace {
 
-constexpr int kCWarps = 7;  // + 1 producer: 8-warp CTAs, two per SM
+// One CTA of 12 warps per SM: three warps per SM sub-partition, so each
+// thread may hold up to 168 registers (the row of 64 entries plus the f32x2
+// operand pairs stay in registers).
+constexpr int kCWarps = 11;    // + 1 producer
+constexpr int kMinBlocks = 1;  // CTAs per SM
 constexpr int kCThreads = kCWarps * 32;
 constexpr int kDThreads = kCThreads + 32;
 constexpr int kMaxStages = 8;
@@ -62,16 +74,25 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, unsigned parity)
                  : "=r"(ok) : "r"(saddr(b)), "r"(parity) : "memory");
     return ok != 0;
 }
-// Wait for the phase of the given parity to complete; false after about a
-// second without progress.
+// Wait for the phase of the given parity to complete, sleeping between
+// tries (exponential back-off up to kMaxSleepNs, so a waiting warp takes
+// few issue slots from the warps that compute); false after about a second
+// without progress.
+template <unsigned kMaxSleepNs>
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, unsigned parity)
 {
     if (mbar_try(b, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try(b, parity))
+    unsigned ns = 64;
+    while (!mbar_try(b, parity)) {
+        __nanosleep(ns);
+        ns = ns < kMaxSleepNs ? 2 * ns : kMaxSleepNs;
         if (clock64() - t0 > kWaitLimit) return false;
+    }
     return true;
 }
+constexpr unsigned kProducerSleep = 2048;  // the producer waits for a stage to drain
+constexpr unsigned kConsumerSleep = 256;   // consumers wait for data to land
 // Bulk copy global -> shared; completion counted in bytes on `bar`.
 // Both addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar)
@@ -94,6 +115,7 @@ __device__ __forceinline__ void cpa_arrive(uint64_t* b)
 }
 
 __host__ __device__ inline int r16(int v) { return (v + 15) & ~15; }
+__host__ __device__ inline int r128(int v) { return (v + 127) & ~127; }
 
 // ---- tile sequence -----------------------------------------------------
 // Tiles are ordered (layer, request, region, row block).  A CTA walks a
@@ -103,7 +125,6 @@ struct TileWalk {
     int l, b, k;    // k: tile within (layer, request)
     bool quant;
     int rbase, n;   // first region row, rows in this tile
-    long long key;  // unit key: (lb, region)
 
     __device__ __forceinline__ void fill(const PoolView& pv, const CallView& cv)
     {
@@ -111,7 +132,6 @@ struct TileWalk {
         rbase = (quant ? k : k - cv.qtiles) * cv.rows_per_tile;
         const int nrows = (quant ? pv.Hq : pv.Hf) * pv.P;
         n = min(cv.rows_per_tile, nrows - rbase);
-        key = lb * 2 + (quant ? 0 : 1);
     }
     __device__ __forceinline__ void start(const PoolView& pv, const CallView& cv, long long t)
     {
@@ -122,8 +142,10 @@ struct TileWalk {
         b = (int)(lb - (long long)l * cv.batch);
         fill(pv, cv);
     }
-    __device__ __forceinline__ void next(const PoolView& pv, const CallView& cv)
+    // Advance; true when the next tile starts a new unit.
+    __device__ __forceinline__ bool next(const PoolView& pv, const CallView& cv)
     {
+        const bool was_quant = quant;
         if (++k == cv.qtiles + cv.ftiles) {
             k = 0;
             ++lb;
@@ -131,12 +153,19 @@ struct TileWalk {
                 b = 0;
                 ++l;
             }
+            fill(pv, cv);
+            return true;
         }
         fill(pv, cv);
+        return quant != was_quant;
     }
 };
 
 // ---- shared-memory geometry (host and device agree on it) --------------
+// Unit buffer: [16 B header: slot, bad][B: G*N f32][C: G*N f32]
+//              [head table: Hpad x float4 {lambda, dt, D, y offset}]
+//              [group table: Hpad x int (g*N)]
+// Stage:       [x: RPT f32, padded to 128 B][payload: codes + meta, or fp rows]
 struct DecodeGeom {
     int S;            // stages
     int RPT;          // rows per tile
@@ -144,9 +173,9 @@ struct DecodeGeom {
     int qcodes_bytes; // codes area of a quantized tile
     int pay_bytes;    // payload area of a stage
     int stage_bytes;
-    int ub_B, ub_C, ub_dt, ub_A, ub_D, unit_bytes;  // unit buffer layout
-    int Hpad;         // floats per lambda array
-    int off_units, off_lam, off_stages, smem_bytes;
+    int ub_B, ub_C, ub_ht, ub_gt, unit_bytes;  // unit buffer layout
+    int Hpad;
+    int off_units, off_stages, smem_bytes;
 };
 
 __host__ __device__ inline DecodeGeom decode_geom(int S, int RPT, int RB, int MB, int fpEB,
@@ -155,38 +184,111 @@ __host__ __device__ inline DecodeGeom decode_geom(int S, int RPT, int RB, int MB
     DecodeGeom g;
     g.S = S;
     g.RPT = RPT;
-    g.x_bytes = r16(RPT * 4);
+    g.x_bytes = r128(RPT * 4);
     g.qcodes_bytes = r16(RPT * RB);
     const int qpay = g.qcodes_bytes + r16(RPT * MB);
     const int fpay = has_fp ? RPT * N * fpEB : 0;
     g.pay_bytes = qpay > fpay ? qpay : fpay;
-    g.stage_bytes = g.x_bytes + g.pay_bytes;
+    g.stage_bytes = r128(g.x_bytes + g.pay_bytes);
     g.Hpad = (H + 3) & ~3;
-    g.ub_B = 16;  // 16-byte header: slot, bad flag
+    g.ub_B = 16;
     g.ub_C = g.ub_B + G * N * 4;
-    g.ub_dt = g.ub_C + G * N * 4;
-    g.ub_A = g.ub_dt + g.Hpad * 4;
-    g.ub_D = g.ub_A + g.Hpad * 4;
-    g.unit_bytes = r16(g.ub_D + g.Hpad * 4);
-    const int bars = r16((2 * kMaxStages + 4) * 8);
+    g.ub_ht = g.ub_C + G * N * 4;
+    g.ub_gt = g.ub_ht + g.Hpad * 16;
+    g.unit_bytes = r128(g.ub_gt + g.Hpad * 4);
+    const int bars = r128((2 * kMaxStages + 4) * 8);
     g.off_units = bars;
-    g.off_lam = g.off_units + 2 * g.unit_bytes;
-    g.off_stages = r16(g.off_lam + kCWarps * 2 * g.Hpad * 4);
+    g.off_stages = g.off_units + 2 * g.unit_bytes;
     g.smem_bytes = g.off_stages + S * g.stage_bytes;
     return g;
 }
 
-// Lane shape of the decode kernel: quantized rows give each lane 64 entries
-// (two lanes per 128-entry row), which halves the per-row and per-tile
-// bookkeeping per entry; fp rows keep 32 entries per lane.
+// Lane shape: quantized rows give each lane 64 entries (two lanes per
+// 128-entry row); fp rows keep 32 entries per lane.
 template <int FMT, int N>
 struct DShape {
     static constexpr int E = Fmt<FMT>::quant ? (N >= 64 ? 64 : N) : (N >= 32 ? 32 : N);
     static constexpr int LPR = N / E;
 };
 
+// A whole quantized row by the formulas verbatim (every fp32 operation one
+// IEEE rounding in the order of the definition), for warps where some row
+// falls outside the magic-number paths: a zero point or scaled values of
+// 2^22 or more in magnitude (rows far from zero relative to their range).  Every lane of the warp
+// calls it together (the row reductions are shuffles).  Codes are read from
+// and written in natural order; B and C come from the interleaved layout.
 template <int FMT, int N>
-__global__ void __launch_bounds__(kDThreads, 2)
+__device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float delta0, float z0,
+                                        float lam, float dtx, const float* __restrict__ gB,
+                                        const float* __restrict__ gC, int j, bool active,
+                                        uint8_t* __restrict__ crow, uint8_t* __restrict__ mrow,
+                                        uint32_t* err)
+{
+    using F = Fmt<FMT>;
+    constexpr int E = DShape<FMT, N>::E, LPR = DShape<FMT, N>::LPR;
+    constexpr int NP = E / 16;
+    constexpr int CB = E * F::bits / 8;
+    float s[E];
+    float lo = 0.0f, hi = 0.0f;
+#pragma unroll 1
+    for (int n = 0; n < E; ++n) {
+        int q;
+        if constexpr (F::bits == 8) {
+            const uint32_t bb = cs[n];
+            q = F::sym ? (int)(int8_t)bb : (int)bb;
+        } else {
+            const uint32_t bb = (cs[n / 2] >> (4 * (n % 2))) & 0xFu;
+            q = F::sym ? (int)((bb ^ 8u) - 8u) : (int)bb;
+        }
+        const float v = __fmul_rn(__fsub_rn((float)q, z0), delta0);
+        const int pc = n / 16, i = (n % 16) / 4, e = n % 4;
+        const int bi = ((i * NP + pc) * LPR + j) * 4 + e;
+        const float w = __fmul_rn(dtx, gB[bi]);
+        const float sv = __fmaf_rn(lam, v, w);
+        s[n] = sv;
+        lo = n == 0 ? sv : fminf(lo, sv);
+        hi = n == 0 ? sv : fmaxf(hi, sv);
+    }
+    const RowParams rp = refit_from_minmax<FMT, LPR>(lo, hi);
+    float acc = 0.0f;
+    uint32_t words[CB / 4];
+#pragma unroll
+    for (int i = 0; i < CB / 4; ++i) words[i] = 0u;
+#pragma unroll 1
+    for (int n = 0; n < E; ++n) {
+        const float rr = rintf(__fmul_rn(s[n], rp.inv));
+        float c, r;
+        if constexpr (F::sym) {
+            c = fminf(fmaxf(rr, -F::qmax), F::qmax);
+            r = c;
+        } else {
+            c = fminf(__fadd_rn(rr, rp.z), F::qmax);
+            r = __fsub_rn(c, rp.z);
+        }
+        const uint32_t code = (uint32_t)(int)c & ((1u << F::bits) - 1u);
+        words[n * F::bits / 32] |= code << ((n * F::bits) % 32);
+        const int pc = n / 16, i = (n % 16) / 4, e = n % 4;
+        const int ci = ((i * NP + pc) * LPR + j) * 4 + e;
+        acc = __fmaf_rn(gC[ci], __fmul_rn(r, rp.delta), acc);
+    }
+    const float ysum = grp_sum<LPR>(acc);
+    if (active) {
+#pragma unroll
+        for (int i = 0; i < CB / 4; ++i) reinterpret_cast<uint32_t*>(crow)[i] = words[i];
+        if (j == 0) {
+            if constexpr (F::sym) {
+                *reinterpret_cast<float*>(mrow) = rp.delta;
+            } else {
+                *reinterpret_cast<float2*>(mrow) = make_float2(rp.delta, rp.z);
+            }
+            if (!rp.finite) atomicOr(err, SSQ_DEVERR_NONFINITE);
+        }
+    }
+    return ysum;
+}
+
+template <int FMT, int N>
+__global__ void __launch_bounds__(kDThreads, kMinBlocks)
 decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv,
               const __grid_constant__ DecodeGeom geo)
 {
@@ -197,9 +299,11 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     constexpr int CB = F::quant ? E * F::bits / 8 : 16;     // code bytes per lane
     constexpr int MB = F::meta_bytes;
     constexpr int FEB = kBf16 ? 2 : 4;                       // fp element bytes
-    constexpr int CPL = E / 4;                               // B/C 16-byte chunks per lane
+    constexpr int NP = E / 16;                               // 16-entry pieces per lane
+    constexpr int PW = F::quant ? Piece<FMT>::words : 1;     // code words per piece
+    constexpr int PB = PW * 4;                               // code bytes per piece
 
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
     uint64_t* ufull = empty + kMaxStages;
@@ -232,21 +336,19 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     if (warp == kCWarps) {
         // ================= producer warp =================
         int si = 0, sph = 0, k = 0, uk = -1;
-        long long prev = -1;
-        bool bad = false, ok = true;
+        bool bad = false, ok = true, newunit = true;
         const uint8_t* codes_u = nullptr;
         const uint8_t* meta_u = nullptr;
         const uint8_t* fp_u = nullptr;
         const float* x_u = nullptr;
         TileWalk ti;
         ti.start(pv, cv, t0);
-        for (long long t = t0; t < t1; ++t, ti.next(pv, cv)) {
+        for (long long t = t0; t < t1; ++t, newunit = ti.next(pv, cv)) {
             const int regbase = ti.quant ? 0 : pv.Hq;
-            if (ti.key != prev) {
-                prev = ti.key;
+            if (newunit) {
                 ++uk;
                 const int u = uk & 1;
-                if (!mbar_wait(&uempty[u], ((uk >> 1) & 1) ^ 1)) { ok = false; break; }
+                if (!mbar_wait<kProducerSleep>(&uempty[u], ((uk >> 1) & 1) ^ 1)) { ok = false; break; }
                 const int slot = cv.slot_idx ? __ldg(cv.slot_idx + ti.b) : ti.b;
                 bad = slot < 0 || slot >= pv.n_slots;
                 uint8_t* ub = units + u * geo.unit_bytes;
@@ -262,32 +364,37 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     meta_u = sb + pv.meta_off + (long long)layer * pv.meta_layer_bytes;
                     fp_u = sb + pv.fp_off + (long long)layer * pv.fp_layer_bytes;
                     x_u = cv.x + ti.lb * H * P;
-                    // B and C in 16-byte chunks.  In quantized units lane j
-                    // of a row owns chunks j*CPL .. j*CPL+CPL-1; chunk i of
-                    // lane j is stored at i*LPR + j, so at each step the
-                    // lanes of a row read consecutive chunks (distinct banks)
-                    // at compile-time offsets from a per-lane base.
+                    // B and C in 16-byte chunks.  In quantized units lane j's
+                    // chunk i of piece pc (its entries 16*pc + 4*i .. +3) is
+                    // stored at (i*NP + pc)*LPR + j, so the lanes of a warp,
+                    // visiting different pieces, read distinct banks.
                     float* dB = reinterpret_cast<float*>(ub + geo.ub_B);
                     float* dC = reinterpret_cast<float*>(ub + geo.ub_C);
                     const float* sB = cv.B + ti.lb * G * N;
                     const float* sC = cv.C + ti.lb * G * N;
                     for (int m = lane; m < G * N / 4; m += 32) {
                         int pos = m;
-                        if (ti.quant) {
+                        if (F::quant && ti.quant) {
                             const int gi = m / (N / 4), mm = m - gi * (N / 4);
-                            const int jj = mm / CPL, ii = mm - jj * CPL;
-                            pos = gi * (N / 4) + ii * LPR + jj;
+                            const int jj = mm / (E / 4), rest = mm - jj * (E / 4);
+                            const int pc = rest / 4, ii = rest - pc * 4;
+                            pos = gi * (N / 4) + (ii * NP + pc) * LPR + jj;
                         }
                         cpa16(dB + 4 * pos, sB + 4 * m);
                         cpa16(dC + 4 * pos, sC + 4 * m);
                     }
-                    float* ddt = reinterpret_cast<float*>(ub + geo.ub_dt);
-                    float* dA = reinterpret_cast<float*>(ub + geo.ub_A);
-                    float* dD = reinterpret_cast<float*>(ub + geo.ub_D);
-                    for (int h = lane; h < H; h += 32) {
-                        cpa4(ddt + h, cv.dt + ti.lb * H + h);
-                        cpa4(dA + h, cv.A + (long long)ti.l * H + h);
-                        cpa4(dD + h, cv.D + (long long)ti.l * H + h);
+                    // head table of the region: lambda = exp(dt*A) once per
+                    // head, dt, D, the head's y offset and B/C group
+                    float4* ht = reinterpret_cast<float4*>(ub + geo.ub_ht);
+                    int* gt = reinterpret_cast<int*>(ub + geo.ub_gt);
+                    const int nreg = ti.quant ? pv.Hq : pv.Hf;
+                    for (int hr = lane; hr < nreg; hr += 32) {
+                        const int h = pv.perm[regbase + hr];
+                        const float dtv = __ldg(cv.dt + ti.lb * H + h);
+                        const float Av = __ldg(cv.A + (long long)ti.l * H + h);
+                        const float Dv = __ldg(cv.D + (long long)ti.l * H + h);
+                        ht[hr] = make_float4(decay(dtv, Av), dtv, Dv, __int_as_float(h * P));
+                        gt[hr] = fdiv(h, pv.mHpg) * N;
                     }
                 }
                 cpa_arrive(&ufull[u]);
@@ -295,7 +402,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 if (lane == 0) mbar_arrive(&ufull[u]);
             }
             if (bad) continue;
-            if (!mbar_wait(&empty[si], sph ^ 1)) { ok = false; break; }
+            if (!mbar_wait<kProducerSleep>(&empty[si], sph ^ 1)) { ok = false; break; }
             uint8_t* st = stages + si * geo.stage_bytes;
             float* sx = reinterpret_cast<float*>(st);
             for (int i = lane; i < ti.n; i += 32) {
@@ -328,20 +435,18 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (lane == 0) {
             for (int jj = (k > S ? k - S : 0); jj < k; ++jj)
-                mbar_wait(&full[jj % S], (jj / S) & 1);
+                mbar_wait<kConsumerSleep>(&full[jj % S], (jj / S) & 1);
         }
         return;
     }
 
     // ================= consumer warps =================
     const int ct = threadIdx.x;
-    const int grow = ct / LPR;
-    const int j = ct % LPR;
+    const int grow = ct / LPR;          // row within the tile
+    const int j = ct % LPR;             // lane within the row
     int si = 0, sph = 0, uk = -1;
-    long long prev = -1;
-    bool bad = false;
+    bool bad = false, newunit = true;
     const uint8_t* ub = units;
-    float* lam = nullptr;
     uint8_t* codes_u = nullptr;
     uint8_t* meta_u = nullptr;
     uint8_t* fp_u = nullptr;
@@ -349,23 +454,21 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
 
     TileWalk ti;
     ti.start(pv, cv, t0);
-    for (long long t = t0; t < t1; ++t, ti.next(pv, cv)) {
-        if (ti.key != prev) {
+    for (long long t = t0; t < t1; ++t, newunit = ti.next(pv, cv)) {
+        if (newunit) {
             if (uk >= 0) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&uempty[uk & 1]);
             }
-            prev = ti.key;
             ++uk;
             const int u = uk & 1;
-            if (!mbar_wait(&ufull[u], (uk >> 1) & 1)) {
+            if (!mbar_wait<kConsumerSleep>(&ufull[u], (uk >> 1) & 1)) {
                 if (lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
                 break;
             }
             ub = units + u * geo.unit_bytes;
             const int slot = reinterpret_cast<const int*>(ub)[0];
             bad = reinterpret_cast<const int*>(ub)[1] != 0;
-            lam = reinterpret_cast<float*>(smem + geo.off_lam) + (warp * 2 + u) * geo.Hpad;
             if (!bad) {
                 const int layer = cv.layer0 + ti.l;
                 uint8_t* sb = pv.pool + pv.header_bytes + (long long)slot * pv.slot_bytes;
@@ -373,60 +476,38 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 meta_u = sb + pv.meta_off + (long long)layer * pv.meta_layer_bytes;
                 fp_u = sb + pv.fp_off + (long long)layer * pv.fp_layer_bytes;
                 y_u = cv.y + ti.lb * H * P;
-                const float* udt = reinterpret_cast<const float*>(ub + geo.ub_dt);
-                const float* uA = reinterpret_cast<const float*>(ub + geo.ub_A);
-                for (int h = lane; h < H; h += 32) lam[h] = decay(udt[h], uA[h]);
-                __syncwarp();
             }
         }
         if (bad) continue;
-        if (!mbar_wait(&full[si], sph)) {
+        if (!mbar_wait<kConsumerSleep>(&full[si], sph)) {
             if (lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
             break;
         }
         const uint8_t* st = stages + si * geo.stage_bytes;
         const float* sx = reinterpret_cast<const float*>(st);
         const uint8_t* pay = st + geo.x_bytes;
-        const int regbase = ti.quant ? 0 : pv.Hq;
         const bool active = grow < ti.n;
         const int rl = active ? grow : 0;          // inactive rows shadow row 0
         const int rr = ti.rbase + rl;
-        const int hrl = fdiv(rr, pv.mP);
-        const int p = rr - hrl * P;
-        const int h = pv.perm[regbase + hrl];
-        const int g = fdiv(h, pv.mHpg);
+        const int hr = fdiv(rr, pv.mP);
+        const int p = rr - hr * P;
+        const float4 hti = reinterpret_cast<const float4*>(ub + geo.ub_ht)[hr];
+        const int gN = reinterpret_cast<const int*>(ub + geo.ub_gt)[hr];
         const float xv = sx[rl];
-        const float lamv = lam[h];
-        const float dtv = reinterpret_cast<const float*>(ub + geo.ub_dt)[h];
-        const float Dv = reinterpret_cast<const float*>(ub + geo.ub_D)[h];
-        const float dtx = __fmul_rn(dtv, xv);
-        const float* gB = reinterpret_cast<const float*>(ub + geo.ub_B) + g * N;
-        const float* gC = reinterpret_cast<const float*>(ub + geo.ub_C) + g * N;
+        const float lamv = hti.x;
+        const float dtx = __fmul_rn(hti.y, xv);
+        const float* gB = reinterpret_cast<const float*>(ub + geo.ub_B) + gN;
+        const float* gC = reinterpret_cast<const float*>(ub + geo.ub_C) + gN;
         float ysum = 0.0f;
         bool done = false;
 
         if constexpr (F::quant) {
             if (ti.quant) {
                 done = true;
-                constexpr int PW = Piece<FMT>::words;        // words per 16 entries
-                constexpr int NP = E / 16;                   // 16-entry pieces per lane
-                uint32_t cw[CB / 4];
-                {
-                    const uint8_t* cs = pay + rl * RB + j * CB;
-                    if constexpr (CB % 16 == 0) {
-#pragma unroll
-                        for (int i = 0; i < CB / 16; ++i) {
-                            const uint4 v = reinterpret_cast<const uint4*>(cs)[i];
-                            cw[4 * i] = v.x; cw[4 * i + 1] = v.y; cw[4 * i + 2] = v.z; cw[4 * i + 3] = v.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < CB / 8; ++i) {
-                            const uint2 v = reinterpret_cast<const uint2*>(cs)[i];
-                            cw[2 * i] = v.x; cw[2 * i + 1] = v.y;
-                        }
-                    }
-                }
+                // this lane's codes and the row's metadata in shared memory
+                const uint8_t* cs = pay + rl * RB + j * CB;
+                uint8_t* crow = codes_u + (long long)rr * RB + j * CB;
+                uint8_t* mrow = meta_u + (long long)rr * MB;
                 float delta0, z0 = 0.0f;
                 {
                     const uint8_t* ms = pay + geo.qcodes_bytes + rl * MB;
@@ -438,101 +519,95 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         z0 = m.y;
                     }
                 }
-                // decode + update, 16 entries at a time, tracking min / max
+                const float4* bl = reinterpret_cast<const float4*>(gB) + j;
+                const float4* cl = reinterpret_cast<const float4*>(gC) + j;
+                // decode + update, one 16-entry piece at a time, with
+                // per-piece min / max.  The decode is exact for |z| < 2^22;
+                // rows beyond that take the exact path below.
                 float s[E];
-                float plo[NP], phi[NP];                      // per-piece min / max
-                const bool dfast = F::sym || __all_sync(0xffffffffu, fabsf(z0) < kFastLimit);
-                const float c0 = __fadd_rn(kTwo23, __fadd_rn(z0, F::bias));
-                const float4* b4 = reinterpret_cast<const float4*>(gB) + j;
-#pragma unroll
-                for (int pc = 0; pc < NP; ++pc) {
-                    float* sp = s + 16 * pc;
-                    if (dfast) {
-                        float f[16];
-                        unpack16_biased<FMT>(cw + PW * pc, f);
-                        const float2 nc02 = make_float2(-c0, -c0);
-                        const float2 d2 = make_float2(delta0, delta0);
-#pragma unroll
-                        for (int n = 0; n < 16; n += 2) {
-                            float2 v = mul2(add2(make_float2(f[n], f[n + 1]), nc02), d2);
-                            sp[n] = v.x; sp[n + 1] = v.y;
-                        }
-                    } else {
-                        int q[16];
-                        unpack16_int<FMT>(cw + PW * pc, q);
-#pragma unroll
-                        for (int n = 0; n < 16; ++n)
-                            sp[n] = __fmul_rn(__fsub_rn((float)q[n], z0), delta0);
-                    }
-                    float Bv[16];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float4 v = b4[(4 * pc + i) * LPR];
-                        Bv[4 * i] = v.x; Bv[4 * i + 1] = v.y; Bv[4 * i + 2] = v.z; Bv[4 * i + 3] = v.w;
-                    }
+                float lo, hi;
+                {
+                    const float c0 = __fadd_rn(kTwo23, __fadd_rn(z0, F::bias));
+                    const float2 nc02 = make_float2(-c0, -c0);
+                    const float2 d2 = make_float2(delta0, delta0);
                     const float2 l2 = make_float2(lamv, lamv);
                     const float2 x2 = make_float2(dtx, dtx);
 #pragma unroll
-                    for (int n = 0; n < 16; n += 2) {
-                        const float2 w = mul2(x2, make_float2(Bv[n], Bv[n + 1]));
-                        const float2 v = fma2(l2, make_float2(sp[n], sp[n + 1]), w);
-                        sp[n] = v.x; sp[n + 1] = v.y;
-                    }
-                    minmax16(sp, plo[pc], phi[pc]);
-                }
-                float lo = plo[0], hi = phi[0];
+                    for (int pc = 0; pc < NP; ++pc) {
+                        uint32_t w[PW];
+                        if constexpr (PW == 4) {
+                            const uint4 v = *reinterpret_cast<const uint4*>(cs + pc * PB);
+                            w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+                        } else {
+                            const uint2 v = *reinterpret_cast<const uint2*>(cs + pc * PB);
+                            w[0] = v.x; w[1] = v.y;
+                        }
+                        float f[16];
+                        unpack16_biased<FMT>(w, f);
+                        const float4* bp = bl + pc * LPR;
+                        float* sp16 = s + 16 * pc;
 #pragma unroll
-                for (int pc = 1; pc < NP; ++pc) {
-                    lo = fminf(lo, plo[pc]);
-                    hi = fmaxf(hi, phi[pc]);
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 bv = bp[i * NP * LPR];
+                            const float2 v0 = mul2(add2(make_float2(f[4 * i], f[4 * i + 1]), nc02), d2);
+                            const float2 v1 = mul2(add2(make_float2(f[4 * i + 2], f[4 * i + 3]), nc02), d2);
+                            const float2 u0 = fma2(l2, v0, mul2(x2, make_float2(bv.x, bv.y)));
+                            const float2 u1 = fma2(l2, v1, mul2(x2, make_float2(bv.z, bv.w)));
+                            sp16[4 * i] = u0.x; sp16[4 * i + 1] = u0.y;
+                            sp16[4 * i + 2] = u1.x; sp16[4 * i + 3] = u1.y;
+                        }
+                        float plo, phi;
+                        minmax16(sp16, plo, phi);
+                        lo = pc == 0 ? plo : fminf(lo, plo);
+                        hi = pc == 0 ? phi : fmaxf(hi, phi);
+                    }
                 }
                 const RowParams rp = refit_from_minmax<FMT, LPR>(lo, hi);
-                const bool fast = __all_sync(0xffffffffu, rp.fast && !rp.clamp);
-                // round, pack and read back, 16 entries at a time
-                const float4* c4 = reinterpret_cast<const float4*>(gC) + j;
-                float2 accp[NP];                             // one accumulator per piece
+                // the magic-number paths are exact for every row of the warp;
+                // rows whose top code must be capped take the clamped loop
+                const bool fast = __all_sync(0xffffffffu, (F::sym || fabsf(z0) < kFastLimit)
+                                                          && rp.fast);
+                if (fast) {
+                    const float2 inv2 = make_float2(rp.inv, rp.inv);
+                    const float2 z2 = make_float2(rp.z, rp.z);
+                    const float mz = F::sym ? -kMagic : -__fadd_rn(kMagic, rp.z);
+                    const float2 mz2 = make_float2(mz, mz);
+                    // round, pack, store and read back, piece by piece; the
+                    // readout sums C (q - z) and scales by Delta once
+                    float2 acc = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
+                    auto piece = [&](auto clamp_tag, int pc) {
+                        float r[16];
+                        uint32_t kk[16];
+                        round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, s + 16 * pc,
+                                                                       r, kk, pv.neg_zero);
+                        uint32_t w[PW];
+                        pack16<FMT>(kk, w);
+                        if (active) {
+                            if constexpr (PW == 4)
+                                __stcs(reinterpret_cast<uint4*>(crow + pc * PB),
+                                       make_uint4(w[0], w[1], w[2], w[3]));
+                            else
+                                __stcs(reinterpret_cast<uint2*>(crow + pc * PB),
+                                       make_uint2(w[0], w[1]));
+                        }
+                        const float4* cp = cl + pc * LPR;
 #pragma unroll
-                for (int pc = 0; pc < NP; ++pc) {
-                    float2& acc = accp[pc];
-                    acc = make_float2(0.0f, 0.0f);
-                    float r[16];
-                    uint32_t kk[16];
-                    if (fast) {
-                        round16_fast<FMT>(rp, s + 16 * pc, r, kk, pv.neg_zero);
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 cv4 = cp[i * NP * LPR];
+                            acc = fma2(make_float2(cv4.x, cv4.y), make_float2(r[4 * i], r[4 * i + 1]), acc);
+                            acc1 = fma2(make_float2(cv4.z, cv4.w), make_float2(r[4 * i + 2], r[4 * i + 3]), acc1);
+                        }
+                    };
+                    if (F::sym || !__any_sync(0xffffffffu, rp.clamp)) {
+#pragma unroll
+                        for (int pc = 0; pc < NP; ++pc) piece(std::false_type{}, pc);
                     } else {
-                        round16_slow<FMT>(rp, s + 16 * pc, r, kk);
 #pragma unroll
-                        for (int n = 0; n < 16; ++n) r[n] = __fmul_rn(r[n], rp.delta);
+                        for (int pc = 0; pc < NP; ++pc) piece(std::true_type{}, pc);
                     }
-                    pack16<FMT>(kk, cw + PW * pc);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float4 v = c4[(4 * pc + i) * LPR];
-                        acc = fma2(make_float2(v.x, v.y), make_float2(r[4 * i], r[4 * i + 1]), acc);
-                        acc = fma2(make_float2(v.z, v.w), make_float2(r[4 * i + 2], r[4 * i + 3]), acc);
-                    }
-                }
-                // fast: acc = sum C (q - z), scaled by Delta once; slow: acc
-                // already sums C * fl((q - z) * Delta)
-                float2 acc = accp[0];
-#pragma unroll
-                for (int pc = 1; pc < NP; ++pc) acc = add2(acc, accp[pc]);
-                const float part = __fadd_rn(acc.x, acc.y);
-                ysum = fast ? __fmul_rn(rp.delta, grp_sum<LPR>(part)) : grp_sum<LPR>(part);
-                if (active) {
-                    uint8_t* crow = codes_u + (long long)rr * RB + j * CB;
-                    if constexpr (CB % 16 == 0) {
-#pragma unroll
-                        for (int i = 0; i < CB / 16; ++i)
-                            __stcs(reinterpret_cast<uint4*>(crow) + i,
-                                   make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]));
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < CB / 8; ++i)
-                            __stcs(reinterpret_cast<uint2*>(crow) + i, make_uint2(cw[2 * i], cw[2 * i + 1]));
-                    }
-                    if (j == 0) {
-                        uint8_t* mrow = meta_u + (long long)rr * MB;
+                    acc = add2(acc, acc1);
+                    ysum = __fmul_rn(rp.delta, grp_sum<LPR>(__fadd_rn(acc.x, acc.y)));
+                    if (active && j == 0) {
                         if constexpr (F::sym) {
                             __stcs(reinterpret_cast<float*>(mrow), rp.delta);
                         } else {
@@ -540,22 +615,29 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         }
                         if (!rp.finite) atomicOr(err, SSQ_DEVERR_NONFINITE);
                     }
+                } else {
+                    ysum = row_exact<FMT, N>(cs, delta0, z0, lamv, dtx, gB, gC, j, active, crow,
+                                             mrow, err);
                 }
             }
         }
         if (!done) {
             // fp row (fp32, or bf16 for the bf16 format), streamed one 16-byte
-            // storage chunk at a time.  Lane j owns chunks LPR*c + j, so the
-            // lanes of a row touch consecutive chunks.
+            // storage chunk at a time.  Lane j owns chunks LPR*c + j; a lane
+            // starts at chunk `rot` so a warp's reads of one step spread over
+            // every bank group while B and C stay within one 128-byte line.
             constexpr int EPC = 16 / FEB;           // elements per chunk
             constexpr int NCH = E / EPC;            // chunks per lane
+            constexpr int RW = (8 / LPR) < NCH ? (8 / LPR) : NCH;   // rotation width
+            const int rot = RW > 1 ? grow % RW : 0;
             const uint8_t* fs = pay + (long long)rl * N * FEB;
             uint8_t* frow = fp_u + (long long)rr * N * FEB;
             const float2 l2 = make_float2(lamv, lamv);
             const float2 x2 = make_float2(dtx, dtx);
             float2 acc = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int c = 0; c < NCH; ++c) {
+            for (int c0 = 0; c0 < NCH; ++c0) {
+                const int c = RW > 1 ? ((c0 + rot) & (NCH - 1)) : c0;
                 const int m = LPR * c + j;
                 const uint4 v = reinterpret_cast<const uint4*>(fs)[m];
                 uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -601,8 +683,8 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             ysum = grp_sum<LPR>(__fadd_rn(acc.x, acc.y));
         }
         if (active && j == 0) {
-            const float yv = __fadd_rn(ysum, __fmul_rn(Dv, xv));
-            __stcs(y_u + h * P + p, yv);
+            const float yv = __fadd_rn(ysum, __fmul_rn(hti.z, xv));
+            __stcs(y_u + __float_as_int(hti.w) + p, yv);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[si]);
@@ -619,8 +701,8 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
     constexpr int RB = F::quant ? N * F::bits / 8 : 0;
     const bool has_fp = pv.Hf > 0;
     const int fpEB = FMT == SSQ_BF16 ? 2 : 4;
-    // stages: as many as fit a budget that leaves room for two CTAs per SM
-    const int budget = 110 * 1024;
+    // stages: as many as fit a budget that leaves room for kMinBlocks CTAs per SM
+    const int budget = (kMinBlocks == 1 ? 200 : 110) * 1024;
     DecodeGeom g = decode_geom(2, RPT, RB, F::meta_bytes, fpEB, has_fp, N, pv.H, pv.G);
     int S = (budget - g.off_stages) / g.stage_bytes;
     if (S > kMaxStages) S = kMaxStages;
@@ -628,22 +710,31 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
     g = decode_geom(S, RPT, RB, F::meta_bytes, fpEB, has_fp, N, pv.H, pv.G);
     if (g.smem_bytes > 227 * 1024) return cudaErrorInvalidConfiguration;
     auto kern = decode_kernel<FMT, N>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         g.smem_bytes);
+    // per-device launch facts, looked up once per kernel instantiation and device
+    thread_local int s_dev = -1, s_grid = 0, s_smem = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    // ask for the largest shared-memory carveout so two CTAs fit per SM
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0, occ = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-        return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kDThreads,
-                                                           g.smem_bytes)) != cudaSuccess)
-        return e;
-    if (occ < 1) return cudaErrorInvalidConfiguration;
-    long long grid = (long long)sms * occ;
+    if (s_dev != dev || s_smem != g.smem_bytes) {
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      g.smem_bytes)) != cudaSuccess)
+            return e;
+        // the largest shared-memory carveout, so two CTAs fit per SM
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                      (int)cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+            return e;
+        int sms = 0, occ = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kDThreads,
+                                                               g.smem_bytes)) != cudaSuccess)
+            return e;
+        if (occ < 1) return cudaErrorInvalidConfiguration;
+        s_dev = dev;
+        s_smem = g.smem_bytes;
+        s_grid = sms * occ;
+    }
+    long long grid = s_grid;
     if (grid > cv.total_tiles) grid = cv.total_tiles;
     kern<<<(int)grid, kDThreads, g.smem_bytes, st>>>(pv, cv, g);
     return cudaGetLastError();
@@ -673,7 +764,7 @@ int decode_rows_per_tile(int fmt, int d_state)
 
 bool decode_fits(int fmt, int d_state, int nheads, int ngroups)
 {
-    // B and C of every group plus the lambda arrays must leave room for two
+    // B and C of every group plus the head tables must leave room for two
     // pipeline stages within one CTA's shared memory
     const int rpt = decode_rows_per_tile(fmt, d_state);
     const DecodeGeom g = decode_geom(2, rpt, d_state, 8, 4, true, d_state, nheads, ngroups);

@@ -205,6 +205,47 @@ def test_decode_step_parity_zoo(fmt):
     check_y(y.cpu().numpy()[0], y_ref, scale, f"zoo {fmt}")
 
 
+@pytest.mark.parametrize("fmt", QFMTS)
+@pytest.mark.parametrize("N", [64, 128])
+def test_decode_crafted_updates(fmt, N):
+    """Updated rows chosen exactly: from the zero state with dt = x = 1 the
+    update is s' = B of the row's group, so each group's B is one of the
+    crafted rows (the top code rounding past the grid, exact half-integer
+    ties, a near-constant row far from zero, a constant row) or a normal
+    row.  Heads of 8 rows put two groups in every warp, so warps mix rows
+    that need the clamped rounding or the exact path with ordinary ones."""
+    ssq = require_gpu()
+    H, P, batch = 12, 8, 2
+    cr = crafted_rows(N)
+    G = 6
+    cfg, L, codec, ocfg = make_cfg(ssq, fmt, 1, batch, H, P, N, G)
+    rng = np.random.default_rng(31 + N)
+    inp = W.Decode("crafted", 3, 1, batch, H, P, N, G, fmt).inputs()
+    inp["dt"][:] = 1.0
+    inp["x"][:] = 1.0
+    for b in range(batch):
+        for g in range(G):
+            k = (g + b) % (cr.shape[0] + 1)
+            inp["B"][0, b, g] = cr[k] if k < cr.shape[0] else \
+                rng.standard_normal(N).astype(np.float32)
+    st = O.State(ocfg, batch)
+    pool = ssq.alloc_pool(cfg)
+    y = torch.empty((1, batch, H, P), device="cuda")
+    ssq.ssq_decode_step(cfg, pool, None, batch, 0, 1, cuda(inp["x"]), cuda(inp["B"]),
+                        cuda(inp["C"]), cuda(inp["dt"]), cuda(inp["A"]), cuda(inp["D"]), y)
+    pre = np.zeros((batch, H * P, N), np.float32)
+    y_ref = np.zeros((batch, H, P), np.float32)
+    for b in range(batch):
+        y_ref[b], pre[b] = O.step(ocfg, st, b, inp["x"][0, b], inp["B"][0, b], inp["C"][0, b],
+                                  inp["dt"][0, b], inp["A"][0], inp["D"][0], want_pre=True)
+    got = download(codec, pool, [(b, 0) for b in range(batch)], ocfg)
+    stats = compare_states(ocfg, got, st, pre, f"crafted {fmt} N{N}")
+    assert stats["code_mismatch"] == 0
+    scale = y_scale(ocfg, st, inp["C"][0], np.repeat(inp["D"], batch, 0), inp["x"][0])
+    check_y(y.cpu().numpy()[0], y_ref, scale, f"crafted {fmt} N{N}")
+    assert ssq.ssq_pool_error(cfg, pool) == 0
+
+
 def test_decode_tiny_multistep_drift():
     """The tiny workload (1 layer, batch 1, 2 heads x 8 x 16, int8 asym, zero
     initial state) for 64 free-running steps: GPU and oracle advance their own
