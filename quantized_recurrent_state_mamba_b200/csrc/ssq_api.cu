@@ -165,12 +165,13 @@ ssq_status need(const void* p, const char* name, size_t align)
         if (_s != SSQ_OK) return _s;       \
     } while (0)
 
-void fill_tiles(const ssq::PoolView& pv, ssq::CallView* cv, int rows_per_tile)
+void fill_tiles(const ssq::PoolView& pv, ssq::CallView* cv, int rows_q, int rows_f)
 {
     const long long qrows = (long long)pv.Hq * pv.P, frows = (long long)pv.Hf * pv.P;
-    cv->rows_per_tile = rows_per_tile;
-    cv->qtiles = (int)((qrows + rows_per_tile - 1) / rows_per_tile);
-    cv->ftiles = (int)((frows + rows_per_tile - 1) / rows_per_tile);
+    cv->rows_per_tile = rows_q;
+    cv->rows_per_tile_f = rows_f;
+    cv->qtiles = (int)((qrows + rows_q - 1) / rows_q);
+    cv->ftiles = (int)((frows + rows_f - 1) / rows_f);
     cv->total_tiles = (long long)cv->nl * cv->batch * (cv->qtiles + cv->ftiles);
 }
 
@@ -259,7 +260,7 @@ ssq_status ssq_quantize_rows(const ssq_config* cfg, void* pool, const int32_t* s
     cv.layer0 = layer0;
     cv.nl = nl;
     cv.S_in = S;
-    fill_tiles(pv, &cv, ssq::rows_per_tile(cfg->d_state));
+    fill_tiles(pv, &cv, ssq::rows_per_tile(cfg->d_state), ssq::rows_per_tile(cfg->d_state));
     cudaError_t e = ssq::launch_quantize(pv, cv, (int)cfg->fmt, stream);
     if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
     return SSQ_OK;
@@ -282,7 +283,7 @@ ssq_status ssq_dequantize_rows(const ssq_config* cfg, const void* pool,
     cv.layer0 = layer0;
     cv.nl = nl;
     cv.S_out = S_out;
-    fill_tiles(pv, &cv, ssq::rows_per_tile(cfg->d_state));
+    fill_tiles(pv, &cv, ssq::rows_per_tile(cfg->d_state), ssq::rows_per_tile(cfg->d_state));
     cudaError_t e = ssq::launch_dequantize(pv, cv, (int)cfg->fmt, stream);
     if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
     return SSQ_OK;
@@ -321,7 +322,9 @@ ssq_status ssq_decode_step(const ssq_config* cfg, void* pool, const int32_t* slo
     if (!ssq::decode_fits((int)cfg->fmt, cfg->d_state, cfg->nheads, cfg->ngroups))
         return fail(SSQ_ERR_UNSUPPORTED, "ngroups*d_state %d too large for the decode kernel",
                     cfg->ngroups * cfg->d_state);
-    fill_tiles(pv, &cv, ssq::decode_rows_per_tile((int)cfg->fmt, cfg->d_state));
+    int rows_q = 0, rows_f = 0;
+    ssq::decode_tile_rows((int)cfg->fmt, cfg->d_state, &rows_q, &rows_f);
+    fill_tiles(pv, &cv, rows_q, rows_f);
     cudaError_t e = ssq::launch_decode(pv, cv, (int)cfg->fmt, stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return SSQ_OK;

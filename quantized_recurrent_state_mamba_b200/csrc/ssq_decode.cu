@@ -21,7 +21,7 @@
 //     consumer row finds everything it needs with two shared loads;
 //   - 11 consumer warps compute from shared memory and store the new rows,
 //     metadata and y straight to global memory.  A row of a quantized head
-//     is held by LPR lanes with E = 64 entries each, streamed 16 at a time;
+//     is held by d_state/64 lanes of 64 entries, streamed 16 at a time;
 //   - B and C are staged with lane j's 16-byte chunks interleaved, so the
 //     lanes of a row read distinct banks;
 //   - waits sleep between tries of the mbarrier, and every wait is
@@ -129,9 +129,10 @@ struct TileWalk {
     __device__ __forceinline__ void fill(const PoolView& pv, const CallView& cv)
     {
         quant = k < cv.qtiles;
-        rbase = (quant ? k : k - cv.qtiles) * cv.rows_per_tile;
+        const int rpt = quant ? cv.rows_per_tile : cv.rows_per_tile_f;
+        rbase = (quant ? k : k - cv.qtiles) * rpt;
         const int nrows = (quant ? pv.Hq : pv.Hf) * pv.P;
-        n = min(cv.rows_per_tile, nrows - rbase);
+        n = min(rpt, nrows - rbase);
     }
     __device__ __forceinline__ void start(const PoolView& pv, const CallView& cv, long long t)
     {
@@ -168,7 +169,7 @@ struct TileWalk {
 // Stage:       [x: RPT f32, padded to 128 B][payload: codes + meta, or fp rows]
 struct DecodeGeom {
     int S;            // stages
-    int RPT;          // rows per tile
+    int RPTq, RPTf;   // rows per tile in the quantized / fp region
     int x_bytes;      // x area of a stage
     int qcodes_bytes; // codes area of a quantized tile
     int pay_bytes;    // payload area of a stage
@@ -178,16 +179,18 @@ struct DecodeGeom {
     int off_units, off_stages, smem_bytes;
 };
 
-__host__ __device__ inline DecodeGeom decode_geom(int S, int RPT, int RB, int MB, int fpEB,
-                                                  bool has_fp, int N, int H, int G)
+__host__ __device__ inline DecodeGeom decode_geom(int S, int RPTq, int RPTf, int RB, int MB,
+                                                  int fpEB, bool has_q, bool has_fp, int N,
+                                                  int H, int G)
 {
     DecodeGeom g;
     g.S = S;
-    g.RPT = RPT;
-    g.x_bytes = r128(RPT * 4);
-    g.qcodes_bytes = r16(RPT * RB);
-    const int qpay = g.qcodes_bytes + r16(RPT * MB);
-    const int fpay = has_fp ? RPT * N * fpEB : 0;
+    g.RPTq = RPTq;
+    g.RPTf = RPTf;
+    g.x_bytes = r128((RPTq > RPTf ? RPTq : RPTf) * 4);
+    g.qcodes_bytes = has_q ? r16(RPTq * RB) : 0;
+    const int qpay = has_q ? g.qcodes_bytes + r16(RPTq * MB) : 0;
+    const int fpay = has_fp ? RPTf * N * fpEB : 0;
     g.pay_bytes = qpay > fpay ? qpay : fpay;
     g.stage_bytes = r128(g.x_bytes + g.pay_bytes);
     g.Hpad = (H + 3) & ~3;
@@ -203,12 +206,25 @@ __host__ __device__ inline DecodeGeom decode_geom(int S, int RPT, int RB, int MB
     return g;
 }
 
-// Lane shape: quantized rows give each lane 64 entries (two lanes per
-// 128-entry row); fp rows keep 32 entries per lane.
-template <int FMT, int N>
-struct DShape {
-    static constexpr int E = Fmt<FMT>::quant ? (N >= 64 ? 64 : N) : (N >= 32 ? 32 : N);
+// Lane shapes.  A quantized row is held by N/kQuantE lanes of kQuantE
+// entries (two lanes for d_state 128): the per-row work (refit, addresses,
+// metadata) is spread over 64 entries while the row and the f32x2 operand
+// pairs still fit the register budget of three warps per SM sub-partition
+// (128 entries per lane needs either spills or fewer warps, both slower).
+// An fp row (the fp32 / bf16 formats, and unmasked heads of the integer
+// formats) is streamed by N/32 lanes of 32 entries.
+constexpr int kQuantE = 64;
+template <int N>
+struct QShape {
+    static constexpr int E = N >= kQuantE ? kQuantE : N;
     static constexpr int LPR = N / E;
+    static constexpr int RPT = kCThreads / LPR;   // rows per tile
+};
+template <int N>
+struct FShape {
+    static constexpr int E = N >= 32 ? 32 : N;
+    static constexpr int LPR = N / E;
+    static constexpr int RPT = kCThreads / LPR;
 };
 
 // A whole quantized row by the formulas verbatim (every fp32 operation one
@@ -225,7 +241,7 @@ __device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float de
                                         uint32_t* err)
 {
     using F = Fmt<FMT>;
-    constexpr int E = DShape<FMT, N>::E, LPR = DShape<FMT, N>::LPR;
+    constexpr int E = QShape<N>::E, LPR = QShape<N>::LPR;
     constexpr int NP = E / 16;
     constexpr int CB = E * F::bits / 8;
     float s[E];
@@ -293,13 +309,15 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
               const __grid_constant__ DecodeGeom geo)
 {
     using F = Fmt<FMT>;
-    constexpr int E = DShape<FMT, N>::E, LPR = DShape<FMT, N>::LPR;
+    // quantized rows: EQ entries per lane, LQ lanes per row; fp rows: EF, LF
+    constexpr int EQ = QShape<N>::E, LQ = QShape<N>::LPR;
+    constexpr int EF = FShape<N>::E, LF = FShape<N>::LPR;
     constexpr bool kBf16 = (FMT == SSQ_BF16);
     constexpr int RB = F::quant ? N * F::bits / 8 : 0;      // code bytes per row
-    constexpr int CB = F::quant ? E * F::bits / 8 : 16;     // code bytes per lane
+    constexpr int CB = F::quant ? EQ * F::bits / 8 : 16;    // code bytes per lane
     constexpr int MB = F::meta_bytes;
     constexpr int FEB = kBf16 ? 2 : 4;                       // fp element bytes
-    constexpr int NP = E / 16;                               // 16-entry pieces per lane
+    constexpr int NP = EQ / 16;                              // 16-entry pieces per lane
     constexpr int PW = F::quant ? Piece<FMT>::words : 1;     // code words per piece
     constexpr int PB = PW * 4;                               // code bytes per piece
 
@@ -376,9 +394,9 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         int pos = m;
                         if (F::quant && ti.quant) {
                             const int gi = m / (N / 4), mm = m - gi * (N / 4);
-                            const int jj = mm / (E / 4), rest = mm - jj * (E / 4);
+                            const int jj = mm / (EQ / 4), rest = mm - jj * (EQ / 4);
                             const int pc = rest / 4, ii = rest - pc * 4;
-                            pos = gi * (N / 4) + (ii * NP + pc) * LPR + jj;
+                            pos = gi * (N / 4) + (ii * NP + pc) * LQ + jj;
                         }
                         cpa16(dB + 4 * pos, sB + 4 * m);
                         cpa16(dC + 4 * pos, sC + 4 * m);
@@ -442,8 +460,6 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
 
     // ================= consumer warps =================
     const int ct = threadIdx.x;
-    const int grow = ct / LPR;          // row within the tile
-    const int j = ct % LPR;             // lane within the row
     int si = 0, sph = 0, uk = -1;
     bool bad = false, newunit = true;
     const uint8_t* ub = units;
@@ -486,6 +502,9 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         const uint8_t* st = stages + si * geo.stage_bytes;
         const float* sx = reinterpret_cast<const float*>(st);
         const uint8_t* pay = st + geo.x_bytes;
+        // row within the tile and lane within the row, by the region's shape
+        const int grow = ti.quant ? ct / LQ : ct / LF;
+        const int j = ti.quant ? ct % LQ : ct % LF;
         const bool active = grow < ti.n;
         const int rl = active ? grow : 0;          // inactive rows shadow row 0
         const int rr = ti.rbase + rl;
@@ -524,7 +543,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 // decode + update, one 16-entry piece at a time, with
                 // per-piece min / max.  The decode is exact for |z| < 2^22;
                 // rows beyond that take the exact path below.
-                float s[E];
+                float s[EQ];
                 float lo, hi;
                 {
                     const float c0 = __fadd_rn(kTwo23, __fadd_rn(z0, F::bias));
@@ -544,11 +563,11 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         }
                         float f[16];
                         unpack16_biased<FMT>(w, f);
-                        const float4* bp = bl + pc * LPR;
+                        const float4* bp = bl + pc * LQ;
                         float* sp16 = s + 16 * pc;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const float4 bv = bp[i * NP * LPR];
+                            const float4 bv = bp[i * NP * LQ];
                             const float2 v0 = mul2(add2(make_float2(f[4 * i], f[4 * i + 1]), nc02), d2);
                             const float2 v1 = mul2(add2(make_float2(f[4 * i + 2], f[4 * i + 3]), nc02), d2);
                             const float2 u0 = fma2(l2, v0, mul2(x2, make_float2(bv.x, bv.y)));
@@ -562,7 +581,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         hi = pc == 0 ? phi : fmaxf(hi, phi);
                     }
                 }
-                const RowParams rp = refit_from_minmax<FMT, LPR>(lo, hi);
+                const RowParams rp = refit_from_minmax<FMT, LQ>(lo, hi);
                 // the magic-number paths are exact for every row of the warp;
                 // rows whose top code must be capped take the clamped loop
                 const bool fast = __all_sync(0xffffffffu, (F::sym || fabsf(z0) < kFastLimit)
@@ -590,10 +609,10 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                                 __stcs(reinterpret_cast<uint2*>(crow + pc * PB),
                                        make_uint2(w[0], w[1]));
                         }
-                        const float4* cp = cl + pc * LPR;
+                        const float4* cp = cl + pc * LQ;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const float4 cv4 = cp[i * NP * LPR];
+                            const float4 cv4 = cp[i * NP * LQ];
                             acc = fma2(make_float2(cv4.x, cv4.y), make_float2(r[4 * i], r[4 * i + 1]), acc);
                             acc1 = fma2(make_float2(cv4.z, cv4.w), make_float2(r[4 * i + 2], r[4 * i + 3]), acc1);
                         }
@@ -606,7 +625,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         for (int pc = 0; pc < NP; ++pc) piece(std::true_type{}, pc);
                     }
                     acc = add2(acc, acc1);
-                    ysum = __fmul_rn(rp.delta, grp_sum<LPR>(__fadd_rn(acc.x, acc.y)));
+                    ysum = __fmul_rn(rp.delta, grp_sum<LQ>(__fadd_rn(acc.x, acc.y)));
                     if (active && j == 0) {
                         if constexpr (F::sym) {
                             __stcs(reinterpret_cast<float*>(mrow), rp.delta);
@@ -623,12 +642,12 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         }
         if (!done) {
             // fp row (fp32, or bf16 for the bf16 format), streamed one 16-byte
-            // storage chunk at a time.  Lane j owns chunks LPR*c + j; a lane
+            // storage chunk at a time.  Lane j owns chunks LF*c + j; a lane
             // starts at chunk `rot` so a warp's reads of one step spread over
             // every bank group while B and C stay within one 128-byte line.
             constexpr int EPC = 16 / FEB;           // elements per chunk
-            constexpr int NCH = E / EPC;            // chunks per lane
-            constexpr int RW = (8 / LPR) < NCH ? (8 / LPR) : NCH;   // rotation width
+            constexpr int NCH = EF / EPC;            // chunks per lane
+            constexpr int RW = (8 / LF) < NCH ? (8 / LF) : NCH;   // rotation width
             const int rot = RW > 1 ? grow % RW : 0;
             const uint8_t* fs = pay + (long long)rl * N * FEB;
             uint8_t* frow = fp_u + (long long)rr * N * FEB;
@@ -638,7 +657,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
 #pragma unroll
             for (int c0 = 0; c0 < NCH; ++c0) {
                 const int c = RW > 1 ? ((c0 + rot) & (NCH - 1)) : c0;
-                const int m = LPR * c + j;
+                const int m = LF * c + j;
                 const uint4 v = reinterpret_cast<const uint4*>(fs)[m];
                 uint32_t w[4] = {v.x, v.y, v.z, v.w};
                 float sv[EPC];
@@ -680,7 +699,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     __stcs(reinterpret_cast<uint4*>(frow) + m, make_uint4(w[0], w[1], w[2], w[3]));
             }
             acc = add2(acc, acc1);
-            ysum = grp_sum<LPR>(__fadd_rn(acc.x, acc.y));
+            ysum = grp_sum<LF>(__fadd_rn(acc.x, acc.y));
         }
         if (active && j == 0) {
             const float yv = __fadd_rn(ysum, __fmul_rn(hti.z, xv));
@@ -696,18 +715,17 @@ template <int FMT, int N>
 cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
 {
     using F = Fmt<FMT>;
-    constexpr int LPR = DShape<FMT, N>::LPR;
-    constexpr int RPT = kCThreads / LPR;
+    constexpr int RPTq = QShape<N>::RPT, RPTf = FShape<N>::RPT;
     constexpr int RB = F::quant ? N * F::bits / 8 : 0;
-    const bool has_fp = pv.Hf > 0;
+    const bool has_q = pv.Hq > 0, has_fp = pv.Hf > 0;
     const int fpEB = FMT == SSQ_BF16 ? 2 : 4;
     // stages: as many as fit a budget that leaves room for kMinBlocks CTAs per SM
     const int budget = (kMinBlocks == 1 ? 200 : 110) * 1024;
-    DecodeGeom g = decode_geom(2, RPT, RB, F::meta_bytes, fpEB, has_fp, N, pv.H, pv.G);
+    DecodeGeom g = decode_geom(2, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G);
     int S = (budget - g.off_stages) / g.stage_bytes;
     if (S > kMaxStages) S = kMaxStages;
     if (S < 2) S = 2;
-    g = decode_geom(S, RPT, RB, F::meta_bytes, fpEB, has_fp, N, pv.H, pv.G);
+    g = decode_geom(S, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G);
     if (g.smem_bytes > 227 * 1024) return cudaErrorInvalidConfiguration;
     auto kern = decode_kernel<FMT, N>;
     // per-device launch facts, looked up once per kernel instantiation and device
@@ -755,19 +773,23 @@ cudaError_t launch_fmt(const PoolView& pv, const CallView& cv, cudaStream_t st)
 
 }  // namespace
 
-int decode_rows_per_tile(int fmt, int d_state)
+void decode_tile_rows(int fmt, int d_state, int* rows_q, int* rows_f)
 {
-    const bool quant = fmt >= SSQ_I8_SYM;
-    const int E = quant ? (d_state >= 64 ? 64 : d_state) : (d_state >= 32 ? 32 : d_state);
-    return kCThreads / (d_state / E);
+    const int eq = d_state >= kQuantE ? kQuantE : d_state;
+    const int ef = d_state >= 32 ? 32 : d_state;
+    *rows_q = kCThreads / (d_state / eq);
+    *rows_f = kCThreads / (d_state / ef);
+    (void)fmt;
 }
 
 bool decode_fits(int fmt, int d_state, int nheads, int ngroups)
 {
     // B and C of every group plus the head tables must leave room for two
-    // pipeline stages within one CTA's shared memory
-    const int rpt = decode_rows_per_tile(fmt, d_state);
-    const DecodeGeom g = decode_geom(2, rpt, d_state, 8, 4, true, d_state, nheads, ngroups);
+    // pipeline stages (of either region) within one CTA's shared memory
+    int rq = 0, rf = 0;
+    decode_tile_rows(fmt, d_state, &rq, &rf);
+    const bool q = fmt >= SSQ_I8_SYM;
+    const DecodeGeom g = decode_geom(2, rq, rf, d_state, 8, 4, q, true, d_state, nheads, ngroups);
     return g.smem_bytes <= 227 * 1024;
 }
 

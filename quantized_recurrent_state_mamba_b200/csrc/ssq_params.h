@@ -28,7 +28,8 @@ struct PoolView {
 struct CallView {
     const int32_t* slot_idx;   // [batch] or null (identity)
     int batch, layer0, nl;
-    int rows_per_tile;         // rows of one region handled per tile
+    int rows_per_tile;         // rows of the quantized region handled per tile
+    int rows_per_tile_f;       // rows of the fp region handled per tile
     int qtiles, ftiles;        // tiles per (layer, request) in each region
     long long total_tiles;
     int T;                     // tokens (scan only)
@@ -64,8 +65,8 @@ ScanPlan scan_plan(int d_state, int headdim, long long batch_heads, int sms);
 cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt, const ScanPlan& sp,
                         cudaStream_t stream);
 
-// Rows per decode tile.
-int decode_rows_per_tile(int fmt, int d_state);
+// Rows per decode tile in the quantized and the fp region.
+void decode_tile_rows(int fmt, int d_state, int* rows_q, int* rows_f);
 // Whether the decode kernel's per-unit shared memory (B and C of every group,
 // per-head arrays) fits one CTA.
 bool decode_fits(int fmt, int d_state, int nheads, int ngroups);
