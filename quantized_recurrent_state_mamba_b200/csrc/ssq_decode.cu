@@ -114,7 +114,41 @@ __device__ __forceinline__ void cpa_arrive(uint64_t* b)
     asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(saddr(b)) : "memory");
 }
 
+// Shared-memory vector loads / stores at 32-bit shared addresses (the
+// quantized path forms its addresses with one XOR each).
+template <int OFF>
+__device__ __forceinline__ uint4 lds128(unsigned a)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a), "n"(OFF) : "memory");
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ uint2 lds64(unsigned a)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2+%3];"
+                 : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF) : "memory");
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ float4 lds128f(unsigned a)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a), "n"(OFF) : "memory");
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ void sts128f(unsigned a, float4 v)
+{
+    asm volatile("st.shared.v4.f32 [%0+%1], {%2, %3, %4, %5};"
+                 :: "r"(a), "n"(OFF), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+}
+
 __host__ __device__ inline int r16(int v) { return (v + 15) & ~15; }
+__host__ __device__ inline int r256(int v) { return (v + 255) & ~255; }
 __host__ __device__ inline int r128(int v) { return (v + 127) & ~127; }
 
 // ---- tile sequence -----------------------------------------------------
@@ -176,49 +210,61 @@ struct DecodeGeom {
     int stage_bytes;
     int ub_B, ub_C, ub_ht, ub_gt, unit_bytes;  // unit buffer layout
     int Hpad;
-    int off_units, off_stages, smem_bytes;
+    int off_units, off_stages, off_scr, scr_warp_bytes, smem_bytes;
 };
 
+// Offsets are from a 256-byte aligned base inside the dynamic shared memory
+// (the launch adds 256 bytes of slack); B, C and every stage start on a
+// 256-byte boundary, so per-lane addresses can be permuted with one XOR.
+// scr_lane_bytes: per lane spill area of a consumer warp (0: none).
 __host__ __device__ inline DecodeGeom decode_geom(int S, int RPTq, int RPTf, int RB, int MB,
                                                   int fpEB, bool has_q, bool has_fp, int N,
-                                                  int H, int G)
+                                                  int H, int G, int scr_lane_bytes)
 {
     DecodeGeom g;
     g.S = S;
     g.RPTq = RPTq;
     g.RPTf = RPTf;
-    g.x_bytes = r128((RPTq > RPTf ? RPTq : RPTf) * 4);
-    g.qcodes_bytes = has_q ? r16(RPTq * RB) : 0;
+    g.x_bytes = r256((RPTq > RPTf ? RPTq : RPTf) * 4);
+    g.qcodes_bytes = has_q ? r256(RPTq * RB) : 0;
     const int qpay = has_q ? g.qcodes_bytes + r16(RPTq * MB) : 0;
     const int fpay = has_fp ? RPTf * N * fpEB : 0;
     g.pay_bytes = qpay > fpay ? qpay : fpay;
-    g.stage_bytes = r128(g.x_bytes + g.pay_bytes);
+    g.stage_bytes = r256(g.x_bytes + g.pay_bytes);
     g.Hpad = (H + 3) & ~3;
-    g.ub_B = 16;
+    g.ub_B = 256;                      // [0, 16): slot, bad flag
     g.ub_C = g.ub_B + G * N * 4;
-    g.ub_ht = g.ub_C + G * N * 4;
+    g.ub_ht = r256(g.ub_C + G * N * 4);
     g.ub_gt = g.ub_ht + g.Hpad * 16;
-    g.unit_bytes = r128(g.ub_gt + g.Hpad * 4);
-    const int bars = r128((2 * kMaxStages + 4) * 8);
+    g.unit_bytes = r256(g.ub_gt + g.Hpad * 4);
+    const int bars = r256((2 * kMaxStages + 4) * 8);
     g.off_units = bars;
     g.off_stages = g.off_units + 2 * g.unit_bytes;
-    g.smem_bytes = g.off_stages + S * g.stage_bytes;
+    g.off_scr = g.off_stages + S * g.stage_bytes;
+    g.scr_warp_bytes = has_q ? 32 * scr_lane_bytes : 0;
+    g.smem_bytes = g.off_scr + kCWarps * g.scr_warp_bytes + 256;
     return g;
 }
 
-// Lane shapes.  A quantized row is held by N/kQuantE lanes of kQuantE
-// entries (two lanes for d_state 128): the per-row work (refit, addresses,
-// metadata) is spread over 64 entries while the row and the f32x2 operand
-// pairs still fit the register budget of three warps per SM sub-partition
-// (128 entries per lane needs either spills or fewer warps, both slower).
-// An fp row (the fp32 / bf16 formats, and unmasked heads of the integer
-// formats) is streamed by N/32 lanes of 32 entries.
-constexpr int kQuantE = 64;
+// Lane shapes.  A quantized row is held by one lane (the whole row for
+// d_state <= 128; two lanes at 256): the per-row work (refit, addresses,
+// metadata, the tile bookkeeping) is spread over 128 entries and the row
+// reductions need no shuffles.  Of the lane's 8 pieces of 16 entries, the
+// first kRegPieces stay in registers between the update and the rounding
+// and the rest wait in a per-lane shared-memory area, which keeps the kernel
+// within the register budget of three warps per SM sub-partition.  An fp
+// row (the fp32 / bf16 formats, and unmasked heads of the integer formats)
+// is streamed by N/32 lanes of 32 entries.
+constexpr int kQuantE = 128;
+constexpr int kRegPieces = 5;
 template <int N>
 struct QShape {
     static constexpr int E = N >= kQuantE ? kQuantE : N;
     static constexpr int LPR = N / E;
     static constexpr int RPT = kCThreads / LPR;   // rows per tile
+    static constexpr int NP = E / 16;             // pieces per lane
+    static constexpr int NREG = NP < kRegPieces ? NP : kRegPieces;
+    static constexpr int SCR = (NP - NREG) * 16 * 4;   // spill bytes per lane
 };
 template <int N>
 struct FShape {
@@ -318,10 +364,12 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     constexpr int MB = F::meta_bytes;
     constexpr int FEB = kBf16 ? 2 : 4;                       // fp element bytes
     constexpr int NP = EQ / 16;                              // 16-entry pieces per lane
+    constexpr int NREG = QShape<N>::NREG;                    // pieces kept in registers
     constexpr int PW = F::quant ? Piece<FMT>::words : 1;     // code words per piece
     constexpr int PB = PW * 4;                               // code bytes per piece
 
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* const smem = smem_raw + ((256u - (saddr(smem_raw) & 255u)) & 255u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
     uint64_t* ufull = empty + kMaxStages;
@@ -523,9 +571,20 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         if constexpr (F::quant) {
             if (ti.quant) {
                 done = true;
-                // this lane's codes and the row's metadata in shared memory
-                const uint8_t* cs = pay + rl * RB + j * CB;
+                // this lane's codes and the row's metadata in shared memory.
+                // The lane visits its pieces in the order pc = sp ^ rot, rot
+                // being its 128-byte line, so the lanes of a warp reading
+                // one step touch every bank group; its code block, B and C
+                // and its row in the pool are aligned so that each permuted
+                // address is a single XOR.
+                const int loff = rl * RB + j * CB;
+                const uint8_t* cs = pay + loff;
+                const unsigned rot = (unsigned)(loff >> 7) & (NP - 1);
+                const unsigned cs_x = saddr(cs) | (rot * PB);
+                const unsigned bx = (saddr(gB) + j * 16) | (rot * LQ * 16);
+                const unsigned cx = (saddr(gC) + j * 16) | (rot * LQ * 16);
                 uint8_t* crow = codes_u + (long long)rr * RB + j * CB;
+                const uintptr_t crow_x = reinterpret_cast<uintptr_t>(crow) | (rot * PB);
                 uint8_t* mrow = meta_u + (long long)rr * MB;
                 float delta0, z0 = 0.0f;
                 {
@@ -538,12 +597,13 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         z0 = m.y;
                     }
                 }
-                const float4* bl = reinterpret_cast<const float4*>(gB) + j;
-                const float4* cl = reinterpret_cast<const float4*>(gC) + j;
+                // pieces NREG.. of the updated row wait in this lane's spill
+                // area: chunk k of lane l at scr + (k * 32 + l) * 16
+                const unsigned scr = saddr(smem + geo.off_scr) + warp * geo.scr_warp_bytes + lane * 16;
                 // decode + update, one 16-entry piece at a time, with
                 // per-piece min / max.  The decode is exact for |z| < 2^22;
                 // rows beyond that take the exact path below.
-                float s[EQ];
+                float s[NREG * 16];
                 float lo, hi;
                 {
                     const float c0 = __fadd_rn(kTwo23, __fadd_rn(z0, F::bias));
@@ -552,33 +612,47 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     const float2 l2 = make_float2(lamv, lamv);
                     const float2 x2 = make_float2(dtx, dtx);
 #pragma unroll
-                    for (int pc = 0; pc < NP; ++pc) {
+                    for (int sp = 0; sp < NP; ++sp) {
                         uint32_t w[PW];
                         if constexpr (PW == 4) {
-                            const uint4 v = *reinterpret_cast<const uint4*>(cs + pc * PB);
+                            const uint4 v = lds128<0>(cs_x ^ (sp * PB));
                             w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
                         } else {
-                            const uint2 v = *reinterpret_cast<const uint2*>(cs + pc * PB);
+                            const uint2 v = lds64<0>(cs_x ^ (sp * PB));
                             w[0] = v.x; w[1] = v.y;
                         }
                         float f[16];
                         unpack16_biased<FMT>(w, f);
-                        const float4* bp = bl + pc * LQ;
-                        float* sp16 = s + 16 * pc;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 bv = bp[i * NP * LQ];
+                        const unsigned bp = bx ^ (sp * LQ * 16);
+                        float v16[16];
+                        auto bq = [&](auto ic) {
+                            constexpr int i = decltype(ic)::value;
+                            const float4 bv = lds128f<i * NP * LQ * 16>(bp);
                             const float2 v0 = mul2(add2(make_float2(f[4 * i], f[4 * i + 1]), nc02), d2);
                             const float2 v1 = mul2(add2(make_float2(f[4 * i + 2], f[4 * i + 3]), nc02), d2);
                             const float2 u0 = fma2(l2, v0, mul2(x2, make_float2(bv.x, bv.y)));
                             const float2 u1 = fma2(l2, v1, mul2(x2, make_float2(bv.z, bv.w)));
-                            sp16[4 * i] = u0.x; sp16[4 * i + 1] = u0.y;
-                            sp16[4 * i + 2] = u1.x; sp16[4 * i + 3] = u1.y;
-                        }
+                            v16[4 * i] = u0.x; v16[4 * i + 1] = u0.y;
+                            v16[4 * i + 2] = u1.x; v16[4 * i + 3] = u1.y;
+                        };
+                        bq(std::integral_constant<int, 0>{});
+                        bq(std::integral_constant<int, 1>{});
+                        bq(std::integral_constant<int, 2>{});
+                        bq(std::integral_constant<int, 3>{});
                         float plo, phi;
-                        minmax16(sp16, plo, phi);
-                        lo = pc == 0 ? plo : fminf(lo, plo);
-                        hi = pc == 0 ? phi : fmaxf(hi, phi);
+                        minmax16(v16, plo, phi);
+                        lo = sp == 0 ? plo : fminf(lo, plo);
+                        hi = sp == 0 ? phi : fmaxf(hi, phi);
+                        if (sp < NREG) {
+#pragma unroll
+                            for (int n = 0; n < 16; ++n) s[(sp < NREG ? sp : 0) * 16 + n] = v16[n];
+                        } else {
+                            const unsigned a = scr + (sp - NREG) * 4 * 512;
+                            sts128f<0>(a, make_float4(v16[0], v16[1], v16[2], v16[3]));
+                            sts128f<512>(a, make_float4(v16[4], v16[5], v16[6], v16[7]));
+                            sts128f<1024>(a, make_float4(v16[8], v16[9], v16[10], v16[11]));
+                            sts128f<1536>(a, make_float4(v16[12], v16[13], v16[14], v16[15]));
+                        }
                     }
                 }
                 const RowParams rp = refit_from_minmax<FMT, LQ>(lo, hi);
@@ -594,35 +668,51 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     // round, pack, store and read back, piece by piece; the
                     // readout sums C (q - z) and scales by Delta once
                     float2 acc = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
-                    auto piece = [&](auto clamp_tag, int pc) {
+                    auto piece = [&](auto clamp_tag, int sp) {
+                        float v16[16];
+                        if (sp < NREG) {
+#pragma unroll
+                            for (int n = 0; n < 16; ++n) v16[n] = s[(sp < NREG ? sp : 0) * 16 + n];
+                        } else {
+                            const unsigned a = scr + (sp - NREG) * 4 * 512;
+                            const float4 q0 = lds128f<0>(a), q1 = lds128f<512>(a);
+                            const float4 q2 = lds128f<1024>(a), q3 = lds128f<1536>(a);
+                            v16[0] = q0.x; v16[1] = q0.y; v16[2] = q0.z; v16[3] = q0.w;
+                            v16[4] = q1.x; v16[5] = q1.y; v16[6] = q1.z; v16[7] = q1.w;
+                            v16[8] = q2.x; v16[9] = q2.y; v16[10] = q2.z; v16[11] = q2.w;
+                            v16[12] = q3.x; v16[13] = q3.y; v16[14] = q3.z; v16[15] = q3.w;
+                        }
                         float r[16];
                         uint32_t kk[16];
-                        round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, s + 16 * pc,
-                                                                       r, kk, pv.neg_zero);
+                        round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, v16, r, kk,
+                                                                       pv.neg_zero);
                         uint32_t w[PW];
                         pack16<FMT>(kk, w);
                         if (active) {
+                            void* dst = reinterpret_cast<void*>(crow_x ^ (uintptr_t)(sp * PB));
                             if constexpr (PW == 4)
-                                __stcs(reinterpret_cast<uint4*>(crow + pc * PB),
-                                       make_uint4(w[0], w[1], w[2], w[3]));
+                                __stcs(reinterpret_cast<uint4*>(dst), make_uint4(w[0], w[1], w[2], w[3]));
                             else
-                                __stcs(reinterpret_cast<uint2*>(crow + pc * PB),
-                                       make_uint2(w[0], w[1]));
+                                __stcs(reinterpret_cast<uint2*>(dst), make_uint2(w[0], w[1]));
                         }
-                        const float4* cp = cl + pc * LQ;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 cv4 = cp[i * NP * LQ];
+                        const unsigned cp = cx ^ (sp * LQ * 16);
+                        auto cq = [&](auto ic) {
+                            constexpr int i = decltype(ic)::value;
+                            const float4 cv4 = lds128f<i * NP * LQ * 16>(cp);
                             acc = fma2(make_float2(cv4.x, cv4.y), make_float2(r[4 * i], r[4 * i + 1]), acc);
                             acc1 = fma2(make_float2(cv4.z, cv4.w), make_float2(r[4 * i + 2], r[4 * i + 3]), acc1);
-                        }
+                        };
+                        cq(std::integral_constant<int, 0>{});
+                        cq(std::integral_constant<int, 1>{});
+                        cq(std::integral_constant<int, 2>{});
+                        cq(std::integral_constant<int, 3>{});
                     };
                     if (F::sym || !__any_sync(0xffffffffu, rp.clamp)) {
 #pragma unroll
-                        for (int pc = 0; pc < NP; ++pc) piece(std::false_type{}, pc);
+                        for (int sp = 0; sp < NP; ++sp) piece(std::false_type{}, sp);
                     } else {
 #pragma unroll
-                        for (int pc = 0; pc < NP; ++pc) piece(std::true_type{}, pc);
+                        for (int sp = 0; sp < NP; ++sp) piece(std::true_type{}, sp);
                     }
                     acc = add2(acc, acc1);
                     ysum = __fmul_rn(rp.delta, grp_sum<LQ>(__fadd_rn(acc.x, acc.y)));
@@ -721,11 +811,12 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
     const int fpEB = FMT == SSQ_BF16 ? 2 : 4;
     // stages: as many as fit a budget that leaves room for kMinBlocks CTAs per SM
     const int budget = (kMinBlocks == 1 ? 200 : 110) * 1024;
-    DecodeGeom g = decode_geom(2, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G);
-    int S = (budget - g.off_stages) / g.stage_bytes;
+    constexpr int SCR = F::quant ? QShape<N>::SCR : 0;
+    DecodeGeom g = decode_geom(2, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G, SCR);
+    int S = (budget - (g.smem_bytes - 2 * g.stage_bytes)) / g.stage_bytes;
     if (S > kMaxStages) S = kMaxStages;
     if (S < 2) S = 2;
-    g = decode_geom(S, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G);
+    g = decode_geom(S, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G, SCR);
     if (g.smem_bytes > 227 * 1024) return cudaErrorInvalidConfiguration;
     auto kern = decode_kernel<FMT, N>;
     // per-device launch facts, looked up once per kernel instantiation and device
@@ -789,7 +880,10 @@ bool decode_fits(int fmt, int d_state, int nheads, int ngroups)
     int rq = 0, rf = 0;
     decode_tile_rows(fmt, d_state, &rq, &rf);
     const bool q = fmt >= SSQ_I8_SYM;
-    const DecodeGeom g = decode_geom(2, rq, rf, d_state, 8, 4, q, true, d_state, nheads, ngroups);
+    const int eq = d_state >= kQuantE ? kQuantE : d_state;
+    const int np = eq / 16, nreg = np < kRegPieces ? np : kRegPieces;
+    const DecodeGeom g = decode_geom(2, rq, rf, d_state, 8, 4, q, true, d_state, nheads, ngroups,
+                                     (np - nreg) * 64);
     return g.smem_bytes <= 227 * 1024;
 }
 
