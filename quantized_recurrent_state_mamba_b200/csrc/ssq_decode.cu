@@ -13,7 +13,8 @@
 //   - work is a sequence of tiles (up to RPT rows of one region of one
 //     (layer, request)); each CTA owns a contiguous range of that sequence;
 //   - a producer warp streams each tile's packed rows and metadata from HBM
-//     into a ring of shared-memory stages with bulk asynchronous copies
+//     (prefetched into L2 as soon as the tile is next in line) into a ring
+//     of shared-memory stages with bulk asynchronous copies
 //     (cp.async.bulk, completion counted in bytes on an mbarrier) and the
 //     tile's x values with cp.async.  Once per (layer, request, region)
 //     "unit" it stages B and C and builds a head table (lambda, dt, D, the
@@ -60,6 +61,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* b)
 {
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
 }
+// Arrive from the lanes where `pred` holds (predicated inside the
+// instruction, so the warp does not branch).
+__device__ __forceinline__ void mbar_arrive_if(uint64_t* b, bool pred)
+{
+    asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n"
+                 " @p mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n}\n"
+                 ::"r"(saddr(b)), "r"((unsigned)pred) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, unsigned bytes)
 {
     asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
@@ -93,6 +102,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, unsigned parity)
 }
 constexpr unsigned kProducerSleep = 2048;  // the producer waits for a stage to drain
 constexpr unsigned kConsumerSleep = 256;   // consumers wait for data to land
+// Bulk prefetch of global memory into L2 (no completion to wait for).
+// Address 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, unsigned bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // Bulk copy global -> shared; completion counted in bytes on `bar`.
 // Both addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar)
@@ -468,6 +483,16 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 if (lane == 0) mbar_arrive(&ufull[u]);
             }
             if (bad) continue;
+            // start the tile's HBM reads into L2 now; the copy into the stage,
+            // issued once the consumers release it, then reads from L2
+            if (lane == 0) {
+                if (F::quant && ti.quant) {
+                    bulk_prefetch_l2(codes_u + (long long)ti.rbase * RB, (unsigned)r16(ti.n * RB));
+                    bulk_prefetch_l2(meta_u + (long long)ti.rbase * MB, (unsigned)r16(ti.n * MB));
+                } else {
+                    bulk_prefetch_l2(fp_u + (long long)ti.rbase * N * FEB, (unsigned)(ti.n * N * FEB));
+                }
+            }
             if (!mbar_wait<kProducerSleep>(&empty[si], sph ^ 1)) { ok = false; break; }
             uint8_t* st = stages + si * geo.stage_bytes;
             float* sx = reinterpret_cast<float*>(st);
@@ -522,7 +547,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         if (newunit) {
             if (uk >= 0) {
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&uempty[uk & 1]);
+                mbar_arrive_if(&uempty[uk & 1], lane == 0);
             }
             ++uk;
             const int u = uk & 1;
@@ -554,7 +579,10 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         const int grow = ti.quant ? ct / LQ : ct / LF;
         const int j = ti.quant ? ct % LQ : ct % LF;
         const bool active = grow < ti.n;
-        const int rl = active ? grow : 0;          // inactive rows shadow row 0
+        // Rows past the end of a partial tile shadow its row 0: they read
+        // row 0's inputs and so compute and store exactly row 0's bytes,
+        // which lets every store go without a branch.
+        const int rl = active ? grow : 0;
         const int rr = ti.rbase + rl;
         const int hr = fdiv(rr, pv.mP);
         const int p = rr - hr * P;
@@ -688,7 +716,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                                                                        pv.neg_zero);
                         uint32_t w[PW];
                         pack16<FMT>(kk, w);
-                        if (active) {
+                        {
                             void* dst = reinterpret_cast<void*>(crow_x ^ (uintptr_t)(sp * PB));
                             if constexpr (PW == 4)
                                 __stcs(reinterpret_cast<uint4*>(dst), make_uint4(w[0], w[1], w[2], w[3]));
@@ -716,14 +744,14 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     }
                     acc = add2(acc, acc1);
                     ysum = __fmul_rn(rp.delta, grp_sum<LQ>(__fadd_rn(acc.x, acc.y)));
-                    if (active && j == 0) {
-                        if constexpr (F::sym) {
-                            __stcs(reinterpret_cast<float*>(mrow), rp.delta);
-                        } else {
-                            __stcs(reinterpret_cast<float2*>(mrow), make_float2(rp.delta, rp.z));
-                        }
-                        if (!rp.finite) atomicOr(err, SSQ_DEVERR_NONFINITE);
+                    // every lane of the row writes the same metadata
+                    if constexpr (F::sym) {
+                        __stcs(reinterpret_cast<float*>(mrow), rp.delta);
+                    } else {
+                        __stcs(reinterpret_cast<float2*>(mrow), make_float2(rp.delta, rp.z));
                     }
+                    if (__any_sync(0xffffffffu, !rp.finite) && lane == 0)
+                        atomicOr(err, SSQ_DEVERR_NONFINITE);
                 } else {
                     ysum = row_exact<FMT, N>(cs, delta0, z0, lamv, dtx, gB, gC, j, active, crow,
                                              mrow, err);
@@ -785,18 +813,16 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
 #pragma unroll
                     for (int n = 0; n < EPC; ++n) w[n] = __float_as_uint(sv[n]);
                 }
-                if (active)
-                    __stcs(reinterpret_cast<uint4*>(frow) + m, make_uint4(w[0], w[1], w[2], w[3]));
+                __stcs(reinterpret_cast<uint4*>(frow) + m, make_uint4(w[0], w[1], w[2], w[3]));
             }
             acc = add2(acc, acc1);
             ysum = grp_sum<LF>(__fadd_rn(acc.x, acc.y));
         }
-        if (active && j == 0) {
-            const float yv = __fadd_rn(ysum, __fmul_rn(hti.z, xv));
-            __stcs(y_u + __float_as_int(hti.w) + p, yv);
-        }
+        // every lane of the row writes the same y (after the row sum all
+        // hold it)
+        __stcs(y_u + __float_as_int(hti.w) + p, __fadd_rn(ysum, __fmul_rn(hti.z, xv)));
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[si]);
+        mbar_arrive_if(&empty[si], lane == 0);
         if (++si == S) { si = 0; sph ^= 1; }
     }
 }
@@ -810,7 +836,7 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
     const bool has_q = pv.Hq > 0, has_fp = pv.Hf > 0;
     const int fpEB = FMT == SSQ_BF16 ? 2 : 4;
     // stages: as many as fit a budget that leaves room for kMinBlocks CTAs per SM
-    const int budget = (kMinBlocks == 1 ? 200 : 110) * 1024;
+    const int budget = (kMinBlocks == 1 ? 225 : 110) * 1024;
     constexpr int SCR = F::quant ? QShape<N>::SCR : 0;
     DecodeGeom g = decode_geom(2, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G, SCR);
     int S = (budget - (g.smem_bytes - 2 * g.stage_bytes)) / g.stage_bytes;
