@@ -153,7 +153,8 @@ def bf16_round(v):
 
 def quantize_row(fmt, v):
     """Refit and round one row.  Returns (codes, delta, zero, pre) where pre
-    is the pre-rounding value fl(v*inv) of each entry."""
+    is the pre-rounding value v*inv of each entry (the exact product,
+    stored as float32)."""
     v = _f32(v)
     N = v.shape[0]
     q = np.zeros(N, np.int32)

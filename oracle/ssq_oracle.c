@@ -88,8 +88,11 @@ static float qmax_of(int fmt)
 
 /* Refit and round one row (ssm-state-quantization README, Setup: per-row
  * scale refit every step, symmetric or asymmetric grid; Findings 1: nearest
- * rounding).  'pre' (optional) receives the pre-rounding value fl(v*inv) of
- * each entry, used by the tests to find entries on a rounding boundary. */
+ * rounding).  Each value is rounded to the nearest integer multiple of the
+ * step as v*inv with the product taken exactly (in double, where the product
+ * of two floats is exact) and one rounding, ties to even; the zero point
+ * likewise.  'pre' (optional) receives the pre-rounding value v*inv of each
+ * entry, used by the tests to find entries on a rounding boundary. */
 void oref_quantize_row_dbg(int fmt, int N, const float* v, int32_t* q,
                            float* delta_out, float* zero_out, float* pre)
 {
@@ -125,13 +128,13 @@ void oref_quantize_row_dbg(int fmt, int N, const float* v, int32_t* q,
     if (!sym) {
         /* Integer zero point: the code of lo is rint(lo*inv) + z = 0.
          * Adding +0 stores a negative zero as +0. */
-        z = rintf(-lo * inv) + 0.0f;
+        z = (float)rint(-(double)lo * (double)inv) + 0.0f;
     }
 
     for (int n = 0; n < N; ++n) {
-        float p = v[n] * inv;          /* one fp32 product */
-        float r = rintf(p);            /* nearest, ties to even */
-        if (pre) pre[n] = p;
+        double p = (double)v[n] * (double)inv;   /* the exact product */
+        float r = (float)rint(p);                 /* nearest, ties to even */
+        if (pre) pre[n] = (float)p;
         float c;
         if (sym) {
             c = r;
@@ -226,7 +229,7 @@ void oref_state_to_f32(const oref_cfg* c, const oref_state* st, float* S)
  *      read from the newly stored state ("ssm-state-quantization", Setup:
  *      the output is read from the quantized state).
  * x[H][P], B/C[G][N], dt/A/D[H], y[H][P].  'pre' (optional, [H*P*N])
- * receives fl(s'*inv) for quantized rows. */
+ * receives s'*inv for quantized rows. */
 void oref_step(const oref_cfg* c, oref_state* st, const float* x,
                const float* B, const float* C, const float* dt,
                const float* A, const float* D, float* y, float* pre)

@@ -29,7 +29,9 @@
  * Readings where the pages are silent (each is listed in the design notes):
  *   - input term dt*B (x) x, the Mamba-2 form; dt arrives already positive;
  *   - group map g(h) = h / (H/G);
- *   - round half to even (rintf under FE_TONEAREST) on fl(s'*inv);
+ *   - round half to even (rint under FE_TONEAREST) on the exact product
+ *     s'*inv (one rounding; the product is formed in double, where the
+ *     product of two floats is exact), and the zero point likewise;
  *   - inv = 1/Delta once per row, then a multiply per entry;
  *   - zero point z = rint(-lo*inv) kept unclamped in an fp32 slot;
  *   - constant row: Delta := |lo|; Delta below FLT_MIN flushes the row to

@@ -128,7 +128,6 @@ ssq_status make_pool_view(const ssq_config* cfg, void* pool, ssq::PoolView* pv,
     pv->hpg = cfg->nheads / cfg->ngroups;
     pv->Hq = L->n_quant_heads;
     pv->Hf = L->n_fp_heads;
-    pv->neg_zero = -0.0f;
     pv->mP = ssq::fdiv_magic(pv->P);
     pv->mHpg = ssq::fdiv_magic(pv->hpg);
     for (int i = 0; i < cfg->nheads; ++i) pv->perm[i] = (uint16_t)perm[i];

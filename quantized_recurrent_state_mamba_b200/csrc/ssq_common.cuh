@@ -32,8 +32,11 @@ constexpr int kThreads = 256;
 // and leaves that integer in the low mantissa bits of the sum.
 constexpr float kMagic = 12582912.0f;
 constexpr float kTwo23 = 8388608.0f;
-// Below 2^22 in magnitude the magic-number paths are exact.
+// Below 2^22 in magnitude the magic-number decode is exact; the rounding
+// path checks its scaled values against 2^21 (a margin for the fp32 product
+// that the check uses).
 constexpr float kFastLimit = 4194304.0f;
+constexpr float kRoundLimit = 2097152.0f;
 
 // ---------------------------------------------------------------------------
 // Format traits
@@ -382,6 +385,15 @@ __device__ __forceinline__ void decode_row(const Chunk<E * Fmt<FMT>::bits / 8>& 
     }
 }
 
+// rint(a*b) with the product exact: formed in double, where the product of
+// two floats is exact, and rounded once to the nearest integer (ties to
+// even).  The magic-number paths below compute the same value in one fp32
+// FMA, fma(a, b, 1.5*2^23) - 1.5*2^23, for |a*b| < 2^21.
+__device__ __forceinline__ float rint_prod(float a, float b)
+{
+    return (float)rint((double)a * (double)b);
+}
+
 // ---------------------------------------------------------------------------
 // Row refit + round.
 //
@@ -389,7 +401,8 @@ __device__ __forceinline__ void decode_row(const Chunk<E * Fmt<FMT>::bits / 8>& 
 // Delta, inv = 1/Delta and z, round every entry, and produce
 //   r[n]  = q_n - z as fp32 (what the stored row decodes to, before * Delta)
 //   k[n]  = a carrier whose low bits are the stored code.
-// Reading of the pages' silent points: ties to even on fl(s'*inv); z =
+// Reading of the pages' silent points: ties to even on the exact product
+// s'*inv (one rounding); z =
 // rint(-lo*inv) unclamped (negative zero stored as +0); a constant row takes
 // Delta = |lo|; Delta below FLT_MIN flushes the row to zero; asym codes
 // clamp at qa (the minimum maps to 0 by construction); the sym clamp never
@@ -441,13 +454,13 @@ __device__ __forceinline__ RowParams refit_from_minmax(float lo, float hi)
     if (delta < 1.17549435e-38f) delta = 0.0f;  // FLT_MIN
     const float inv = (delta == 0.0f) ? 0.0f : __frcp_rn(delta);
     float z = 0.0f;
-    if constexpr (!F::sym) z = __fadd_rn(rintf(__fmul_rn(-lo, inv)), 0.0f);
+    if constexpr (!F::sym) z = __fadd_rn(rint_prod(-lo, inv), 0.0f);
     const float plo = __fmul_rn(lo, inv), phi = __fmul_rn(hi, inv);
     rp.delta = delta;
     rp.inv = inv;
     rp.z = z;
-    rp.fast = fmaxf(fabsf(plo), fabsf(phi)) < kFastLimit && fabsf(z) < kFastLimit;
-    rp.clamp = (!F::sym) && (__fadd_rn(rintf(phi), z) > F::qmax);
+    rp.fast = fmaxf(fabsf(plo), fabsf(phi)) < kRoundLimit && fabsf(z) < kRoundLimit;
+    rp.clamp = (!F::sym) && (__fadd_rn(rint_prod(hi, inv), z) > F::qmax);
     return rp;
 }
 
@@ -489,21 +502,19 @@ __device__ __forceinline__ RowParams refit_row(const float (&s)[E])
 }
 
 // Fast rounding of 16 entries (valid when the warp's rows all passed the
-// fast test): r = rint(fl(s*inv)) exactly, k carries the stored code.
+// fast test): r = rint(s*inv) (exact product) exactly, k carries the stored code.
 template <int FMT>
 __device__ __forceinline__ void round16_fast(const RowParams& rp, const float* s, float* r,
-                                             uint32_t (&k)[16], float nz)
+                                             uint32_t (&k)[16])
 {
     using F = Fmt<FMT>;
-    const float2 nz2 = make_float2(nz, nz);
     const float2 inv2 = make_float2(rp.inv, rp.inv);
     const float2 m2 = make_float2(kMagic, kMagic);
     const float2 nm2 = make_float2(-kMagic, -kMagic);
     const float2 z2 = make_float2(rp.z, rp.z);
 #pragma unroll
     for (int n = 0; n < 16; n += 2) {
-        float2 p = fma2(make_float2(s[n], s[n + 1]), inv2, nz2);
-        float2 t = add2(p, m2);
+        float2 t = fma2(make_float2(s[n], s[n + 1]), inv2, m2);   // 1.5*2^23 + rint(s*inv)
         float2 rr = add2(t, nm2);
         r[n] = rr.x; r[n + 1] = rr.y;
         if constexpr (F::sym) {
@@ -525,16 +536,16 @@ __device__ __forceinline__ void round16_fast(const RowParams& rp, const float* s
 // below 2^24 in magnitude.
 template <int FMT, bool CLAMP>
 __device__ __forceinline__ void round16_carry(float2 inv2, float2 z2, float2 mz2, float* s,
-                                              float* r, uint32_t (&k)[16], float nz)
+                                              float* r, uint32_t (&k)[16])
 {
     using F = Fmt<FMT>;
-    const float2 nz2 = make_float2(nz, nz);
     const float2 m2 = make_float2(kMagic, kMagic);
     constexpr float kTop = kMagic + F::qmax;   // carrier of code qa
 #pragma unroll
     for (int n = 0; n < 16; n += 2) {
-        const float2 p = fma2(make_float2(s[n], s[n + 1]), inv2, nz2);
-        const float2 t = add2(p, m2);                  // 1.5*2^23 + rint(p)
+        // 1.5*2^23 + rint(s*inv): the exact product and the magic number
+        // rounded together, once
+        const float2 t = fma2(make_float2(s[n], s[n + 1]), inv2, m2);
         if constexpr (F::sym) {
             const float2 rr = add2(t, mz2);            // rint(p), exact
             r[n] = rr.x; r[n + 1] = rr.y;
@@ -562,7 +573,7 @@ __device__ __forceinline__ void round16_slow(const RowParams& rp, const float* s
     using F = Fmt<FMT>;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
-        const float rr = rintf(__fmul_rn(s[n], rp.inv));
+        const float rr = rint_prod(s[n], rp.inv);
         float c;
         if constexpr (F::sym) {
             c = fminf(fmaxf(rr, -F::qmax), F::qmax);
@@ -579,20 +590,18 @@ __device__ __forceinline__ void round16_slow(const RowParams& rp, const float* s
 // the choice is warp-uniform and every lane of the warp must call this.
 template <int FMT, int E>
 __device__ __forceinline__ bool round_row(const RowParams& rp, const float (&s)[E],
-                                          float (&r)[E], uint32_t (&k)[E], float nz)
+                                          float (&r)[E], uint32_t (&k)[E])
 {
     using F = Fmt<FMT>;
     const bool fast = __all_sync(0xffffffffu, rp.fast && !rp.clamp);
     if (fast) {
-        const float2 nz2 = make_float2(nz, nz);
         const float2 inv2 = make_float2(rp.inv, rp.inv);
         const float2 m2 = make_float2(kMagic, kMagic);
         const float2 nm2 = make_float2(-kMagic, -kMagic);
         const float2 z2 = make_float2(rp.z, rp.z);
 #pragma unroll
         for (int n = 0; n < E; n += 2) {
-            float2 p = fma2(make_float2(s[n], s[n + 1]), inv2, nz2);
-            float2 t = add2(p, m2);            // 1.5*2^23 + rint(p)
+            float2 t = fma2(make_float2(s[n], s[n + 1]), inv2, m2);   // 1.5*2^23 + rint(s*inv)
             float2 rr = add2(t, nm2);          // rint(p), exact
             r[n] = rr.x; r[n + 1] = rr.y;
             if constexpr (F::sym) {
@@ -608,7 +617,7 @@ __device__ __forceinline__ bool round_row(const RowParams& rp, const float (&s)[
         // The scalar formulas verbatim.
 #pragma unroll
         for (int n = 0; n < E; ++n) {
-            const float rr = rintf(__fmul_rn(s[n], rp.inv));
+            const float rr = rint_prod(s[n], rp.inv);
             float c;
             if constexpr (F::sym) {
                 c = fminf(fmaxf(rr, -F::qmax), F::qmax);

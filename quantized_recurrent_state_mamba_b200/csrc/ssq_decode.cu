@@ -333,7 +333,7 @@ __device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float de
     for (int i = 0; i < CB / 4; ++i) words[i] = 0u;
 #pragma unroll 1
     for (int n = 0; n < E; ++n) {
-        const float rr = rintf(__fmul_rn(s[n], rp.inv));
+        const float rr = rint_prod(s[n], rp.inv);
         float c, r;
         if constexpr (F::sym) {
             c = fminf(fmaxf(rr, -F::qmax), F::qmax);
@@ -712,8 +712,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         }
                         float r[16];
                         uint32_t kk[16];
-                        round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, v16, r, kk,
-                                                                       pv.neg_zero);
+                        round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, v16, r, kk);
                         uint32_t w[PW];
                         pack16<FMT>(kk, w);
                         {

@@ -18,7 +18,6 @@ struct PoolView {
     int n_slots, n_layers;
     int H, P, N, G, hpg;       // heads, head_dim, d_state, groups, heads/group
     int Hq, Hf;                // heads in the quantized / fp region
-    float neg_zero;            // -0.0f, opaque to the compiler (see round_row)
     // n / P and h / hpg as (n * m) >> 32 with m = floor(2^32 / d) + 1: exact
     // for n < 2^32 / d (row and head indices are far below that)
     unsigned long long mP, mHpg;

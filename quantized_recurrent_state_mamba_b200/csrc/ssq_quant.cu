@@ -83,7 +83,7 @@ rows_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
                 const RowParams rp = refit_row<FMT, E, LPR>(s);
                 float rq[E];
                 uint32_t k[E];
-                round_row<FMT, E>(rp, s, rq, k, pv.neg_zero);
+                round_row<FMT, E>(rp, s, rq, k);
                 pack_codes<FMT, E>(k, c);
                 if (active) {
                     store_chunk<CB>(crow, c);

@@ -69,14 +69,14 @@ __host__ __device__ inline int scan_entries(int N, bool wide)
     return wide ? 64 : 32;
 }
 
-// Round 16 entries of a row on the fast path: s <- fl(rint(fl(s*inv)) *
-// Delta); with CODES also the carriers of the stored codes.
+// Round 16 entries of a row on the fast path: s <- fl(rint(s*inv) * Delta),
+// the product s*inv exact (one FMA with the magic number); with CODES also
+// the carriers of the stored codes.
 template <int FMT, bool CODES>
 __device__ __forceinline__ void round_piece_fast(const RowParams& rp, float* s,
-                                                 uint32_t (&k)[16], float nz)
+                                                 uint32_t (&k)[16])
 {
     using F = Fmt<FMT>;
-    const float2 nz2 = make_float2(nz, nz);
     const float2 inv2 = make_float2(rp.inv, rp.inv);
     const float2 d2 = make_float2(rp.delta, rp.delta);
     const float2 m2 = make_float2(kMagic, kMagic);
@@ -84,8 +84,7 @@ __device__ __forceinline__ void round_piece_fast(const RowParams& rp, float* s,
     const float2 z2 = make_float2(rp.z, rp.z);
 #pragma unroll
     for (int n = 0; n < 16; n += 2) {
-        const float2 p = fma2(make_float2(s[n], s[n + 1]), inv2, nz2);
-        const float2 t = add2(p, m2);          // 1.5*2^23 + rint(p)
+        const float2 t = fma2(make_float2(s[n], s[n + 1]), inv2, m2);   // 1.5*2^23 + rint(s*inv)
         const float2 r = add2(t, nm2);         // rint(p) = q - z, exact
         const float2 v = mul2(r, d2);
         s[n] = v.x; s[n + 1] = v.y;
@@ -110,7 +109,7 @@ __device__ __forceinline__ void round_piece_slow(const RowParams& rp, float* s,
     using F = Fmt<FMT>;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
-        const float rr = rintf(__fmul_rn(s[n], rp.inv));
+        const float rr = rint_prod(s[n], rp.inv);
         float c, r;
         if constexpr (F::sym) {
             c = fminf(fmaxf(rr, -F::qmax), F::qmax);
@@ -336,7 +335,7 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
             if (__all_sync(0xffffffffu, rp.fast && !rp.clamp)) {
 #pragma unroll
                 for (int pc = 0; pc < NP; ++pc) {
-                    round_piece_fast<FMT, CODES>(rp, s + 16 * pc, kc, pv.neg_zero);
+                    round_piece_fast<FMT, CODES>(rp, s + 16 * pc, kc);
                     if constexpr (CODES) pack16<FMT>(kc, cw + PW * pc);
                 }
             } else {

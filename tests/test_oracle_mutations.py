@@ -18,7 +18,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "ssq_oracle.c")
 
 MUTATIONS = {
-    "z_sign": ("z = rintf(-lo * inv) + 0.0f;", "z = rintf(lo * inv) + 0.0f;"),
+    "z_sign": ("z = (float)rint(-(double)lo * (double)inv) + 0.0f;",
+               "z = (float)rint((double)lo * (double)inv) + 0.0f;"),
     "asym_levels_2b": ("return (float)((1 << b) - 1);", "return (float)(1 << b);"),
     "sym_levels_2b1": ("return (float)((1 << (b - 1)) - 1);",
                        "return (float)(1 << (b - 1));"),
@@ -26,12 +27,12 @@ MUTATIONS = {
     "decay_not_exp": ("double e = exp((double)dA);", "double e = 1.0 + (double)dA;"),
     "group_map": ("const int g = h / heads_per_group;",
                   "const int g = h % G;"),
-    "round_half_away": ("float r = rintf(p);", "float r = roundf(p);"),
+    "round_half_away": ("float r = (float)rint(p);", "float r = (float)round(p);"),
     "y_before_rounding": ("acc += (double)Cg[n] * (double)stored[n];",
                           "acc += (double)Cg[n] * (double)sn[n];"),
     "no_skip_term": ("acc += (double)D[h] * (double)x[r];", "acc += 0.0;"),
     "no_clamp": ("if (c > qm) c = qm;\n        }", "}"),
-    "truncate": ("float r = rintf(p);", "float r = truncf(p);"),
+    "truncate": ("float r = (float)rint(p);", "float r = (float)trunc(p);"),
     "deq_drop_zero": ("float d = (float)q[n] - zero;", "float d = (float)q[n];"),
     "swap_B_C": ("float w = dtx * Bg[n];", "float w = dtx * Cg[n];"),
     "constant_row_step": ("if (delta == 0.0f) delta = fabsf(lo);",
