@@ -44,7 +44,7 @@ METRIC = "quantized state-update HBM GB/s (% of B200 peak) and request-steps/s/l
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 SM_MAX_MHZ = 1965.0        # B200 maximum SM clock, used when NVML is unavailable
-SCAN_FP32_OPS = 7          # algorithmic fp32 operations per element-token of the scan
+SCAN_FP32_OPS = 6          # algorithmic fp32 operations per element-token of the scan
 
 
 # ---------------------------------------------------------------------------
@@ -520,7 +520,8 @@ def run_ours(args, wl, name):
         # The scan reads each input once and keeps the state on chip: its
         # bound is the FP32 pipe, not HBM.  Algorithmic fp32 operations per
         # element-token (each add / mul / fma one): w = dtx*B, s' = fma,
-        # p = s'*inv, +M and -M (round to nearest), r*Delta, C*r = 7.
+        # fma(s', inv, M) and -M (round the exact product to nearest),
+        # r*Delta, C*r = 6.
         # Peak: 148 SMs x 128 FP32 lanes x the maximum SM clock.
         ops = SCAN_FP32_OPS * elem_steps(wl)
         sm_max = clocks.get("sm_max_mhz") or SM_MAX_MHZ
