@@ -454,13 +454,24 @@ __device__ __forceinline__ RowParams refit_from_minmax(float lo, float hi)
     if (delta < 1.17549435e-38f) delta = 0.0f;  // FLT_MIN
     const float inv = (delta == 0.0f) ? 0.0f : __frcp_rn(delta);
     float z = 0.0f;
-    if constexpr (!F::sym) z = __fadd_rn(rint_prod(-lo, inv), 0.0f);
     const float plo = __fmul_rn(lo, inv), phi = __fmul_rn(hi, inv);
+    // Below 2^21 the exact-product rounding is one FMA with the magic
+    // number; rows beyond it (rare: far from zero relative to their range)
+    // take it in double.
+    const bool small = fmaxf(fabsf(plo), fabsf(phi)) < kRoundLimit;
+    float rhi;
+    if (small) {
+        if constexpr (!F::sym) z = __fadd_rn(__fsub_rn(__fmaf_rn(-lo, inv, kMagic), kMagic), 0.0f);
+        rhi = __fsub_rn(__fmaf_rn(hi, inv, kMagic), kMagic);
+    } else {
+        if constexpr (!F::sym) z = __fadd_rn(rint_prod(-lo, inv), 0.0f);
+        rhi = rint_prod(hi, inv);
+    }
     rp.delta = delta;
     rp.inv = inv;
     rp.z = z;
-    rp.fast = fmaxf(fabsf(plo), fabsf(phi)) < kRoundLimit && fabsf(z) < kRoundLimit;
-    rp.clamp = (!F::sym) && (__fadd_rn(rint_prod(hi, inv), z) > F::qmax);
+    rp.fast = small && fabsf(z) < kRoundLimit;
+    rp.clamp = (!F::sym) && (__fadd_rn(rhi, z) > F::qmax);
     return rp;
 }
 

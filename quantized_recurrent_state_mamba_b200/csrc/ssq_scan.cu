@@ -16,7 +16,8 @@
 // i of lane j at position i * LPR + j), so the lanes of a warp read
 // consecutive 16-byte words.  lambda = exp(dt * A) is computed once per
 // token per CTA.  The token loop streams each lane's entries in pieces of 16:
-// update and min / max, refit, then round, rescale and read out.
+// the readout of the previous token and the update of this one in one pass,
+// min / max, refit, then round and rescale.
 #include "ssq_common.cuh"
 #include "ssq_params.h"
 
@@ -53,6 +54,12 @@ struct SGeom {
     static constexpr int NP = E / 16;                 // 16-entry pieces per lane
     static_assert(E % 16 == 0 && N % E == 0 && LPR <= 32, "bad scan shape");
 };
+
+// Staging buffers: chunk c is read from buffer c % 3 while chunk c + 1 is
+// staged into the next; the third keeps chunk c - 1, whose last token's C the
+// first token of chunk c still reads (the readout of token t is fused into
+// the update of token t + 1).
+constexpr int kScanBufs = 3;
 
 // Floats of one staging buffer: B, C [K][N]; x [K][rows]; dt, lambda [K].
 __host__ __device__ inline int scan_buf_floats(int N, int K, int rows)
@@ -124,7 +131,7 @@ __device__ __forceinline__ void round_piece_slow(const RowParams& rp, float* s,
 }
 
 template <int FMT, int N, int E>
-__global__ void __launch_bounds__(64)
+__global__ void __launch_bounds__(64, E >= 64 ? 6 : 8)
 scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv)
 {
     using F = Fmt<FMT>;
@@ -251,14 +258,43 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
     float* const yrow = cv.y + (bT * H + h) * P + p;   // y of this row at token 0
     const bool ylane = active && j == 0;
     const int nchunks = (T + K - 1) / K;
+    // The readout of token t, y_t = C_t . s_t + D x_t, is formed while token
+    // t + 1 updates the state: one pass over the entries reads s_t for both,
+    // and the row sum of y_t overlaps the refit of token t + 1.
+    const float* cprev = nullptr;     // C row of token t - 1 in shared memory
+    float xprev = 0.0f;               // x of this row at token t - 1
+    auto emit_y = [&](int t, float ysum, float xv) {
+        if (ylane) __stcs(yrow + (long long)t * HP, __fadd_rn(ysum, __fmul_rn(Dv, xv)));
+    };
+    // C . s over the lane's entries, reduced over the row's lanes
+    auto readout = [&](const float* crow_s) {
+        const float4* c4 = reinterpret_cast<const float4*>(crow_s) + j;
+        float2 accp[NP];
+#pragma unroll
+        for (int pc = 0; pc < NP; ++pc) {
+            const float* sp = s + 16 * pc;
+            float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 v = c4[(4 * pc + i) * LPR];
+                acc = fma2(make_float2(v.x, v.y), make_float2(sp[4 * i], sp[4 * i + 1]), acc);
+                acc = fma2(make_float2(v.z, v.w), make_float2(sp[4 * i + 2], sp[4 * i + 3]), acc);
+            }
+            accp[pc] = acc;
+        }
+        float2 acc = accp[0];
+#pragma unroll
+        for (int pc = 1; pc < NP; ++pc) acc = add2(acc, accp[pc]);
+        return grp_sum<LPR>(__fadd_rn(acc.x, acc.y));
+    };
     stage(0, 0);
     for (int c = 0; c < nchunks; ++c) {
-        const int bi = c & 1;
+        const int bi = c % kScanBufs;
         const int t0 = c * K;
         const int nt = min(K, T - t0);
         cp_async_wait_all();
-        __syncthreads();   // chunk c visible to all; everyone is done with chunk c-1
-        if (c + 1 < nchunks) stage(t0 + K, bi ^ 1);
+        __syncthreads();   // chunk c visible to all; everyone is done with chunk c-2
+        if (c + 1 < nchunks) stage(t0 + K, (c + 1) % kScanBufs);
         const float* sB = smem + bi * bufsz;
         const float* sC = sB + K * N;
         const float* sx = sC + K * N;
@@ -267,68 +303,76 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
         if (tid < nt) slam[tid] = decay(sdt[tid], Av);
         __syncthreads();
 
-        float* const yc = yrow + (long long)t0 * HP;
-        // update + min / max of one token's B over the lane's entries
-        auto update_q = [&](int tt, float& lo, float& hi) {
+        // Update one token's state (s <- lambda s + dt x B) with the min /
+        // max of the result; with READ also the readout of the previous
+        // token from the state before the update.  Returns x of this row.
+        auto update = [&](auto read_tag, auto quant_tag, int tt, float& lo, float& hi,
+                          float& yprev) {
+            constexpr bool READ = decltype(read_tag)::value;
+            constexpr bool MINMAX = decltype(quant_tag)::value;
             const float xv = sx[tt * rows + rowe];
             const float dtx = __fmul_rn(sdt[tt], xv);
             const float2 l2 = make_float2(slam[tt], slam[tt]);
             const float2 x2 = make_float2(dtx, dtx);
             const float4* b4 = reinterpret_cast<const float4*>(sB + tt * N) + j;
+            const float4* c4 = reinterpret_cast<const float4*>(cprev) + j;
             float plo[NP], phi[NP];
-#pragma unroll
-            for (int pc = 0; pc < NP; ++pc) {
-                float* sp = s + 16 * pc;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 v = b4[(4 * pc + i) * LPR];
-                    const float2 w0 = mul2(x2, make_float2(v.x, v.y));
-                    const float2 w1 = mul2(x2, make_float2(v.z, v.w));
-                    const float2 u0 = fma2(l2, make_float2(sp[4 * i], sp[4 * i + 1]), w0);
-                    const float2 u1 = fma2(l2, make_float2(sp[4 * i + 2], sp[4 * i + 3]), w1);
-                    sp[4 * i] = u0.x; sp[4 * i + 1] = u0.y;
-                    sp[4 * i + 2] = u1.x; sp[4 * i + 3] = u1.y;
-                }
-                minmax16(sp, plo[pc], phi[pc]);
-            }
-            lo = plo[0];
-            hi = phi[0];
-#pragma unroll
-            for (int pc = 1; pc < NP; ++pc) {
-                lo = fminf(lo, plo[pc]);
-                hi = fmaxf(hi, phi[pc]);
-            }
-            return xv;
-        };
-        // C . s over the lane's entries
-        auto readout = [&](int tt) {
-            const float4* c4 = reinterpret_cast<const float4*>(sC + tt * N) + j;
             float2 accp[NP];
 #pragma unroll
             for (int pc = 0; pc < NP; ++pc) {
-                const float* sp = s + 16 * pc;
+                float* sp = s + 16 * pc;
                 float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float4 v = c4[(4 * pc + i) * LPR];
-                    acc = fma2(make_float2(v.x, v.y), make_float2(sp[4 * i], sp[4 * i + 1]), acc);
-                    acc = fma2(make_float2(v.z, v.w), make_float2(sp[4 * i + 2], sp[4 * i + 3]), acc);
+                    const float4 v = b4[(4 * pc + i) * LPR];
+                    const float2 s0 = make_float2(sp[4 * i], sp[4 * i + 1]);
+                    const float2 s1 = make_float2(sp[4 * i + 2], sp[4 * i + 3]);
+                    if constexpr (READ) {
+                        const float4 cq = c4[(4 * pc + i) * LPR];
+                        acc = fma2(make_float2(cq.x, cq.y), s0, acc);
+                        acc = fma2(make_float2(cq.z, cq.w), s1, acc);
+                    }
+                    float2 u0 = fma2(l2, s0, mul2(x2, make_float2(v.x, v.y)));
+                    float2 u1 = fma2(l2, s1, mul2(x2, make_float2(v.z, v.w)));
+                    if constexpr (kBf16) {
+                        u0 = __bfloat1622float2(__float22bfloat162_rn(u0));
+                        u1 = __bfloat1622float2(__float22bfloat162_rn(u1));
+                    }
+                    sp[4 * i] = u0.x; sp[4 * i + 1] = u0.y;
+                    sp[4 * i + 2] = u1.x; sp[4 * i + 3] = u1.y;
                 }
                 accp[pc] = acc;
+                if constexpr (MINMAX) minmax16(sp, plo[pc], phi[pc]);
             }
-            float2 acc = accp[0];
+            if constexpr (MINMAX) {
+                lo = plo[0];
+                hi = phi[0];
 #pragma unroll
-            for (int pc = 1; pc < NP; ++pc) acc = add2(acc, accp[pc]);
-            return grp_sum<LPR>(__fadd_rn(acc.x, acc.y));
-        };
-        auto emit_y = [&](int tt, float ysum, float xv) {
-            if (ylane) __stcs(yc + (long long)tt * HP, __fadd_rn(ysum, __fmul_rn(Dv, xv)));
+                for (int pc = 1; pc < NP; ++pc) {
+                    lo = fminf(lo, plo[pc]);
+                    hi = fmaxf(hi, phi[pc]);
+                }
+            }
+            if constexpr (READ) {
+                float2 acc = accp[0];
+#pragma unroll
+                for (int pc = 1; pc < NP; ++pc) acc = add2(acc, accp[pc]);
+                yprev = grp_sum<LPR>(__fadd_rn(acc.x, acc.y));
+            }
+            return xv;
         };
         // one token of a quantized row; CODES: also pack the stored codes
         auto qtoken = [&](auto codes_tag, int tt) {
             constexpr bool CODES = decltype(codes_tag)::value;
-            float lo, hi;
-            const float xv = update_q(tt, lo, hi);
+            float lo, hi, yprev = 0.0f;
+            const int t = t0 + tt;
+            float xv;
+            if (t > 0) {
+                xv = update(std::true_type{}, std::true_type{}, tt, lo, hi, yprev);
+                emit_y(t - 1, yprev, xprev);
+            } else {
+                xv = update(std::false_type{}, std::true_type{}, tt, lo, hi, yprev);
+            }
             rp = refit_from_minmax<FMT, LPR>(lo, hi);
             finite_all = finite_all && rp.finite;
             uint32_t kc[16];
@@ -345,34 +389,22 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
                     if constexpr (CODES) pack16<FMT>(kc, cw + PW * pc);
                 }
             }
-            emit_y(tt, readout(tt), xv);
+            cprev = sC + tt * N;
+            xprev = xv;
         };
         // one token of an fp row (fp32 update, rounded to bf16 for bf16)
         auto ftoken = [&](int tt) {
-            const float xv = sx[tt * rows + rowe];
-            const float dtx = __fmul_rn(sdt[tt], xv);
-            const float2 l2 = make_float2(slam[tt], slam[tt]);
-            const float2 x2 = make_float2(dtx, dtx);
-            const float4* b4 = reinterpret_cast<const float4*>(sB + tt * N) + j;
-#pragma unroll
-            for (int pc = 0; pc < NP; ++pc) {
-                float* sp = s + 16 * pc;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 v = b4[(4 * pc + i) * LPR];
-                    const float2 w0 = mul2(x2, make_float2(v.x, v.y));
-                    const float2 w1 = mul2(x2, make_float2(v.z, v.w));
-                    float2 u0 = fma2(l2, make_float2(sp[4 * i], sp[4 * i + 1]), w0);
-                    float2 u1 = fma2(l2, make_float2(sp[4 * i + 2], sp[4 * i + 3]), w1);
-                    if constexpr (kBf16) {
-                        u0 = __bfloat1622float2(__float22bfloat162_rn(u0));
-                        u1 = __bfloat1622float2(__float22bfloat162_rn(u1));
-                    }
-                    sp[4 * i] = u0.x; sp[4 * i + 1] = u0.y;
-                    sp[4 * i + 2] = u1.x; sp[4 * i + 3] = u1.y;
-                }
+            float lo, hi, yprev = 0.0f;
+            const int t = t0 + tt;
+            float xv;
+            if (t > 0) {
+                xv = update(std::true_type{}, std::false_type{}, tt, lo, hi, yprev);
+                emit_y(t - 1, yprev, xprev);
+            } else {
+                xv = update(std::false_type{}, std::false_type{}, tt, lo, hi, yprev);
             }
-            emit_y(tt, readout(tt), xv);
+            cprev = sC + tt * N;
+            xprev = xv;
         };
 
         bool qdone = false;
@@ -388,6 +420,8 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
         if (!qdone)
             for (int tt = 0; tt < nt; ++tt) ftoken(tt);
     }
+    // the readout of the last token
+    emit_y(T - 1, readout(cprev), xprev);
 
     // The final state back to the pool.
     if (!active) return;
@@ -429,7 +463,7 @@ cudaError_t launch_scan_ne(const PoolView& pv, const CallView& cv, int warps, in
 {
     using SG = SGeom<N, E>;
     const size_t smem =
-        2 * (size_t)scan_buf_floats(N, cv.scan_chunk, warps * SG::RPW) * sizeof(float);
+        kScanBufs * (size_t)scan_buf_floats(N, cv.scan_chunk, warps * SG::RPW) * sizeof(float);
     auto kern = scan_kernel<FMT, N, E>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -482,7 +516,7 @@ ScanPlan scan_plan(int d_state, int headdim, long long batch_heads, int sms)
     // Tokens per staged chunk: two buffers of B and C of K tokens stay near
     // 16 KB per CTA.
     sp.chunk = N <= 128 ? 8 : 4;
-    sp.smem_bytes = 2 * (size_t)scan_buf_floats(N, sp.chunk, sp.rows) * sizeof(float);
+    sp.smem_bytes = kScanBufs * (size_t)scan_buf_floats(N, sp.chunk, sp.rows) * sizeof(float);
     return sp;
 }
 
