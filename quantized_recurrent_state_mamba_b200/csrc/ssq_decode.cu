@@ -164,7 +164,6 @@ __device__ __forceinline__ void sts128f(unsigned a, float4 v)
 
 __host__ __device__ inline int r16(int v) { return (v + 15) & ~15; }
 __host__ __device__ inline int r256(int v) { return (v + 255) & ~255; }
-__host__ __device__ inline int r128(int v) { return (v + 127) & ~127; }
 
 // ---- tile sequence -----------------------------------------------------
 // Tiles are ordered (layer, request, region, row block).  A CTA walks a

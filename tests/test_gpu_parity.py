@@ -399,11 +399,11 @@ def test_scan_groups_and_ragged_tiles(fmt):
 
 def _wide_scan_batch(H, P, N):
     """Requests that make the scan give each lane 64 entries of a row: at
-    least three warps per SM sub-partition at 32 / (N / 64) rows per warp."""
+    least one warp per SM sub-partition at 32 / (N / 64) rows per warp."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     rpw = 32 // (N // 64)
     per_request = H * -(-P // rpw)
-    return -(-3 * 4 * sms // per_request)
+    return -(-4 * sms // per_request)
 
 
 @pytest.mark.parametrize("fmt,H,N", [("i8a", 32, 128), ("i4s", 32, 128), ("bf16", 32, 128),
