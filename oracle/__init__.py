@@ -231,6 +231,22 @@ def scan(cfg: Cfg, st: State, i, x, B, C, dt, A, D):
     return y
 
 
+def prefill(cfg: Cfg, st: State, i, x, B, C, dt, A, D):
+    """Prefill hand-off on state pair i: T tokens of the fp32 recurrence with
+    no rounding between tokens, y from the fp32 state, one quantization of
+    the final state.  x[T][H][P], B/C[T][G][N], dt[T][H]."""
+    x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))
+    T = x.shape[0]
+    y = np.zeros((T, cfg.nheads, cfg.headdim), np.float32)
+    c = cfg.c()
+    lib().oref_prefill(ctypes.byref(c), ctypes.byref(st.c(i)), T,
+                       _p(x, ctypes.c_float), _p(B, ctypes.c_float),
+                       _p(C, ctypes.c_float), _p(dt, ctypes.c_float),
+                       _p(A, ctypes.c_float), _p(D, ctypes.c_float),
+                       _p(y, ctypes.c_float))
+    return y
+
+
 def scan_f64(cfg: Cfg, S0, x, B, C, dt, A, D):
     """Unquantized fp64 trajectory from S0[H][P][N]; returns (S_T, y[T])."""
     x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))

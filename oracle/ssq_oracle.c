@@ -306,6 +306,65 @@ void oref_scan(const oref_cfg* c, oref_state* st, int T, const float* x,
     }
 }
 
+/* Prefill hand-off ("Mamba state quantization for inference", phase-aware
+ * benchmarks: prefill computes in FP32 and writes its final state into the
+ * packed cache): from the stored state, T tokens of the fp32 recurrence
+ * s'_n = fma(lambda, s_n, fl(dt*x) * B_n) with no rounding between tokens,
+ * y_t read from the fp32 state (accumulated in double), and the state
+ * quantized (or stored, bf16-rounded for the bf16 format) once after the
+ * last token.  x[T][H][P], B/C[T][G][N], dt[T][H], A/D[H], y[T][H][P]. */
+void oref_prefill(const oref_cfg* c, oref_state* st, int T, const float* x,
+                  const float* B, const float* C, const float* dt,
+                  const float* A, const float* D, float* y)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state, G = c->ngroups;
+    const int hpg = H / G;
+    const size_t HP = (size_t)H * P;
+    const size_t GN = (size_t)G * N;
+    float* s = (float*)malloc(sizeof(float) * (size_t)N);
+    for (int h = 0; h < H; ++h) {
+        const int g = h / hpg;
+        const int quant = oref_row_is_quant(c, h);
+        for (int p = 0; p < P; ++p) {
+            const size_t r = (size_t)h * P + p;
+            /* the stored state, decoded once */
+            if (quant) {
+                oref_dequantize_row(c->fmt, N, st->q + r * N, st->delta[r],
+                                    st->zero[r], s);
+            } else {
+                memcpy(s, st->val + r * N, sizeof(float) * (size_t)N);
+            }
+            for (int t = 0; t < T; ++t) {
+                const float lam = oref_lambda(dt[(size_t)t * H + h], A[h]);
+                const float* Bg = B + t * GN + (size_t)g * N;
+                const float* Cg = C + t * GN + (size_t)g * N;
+                const float xv = x[t * HP + r];
+                const float dtx = dt[(size_t)t * H + h] * xv;
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    float w = dtx * Bg[n];
+                    s[n] = fmaf(lam, s[n], w);
+                    acc += (double)Cg[n] * (double)s[n];
+                }
+                acc += (double)D[h] * (double)xv;
+                y[t * HP + r] = (float)acc;
+            }
+            /* the hand-off: one refit and rounding of the final state */
+            if (quant) {
+                oref_quantize_row(c->fmt, N, s, st->q + r * N, st->delta + r,
+                                  st->zero + r);
+            } else {
+                for (int n = 0; n < N; ++n) {
+                    float v = s[n];
+                    if (c->fmt == OREF_BF16) v = oref_bf16_round(v);
+                    st->val[r * N + n] = v;
+                }
+            }
+        }
+    }
+    free(s);
+}
+
 /* Unquantized trajectory in double, used only to report drift: the exact
  * recurrence S_t = A_t S_(t-1) + W_t of "Mamba state quantization for
  * inference" (no residual R_t), with lambda = exp(dt*A) and W = dt*B(x)x,

@@ -101,6 +101,10 @@ void  oref_scan(const oref_cfg* c, oref_state* st, int T, const float* x,
                 const float* B, const float* C, const float* dt,
                 const float* A, const float* D, float* y);
 
+void  oref_prefill(const oref_cfg* c, oref_state* st, int T, const float* x,
+                   const float* B, const float* C, const float* dt,
+                   const float* A, const float* D, float* y);
+
 void  oref_scan_f64(const oref_cfg* c, double* S, int T, const float* x,
                     const float* B, const float* C, const float* dt,
                     const float* A, const float* D, double* y);

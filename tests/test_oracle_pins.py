@@ -503,3 +503,90 @@ def test_output_read_from_quantized_state(oref, fmt):
     sf = O.state_from_f32(cf, Sdeq)
     y_f = O.step(cf, sf, 0, x, B, C, dt, A, D)
     assert np.max(np.abs(y_f - y) / scale) > 1e-5
+
+
+# ---------------------------------------------------------------------------
+# Prefill hand-off ("Mamba state quantization for inference", phase-aware
+# benchmarks: prefill in FP32, then the final state written into the packed
+# cache)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [O.F32] + QFMTS)
+def test_prefill_matches_unrolled_closed_form(oref, fmt):
+    """T=64 tokens of the prefill from an N(0,1) state: every y_t equals the
+    unrolled fp64 recurrence within 1e-5 normwise (y is read from the fp32
+    state, not the codes), and the stored state is the closed-form S_T
+    quantized once: within half a step of S_T per entry (fp32 format: within
+    1e-5 normwise)."""
+    G, H, P, N, T = 2, 4, 8, 16, 64
+    wl = W.Scan("pin", seed=6, batch=1, T=T, nheads=H, headdim=P,
+                d_state=N, ngroups=G, fmt="f32")
+    inp = wl.inputs()
+    x, B, C, dt = (inp[k][0] for k in ("x", "B", "C", "dt"))
+    A, D = inp["A"], inp["D"]
+    S0 = W.state_pair(6, 0, 0, H * P, N).reshape(H, P, N)
+    # the starting state is what the pool holds: S0 in the target format
+    cfg = O.Cfg(fmt, H, P, N, G)
+    st = O.state_from_f32(cfg, S0)
+    S0_stored = O.state_to_f32(st)[0]
+    y = O.prefill(cfg, st, 0, x, B, C, dt, A, D)
+    S_ref, y_ref = _closed_form(S0_stored, x, B, C, dt, A, D, G)
+    for t in range(T):
+        assert np.linalg.norm(y[t] - y_ref[t]) <= 1e-5 * np.linalg.norm(y_ref[t]) + 1e-6
+    S_T = O.state_to_f32(st)[0]
+    if fmt == O.F32:
+        assert np.linalg.norm(S_T - S_ref) <= 1e-5 * np.linalg.norm(S_ref)
+    else:
+        half = st.delta[0].reshape(H, P, 1) / 2
+        rng = np.abs(S_ref).max(axis=-1, keepdims=True)
+        assert np.all(np.abs(S_T - S_ref) <= half * (1 + 1e-3) + 1e-5 * rng)
+
+
+@pytest.mark.parametrize("fmt", QFMTS)
+def test_prefill_one_token_from_zero(oref, fmt):
+    """One token from the zero state: the fp32 state is w = fl(dt x) B
+    exactly, so the stored codes are the quantizer applied to that row and
+    y = (dt x)(C . B) + D x within fp64 accumulation of fp32 terms."""
+    H, P, N = 4, 8, 16
+    wl = W.Scan("pin", seed=10, batch=1, T=1, nheads=H, headdim=P,
+                d_state=N, ngroups=1, fmt="f32")
+    inp = wl.inputs()
+    x, B, C, dt = (inp[k][0] for k in ("x", "B", "C", "dt"))
+    A, D = inp["A"], inp["D"]
+    cfg = O.Cfg(fmt, H, P, N, 1)
+    st = O.State(cfg)
+    y = O.prefill(cfg, st, 0, x, B, C, dt, A, D)
+    for h in range(H):
+        for p in range(P):
+            dtx = np.float32(dt[0, h]) * np.float32(x[0, h, p])
+            w = (dtx * B[0, 0]).astype(np.float32)
+            q, d, z, _ = O.quantize_row(fmt, w)
+            r = h * P + p
+            assert np.array_equal(st.q[0, r], q)
+            assert st.delta[0, r] == d and st.zero[0, r] == z
+            yref = float(np.dot(C[0, 0].astype(np.float64), w.astype(np.float64))) \
+                + float(D[h]) * float(x[0, h, p])
+            assert abs(float(y[0, h, p]) - yref) <= 1e-6 * (abs(yref) + 1.0)
+
+
+def test_prefill_closer_to_exact_than_rounding_every_token(oref):
+    """The point of the FP32 prefill: over T=256 tokens its final state is
+    nearer the exact trajectory than the per-token rounded scan (int4, where
+    the per-step rounding error is large): no worse on any head (a fast-
+    decaying head forgets all but the last rounding either way) and clearly
+    better on average."""
+    H, P, N, T = 4, 8, 32, 256
+    wl = W.Scan("pin", seed=12, batch=1, T=T, nheads=H, headdim=P,
+                d_state=N, ngroups=1, fmt="f32")
+    inp = wl.inputs()
+    x, B, C, dt = (inp[k][0] for k in ("x", "B", "C", "dt"))
+    A, D = inp["A"], inp["D"]
+    cfg = O.Cfg(O.I4_ASYM, H, P, N, 1)
+    st_p, st_s = O.State(cfg), O.State(cfg)
+    O.prefill(cfg, st_p, 0, x, B, C, dt, A, D)
+    O.scan(cfg, st_s, 0, x, B, C, dt, A, D)
+    S64, _ = O.scan_f64(cfg, np.zeros((H, P, N)), x, B, C, dt, A, D)
+    ep = np.abs(O.state_to_f32(st_p)[0] - S64).reshape(H, -1).mean(axis=1)
+    es = np.abs(O.state_to_f32(st_s)[0] - S64).reshape(H, -1).mean(axis=1)
+    assert np.all(ep <= es * 1.01), (ep, es)
+    assert ep.mean() < 0.9 * es.mean(), (ep, es)
