@@ -45,6 +45,7 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 SM_MAX_MHZ = 1965.0        # B200 maximum SM clock, used when NVML is unavailable
 SCAN_FP32_OPS = 6          # algorithmic fp32 operations per element-token of the scan
+PREFILL_FP32_OPS = 3       # ... of the prefill hand-off: w = dtx*B, the fma, C*s
 
 
 # ---------------------------------------------------------------------------
@@ -69,6 +70,8 @@ def workload(name):
         "sweep_i4a": lambda: W.sweep_serving("i4a"),
         "scan_370m_all": lambda: W.scan_370m("all"),
         "scan_370m_mid": lambda: W.scan_370m("mid"),
+        "prefill_370m_all": lambda: W.scan_370m("all"),
+        "prefill_370m_mid": lambda: W.scan_370m("mid"),
     }
     if name not in table:
         raise SystemExit(f"unknown workload {name}; choose from {sorted(table)}")
@@ -289,16 +292,17 @@ def oracle_decode_sample(wl, budget_s):
     return sec, per_pair * npairs, npairs
 
 
-def oracle_scan_sample(wl, budget_s):
+def oracle_scan_sample(wl, budget_s, prefill=False):
     import oracle as O
     H, P, N = wl.nheads, wl.headdim, wl.d_state
     inp = wl.inputs()
     ocfg = O.Cfg(O.FORMATS[wl.fmt], H, P, N, wl.ngroups, wl.head_mask)
     t = time.perf_counter()
     st = O.State(ocfg, 1)
+    run = O.prefill if prefill else O.scan
     T1 = min(wl.T, 8)
-    O.scan(ocfg, st, 0, inp["x"][0, :T1], inp["B"][0, :T1], inp["C"][0, :T1],
-           inp["dt"][0, :T1], inp["A"], inp["D"])
+    run(ocfg, st, 0, inp["x"][0, :T1], inp["B"][0, :T1], inp["C"][0, :T1],
+        inp["dt"][0, :T1], inp["A"], inp["D"])
     per_tok = max((time.perf_counter() - t) / T1, 1e-6)
     ntok = int(max(1, min(wl.T * wl.batch, budget_s / per_tok)))
     st = O.State(ocfg, 1)
@@ -306,8 +310,8 @@ def oracle_scan_sample(wl, budget_s):
     t = time.perf_counter()
     while done < ntok:
         n = min(wl.T, ntok - done)
-        O.scan(ocfg, st, 0, inp["x"][b, :n], inp["B"][b, :n], inp["C"][b, :n],
-               inp["dt"][b, :n], inp["A"], inp["D"])
+        run(ocfg, st, 0, inp["x"][b, :n], inp["B"][b, :n], inp["C"][b, :n],
+            inp["dt"][b, :n], inp["A"], inp["D"])
         done += n
         b = (b + 1) % wl.batch
     sec = time.perf_counter() - t
@@ -315,10 +319,12 @@ def oracle_scan_sample(wl, budget_s):
     return sec, scan_bytes(wl) * frac, ntok
 
 
-def cpu_leg(wl, budget_s):
+def cpu_leg(wl, budget_s, name=""):
     if isinstance(wl, W.Scan):
-        sec, nbytes, n = oracle_scan_sample(wl, budget_s)
-        sample = f"{n} request-tokens of the scan (request 0 onward), single thread"
+        pf = name.startswith("prefill")
+        sec, nbytes, n = oracle_scan_sample(wl, budget_s, prefill=pf)
+        sample = (f"{n} request-tokens of the {'prefill' if pf else 'scan'} "
+                  f"(request 0 onward), single thread")
         rsps = n / sec
     else:
         sec, nbytes, n = oracle_decode_sample(wl, budget_s)
@@ -337,10 +343,10 @@ def run_reference(args, wl, name):
     steps, warm = args.steps, args.warmup
     budget = max(0.5, 120.0 / max(1, steps + warm))
     for _ in range(warm):
-        cpu_leg(wl, budget)
+        cpu_leg(wl, budget, name)
     vals, secs = [], 0.0
     for _ in range(steps):
-        r = cpu_leg(wl, budget)
+        r = cpu_leg(wl, budget, name)
         vals.append(r["value"])
         secs += r["seconds"]
     value = statistics.mean(vals)
@@ -398,13 +404,16 @@ def run_ours(args, wl, name):
                                   torch.from_numpy(S).to(dev))
         torch.cuda.synchronize()
 
+    # the prefill hand-off runs the scan's shape with the state in fp32
+    # between tokens and one quantization at the end
+    scan_fn = ssq.ssq_prefill if name.startswith("prefill") else ssq.ssq_scan
     if is_scan:
         y = torch.empty((wl.batch, wl.T, H, P), device=dev)
         nbytes = scan_bytes(wl)
 
         def step():
-            ssq.ssq_scan(cfg, pool, None, wl.batch, 0, wl.T, d["x"], d["B"], d["C"], d["dt"],
-                         d["A"], d["D"], y)
+            scan_fn(cfg, pool, None, wl.batch, 0, wl.T, d["x"], d["B"], d["C"], d["dt"],
+                    d["A"], d["D"], y)
         units = wl.batch * wl.T          # request-tokens
     else:
         y = torch.empty((wl.nl, wl.batch, H, P), device=dev)
@@ -479,8 +488,8 @@ def run_ours(args, wl, name):
             s_c.wait_event(ev_out[kk])
         t = din[kk]
         if is_scan:
-            ssq.ssq_scan(cfg, pool, None, wl.batch, 0, wl.T, t["x"], t["B"], t["C"], t["dt"],
-                         d["A"], d["D"], yb[kk], stream=s_c)
+            scan_fn(cfg, pool, None, wl.batch, 0, wl.T, t["x"], t["B"], t["C"], t["dt"],
+                    d["A"], d["D"], yb[kk], stream=s_c)
         else:
             ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, t["x"], t["B"], t["C"],
                                 t["dt"], d["A"], d["D"], yb[kk], stream=s_c)
@@ -523,7 +532,8 @@ def run_ours(args, wl, name):
         # fma(s', inv, M) and -M (round the exact product to nearest),
         # r*Delta, C*r = 6.
         # Peak: 148 SMs x 128 FP32 lanes x the maximum SM clock.
-        ops = SCAN_FP32_OPS * elem_steps(wl)
+        ops = (PREFILL_FP32_OPS if name.startswith("prefill") else SCAN_FP32_OPS) \
+            * elem_steps(wl)
         sm_max = clocks.get("sm_max_mhz") or SM_MAX_MHZ
         alu_peak = 148 * 128 * sm_max * 1e6 / 1e12
         alu_ach = ops / (kern_ms / 1e3) / 1e12
@@ -563,7 +573,7 @@ def run_ours(args, wl, name):
         "device_error_word": err,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_leg(wl, args.cpu_budget)
+        out["cpu_baseline"] = cpu_leg(wl, args.cpu_budget, name)
     if rank == 0:
         print(json.dumps(out))
     if world > 1:

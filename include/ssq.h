@@ -237,6 +237,22 @@ SSQ_API ssq_status ssq_scan(const ssq_config* cfg, void* pool,
                     const float* dt, const float* A, const float* D,
                     float* y, cudaStream_t stream);
 
+/* Prefill hand-off ("Mamba state quantization for inference", phase-aware
+ * benchmarks: prefill computes in FP32 and writes its final state into the
+ * packed cache).  T tokens of one layer from the stored state with the
+ * recurrence in fp32 and no rounding between tokens; y_t is read from the
+ * fp32 state; after the last token the state is refit and quantized once
+ * (quantized heads; fp heads are stored as fp32, or rounded to bf16 for
+ * SSQ_BF16) and written to the pool.  Arguments, layouts, ownership and
+ * errors as ssq_scan.  A fresh request starts from a zero slot
+ * (ssq_pool_init, or ssq_quantize_rows of zeros); a chunked prefill passes
+ * each chunk in turn (the state is requantized between chunks). */
+SSQ_API ssq_status ssq_prefill(const ssq_config* cfg, void* pool,
+                       const int32_t* slot_idx, int batch, int layer, int T,
+                       const float* x, const float* B, const float* C,
+                       const float* dt, const float* A, const float* D,
+                       float* y, cudaStream_t stream);
+
 /* Static string for a status code. */
 SSQ_API const char* ssq_status_string(ssq_status s);
 

@@ -329,10 +329,16 @@ ssq_status ssq_decode_step(const ssq_config* cfg, void* pool, const int32_t* slo
     return SSQ_OK;
 }
 
-ssq_status ssq_scan(const ssq_config* cfg, void* pool, const int32_t* slot_idx, int batch,
-                    int layer, int T, const float* x, const float* B, const float* C,
-                    const float* dt, const float* A, const float* D, float* y,
-                    cudaStream_t stream)
+}  // extern "C"
+
+namespace {
+
+// ssq_scan and ssq_prefill: the same launch geometry; prefill keeps the state
+// fp32 across the tokens and quantizes it once at the end.
+ssq_status scan_common(const ssq_config* cfg, void* pool, const int32_t* slot_idx, int batch,
+                       int layer, int T, const float* x, const float* B, const float* C,
+                       const float* dt, const float* A, const float* D, float* y,
+                       bool prefill, cudaStream_t stream)
 {
     ssq::PoolView pv;
     ssq_layout L;
@@ -372,9 +378,31 @@ ssq_status ssq_scan(const ssq_config* cfg, void* pool, const int32_t* slot_idx, 
     cv.qtiles = pv.Hq * sp.tiles_per_head;
     cv.ftiles = pv.Hf * sp.tiles_per_head;
     cv.total_tiles = (long long)batch * (cv.qtiles + cv.ftiles);
-    e = ssq::launch_scan(pv, cv, (int)cfg->fmt, sp, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    e = ssq::launch_scan(pv, cv, (int)cfg->fmt, sp, prefill, stream);
+    if (e != cudaSuccess) return cuda_fail(e, prefill ? "prefill launch" : "scan launch");
     return SSQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ssq_status ssq_scan(const ssq_config* cfg, void* pool, const int32_t* slot_idx, int batch,
+                    int layer, int T, const float* x, const float* B, const float* C,
+                    const float* dt, const float* A, const float* D, float* y,
+                    cudaStream_t stream)
+{
+    return scan_common(cfg, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y, false,
+                       stream);
+}
+
+ssq_status ssq_prefill(const ssq_config* cfg, void* pool, const int32_t* slot_idx, int batch,
+                       int layer, int T, const float* x, const float* B, const float* C,
+                       const float* dt, const float* A, const float* D, float* y,
+                       cudaStream_t stream)
+{
+    return scan_common(cfg, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y, true,
+                       stream);
 }
 
 }  // extern "C"

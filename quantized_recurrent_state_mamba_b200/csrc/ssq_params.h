@@ -61,8 +61,10 @@ struct ScanPlan {
     size_t smem_bytes;
 };
 ScanPlan scan_plan(int d_state, int headdim, long long batch_heads, int sms);
+// prefill: keep the state fp32 over all T tokens and quantize it once at
+// the end (the prefill hand-off) instead of rounding at every token.
 cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt, const ScanPlan& sp,
-                        cudaStream_t stream);
+                        bool prefill, cudaStream_t stream);
 
 // Rows per decode tile in the quantized and the fp region.
 void decode_tile_rows(int fmt, int d_state, int* rows_q, int* rows_f);

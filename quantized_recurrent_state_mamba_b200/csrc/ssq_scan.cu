@@ -130,7 +130,9 @@ __device__ __forceinline__ void round_piece_slow(const RowParams& rp, float* s,
     }
 }
 
-template <int FMT, int N, int E>
+// PF (prefill hand-off): the state stays fp32 for all T tokens (y read from
+// it) and is quantized, or bf16-rounded, once after the last token.
+template <int FMT, int N, int E, bool PF>
 __global__ void __launch_bounds__(64, E >= 64 ? 6 : 8)
 scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv)
 {
@@ -334,7 +336,7 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
                     }
                     float2 u0 = fma2(l2, s0, mul2(x2, make_float2(v.x, v.y)));
                     float2 u1 = fma2(l2, s1, mul2(x2, make_float2(v.z, v.w)));
-                    if constexpr (kBf16) {
+                    if constexpr (kBf16 && !PF) {
                         u0 = __bfloat1622float2(__float22bfloat162_rn(u0));
                         u1 = __bfloat1622float2(__float22bfloat162_rn(u1));
                     }
@@ -408,7 +410,7 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
         };
 
         bool qdone = false;
-        if constexpr (F::quant) {
+        if constexpr (F::quant && !PF) {
             if (qrow) {
                 qdone = true;
                 // the final token also packs the codes that go back to the pool
@@ -422,6 +424,37 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
     }
     // the readout of the last token
     emit_y(T - 1, readout(cprev), xprev);
+
+    if constexpr (PF && F::quant) {
+        // the hand-off: one refit and rounding of the final fp32 state (all
+        // lanes of the warp take part in the row reductions)
+        if (qrow) {
+            float lo = s[0], hi = s[0];
+#pragma unroll
+            for (int pc = 0; pc < NP; ++pc) {
+                float plo, phi;
+                minmax16(s + 16 * pc, plo, phi);
+                lo = fminf(lo, plo);
+                hi = fmaxf(hi, phi);
+            }
+            rp = refit_from_minmax<FMT, LPR>(lo, hi);
+            finite_all = rp.finite;
+            uint32_t kc[16];
+            if (__all_sync(0xffffffffu, rp.fast && !rp.clamp)) {
+#pragma unroll
+                for (int pc = 0; pc < NP; ++pc) {
+                    round_piece_fast<FMT, true>(rp, s + 16 * pc, kc);
+                    pack16<FMT>(kc, cw + PW * pc);
+                }
+            } else {
+#pragma unroll
+                for (int pc = 0; pc < NP; ++pc) {
+                    round_piece_slow<FMT>(rp, s + 16 * pc, kc);
+                    pack16<FMT>(kc, cw + PW * pc);
+                }
+            }
+        }
+    }
 
     // The final state back to the pool.
     if (!active) return;
@@ -457,14 +490,14 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
     }
 }
 
-template <int FMT, int N, int E>
+template <int FMT, int N, int E, bool PF>
 cudaError_t launch_scan_ne(const PoolView& pv, const CallView& cv, int warps, int grid,
                            cudaStream_t st)
 {
     using SG = SGeom<N, E>;
     const size_t smem =
         kScanBufs * (size_t)scan_buf_floats(N, cv.scan_chunk, warps * SG::RPW) * sizeof(float);
-    auto kern = scan_kernel<FMT, N, E>;
+    auto kern = scan_kernel<FMT, N, E, PF>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -474,22 +507,37 @@ cudaError_t launch_scan_ne(const PoolView& pv, const CallView& cv, int warps, in
     return cudaGetLastError();
 }
 
-template <int FMT>
+template <int FMT, bool PF>
 cudaError_t launch_scan_fmt(const PoolView& pv, const CallView& cv, int E, int warps,
                             int grid, cudaStream_t st)
 {
     switch (pv.N) {
-    case 16: return launch_scan_ne<FMT, 16, 16>(pv, cv, warps, grid, st);
-    case 32: return launch_scan_ne<FMT, 32, 32>(pv, cv, warps, grid, st);
+    case 16: return launch_scan_ne<FMT, 16, 16, PF>(pv, cv, warps, grid, st);
+    case 32: return launch_scan_ne<FMT, 32, 32, PF>(pv, cv, warps, grid, st);
     case 64:
-        return E == 64 ? launch_scan_ne<FMT, 64, 64>(pv, cv, warps, grid, st)
-                       : launch_scan_ne<FMT, 64, 32>(pv, cv, warps, grid, st);
+        return E == 64 ? launch_scan_ne<FMT, 64, 64, PF>(pv, cv, warps, grid, st)
+                       : launch_scan_ne<FMT, 64, 32, PF>(pv, cv, warps, grid, st);
     case 128:
-        return E == 64 ? launch_scan_ne<FMT, 128, 64>(pv, cv, warps, grid, st)
-                       : launch_scan_ne<FMT, 128, 32>(pv, cv, warps, grid, st);
+        return E == 64 ? launch_scan_ne<FMT, 128, 64, PF>(pv, cv, warps, grid, st)
+                       : launch_scan_ne<FMT, 128, 32, PF>(pv, cv, warps, grid, st);
     case 256:
-        return E == 64 ? launch_scan_ne<FMT, 256, 64>(pv, cv, warps, grid, st)
-                       : launch_scan_ne<FMT, 256, 32>(pv, cv, warps, grid, st);
+        return E == 64 ? launch_scan_ne<FMT, 256, 64, PF>(pv, cv, warps, grid, st)
+                       : launch_scan_ne<FMT, 256, 32, PF>(pv, cv, warps, grid, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <bool PF>
+cudaError_t launch_scan_pf(const PoolView& pv, const CallView& cv, int fmt, int E, int w,
+                           int g, cudaStream_t st)
+{
+    switch (fmt) {
+    case SSQ_F32: return launch_scan_fmt<SSQ_F32, PF>(pv, cv, E, w, g, st);
+    case SSQ_BF16: return launch_scan_fmt<SSQ_BF16, PF>(pv, cv, E, w, g, st);
+    case SSQ_I8_SYM: return launch_scan_fmt<SSQ_I8_SYM, PF>(pv, cv, E, w, g, st);
+    case SSQ_I8_ASYM: return launch_scan_fmt<SSQ_I8_ASYM, PF>(pv, cv, E, w, g, st);
+    case SSQ_I4_SYM: return launch_scan_fmt<SSQ_I4_SYM, PF>(pv, cv, E, w, g, st);
+    case SSQ_I4_ASYM: return launch_scan_fmt<SSQ_I4_ASYM, PF>(pv, cv, E, w, g, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -523,21 +571,14 @@ ScanPlan scan_plan(int d_state, int headdim, long long batch_heads, int sms)
 }
 
 cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt, const ScanPlan& sp,
-                        cudaStream_t st)
+                        bool prefill, cudaStream_t st)
 {
     const long long grid = (long long)cv.batch * (cv.qtiles + cv.ftiles);
     if (grid <= 0) return cudaSuccess;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int g = (int)grid, E = sp.E, w = sp.warps;
-    switch (fmt) {
-    case SSQ_F32: return launch_scan_fmt<SSQ_F32>(pv, cv, E, w, g, st);
-    case SSQ_BF16: return launch_scan_fmt<SSQ_BF16>(pv, cv, E, w, g, st);
-    case SSQ_I8_SYM: return launch_scan_fmt<SSQ_I8_SYM>(pv, cv, E, w, g, st);
-    case SSQ_I8_ASYM: return launch_scan_fmt<SSQ_I8_ASYM>(pv, cv, E, w, g, st);
-    case SSQ_I4_SYM: return launch_scan_fmt<SSQ_I4_SYM>(pv, cv, E, w, g, st);
-    case SSQ_I4_ASYM: return launch_scan_fmt<SSQ_I4_ASYM>(pv, cv, E, w, g, st);
-    default: return cudaErrorInvalidValue;
-    }
+    return prefill ? launch_scan_pf<true>(pv, cv, fmt, E, w, g, st)
+                   : launch_scan_pf<false>(pv, cv, fmt, E, w, g, st);
 }
 
 }  // namespace ssq

@@ -69,8 +69,9 @@ _lib.ssq_quantize_rows.argtypes = [_CFG, _P, _P, _I, _I, _I, _P, _P]
 _lib.ssq_dequantize_rows.argtypes = [_CFG, _P, _P, _I, _I, _I, _P, _P]
 _lib.ssq_decode_step.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
 _lib.ssq_scan.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
+_lib.ssq_prefill.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
 for _f in ("ssq_pool_layout", "ssq_pool_init", "ssq_pool_error", "ssq_quantize_rows",
-           "ssq_dequantize_rows", "ssq_decode_step", "ssq_scan"):
+           "ssq_dequantize_rows", "ssq_decode_step", "ssq_scan", "ssq_prefill"):
     getattr(_lib, _f).restype = _I
 
 
@@ -209,6 +210,20 @@ def ssq_scan(cfg: Config, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y,
     H, P, N, G = cfg.nheads, cfg.headdim, cfg.d_state, cfg.ngroups
     f = torch.float32
     _check(_lib.ssq_scan(
+        cfg.ref, _pool_ptr(cfg, pool), _slots(slot_idx, batch), batch, layer, T,
+        _ptr(x, "x", f, batch * T * H * P), _ptr(B, "B", f, batch * T * G * N),
+        _ptr(C, "C", f, batch * T * G * N), _ptr(dt, "dt", f, batch * T * H),
+        _ptr(A, "A", f, H), _ptr(D, "D", f, H), _ptr(y, "y", f, batch * T * H * P),
+        _stream(stream)))
+
+
+def ssq_prefill(cfg: Config, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y,
+                stream=None):
+    """Prefill hand-off: T tokens of one layer in fp32, the final state
+    quantized once.  Layouts as ssq_scan."""
+    H, P, N, G = cfg.nheads, cfg.headdim, cfg.d_state, cfg.ngroups
+    f = torch.float32
+    _check(_lib.ssq_prefill(
         cfg.ref, _pool_ptr(cfg, pool), _slots(slot_idx, batch), batch, layer, T,
         _ptr(x, "x", f, batch * T * H * P), _ptr(B, "B", f, batch * T * G * N),
         _ptr(C, "C", f, batch * T * G * N), _ptr(dt, "dt", f, batch * T * H),
