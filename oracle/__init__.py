@@ -71,6 +71,8 @@ def lib():
         _lib.oref_lambda.argtypes = [ctypes.c_float, ctypes.c_float]
         _lib.oref_bf16_round.restype = ctypes.c_float
         _lib.oref_bf16_round.argtypes = [ctypes.c_float]
+        _lib.oref_sr_u16.restype = ctypes.c_uint32
+        _lib.oref_sr_u16.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     return _lib
 
 
@@ -228,6 +230,71 @@ def scan(cfg: Cfg, st: State, i, x, B, C, dt, A, D):
                     _p(C, ctypes.c_float), _p(dt, ctypes.c_float),
                     _p(A, ctypes.c_float), _p(D, ctypes.c_float),
                     _p(y, ctypes.c_float))
+    return y
+
+
+class _SR(ctypes.Structure):
+    _fields_ = [("seed", ctypes.c_uint64), ("step", ctypes.c_uint32),
+                ("layer", ctypes.c_uint32), ("slot", ctypes.c_uint32)]
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32-10 of a 4-word counter and 2-word key (uint32 each)."""
+    c = (ctypes.c_uint32 * 4)(*[int(v) & 0xFFFFFFFF for v in ctr])
+    k = (ctypes.c_uint32 * 2)(*[int(v) & 0xFFFFFFFF for v in key])
+    out = (ctypes.c_uint32 * 4)()
+    lib().oref_philox4x32_10(c, k, out)
+    return [int(v) for v in out]
+
+
+def sr_draws(seed, step, layer, slot, rows, N):
+    """The 16-bit draws of every entry of `rows` rows: uint32 [rows][N]."""
+    r = _SR(seed, step, layer, slot)
+    u = np.zeros((rows, N), np.uint32)
+    for row in range(rows):
+        for n in range(N):
+            u[row, n] = lib().oref_sr_u16(ctypes.byref(r), row, n, N)
+    return u
+
+
+def quantize_row_sr(fmt, v, u16):
+    """Refit one row and round it stochastically with the given 16-bit
+    draws.  Returns (codes, delta, zero)."""
+    v = _f32(v)
+    N = v.shape[0]
+    u = np.ascontiguousarray(u16, dtype=np.uint32)
+    q = np.zeros(N, np.int32)
+    d = ctypes.c_float()
+    z = ctypes.c_float()
+    lib().oref_quantize_row_sr(fmt, N, _p(v, ctypes.c_float), _p(u, ctypes.c_uint32),
+                               _p(q, ctypes.c_int32), ctypes.byref(d), ctypes.byref(z))
+    return q, np.float32(d.value), np.float32(z.value)
+
+
+def step_sr(cfg: Cfg, st: State, i, x, B, C, dt, A, D, seed, step, layer, slot):
+    """One decode step on pair i with stochastic rounding."""
+    x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))
+    y = np.zeros((cfg.nheads, cfg.headdim), np.float32)
+    r = _SR(seed, step, layer, slot)
+    c = cfg.c()
+    lib().oref_step_sr(ctypes.byref(c), ctypes.byref(st.c(i)), ctypes.byref(r),
+                       _p(x, ctypes.c_float), _p(B, ctypes.c_float), _p(C, ctypes.c_float),
+                       _p(dt, ctypes.c_float), _p(A, ctypes.c_float), _p(D, ctypes.c_float),
+                       _p(y, ctypes.c_float))
+    return y
+
+
+def scan_sr(cfg: Cfg, st: State, i, x, B, C, dt, A, D, seed, step0, layer, slot):
+    """T steps on pair i with stochastic rounding, token t at step0 + t."""
+    x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))
+    T = x.shape[0]
+    y = np.zeros((T, cfg.nheads, cfg.headdim), np.float32)
+    r = _SR(seed, step0, layer, slot)
+    c = cfg.c()
+    lib().oref_scan_sr(ctypes.byref(c), ctypes.byref(st.c(i)), ctypes.byref(r), T,
+                       _p(x, ctypes.c_float), _p(B, ctypes.c_float), _p(C, ctypes.c_float),
+                       _p(dt, ctypes.c_float), _p(A, ctypes.c_float), _p(D, ctypes.c_float),
+                       _p(y, ctypes.c_float))
     return y
 
 

@@ -306,6 +306,150 @@ void oref_scan(const oref_cfg* c, oref_state* st, int T, const float* x,
     }
 }
 
+/* ---------------------------------------------------------------------------
+ * Stochastic rounding ("ssm-state-quantization" README, Findings 9: SR of the
+ * state keeps 8 bits within 0.4 ppl of the control).  Each entry rounds down
+ * or up to a neighbouring grid level with probability given by its distance:
+ * code = floor(v*inv + u) (+ z), u uniform in [0, 1) on a 2^-16 grid, the
+ * product exact and the sum exact (both in double), then clamped to the
+ * code range (the minimum can now round down one level, the maximum up one).
+ * The grid (Delta, z) is refit as for nearest rounding.
+ * Parity: the rounding rule is pinned by the tests (neighbours only, grid
+ * points fixed, unbiased on average); the generator by statistics only.
+ * ------------------------------------------------------------------------- */
+
+/* Philox4x32-10 from its definition: ten rounds of two 32x32->64-bit
+ * multiplications by fixed constants, the high halves XORed with the other
+ * two counter words and the key, the key bumped by two Weyl constants after
+ * each round. */
+void oref_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)c2;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        c0 = hi1 ^ c1 ^ k0;
+        c1 = lo1;
+        c2 = hi0 ^ c3 ^ k1;
+        c3 = lo0;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+uint32_t oref_sr_u16(const oref_sr* r, int row, int n, int N)
+{
+    const uint32_t ctr[4] = {(uint32_t)row * (uint32_t)(N / 8) + (uint32_t)(n / 8),
+                             r->layer, r->slot, r->step};
+    const uint32_t key[2] = {(uint32_t)r->seed, (uint32_t)(r->seed >> 32)};
+    uint32_t out[4];
+    oref_philox4x32_10(ctr, key, out);
+    return (out[(n % 8) / 2] >> (16 * (n % 2))) & 0xFFFFu;
+}
+
+void oref_quantize_row_sr(int fmt, int N, const float* v, const uint32_t* u16,
+                          int32_t* q, float* delta_out, float* zero_out)
+{
+    /* the grid: as for nearest rounding */
+    int32_t* tmp = (int32_t*)malloc(sizeof(int32_t) * (size_t)N);
+    oref_quantize_row(fmt, N, v, tmp, delta_out, zero_out);
+    free(tmp);
+    const float delta = *delta_out, z = *zero_out;
+    const float qm = qmax_of(fmt);
+    const int sym = oref_is_sym(fmt);
+    const float inv = (delta == 0.0f) ? 0.0f : 1.0f / delta;
+    for (int n = 0; n < N; ++n) {
+        const double p = (double)v[n] * (double)inv;       /* exact */
+        const double k = floor(p + (double)u16[n] / 65536.0); /* exact sum */
+        float c = (float)k;
+        if (sym) {
+            if (c > qm) c = qm;
+            if (c < -qm) c = -qm;
+        } else {
+            c = c + z;
+            if (c > qm) c = qm;
+            if (c < 0.0f) c = 0.0f;
+        }
+        q[n] = (int32_t)c;
+    }
+}
+
+/* One decode step with stochastic rounding of the quantized rows (steps 1,
+ * 2 and 6 as oref_step). */
+void oref_step_sr(const oref_cfg* c, oref_state* st, const oref_sr* r,
+                  const float* x, const float* B, const float* C,
+                  const float* dt, const float* A, const float* D, float* y)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state, G = c->ngroups;
+    const int heads_per_group = H / G;
+    float* s = (float*)malloc(sizeof(float) * (size_t)N);
+    float* sn = (float*)malloc(sizeof(float) * (size_t)N);
+    float* stored = (float*)malloc(sizeof(float) * (size_t)N);
+    uint32_t* u = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)N);
+    for (int h = 0; h < H; ++h) {
+        const int g = h / heads_per_group;
+        const float lam = oref_lambda(dt[h], A[h]);
+        const float* Bg = B + (size_t)g * N;
+        const float* Cg = C + (size_t)g * N;
+        const int quant = oref_row_is_quant(c, h);
+        for (int p = 0; p < P; ++p) {
+            const int row = h * P + p;
+            if (quant) {
+                oref_dequantize_row(c->fmt, N, st->q + (size_t)row * N,
+                                    st->delta[row], st->zero[row], s);
+            } else {
+                memcpy(s, st->val + (size_t)row * N, sizeof(float) * (size_t)N);
+            }
+            const float dtx = dt[h] * x[row];
+            for (int n = 0; n < N; ++n) {
+                float w = dtx * Bg[n];
+                sn[n] = fmaf(lam, s[n], w);
+            }
+            if (quant) {
+                for (int n = 0; n < N; ++n) u[n] = oref_sr_u16(r, row, n, N);
+                int32_t* qr = st->q + (size_t)row * N;
+                oref_quantize_row_sr(c->fmt, N, sn, u, qr, st->delta + row, st->zero + row);
+                oref_dequantize_row(c->fmt, N, qr, st->delta[row], st->zero[row], stored);
+            } else {
+                for (int n = 0; n < N; ++n) {
+                    float v = sn[n];
+                    if (c->fmt == OREF_BF16) v = oref_bf16_round(v);
+                    st->val[(size_t)row * N + n] = v;
+                    stored[n] = v;
+                }
+            }
+            double acc = 0.0;
+            for (int n = 0; n < N; ++n)
+                acc += (double)Cg[n] * (double)stored[n];
+            acc += (double)D[h] * (double)x[row];
+            y[row] = (float)acc;
+        }
+    }
+    free(s);
+    free(sn);
+    free(stored);
+    free(u);
+}
+
+/* T steps with stochastic rounding; token t draws with step r->step + t. */
+void oref_scan_sr(const oref_cfg* c, oref_state* st, const oref_sr* r, int T,
+                  const float* x, const float* B, const float* C,
+                  const float* dt, const float* A, const float* D, float* y)
+{
+    const size_t HP = (size_t)c->nheads * c->headdim;
+    const size_t GN = (size_t)c->ngroups * c->d_state;
+    oref_sr rt = *r;
+    for (int t = 0; t < T; ++t) {
+        rt.step = r->step + (uint32_t)t;
+        oref_step_sr(c, st, &rt, x + t * HP, B + t * GN, C + t * GN,
+                     dt + (size_t)t * c->nheads, A, D, y + t * HP);
+    }
+}
+
 /* Prefill hand-off ("Mamba state quantization for inference", phase-aware
  * benchmarks: prefill computes in FP32 and writes its final state into the
  * packed cache): from the stored state, T tokens of the fp32 recurrence

@@ -101,6 +101,29 @@ void  oref_scan(const oref_cfg* c, oref_state* st, int T, const float* x,
                 const float* B, const float* C, const float* dt,
                 const float* A, const float* D, float* y);
 
+/* Stochastic rounding.  The random draw of entry n of row r (= h*P + p) at
+ * a step is 16 bits of Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel
+ * random numbers: as easy as 1, 2, 3", SC 2011) with key (seed low, seed
+ * high) and counter (r*(N/8) + n/8, layer, slot, step): word (n%8)/2 of the
+ * output, low half for even n, high half for odd n. */
+typedef struct {
+    uint64_t seed;
+    uint32_t step;   /* token counter: decode position, or the first token of a scan */
+    uint32_t layer;
+    uint32_t slot;
+} oref_sr;
+
+void  oref_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+uint32_t oref_sr_u16(const oref_sr* r, int row, int n, int N);
+void  oref_quantize_row_sr(int fmt, int N, const float* v, const uint32_t* u16,
+                           int32_t* q, float* delta, float* zero);
+void  oref_step_sr(const oref_cfg* c, oref_state* st, const oref_sr* r,
+                   const float* x, const float* B, const float* C,
+                   const float* dt, const float* A, const float* D, float* y);
+void  oref_scan_sr(const oref_cfg* c, oref_state* st, const oref_sr* r, int T,
+                   const float* x, const float* B, const float* C,
+                   const float* dt, const float* A, const float* D, float* y);
+
 void  oref_prefill(const oref_cfg* c, oref_state* st, int T, const float* x,
                    const float* B, const float* C, const float* dt,
                    const float* A, const float* D, float* y);

@@ -37,6 +37,9 @@ MUTATIONS = {
     "swap_B_C": ("float w = dtx * Bg[n];", "float w = dtx * Cg[n];"),
     "constant_row_step": ("if (delta == 0.0f) delta = fabsf(lo);",
                           "if (delta == 0.0f) delta = 1.0f;"),
+    "sr_ignores_draw": ("const double k = floor(p + (double)u16[n] / 65536.0);",
+                        "const double k = floor(p + 0.5);"),
+    "sr_no_low_clamp": ("            if (c < 0.0f) c = 0.0f;\n", ""),
 }
 
 

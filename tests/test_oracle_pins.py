@@ -590,3 +590,129 @@ def test_prefill_closer_to_exact_than_rounding_every_token(oref):
     es = np.abs(O.state_to_f32(st_s)[0] - S64).reshape(H, -1).mean(axis=1)
     assert np.all(ep <= es * 1.01), (ep, es)
     assert ep.mean() < 0.9 * es.mean(), (ep, es)
+
+
+# ---------------------------------------------------------------------------
+# Stochastic rounding ("ssm-state-quantization" README, Findings 9)
+# ---------------------------------------------------------------------------
+
+def _levels(fmt, delta, z):
+    qm = {O.I8_ASYM: 255, O.I4_ASYM: 15, O.I8_SYM: 127, O.I4_SYM: 7}[fmt]
+    codes = np.arange(-qm, qm + 1) if fmt in (O.I8_SYM, O.I4_SYM) else np.arange(0, qm + 1)
+    deq = np.array([O.dequantize_row(fmt, np.array([c], np.int32), delta, z)[0]
+                    for c in codes], np.float64)
+    return codes, deq
+
+
+@pytest.mark.parametrize("fmt", QFMTS)
+def test_sr_rounds_to_a_bracketing_level(oref, fmt):
+    """Every stochastically rounded entry lands on one of the two grid
+    levels around it (or the end of the code range), whatever the draw."""
+    rng = np.random.default_rng(41)
+    for trial in range(40):
+        v = (rng.standard_normal(32) * rng.uniform(0.01, 10)).astype(np.float32)
+        if trial % 4 == 1:
+            v = np.abs(v) + 1.0
+        u = rng.integers(0, 65536, 32).astype(np.uint32)
+        q, d, z = O.quantize_row_sr(fmt, v, u)
+        codes, deq = _levels(fmt, d, z)
+        for n in range(32):
+            below = deq[deq <= v[n] * (1 + 1e-6) + 1e-30]
+            above = deq[deq >= v[n] * (1 - 1e-6) - 1e-30]
+            lo = below.max() if below.size else deq.min()
+            hi = above.min() if above.size else deq.max()
+            got = O.dequantize_row(fmt, q[n:n + 1], d, z)[0]
+            assert lo - 1e-6 * abs(lo) <= got <= hi + 1e-6 * abs(hi), (fmt, n, v[n], got, lo, hi)
+
+
+@pytest.mark.parametrize("fmt", QFMTS)
+def test_sr_with_half_draw_is_nearest_off_ties(oref, fmt):
+    """A draw of exactly 1/2 turns floor(p + u) into round-half-up: equal to
+    the nearest rounding on every entry that is not an exact tie."""
+    rng = np.random.default_rng(43)
+    for _ in range(30):
+        v = (rng.standard_normal(64) * 3).astype(np.float32)
+        q_rtn, d, z, pre = O.quantize_row(fmt, v)
+        q_sr, d2, z2 = O.quantize_row_sr(fmt, v, np.full(64, 32768, np.uint32))
+        assert d == d2 and z == z2
+        ties = np.abs(np.abs(pre - np.floor(pre)) - 0.5) == 0
+        assert np.array_equal(q_rtn[~ties], q_sr[~ties])
+
+
+@pytest.mark.parametrize("fmt", [O.I8_ASYM, O.I4_ASYM])
+def test_sr_keeps_grid_points(oref, fmt):
+    """Rows built on the grid reconstruct exactly under any draws (the
+    fractional part is 0, so floor(p + u) = p)."""
+    qa = 255 if fmt == O.I8_ASYM else 15
+    rng = np.random.default_rng(45)
+    e = -6
+    codes = rng.integers(0, qa + 1, 48)
+    codes[0], codes[1] = 0, qa
+    k = 37
+    v = ((codes - k) * 2.0 ** e).astype(np.float32)
+    for _ in range(5):
+        u = rng.integers(0, 65536, 48).astype(np.uint32)
+        q, d, z = O.quantize_row_sr(fmt, v, u)
+        assert np.array_equal(O.dequantize_row(fmt, q, d, z), v)
+
+
+@pytest.mark.parametrize("fmt", QFMTS)
+def test_sr_is_unbiased(oref, fmt):
+    """Averaged over independent draws (Philox at 3000 steps) the
+    stochastically rounded row equals the row: within 5 standard errors
+    (each draw errs by at most one step), for every entry between the end
+    levels of the grid.  (An extreme entry beyond the last level, which the
+    integer zero point allows by up to half a step, is clamped and so
+    biased by as much.)"""
+    rng = np.random.default_rng(47)
+    N = 32
+    v = (rng.standard_normal(N) * 2).astype(np.float32)
+    K = 3000
+    acc = np.zeros(N)
+    for step in range(K):
+        u = O.sr_draws(123, step, 0, 0, 1, N)[0]
+        q, d, z = O.quantize_row_sr(fmt, v, u)
+        acc += O.dequantize_row(fmt, q, d, z)
+    _, d, z, _ = O.quantize_row(fmt, v)
+    _, deq = _levels(fmt, d, z)
+    inside = (v >= deq.min()) & (v <= deq.max())
+    assert inside.sum() >= N - 2
+    mean = acc / K
+    err = np.abs(mean - v)[inside]
+    assert np.all(err <= 5 * (float(d) / 2) / np.sqrt(K)), err.max()
+
+
+def test_sr_draws_are_uniform_and_keyed(oref):
+    """The 16-bit draws: uniform over 16 bins (chi-square, 15 dof, p > 1e-4),
+    mean within 5 sigma, and different for a different seed, step, layer,
+    slot or row."""
+    u = O.sr_draws(7, 11, 2, 5, 64, 128).reshape(-1).astype(np.float64)
+    n = u.size
+    assert abs(u.mean() - 32767.5) <= 5 * 18918.6 / np.sqrt(n)
+    counts = np.bincount((u // 4096).astype(int), minlength=16)
+    chi2 = float(((counts - n / 16) ** 2 / (n / 16)).sum())
+    assert chi2 < 50.0, chi2                      # 15 dof: p(chi2 > 50) < 1e-5
+    base = O.sr_draws(7, 11, 2, 5, 2, 16)
+    for other in (O.sr_draws(8, 11, 2, 5, 2, 16), O.sr_draws(7, 12, 2, 5, 2, 16),
+                  O.sr_draws(7, 11, 3, 5, 2, 16), O.sr_draws(7, 11, 2, 6, 2, 16)):
+        assert np.mean(other == base) < 0.01
+    assert np.mean(base[0] == base[1]) < 0.2
+
+
+def test_sr_scan_is_steps_with_advancing_counter(oref):
+    """T tokens of the SR scan equal T SR decode steps at steps step0 .. step0+T-1."""
+    H, P, N, T = 2, 8, 16, 12
+    wl = W.Scan("pin", seed=13, batch=1, T=T, nheads=H, headdim=P, d_state=N,
+                ngroups=1, fmt="i8a")
+    inp = wl.inputs()
+    x, B, C, dt = (inp[k][0] for k in ("x", "B", "C", "dt"))
+    cfg = O.Cfg(O.I8_ASYM, H, P, N, 1)
+    a, b = O.State(cfg), O.State(cfg)
+    ya = O.scan_sr(cfg, a, 0, x, B, C, dt, inp["A"], inp["D"], 99, 1000, 3, 4)
+    yb = np.stack([O.step_sr(cfg, b, 0, x[t], B[t], C[t], dt[t], inp["A"], inp["D"],
+                             99, 1000 + t, 3, 4) for t in range(T)])
+    assert np.array_equal(a.q, b.q) and np.array_equal(ya, yb)
+    # and it differs from nearest rounding somewhere
+    c = O.State(cfg)
+    O.scan(cfg, c, 0, x, B, C, dt, inp["A"], inp["D"])
+    assert not np.array_equal(a.q, c.q)
