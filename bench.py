@@ -56,6 +56,7 @@ def workload(name):
     table = {
         "decode_130m": lambda: W.decode_130m("i8a"),
         "decode_130m_f32": lambda: W.decode_130m("f32"),
+        "decode_130m_sr": lambda: W.decode_130m("i8a"),
         "decode_8b_b1_i8a": lambda: W.decode_8b("i8a", 1),
         "decode_8b_b16_i8a": lambda: W.decode_8b("i8a", 16),
         "decode_8b_b64_i8a": lambda: W.decode_8b("i8a", 64),
@@ -419,9 +420,18 @@ def run_ours(args, wl, name):
         y = torch.empty((wl.nl, wl.batch, H, P), device=dev)
         nbytes = decode_bytes(wl)
 
+        # the stochastic-rounding variant draws fresh randomness every step
+        sr = name.endswith("_sr")
+        nstep = [0]
+
         def step():
-            ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, d["x"], d["B"], d["C"],
-                                d["dt"], d["A"], d["D"], y)
+            if sr:
+                nstep[0] += 1
+                ssq.ssq_decode_step_sr(cfg, pool, None, wl.batch, 0, wl.nl, d["x"], d["B"],
+                                       d["C"], d["dt"], d["A"], d["D"], y, 12345, nstep[0])
+            else:
+                ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, d["x"], d["B"],
+                                    d["C"], d["dt"], d["A"], d["D"], y)
         units = wl.batch * wl.nl         # request-layer steps
 
     stream = torch.cuda.current_stream(dev)

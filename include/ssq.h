@@ -220,6 +220,23 @@ SSQ_API ssq_status ssq_decode_step(const ssq_config* cfg, void* pool,
                            const float* C, const float* dt, const float* A,
                            const float* D, float* y, cudaStream_t stream);
 
+/* ssq_decode_step with stochastic rounding of the quantized rows
+ * ("ssm-state-quantization" README, Findings 9: stochastic rounding of the
+ * state keeps 8 bits within 0.4 ppl of the control).  Entry n of row r =
+ * h*headdim + p rounds to floor(s'*inv + u) (+ z), clamped to the code
+ * range, on the grid refit as for nearest rounding; u = d/65536 with d 16
+ * bits of Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC 2011) under key
+ * (seed low word, seed high word) and counter (r*(d_state/8) + n/8, layer,
+ * slot, step): word (n%8)/2 of the output, low half for even n.  Pass a new
+ * step (e.g. the token position) at every call for fresh draws.  fp32 /
+ * bf16 rows are unaffected.  Other arguments as ssq_decode_step. */
+SSQ_API ssq_status ssq_decode_step_sr(const ssq_config* cfg, void* pool,
+                              const int32_t* slot_idx, int batch, int layer0,
+                              int nl, const float* x, const float* B,
+                              const float* C, const float* dt, const float* A,
+                              const float* D, float* y, uint64_t seed,
+                              uint32_t step, cudaStream_t stream);
+
 /* T tokens of one layer with the state rounded at every token and held on
  * chip between tokens ("ssm-state-quantization", Setup: a sequential
  * per-token scan in place of the chunked scan, so the state can be rounded
@@ -236,6 +253,16 @@ SSQ_API ssq_status ssq_scan(const ssq_config* cfg, void* pool,
                     const float* x, const float* B, const float* C,
                     const float* dt, const float* A, const float* D,
                     float* y, cudaStream_t stream);
+
+/* ssq_scan with stochastic rounding at every token, token t drawing with
+ * step counter step0 + t (draws as ssq_decode_step_sr); equal to T calls of
+ * ssq_decode_step_sr with nl = 1 and steps step0 .. step0+T-1. */
+SSQ_API ssq_status ssq_scan_sr(const ssq_config* cfg, void* pool,
+                       const int32_t* slot_idx, int batch, int layer, int T,
+                       const float* x, const float* B, const float* C,
+                       const float* dt, const float* A, const float* D,
+                       float* y, uint64_t seed, uint32_t step0,
+                       cudaStream_t stream);
 
 /* Prefill hand-off ("Mamba state quantization for inference", phase-aware
  * benchmarks: prefill computes in FP32 and writes its final state into the

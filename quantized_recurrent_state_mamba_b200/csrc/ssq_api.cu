@@ -288,10 +288,16 @@ ssq_status ssq_dequantize_rows(const ssq_config* cfg, const void* pool,
     return SSQ_OK;
 }
 
-ssq_status ssq_decode_step(const ssq_config* cfg, void* pool, const int32_t* slot_idx,
-                           int batch, int layer0, int nl, const float* x, const float* B,
-                           const float* C, const float* dt, const float* A, const float* D,
-                           float* y, cudaStream_t stream)
+}  // extern "C"
+
+namespace {
+
+// ssq_decode_step and ssq_decode_step_sr: sr rounds the quantized rows
+// stochastically with draws keyed by seed at step counter `step`.
+ssq_status decode_common(const ssq_config* cfg, void* pool, const int32_t* slot_idx,
+                         int batch, int layer0, int nl, const float* x, const float* B,
+                         const float* C, const float* dt, const float* A, const float* D,
+                         float* y, bool sr, uint64_t seed, uint32_t step, cudaStream_t stream)
 {
     ssq::PoolView pv;
     ssq_layout L;
@@ -318,27 +324,29 @@ ssq_status ssq_decode_step(const ssq_config* cfg, void* pool, const int32_t* slo
     cv.A = A;
     cv.D = D;
     cv.y = y;
+    cv.sr_seed = seed;
+    cv.sr_step = step;
     if (!ssq::decode_fits((int)cfg->fmt, cfg->d_state, cfg->nheads, cfg->ngroups))
         return fail(SSQ_ERR_UNSUPPORTED, "ngroups*d_state %d too large for the decode kernel",
                     cfg->ngroups * cfg->d_state);
     int rows_q = 0, rows_f = 0;
     ssq::decode_tile_rows((int)cfg->fmt, cfg->d_state, &rows_q, &rows_f);
     fill_tiles(pv, &cv, rows_q, rows_f);
-    cudaError_t e = ssq::launch_decode(pv, cv, (int)cfg->fmt, stream);
+    cudaError_t e = ssq::launch_decode(pv, cv, (int)cfg->fmt, sr, stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return SSQ_OK;
 }
 
-}  // extern "C"
 
-namespace {
-
-// ssq_scan and ssq_prefill: the same launch geometry; prefill keeps the state
-// fp32 across the tokens and quantizes it once at the end.
+// ssq_scan, ssq_scan_sr and ssq_prefill: the same launch geometry; prefill
+// keeps the state fp32 across the tokens and quantizes it once at the end;
+// sr rounds stochastically at every token (token t at step counter
+// step0 + t).
 ssq_status scan_common(const ssq_config* cfg, void* pool, const int32_t* slot_idx, int batch,
                        int layer, int T, const float* x, const float* B, const float* C,
                        const float* dt, const float* A, const float* D, float* y,
-                       bool prefill, cudaStream_t stream)
+                       bool prefill, bool sr, uint64_t seed, uint32_t step0,
+                       cudaStream_t stream)
 {
     ssq::PoolView pv;
     ssq_layout L;
@@ -367,6 +375,8 @@ ssq_status scan_common(const ssq_config* cfg, void* pool, const int32_t* slot_id
     cv.A = A;
     cv.D = D;
     cv.y = y;
+    cv.sr_seed = seed;
+    cv.sr_step = step0;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -378,7 +388,7 @@ ssq_status scan_common(const ssq_config* cfg, void* pool, const int32_t* slot_id
     cv.qtiles = pv.Hq * sp.tiles_per_head;
     cv.ftiles = pv.Hf * sp.tiles_per_head;
     cv.total_tiles = (long long)batch * (cv.qtiles + cv.ftiles);
-    e = ssq::launch_scan(pv, cv, (int)cfg->fmt, sp, prefill, stream);
+    e = ssq::launch_scan(pv, cv, (int)cfg->fmt, sp, prefill, sr, stream);
     if (e != cudaSuccess) return cuda_fail(e, prefill ? "prefill launch" : "scan launch");
     return SSQ_OK;
 }
@@ -387,13 +397,41 @@ ssq_status scan_common(const ssq_config* cfg, void* pool, const int32_t* slot_id
 
 extern "C" {
 
+ssq_status ssq_decode_step(const ssq_config* cfg, void* pool, const int32_t* slot_idx,
+                           int batch, int layer0, int nl, const float* x, const float* B,
+                           const float* C, const float* dt, const float* A, const float* D,
+                           float* y, cudaStream_t stream)
+{
+    return decode_common(cfg, pool, slot_idx, batch, layer0, nl, x, B, C, dt, A, D, y, false,
+                         0, 0, stream);
+}
+
+ssq_status ssq_decode_step_sr(const ssq_config* cfg, void* pool, const int32_t* slot_idx,
+                              int batch, int layer0, int nl, const float* x, const float* B,
+                              const float* C, const float* dt, const float* A,
+                              const float* D, float* y, uint64_t seed, uint32_t step,
+                              cudaStream_t stream)
+{
+    return decode_common(cfg, pool, slot_idx, batch, layer0, nl, x, B, C, dt, A, D, y, true,
+                         seed, step, stream);
+}
+
 ssq_status ssq_scan(const ssq_config* cfg, void* pool, const int32_t* slot_idx, int batch,
                     int layer, int T, const float* x, const float* B, const float* C,
                     const float* dt, const float* A, const float* D, float* y,
                     cudaStream_t stream)
 {
     return scan_common(cfg, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y, false,
-                       stream);
+                       false, 0, 0, stream);
+}
+
+ssq_status ssq_scan_sr(const ssq_config* cfg, void* pool, const int32_t* slot_idx, int batch,
+                       int layer, int T, const float* x, const float* B, const float* C,
+                       const float* dt, const float* A, const float* D, float* y,
+                       uint64_t seed, uint32_t step0, cudaStream_t stream)
+{
+    return scan_common(cfg, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y, false,
+                       true, seed, step0, stream);
 }
 
 ssq_status ssq_prefill(const ssq_config* cfg, void* pool, const int32_t* slot_idx, int batch,
@@ -402,7 +440,7 @@ ssq_status ssq_prefill(const ssq_config* cfg, void* pool, const int32_t* slot_id
                        cudaStream_t stream)
 {
     return scan_common(cfg, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y, true,
-                       stream);
+                       false, 0, 0, stream);
 }
 
 }  // extern "C"

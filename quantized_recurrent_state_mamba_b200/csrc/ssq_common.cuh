@@ -576,6 +576,118 @@ __device__ __forceinline__ void round16_carry(float2 inv2, float2 z2, float2 mz2
     }
 }
 
+// ---------------------------------------------------------------------------
+// Stochastic rounding ("ssm-state-quantization" README, Findings 9).
+//
+// An entry rounds to floor(s*inv + u) (plus z, clamped to the code range),
+// u = d * 2^-16 with d a 16-bit draw of Philox4x32-10 (Salmon, Moraes, Dror,
+// Shaw, SC 2011) keyed by the caller's seed, counter (r*(N/8) + n/8, layer,
+// slot, step) for entry n of row r = h*P + p: word (n%8)/2 of the output,
+// low half for even n.  floor of the exact s*inv + u is formed as
+// fma rounded toward -inf (floor of that float is floor of the exact sum)
+// and an add of 1.5*2^23 rounded toward -inf.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k)
+{
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+        c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+        k.x += 0x9E3779B9u;
+        k.y += 0xBB67AE85u;
+    }
+    return c;
+}
+
+// Counter words of a stochastic-rounding draw: y = layer, z = slot, w = step;
+// x is set per 8-entry block.
+struct SrKey {
+    uint2 key;
+    uint32_t layer, slot, step;
+    uint32_t row_block;   // r * (N/8): the first block of this row
+};
+
+// u = d * 2^-16 for the 16 entries [n0, n0 + 16) of a row (n0 a multiple of
+// 16): two Philox blocks.
+__device__ __forceinline__ void sr_draws16(const SrKey& k, int n0, float (&u)[16])
+{
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+        const uint4 w = philox4x32_10(
+            make_uint4(k.row_block + (uint32_t)(n0 / 8 + b), k.layer, k.slot, k.step), k.key);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // 1 + d*2^-16 has the 16 draw bits on top of the mantissa
+            u[8 * b + 2 * i] = __uint_as_float(0x3F800000u | ((ww[i] & 0xFFFFu) << 7)) - 1.0f;
+            u[8 * b + 2 * i + 1] = __uint_as_float(0x3F800000u | ((ww[i] >> 16) << 7)) - 1.0f;
+        }
+    }
+}
+
+__device__ __forceinline__ float2 fma2_rm(float2 a, float2 b, float2 c)
+{
+    unsigned long long d;
+    asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(d)
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+          "l"(*reinterpret_cast<unsigned long long*>(&b)),
+          "l"(*reinterpret_cast<unsigned long long*>(&c)));
+    return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 add2_rm(float2 a, float2 b)
+{
+    unsigned long long d;
+    asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d)
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+          "l"(*reinterpret_cast<unsigned long long*>(&b)));
+    return *reinterpret_cast<float2*>(&d);
+}
+
+// Stochastic rounding of 16 entries on the fast path (|s*inv| < 2^21):
+// r = q - z (asym) or q (sym) exactly, k carries the stored code.  mz2 holds
+// -(1.5*2^23 + z) (asym) or -1.5*2^23 (sym).
+template <int FMT>
+__device__ __forceinline__ void round16_sr(float2 inv2, float2 z2, float2 mz2, const float* s,
+                                           const float (&u)[16], float* r, uint32_t (&k)[16])
+{
+    using F = Fmt<FMT>;
+    const float2 m2 = make_float2(kMagic, kMagic);
+    constexpr float kLo = F::sym ? kMagic - F::qmax : kMagic;
+    constexpr float kHi = kMagic + F::qmax;
+#pragma unroll
+    for (int n = 0; n < 16; n += 2) {
+        const float2 v = fma2_rm(make_float2(s[n], s[n + 1]), inv2, make_float2(u[n], u[n + 1]));
+        float2 t = add2_rm(v, m2);                     // 1.5*2^23 + floor(s*inv + u)
+        if constexpr (!F::sym) t = add2(t, z2);        // 1.5*2^23 + q before the clamp
+        t.x = fminf(fmaxf(t.x, kLo), kHi);
+        t.y = fminf(fmaxf(t.y, kLo), kHi);
+        const float2 rr = add2(t, mz2);
+        r[n] = rr.x; r[n + 1] = rr.y;
+        k[n] = __float_as_uint(t.x);
+        k[n + 1] = __float_as_uint(t.y);
+    }
+}
+
+// The same by the formulas verbatim (exact sum in double), for rows outside
+// the fast range.
+template <int FMT>
+__device__ __forceinline__ float round1_sr_exact(float s, float inv, float z, float u,
+                                                 float* r)
+{
+    using F = Fmt<FMT>;
+    const double kf = floor((double)s * (double)inv + (double)u);
+    float c = (float)kf;
+    if constexpr (F::sym) {
+        c = fminf(fmaxf(c, -F::qmax), F::qmax);
+        *r = c;
+    } else {
+        c = fminf(fmaxf(__fadd_rn(c, z), 0.0f), F::qmax);
+        *r = __fsub_rn(c, z);
+    }
+    return c;
+}
+
 // Exact scalar rounding of 16 entries (the definition verbatim).
 template <int FMT>
 __device__ __forceinline__ void round16_slow(const RowParams& rp, const float* s, float* r,

@@ -293,12 +293,12 @@ struct FShape {
 // 2^22 or more in magnitude (rows far from zero relative to their range).  Every lane of the warp
 // calls it together (the row reductions are shuffles).  Codes are read from
 // and written in natural order; B and C come from the interleaved layout.
-template <int FMT, int N>
+template <int FMT, int N, bool SR>
 __device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float delta0, float z0,
                                         float lam, float dtx, const float* __restrict__ gB,
                                         const float* __restrict__ gC, int j, bool active,
                                         uint8_t* __restrict__ crow, uint8_t* __restrict__ mrow,
-                                        uint32_t* err)
+                                        uint32_t* err, SrKey srk)
 {
     using F = Fmt<FMT>;
     constexpr int E = QShape<N>::E, LPR = QShape<N>::LPR;
@@ -332,14 +332,24 @@ __device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float de
     for (int i = 0; i < CB / 4; ++i) words[i] = 0u;
 #pragma unroll 1
     for (int n = 0; n < E; ++n) {
-        const float rr = rint_prod(s[n], rp.inv);
         float c, r;
-        if constexpr (F::sym) {
-            c = fminf(fmaxf(rr, -F::qmax), F::qmax);
-            r = c;
+        if constexpr (SR) {
+            const int ng = j * E + n;                   // entry within the row
+            const uint4 w = philox4x32_10(
+                make_uint4(srk.row_block + (uint32_t)(ng / 8), srk.layer, srk.slot, srk.step),
+                srk.key);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            const uint32_t d = (ww[(ng % 8) / 2] >> (16 * (ng % 2))) & 0xFFFFu;
+            c = round1_sr_exact<FMT>(s[n], rp.inv, rp.z, (float)d * (1.0f / 65536.0f), &r);
         } else {
-            c = fminf(__fadd_rn(rr, rp.z), F::qmax);
-            r = __fsub_rn(c, rp.z);
+            const float rr = rint_prod(s[n], rp.inv);
+            if constexpr (F::sym) {
+                c = fminf(fmaxf(rr, -F::qmax), F::qmax);
+                r = c;
+            } else {
+                c = fminf(__fadd_rn(rr, rp.z), F::qmax);
+                r = __fsub_rn(c, rp.z);
+            }
         }
         const uint32_t code = (uint32_t)(int)c & ((1u << F::bits) - 1u);
         words[n * F::bits / 32] |= code << ((n * F::bits) % 32);
@@ -363,7 +373,9 @@ __device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float de
     return ysum;
 }
 
-template <int FMT, int N>
+// SR: round the quantized rows stochastically (draws keyed by cv.sr_seed
+// and countered by row block, layer, slot and cv.sr_step).
+template <int FMT, int N, bool SR>
 __global__ void __launch_bounds__(kDThreads, kMinBlocks)
 decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv,
               const __grid_constant__ DecodeGeom geo)
@@ -539,6 +551,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     uint8_t* meta_u = nullptr;
     uint8_t* fp_u = nullptr;
     float* y_u = nullptr;
+    int cur_slot = 0;
 
     TileWalk ti;
     ti.start(pv, cv, t0);
@@ -556,6 +569,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             }
             ub = units + u * geo.unit_bytes;
             const int slot = reinterpret_cast<const int*>(ub)[0];
+            cur_slot = slot;
             bad = reinterpret_cast<const int*>(ub)[1] != 0;
             if (!bad) {
                 const int layer = cv.layer0 + ti.l;
@@ -687,6 +701,15 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 // rows whose top code must be capped take the clamped loop
                 const bool fast = __all_sync(0xffffffffu, (F::sym || fabsf(z0) < kFastLimit)
                                                           && rp.fast);
+                // the stochastic-rounding key of this row (unused for RTN)
+                SrKey srk;
+                if constexpr (SR) {
+                    srk.key = make_uint2((uint32_t)cv.sr_seed, (uint32_t)(cv.sr_seed >> 32));
+                    srk.layer = (uint32_t)(cv.layer0 + ti.l);
+                    srk.slot = (uint32_t)cur_slot;
+                    srk.step = cv.sr_step;
+                    srk.row_block = (uint32_t)(__float_as_int(hti.w) + p) * (uint32_t)(N / 8);
+                }
                 if (fast) {
                     const float2 inv2 = make_float2(rp.inv, rp.inv);
                     const float2 z2 = make_float2(rp.z, rp.z);
@@ -711,7 +734,13 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         }
                         float r[16];
                         uint32_t kk[16];
-                        round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, v16, r, kk);
+                        if constexpr (SR) {
+                            float u[16];
+                            sr_draws16(srk, j * EQ + 16 * (int)((unsigned)sp ^ rot), u);
+                            round16_sr<FMT>(inv2, z2, mz2, v16, u, r, kk);
+                        } else {
+                            round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, v16, r, kk);
+                        }
                         uint32_t w[PW];
                         pack16<FMT>(kk, w);
                         {
@@ -733,7 +762,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         cq(std::integral_constant<int, 2>{});
                         cq(std::integral_constant<int, 3>{});
                     };
-                    if (F::sym || !__any_sync(0xffffffffu, rp.clamp)) {
+                    if (SR || F::sym || !__any_sync(0xffffffffu, rp.clamp)) {
 #pragma unroll
                         for (int sp = 0; sp < NP; ++sp) piece(std::false_type{}, sp);
                     } else {
@@ -751,8 +780,8 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     if (__any_sync(0xffffffffu, !rp.finite) && lane == 0)
                         atomicOr(err, SSQ_DEVERR_NONFINITE);
                 } else {
-                    ysum = row_exact<FMT, N>(cs, delta0, z0, lamv, dtx, gB, gC, j, active, crow,
-                                             mrow, err);
+                    ysum = row_exact<FMT, N, SR>(cs, delta0, z0, lamv, dtx, gB, gC, j, active,
+                                                 crow, mrow, err, srk);
                 }
             }
         }
@@ -825,7 +854,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     }
 }
 
-template <int FMT, int N>
+template <int FMT, int N, bool SR>
 cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
 {
     using F = Fmt<FMT>;
@@ -842,7 +871,7 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
     if (S < 2) S = 2;
     g = decode_geom(S, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G, SCR);
     if (g.smem_bytes > 227 * 1024) return cudaErrorInvalidConfiguration;
-    auto kern = decode_kernel<FMT, N>;
+    auto kern = decode_kernel<FMT, N, SR>;
     // per-device launch facts, looked up once per kernel instantiation and device
     thread_local int s_dev = -1, s_grid = 0, s_smem = 0;
     int dev = 0;
@@ -873,15 +902,15 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <int FMT>
+template <int FMT, bool SR>
 cudaError_t launch_fmt(const PoolView& pv, const CallView& cv, cudaStream_t st)
 {
     switch (pv.N) {
-    case 16: return launch_n<FMT, 16>(pv, cv, st);
-    case 32: return launch_n<FMT, 32>(pv, cv, st);
-    case 64: return launch_n<FMT, 64>(pv, cv, st);
-    case 128: return launch_n<FMT, 128>(pv, cv, st);
-    case 256: return launch_n<FMT, 256>(pv, cv, st);
+    case 16: return launch_n<FMT, 16, SR>(pv, cv, st);
+    case 32: return launch_n<FMT, 32, SR>(pv, cv, st);
+    case 64: return launch_n<FMT, 64, SR>(pv, cv, st);
+    case 128: return launch_n<FMT, 128, SR>(pv, cv, st);
+    case 256: return launch_n<FMT, 256, SR>(pv, cv, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -911,16 +940,21 @@ bool decode_fits(int fmt, int d_state, int nheads, int ngroups)
     return g.smem_bytes <= 227 * 1024;
 }
 
-cudaError_t launch_decode(const PoolView& pv, const CallView& cv, int fmt,
+cudaError_t launch_decode(const PoolView& pv, const CallView& cv, int fmt, bool sr,
                           cudaStream_t st)
 {
+    // stochastic rounding changes only the integer formats
     switch (fmt) {
-    case SSQ_F32: return launch_fmt<SSQ_F32>(pv, cv, st);
-    case SSQ_BF16: return launch_fmt<SSQ_BF16>(pv, cv, st);
-    case SSQ_I8_SYM: return launch_fmt<SSQ_I8_SYM>(pv, cv, st);
-    case SSQ_I8_ASYM: return launch_fmt<SSQ_I8_ASYM>(pv, cv, st);
-    case SSQ_I4_SYM: return launch_fmt<SSQ_I4_SYM>(pv, cv, st);
-    case SSQ_I4_ASYM: return launch_fmt<SSQ_I4_ASYM>(pv, cv, st);
+    case SSQ_F32: return launch_fmt<SSQ_F32, false>(pv, cv, st);
+    case SSQ_BF16: return launch_fmt<SSQ_BF16, false>(pv, cv, st);
+    case SSQ_I8_SYM:
+        return sr ? launch_fmt<SSQ_I8_SYM, true>(pv, cv, st) : launch_fmt<SSQ_I8_SYM, false>(pv, cv, st);
+    case SSQ_I8_ASYM:
+        return sr ? launch_fmt<SSQ_I8_ASYM, true>(pv, cv, st) : launch_fmt<SSQ_I8_ASYM, false>(pv, cv, st);
+    case SSQ_I4_SYM:
+        return sr ? launch_fmt<SSQ_I4_SYM, true>(pv, cv, st) : launch_fmt<SSQ_I4_SYM, false>(pv, cv, st);
+    case SSQ_I4_ASYM:
+        return sr ? launch_fmt<SSQ_I4_ASYM, true>(pv, cv, st) : launch_fmt<SSQ_I4_ASYM, false>(pv, cv, st);
     default: return cudaErrorInvalidValue;
     }
 }

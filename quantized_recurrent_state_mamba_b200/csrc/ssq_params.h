@@ -34,6 +34,8 @@ struct CallView {
     int T;                     // tokens (scan only)
     int tiles_per_head;        // scan: CTAs per head
     int scan_chunk;            // scan: tokens staged per shared-memory buffer
+    unsigned long long sr_seed;  // stochastic rounding: Philox key
+    unsigned sr_step;            // stochastic rounding: step counter (first token)
     const float* x;
     const float* B;
     const float* C;
@@ -48,7 +50,8 @@ struct CallView {
 // Host-side launchers (one per kernel family); each returns the CUDA error of
 // its launch.  The decode and rows kernels run a grid-stride loop over tiles
 // on a grid sized to the device's resident capacity.
-cudaError_t launch_decode(const PoolView& pv, const CallView& cv, int fmt,
+// sr: stochastic rounding of the quantized rows (cv.sr_seed, cv.sr_step)
+cudaError_t launch_decode(const PoolView& pv, const CallView& cv, int fmt, bool sr,
                           cudaStream_t stream);
 cudaError_t launch_quantize(const PoolView& pv, const CallView& cv, int fmt,
                             cudaStream_t stream);
@@ -63,8 +66,9 @@ struct ScanPlan {
 ScanPlan scan_plan(int d_state, int headdim, long long batch_heads, int sms);
 // prefill: keep the state fp32 over all T tokens and quantize it once at
 // the end (the prefill hand-off) instead of rounding at every token.
+// sr: stochastic rounding at every token (not with prefill)
 cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt, const ScanPlan& sp,
-                        bool prefill, cudaStream_t stream);
+                        bool prefill, bool sr, cudaStream_t stream);
 
 // Rows per decode tile in the quantized and the fp region.
 void decode_tile_rows(int fmt, int d_state, int* rows_q, int* rows_f);

@@ -108,6 +108,47 @@ __device__ __forceinline__ void round_piece_fast(const RowParams& rp, float* s,
     }
 }
 
+// Stochastic rounding of 16 entries on the fast path (see round16_sr): s <-
+// fl((q - z) * Delta) with q = clamp(floor(s*inv + u) (+ z)); with CODES also
+// the carriers of the stored codes.
+template <int FMT, bool CODES>
+__device__ __forceinline__ void round_piece_sr(const RowParams& rp, float* s,
+                                               const float (&u)[16], uint32_t (&k)[16])
+{
+    using F = Fmt<FMT>;
+    const float2 inv2 = make_float2(rp.inv, rp.inv);
+    const float2 z2 = make_float2(rp.z, rp.z);
+    const float mz = F::sym ? -kMagic : -__fadd_rn(kMagic, rp.z);
+    const float2 mz2 = make_float2(mz, mz);
+    const float2 d2 = make_float2(rp.delta, rp.delta);
+    float r[16];
+    uint32_t kk[16];
+    round16_sr<FMT>(inv2, z2, mz2, s, u, r, kk);
+#pragma unroll
+    for (int n = 0; n < 16; n += 2) {
+        const float2 v = mul2(make_float2(r[n], r[n + 1]), d2);
+        s[n] = v.x; s[n + 1] = v.y;
+        if constexpr (CODES) {
+            k[n] = kk[n];
+            k[n + 1] = kk[n + 1];
+        }
+    }
+}
+
+// The stochastic rounding by the formulas verbatim.
+template <int FMT>
+__device__ __forceinline__ void round_piece_sr_slow(const RowParams& rp, float* s,
+                                                    const float (&u)[16], uint32_t (&k)[16])
+{
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        float r;
+        const float c = round1_sr_exact<FMT>(s[n], rp.inv, rp.z, u[n], &r);
+        s[n] = __fmul_rn(r, rp.delta);
+        k[n] = (uint32_t)(int)c;
+    }
+}
+
 // The scalar formulas verbatim, for rows the fast path does not cover.
 template <int FMT>
 __device__ __forceinline__ void round_piece_slow(const RowParams& rp, float* s,
@@ -132,7 +173,9 @@ __device__ __forceinline__ void round_piece_slow(const RowParams& rp, float* s,
 
 // PF (prefill hand-off): the state stays fp32 for all T tokens (y read from
 // it) and is quantized, or bf16-rounded, once after the last token.
-template <int FMT, int N, int E, bool PF>
+// SR: round stochastically at every token (draws keyed by cv.sr_seed,
+// countered by row block, layer, slot and cv.sr_step + t).
+template <int FMT, int N, int E, bool PF, bool SR>
 __global__ void __launch_bounds__(64, E >= 64 ? 6 : 8)
 scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv)
 {
@@ -180,6 +223,14 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
     const float Av = __ldg(cv.A + h);
     const float Dv = __ldg(cv.D + h);
     const long long bT = (long long)b * T;
+    SrKey srk;
+    if constexpr (SR) {
+        srk.key = make_uint2((uint32_t)cv.sr_seed, (uint32_t)(cv.sr_seed >> 32));
+        srk.layer = (uint32_t)cv.layer0;
+        srk.slot = (uint32_t)slot;
+        srk.step = cv.sr_step;
+        srk.row_block = (uint32_t)(h * P + p) * (uint32_t)(N / 8);
+    }
 
     // Stage tokens [t0, t0 + nt) into buffer `bi`.
     auto stage = [&](int t0, int bi) {
@@ -378,7 +429,20 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
             rp = refit_from_minmax<FMT, LPR>(lo, hi);
             finite_all = finite_all && rp.finite;
             uint32_t kc[16];
-            if (__all_sync(0xffffffffu, rp.fast && !rp.clamp)) {
+            if constexpr (SR) {
+                srk.step = cv.sr_step + (uint32_t)t;
+                const bool sfast = __all_sync(0xffffffffu, rp.fast);
+#pragma unroll
+                for (int pc = 0; pc < NP; ++pc) {
+                    float u[16];
+                    sr_draws16(srk, j * E + 16 * pc, u);
+                    if (sfast)
+                        round_piece_sr<FMT, CODES>(rp, s + 16 * pc, u, kc);
+                    else
+                        round_piece_sr_slow<FMT>(rp, s + 16 * pc, u, kc);
+                    if constexpr (CODES) pack16<FMT>(kc, cw + PW * pc);
+                }
+            } else if (__all_sync(0xffffffffu, rp.fast && !rp.clamp)) {
 #pragma unroll
                 for (int pc = 0; pc < NP; ++pc) {
                     round_piece_fast<FMT, CODES>(rp, s + 16 * pc, kc);
@@ -490,14 +554,14 @@ scan_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
     }
 }
 
-template <int FMT, int N, int E, bool PF>
+template <int FMT, int N, int E, bool PF, bool SR>
 cudaError_t launch_scan_ne(const PoolView& pv, const CallView& cv, int warps, int grid,
                            cudaStream_t st)
 {
     using SG = SGeom<N, E>;
     const size_t smem =
         kScanBufs * (size_t)scan_buf_floats(N, cv.scan_chunk, warps * SG::RPW) * sizeof(float);
-    auto kern = scan_kernel<FMT, N, E, PF>;
+    auto kern = scan_kernel<FMT, N, E, PF, SR>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -507,22 +571,22 @@ cudaError_t launch_scan_ne(const PoolView& pv, const CallView& cv, int warps, in
     return cudaGetLastError();
 }
 
-template <int FMT, bool PF>
+template <int FMT, bool PF, bool SR>
 cudaError_t launch_scan_fmt(const PoolView& pv, const CallView& cv, int E, int warps,
                             int grid, cudaStream_t st)
 {
     switch (pv.N) {
-    case 16: return launch_scan_ne<FMT, 16, 16, PF>(pv, cv, warps, grid, st);
-    case 32: return launch_scan_ne<FMT, 32, 32, PF>(pv, cv, warps, grid, st);
+    case 16: return launch_scan_ne<FMT, 16, 16, PF, SR>(pv, cv, warps, grid, st);
+    case 32: return launch_scan_ne<FMT, 32, 32, PF, SR>(pv, cv, warps, grid, st);
     case 64:
-        return E == 64 ? launch_scan_ne<FMT, 64, 64, PF>(pv, cv, warps, grid, st)
-                       : launch_scan_ne<FMT, 64, 32, PF>(pv, cv, warps, grid, st);
+        return E == 64 ? launch_scan_ne<FMT, 64, 64, PF, SR>(pv, cv, warps, grid, st)
+                       : launch_scan_ne<FMT, 64, 32, PF, SR>(pv, cv, warps, grid, st);
     case 128:
-        return E == 64 ? launch_scan_ne<FMT, 128, 64, PF>(pv, cv, warps, grid, st)
-                       : launch_scan_ne<FMT, 128, 32, PF>(pv, cv, warps, grid, st);
+        return E == 64 ? launch_scan_ne<FMT, 128, 64, PF, SR>(pv, cv, warps, grid, st)
+                       : launch_scan_ne<FMT, 128, 32, PF, SR>(pv, cv, warps, grid, st);
     case 256:
-        return E == 64 ? launch_scan_ne<FMT, 256, 64, PF>(pv, cv, warps, grid, st)
-                       : launch_scan_ne<FMT, 256, 32, PF>(pv, cv, warps, grid, st);
+        return E == 64 ? launch_scan_ne<FMT, 256, 64, PF, SR>(pv, cv, warps, grid, st)
+                       : launch_scan_ne<FMT, 256, 32, PF, SR>(pv, cv, warps, grid, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -532,13 +596,26 @@ cudaError_t launch_scan_pf(const PoolView& pv, const CallView& cv, int fmt, int 
                            int g, cudaStream_t st)
 {
     switch (fmt) {
-    case SSQ_F32: return launch_scan_fmt<SSQ_F32, PF>(pv, cv, E, w, g, st);
-    case SSQ_BF16: return launch_scan_fmt<SSQ_BF16, PF>(pv, cv, E, w, g, st);
-    case SSQ_I8_SYM: return launch_scan_fmt<SSQ_I8_SYM, PF>(pv, cv, E, w, g, st);
-    case SSQ_I8_ASYM: return launch_scan_fmt<SSQ_I8_ASYM, PF>(pv, cv, E, w, g, st);
-    case SSQ_I4_SYM: return launch_scan_fmt<SSQ_I4_SYM, PF>(pv, cv, E, w, g, st);
-    case SSQ_I4_ASYM: return launch_scan_fmt<SSQ_I4_ASYM, PF>(pv, cv, E, w, g, st);
+    case SSQ_F32: return launch_scan_fmt<SSQ_F32, PF, false>(pv, cv, E, w, g, st);
+    case SSQ_BF16: return launch_scan_fmt<SSQ_BF16, PF, false>(pv, cv, E, w, g, st);
+    case SSQ_I8_SYM: return launch_scan_fmt<SSQ_I8_SYM, PF, false>(pv, cv, E, w, g, st);
+    case SSQ_I8_ASYM: return launch_scan_fmt<SSQ_I8_ASYM, PF, false>(pv, cv, E, w, g, st);
+    case SSQ_I4_SYM: return launch_scan_fmt<SSQ_I4_SYM, PF, false>(pv, cv, E, w, g, st);
+    case SSQ_I4_ASYM: return launch_scan_fmt<SSQ_I4_ASYM, PF, false>(pv, cv, E, w, g, st);
     default: return cudaErrorInvalidValue;
+    }
+}
+
+// stochastic rounding at every token: the integer formats only
+cudaError_t launch_scan_sr(const PoolView& pv, const CallView& cv, int fmt, int E, int w,
+                           int g, cudaStream_t st)
+{
+    switch (fmt) {
+    case SSQ_I8_SYM: return launch_scan_fmt<SSQ_I8_SYM, false, true>(pv, cv, E, w, g, st);
+    case SSQ_I8_ASYM: return launch_scan_fmt<SSQ_I8_ASYM, false, true>(pv, cv, E, w, g, st);
+    case SSQ_I4_SYM: return launch_scan_fmt<SSQ_I4_SYM, false, true>(pv, cv, E, w, g, st);
+    case SSQ_I4_ASYM: return launch_scan_fmt<SSQ_I4_ASYM, false, true>(pv, cv, E, w, g, st);
+    default: return launch_scan_pf<false>(pv, cv, fmt, E, w, g, st);
     }
 }
 
@@ -571,12 +648,13 @@ ScanPlan scan_plan(int d_state, int headdim, long long batch_heads, int sms)
 }
 
 cudaError_t launch_scan(const PoolView& pv, const CallView& cv, int fmt, const ScanPlan& sp,
-                        bool prefill, cudaStream_t st)
+                        bool prefill, bool sr, cudaStream_t st)
 {
     const long long grid = (long long)cv.batch * (cv.qtiles + cv.ftiles);
     if (grid <= 0) return cudaSuccess;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int g = (int)grid, E = sp.E, w = sp.warps;
+    if (sr) return launch_scan_sr(pv, cv, fmt, E, w, g, st);
     return prefill ? launch_scan_pf<true>(pv, cv, fmt, E, w, g, st)
                    : launch_scan_pf<false>(pv, cv, fmt, E, w, g, st);
 }

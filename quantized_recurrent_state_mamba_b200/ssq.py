@@ -70,8 +70,11 @@ _lib.ssq_dequantize_rows.argtypes = [_CFG, _P, _P, _I, _I, _I, _P, _P]
 _lib.ssq_decode_step.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
 _lib.ssq_scan.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
 _lib.ssq_prefill.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
+_lib.ssq_decode_step_sr.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [ctypes.c_uint64, ctypes.c_uint32, _P]
+_lib.ssq_scan_sr.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [ctypes.c_uint64, ctypes.c_uint32, _P]
 for _f in ("ssq_pool_layout", "ssq_pool_init", "ssq_pool_error", "ssq_quantize_rows",
-           "ssq_dequantize_rows", "ssq_decode_step", "ssq_scan", "ssq_prefill"):
+           "ssq_dequantize_rows", "ssq_decode_step", "ssq_scan", "ssq_prefill",
+           "ssq_decode_step_sr", "ssq_scan_sr"):
     getattr(_lib, _f).restype = _I
 
 
@@ -215,6 +218,32 @@ def ssq_scan(cfg: Config, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y,
         _ptr(C, "C", f, batch * T * G * N), _ptr(dt, "dt", f, batch * T * H),
         _ptr(A, "A", f, H), _ptr(D, "D", f, H), _ptr(y, "y", f, batch * T * H * P),
         _stream(stream)))
+
+
+def ssq_decode_step_sr(cfg: Config, pool, slot_idx, batch, layer0, nl, x, B, C, dt, A, D, y,
+                       seed, step, stream=None):
+    """ssq_decode_step with stochastic rounding (draws keyed by seed, step)."""
+    H, P, N, G = cfg.nheads, cfg.headdim, cfg.d_state, cfg.ngroups
+    f = torch.float32
+    _check(_lib.ssq_decode_step_sr(
+        cfg.ref, _pool_ptr(cfg, pool), _slots(slot_idx, batch), batch, layer0, nl,
+        _ptr(x, "x", f, nl * batch * H * P), _ptr(B, "B", f, nl * batch * G * N),
+        _ptr(C, "C", f, nl * batch * G * N), _ptr(dt, "dt", f, nl * batch * H),
+        _ptr(A, "A", f, nl * H), _ptr(D, "D", f, nl * H), _ptr(y, "y", f, nl * batch * H * P),
+        ctypes.c_uint64(int(seed)), ctypes.c_uint32(int(step)), _stream(stream)))
+
+
+def ssq_scan_sr(cfg: Config, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y, seed,
+                step0, stream=None):
+    """ssq_scan with stochastic rounding, token t at step0 + t."""
+    H, P, N, G = cfg.nheads, cfg.headdim, cfg.d_state, cfg.ngroups
+    f = torch.float32
+    _check(_lib.ssq_scan_sr(
+        cfg.ref, _pool_ptr(cfg, pool), _slots(slot_idx, batch), batch, layer, T,
+        _ptr(x, "x", f, batch * T * H * P), _ptr(B, "B", f, batch * T * G * N),
+        _ptr(C, "C", f, batch * T * G * N), _ptr(dt, "dt", f, batch * T * H),
+        _ptr(A, "A", f, H), _ptr(D, "D", f, H), _ptr(y, "y", f, batch * T * H * P),
+        ctypes.c_uint64(int(seed)), ctypes.c_uint32(int(step0)), _stream(stream)))
 
 
 def ssq_prefill(cfg: Config, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y,
