@@ -262,6 +262,24 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: every rank contributes its own device-timed
+    milliseconds and gets the maximum back (a no-op on one rank)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step, steps, world, ms):
+    """Whole-job GB/s: every rank runs its own replica of the step, so the
+    job moves world x steps x bytes in the slowest rank's time."""
+    return bytes_per_step * steps * world / (ms / 1e3) / 1e9
+
+
 # ---------------------------------------------------------------------------
 # The CPU oracle leg (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
@@ -461,11 +479,8 @@ def run_ours(args, wl, name):
     region_ms = ev[0][0].elapsed_time(ev[-1][1])
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     kern_ms = statistics.mean(launch_ms)
-    if world > 1:
-        tt = torch.tensor([region_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        region_ms = float(tt.item())
-    value = nbytes * K * world / (region_ms / 1e3) / 1e9
+    region_ms = max_over_ranks(region_ms, world, dev)
+    value = job_throughput(nbytes, K, world, region_ms)
     ms_per_step = region_ms / K
 
     # End to end through the public API: every step copies that step's inputs
@@ -523,11 +538,8 @@ def run_ours(args, wl, name):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = nbytes * K * world / (e2e_ms / 1e3) / 1e9
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    e2e_value = job_throughput(nbytes, K, world, e2e_ms)
     e2e_launches = K
     err = ssq.ssq_pool_error(cfg, pool)
 

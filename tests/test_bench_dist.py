@@ -1,0 +1,85 @@
+"""The multi-rank plumbing of bench.py on CPU: two gloo ranks (127.0.0.1),
+each with its own device time, agree on the slowest rank's time and on the
+whole-job throughput; the reference arm works on rank 0 only."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, times, out):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
+                      RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w, r, local = bench.dist_setup()
+        ms = bench.max_over_ranks(times[rank], w, "cpu")
+        value = bench.job_throughput(1e9, 4, w, ms)
+        out[rank] = (w, r, local, ms, value)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_time_and_the_whole_job_bytes():
+    world, port = 2, _free_port()
+    times = [3.0, 5.0]
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_rank, args=(world, port, times, out), nprocs=world,
+                           start_method="spawn")
+        res = dict(out)
+    assert sorted(res) == [0, 1]
+    for rank in (0, 1):
+        w, r, local, ms, value = res[rank]
+        assert (w, r, local) == (2, rank, rank)
+        assert ms == 5.0                                  # the slowest rank
+        assert value == pytest.approx(1e9 * 4 * 2 / 5e-3 / 1e9)
+
+
+def test_single_rank_is_a_no_op():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(2.5, 1, "cpu") == 2.5
+    assert bench.job_throughput(2e9, 10, 1, 1000.0) == pytest.approx(20.0)
+
+
+def _ref_rank(rank, world, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import argparse
+    import io
+    import contextlib
+    import bench
+    from quantized_recurrent_state_mamba_b200 import workloads as W
+    wl = W.tiny()
+    args = argparse.Namespace(steps=1, warmup=0, cpu_budget=0.5)
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        rc = bench.run_reference(args, wl, "tiny")
+    out[rank] = (rc, buf.getvalue())
+
+
+def test_reference_arm_runs_on_rank_0_only():
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_ref_rank, args=(2, out), nprocs=2, start_method="spawn")
+        res = dict(out)
+    assert res[0][0] == 0 and res[1][0] == 0
+    assert '"impl": "reference"' in res[0][1]
+    assert res[1][1] == ""
