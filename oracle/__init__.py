@@ -233,6 +233,19 @@ def scan(cfg: Cfg, st: State, i, x, B, C, dt, A, D):
     return y
 
 
+def step_diag(cfg: Cfg, st: State, i, x, B, C, dt, A, D):
+    """Diagnostics of the decode step pair i would take (state unchanged):
+    [H][P][4] = reversals, readout reversal error, readout rounding error,
+    readout signal."""
+    x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))
+    out = np.zeros((cfg.nheads, cfg.headdim, 4), np.float32)
+    c = cfg.c()
+    lib().oref_step_diag(ctypes.byref(c), ctypes.byref(st.c(i)), _p(x, ctypes.c_float),
+                         _p(B, ctypes.c_float), _p(C, ctypes.c_float), _p(dt, ctypes.c_float),
+                         _p(A, ctypes.c_float), _p(D, ctypes.c_float), _p(out, ctypes.c_float))
+    return out
+
+
 class _SR(ctypes.Structure):
     _fields_ = [("seed", ctypes.c_uint64), ("step", ctypes.c_uint32),
                 ("layer", ctypes.c_uint32), ("slot", ctypes.c_uint32)]

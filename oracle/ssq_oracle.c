@@ -450,6 +450,80 @@ void oref_scan_sr(const oref_cfg* c, oref_state* st, const oref_sr* r, int T,
     }
 }
 
+/* Diagnostics of one decode step ("ssm-state-quantization" README, Findings
+ * 4 and 5): for every row, without changing the state, the step that
+ * oref_step would take is evaluated and
+ *   diag[4r+0] = reversals: entries whose applied increment e + w opposes
+ *                the new input w = fl(dt*x)*B_n (w != 0 and e + w of the
+ *                other sign), e = fl(deq - s') the rounding error, e + w in
+ *                fp32 (the decision is taken in fp32 on both sides);
+ *   diag[4r+1] = sum over reversed entries of C_n * e_n (the reversal error
+ *                seen by the readout);
+ *   diag[4r+2] = sum over all entries of C_n * e_n (the readout-visible
+ *                rounding error: y from the stored state minus y from s');
+ *   diag[4r+3] = sum over all entries of C_n * s'_n (the readout signal).
+ * Sums in double.  fp rows are not rounded: zeros but the signal. */
+void oref_step_diag(const oref_cfg* c, const oref_state* st, const float* x,
+                    const float* B, const float* C, const float* dt,
+                    const float* A, const float* D, float* diag)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state, G = c->ngroups;
+    const int heads_per_group = H / G;
+    float* s = (float*)malloc(sizeof(float) * (size_t)N);
+    float* sn = (float*)malloc(sizeof(float) * (size_t)N);
+    float* w = (float*)malloc(sizeof(float) * (size_t)N);
+    float* deq = (float*)malloc(sizeof(float) * (size_t)N);
+    int32_t* q = (int32_t*)malloc(sizeof(int32_t) * (size_t)N);
+    (void)D;
+    for (int h = 0; h < H; ++h) {
+        const int g = h / heads_per_group;
+        const float lam = oref_lambda(dt[h], A[h]);
+        const float* Bg = B + (size_t)g * N;
+        const float* Cg = C + (size_t)g * N;
+        const int quant = oref_row_is_quant(c, h);
+        for (int p = 0; p < P; ++p) {
+            const int r = h * P + p;
+            if (quant) {
+                oref_dequantize_row(c->fmt, N, st->q + (size_t)r * N, st->delta[r],
+                                    st->zero[r], s);
+            } else {
+                memcpy(s, st->val + (size_t)r * N, sizeof(float) * (size_t)N);
+            }
+            const float dtx = dt[h] * x[r];
+            for (int n = 0; n < N; ++n) {
+                w[n] = dtx * Bg[n];
+                sn[n] = fmaf(lam, s[n], w[n]);
+            }
+            double rev = 0.0, rev_err = 0.0, tot_err = 0.0, signal = 0.0;
+            for (int n = 0; n < N; ++n) signal += (double)Cg[n] * (double)sn[n];
+            if (quant) {
+                float dl, z;
+                oref_quantize_row(c->fmt, N, sn, q, &dl, &z);
+                oref_dequantize_row(c->fmt, N, q, dl, z, deq);
+                for (int n = 0; n < N; ++n) {
+                    const float e = deq[n] - sn[n];
+                    const float inc = e + w[n];
+                    const int reversed = (w[n] > 0.0f && inc < 0.0f) || (w[n] < 0.0f && inc > 0.0f);
+                    tot_err += (double)Cg[n] * (double)e;
+                    if (reversed) {
+                        rev += 1.0;
+                        rev_err += (double)Cg[n] * (double)e;
+                    }
+                }
+            }
+            diag[4 * (size_t)r + 0] = (float)rev;
+            diag[4 * (size_t)r + 1] = (float)rev_err;
+            diag[4 * (size_t)r + 2] = (float)tot_err;
+            diag[4 * (size_t)r + 3] = (float)signal;
+        }
+    }
+    free(s);
+    free(sn);
+    free(w);
+    free(deq);
+    free(q);
+}
+
 /* Prefill hand-off ("Mamba state quantization for inference", phase-aware
  * benchmarks: prefill computes in FP32 and writes its final state into the
  * packed cache): from the stored state, T tokens of the fp32 recurrence

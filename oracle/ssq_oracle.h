@@ -101,6 +101,10 @@ void  oref_scan(const oref_cfg* c, oref_state* st, int T, const float* x,
                 const float* B, const float* C, const float* dt,
                 const float* A, const float* D, float* y);
 
+void  oref_step_diag(const oref_cfg* c, const oref_state* st, const float* x,
+                     const float* B, const float* C, const float* dt,
+                     const float* A, const float* D, float* diag);
+
 /* Stochastic rounding.  The random draw of entry n of row r (= h*P + p) at
  * a step is 16 bits of Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel
  * random numbers: as easy as 1, 2, 3", SC 2011) with key (seed low, seed

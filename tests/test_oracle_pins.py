@@ -716,3 +716,87 @@ def test_sr_scan_is_steps_with_advancing_counter(oref):
     c = O.State(cfg)
     O.scan(cfg, c, 0, x, B, C, dt, inp["A"], inp["D"])
     assert not np.array_equal(a.q, c.q)
+
+
+# ---------------------------------------------------------------------------
+# Step diagnostics ("ssm-state-quantization" README, Findings 4 and 5)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", QFMTS)
+def test_diag_readout_error_is_the_y_difference(oref, fmt):
+    """The readout-visible rounding error of a row is y read from the stored
+    state minus y read from the unrounded update (the step's y and the f32
+    state's y), and the signal is the latter minus D x."""
+    H, P, N = 3, 8, 32
+    wl = W.Decode("pin", 21, 1, 1, H, P, N, 1, "i8a")
+    inp = wl.inputs()
+    S0 = W.state_pair(21, 0, 0, H * P, N).reshape(1, H, P, N)
+    cfg = O.Cfg(fmt, H, P, N, 1)
+    st = O.state_from_f32(cfg, S0)
+    x, B, C, dt = (inp[k][0, 0] for k in ("x", "B", "C", "dt"))
+    A, D = inp["A"][0], inp["D"][0]
+    diag = O.step_diag(cfg, st, 0, x, B, C, dt, A, D)
+    # the unrounded update: the same step with an f32 state holding deq(q)
+    cf = O.Cfg(O.F32, H, P, N, 1)
+    sf = O.state_from_f32(cf, O.state_to_f32(st))
+    y_unrounded = O.step(cf, sf, 0, x, B, C, dt, A, D)
+    y_stored = O.step(cfg, st, 0, x, B, C, dt, A, D)
+    scale = np.abs(y_unrounded) + 1e-3
+    assert np.all(np.abs((y_stored - y_unrounded) - diag[..., 2]) <= 1e-4 * scale)
+    assert np.all(np.abs(y_unrounded - D[:, None] * x - diag[..., 3]) <= 1e-4 * scale)
+    assert np.all(np.abs(diag[..., 1]) <= np.abs(C).sum() * st.delta.max() + 1e-6)
+
+
+def test_diag_reversal_cases(oref):
+    """Hand-built rows on the int8 asymmetric grid: with the zero state
+    (lambda irrelevant) the update is s' = w, the applied increment is
+    e + w = deq(s') and a reversal is deq of the other sign than w: never,
+    since rounding keeps signs on a grid through 0.  A pure requantize
+    (dt = 0, so w = 0) has no reversals by definition."""
+    H, P, N = 1, 1, 16
+    cfg = O.Cfg(O.I8_ASYM, H, P, N, 1)
+    x = np.ones((H, P), np.float32)
+    A = np.full(H, -1.0, np.float32)
+    D = np.zeros(H, np.float32)
+    C = np.ones((1, N), np.float32)
+    dt = np.ones(H, np.float32)
+    rng = np.random.default_rng(3)
+    B = rng.standard_normal((1, N)).astype(np.float32)
+    st = O.State(cfg)
+    diag = O.step_diag(cfg, st, 0, x, B, C, dt, A, D)
+    assert diag[0, 0, 0] == 0
+    st2 = O.state_from_f32(cfg, rng.standard_normal((1, H, P, N)).astype(np.float32))
+    diag2 = O.step_diag(cfg, st2, 0, x, B, C, np.zeros(H, np.float32), A, D)
+    assert diag2[0, 0, 0] == 0 and diag2[0, 0, 1] == 0
+
+
+@pytest.mark.parametrize("fmt", QFMTS)
+def test_diag_reversals_from_the_step_results(oref, fmt):
+    """Reversal count and reversal readout error recomputed from what the
+    plain step produces (the stored state after oref_step, the unrounded
+    update of an f32 state, and w = fl(dt x) B): an entry reverses when the
+    applied increment (stored - s') + w has the other sign than w."""
+    H, P, N = 4, 8, 32
+    wl = W.Decode("pin", 22, 1, 1, H, P, N, 1, "i8a")
+    inp = wl.inputs()
+    S0 = (W.state_pair(22, 0, 0, H * P, N).reshape(1, H, P, N) * 0.05).astype(np.float32)
+    cfg = O.Cfg(fmt, H, P, N, 1)
+    st = O.state_from_f32(cfg, S0)
+    x, B, C, dt = (inp[k][0, 0] for k in ("x", "B", "C", "dt"))
+    A, D = inp["A"][0], inp["D"][0]
+    diag = O.step_diag(cfg, st, 0, x, B, C, dt, A, D)
+    cf = O.Cfg(O.F32, H, P, N, 1)
+    sf = O.state_from_f32(cf, O.state_to_f32(st))
+    O.step(cf, sf, 0, x, B, C, dt, A, D)
+    s_new = O.state_to_f32(sf)[0]                       # s' per entry
+    O.step(cfg, st, 0, x, B, C, dt, A, D)
+    stored = O.state_to_f32(st)[0]
+    w = (dt[:, None].astype(np.float32) * x).astype(np.float32)[..., None] * B[0][None, None, :]
+    w = w.astype(np.float32)
+    e = (stored - s_new).astype(np.float32)
+    inc = (e + w).astype(np.float32)
+    rev = ((w > 0) & (inc < 0)) | ((w < 0) & (inc > 0))
+    assert np.array_equal(rev.sum(axis=-1), diag[..., 0].astype(int))
+    rev_err = np.where(rev, C[0][None, None, :].astype(np.float64) * e, 0.0).sum(axis=-1)
+    assert np.all(np.abs(rev_err - diag[..., 1]) <= 1e-5 * (np.abs(diag[..., 3]) + 1e-3))
+    assert rev.sum() > 0                     # the small state makes reversals common
