@@ -198,6 +198,31 @@ SSQ_API ssq_status ssq_dequantize_rows(const ssq_config* cfg, const void* pool,
                                int layer0, int nl, float* S_out,
                                cudaStream_t stream);
 
+/* Diagnostics of one decode step, read-only ("ssm-state-quantization"
+ * README, Findings 4 and 5: a reversal is a step where rounding moves a
+ * state entry against the new input; the reversal error as seen by the
+ * readout, relative to the readout signal, is the reported correlate).  For
+ * every row the step ssq_decode_step would take is evaluated (same update
+ * s' = fma(lambda, s, w), w = fl(fl(dt*x)*B_n), same refit and nearest
+ * rounding) and, with e_n = fl(deq_n - s'_n) the rounding error, four fp32
+ * numbers are written:
+ *   [0] reversals: entries with w_n != 0 whose increment fl(e_n + w_n) has
+ *       the other sign than w_n
+ *   [1] sum over the reversed entries of C_n e_n
+ *   [2] sum over all entries of C_n e_n
+ *   [3] the readout signal, sum over all entries of C_n s'_n
+ * Rows stored as fp32 / bf16 are not rounded: [0..2] = 0.  The pool is not
+ * changed; y and D are not involved (the D*x term does not see the state).
+ *   x, B, C, dt, A, slot_idx  as ssq_decode_step
+ *   diag  device fp32 [nl][batch][nheads][headdim][4], natural head order,
+ *         16-byte aligned; rows of a request whose slot index is out of
+ *         range are not written (the pool's error word records it). */
+SSQ_API ssq_status ssq_decode_diag(const ssq_config* cfg, const void* pool,
+                           const int32_t* slot_idx, int batch, int layer0,
+                           int nl, const float* x, const float* B,
+                           const float* C, const float* dt, const float* A,
+                           float* diag, cudaStream_t stream);
+
 /* One decode token for a batch of live requests over nl layers, in one
  * launch: the fused read -> recurrence -> refit -> requantize -> write-back
  * -> readout of "Mamba state quantization for inference" (mixed-precision

@@ -288,6 +288,39 @@ ssq_status ssq_dequantize_rows(const ssq_config* cfg, const void* pool,
     return SSQ_OK;
 }
 
+ssq_status ssq_decode_diag(const ssq_config* cfg, const void* pool, const int32_t* slot_idx,
+                           int batch, int layer0, int nl, const float* x, const float* B,
+                           const float* C, const float* dt, const float* A, float* diag,
+                           cudaStream_t stream)
+{
+    ssq::PoolView pv;
+    ssq_layout L;
+    SSQ_TRY(make_pool_view(cfg, const_cast<void*>(pool), &pv, &L));
+    SSQ_TRY(check_batch(cfg, slot_idx, batch, layer0, nl));
+    SSQ_TRY(need(x, "x", 4));
+    SSQ_TRY(need(B, "B", 16));
+    SSQ_TRY(need(C, "C", 16));
+    SSQ_TRY(need(dt, "dt", 4));
+    SSQ_TRY(need(A, "A", 4));
+    SSQ_TRY(need(diag, "diag", 16));
+    if (batch == 0) return SSQ_OK;
+    ssq::CallView cv;
+    memset(&cv, 0, sizeof(cv));
+    cv.slot_idx = slot_idx;
+    cv.batch = batch;
+    cv.layer0 = layer0;
+    cv.nl = nl;
+    cv.x = x;
+    cv.B = B;
+    cv.C = C;
+    cv.dt = dt;
+    cv.A = A;
+    fill_tiles(pv, &cv, ssq::rows_per_tile(cfg->d_state), ssq::rows_per_tile(cfg->d_state));
+    cudaError_t e = ssq::launch_diag(pv, cv, (int)cfg->fmt, diag, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "diag launch");
+    return SSQ_OK;
+}
+
 }  // extern "C"
 
 namespace {

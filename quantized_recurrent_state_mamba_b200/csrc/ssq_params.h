@@ -57,6 +57,10 @@ cudaError_t launch_quantize(const PoolView& pv, const CallView& cv, int fmt,
                             cudaStream_t stream);
 cudaError_t launch_dequantize(const PoolView& pv, const CallView& cv, int fmt,
                               cudaStream_t stream);
+// Step diagnostics (read-only): per row {reversals, reversal error, total
+// rounding error, readout signal} as float4 in [nl][batch][H][P] order.
+cudaError_t launch_diag(const PoolView& pv, const CallView& cv, int fmt, float* diag,
+                        cudaStream_t stream);
 // How the scan splits its rows: entries per lane, warps per CTA, rows per
 // CTA, CTAs per head, tokens per staged chunk, dynamic shared memory.
 struct ScanPlan {

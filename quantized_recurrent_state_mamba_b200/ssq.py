@@ -72,9 +72,10 @@ _lib.ssq_scan.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
 _lib.ssq_prefill.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
 _lib.ssq_decode_step_sr.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [ctypes.c_uint64, ctypes.c_uint32, _P]
 _lib.ssq_scan_sr.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [ctypes.c_uint64, ctypes.c_uint32, _P]
+_lib.ssq_decode_diag.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 6 + [_P]
 for _f in ("ssq_pool_layout", "ssq_pool_init", "ssq_pool_error", "ssq_quantize_rows",
            "ssq_dequantize_rows", "ssq_decode_step", "ssq_scan", "ssq_prefill",
-           "ssq_decode_step_sr", "ssq_scan_sr"):
+           "ssq_decode_step_sr", "ssq_scan_sr", "ssq_decode_diag"):
     getattr(_lib, _f).restype = _I
 
 
@@ -205,6 +206,21 @@ def ssq_decode_step(cfg: Config, pool, slot_idx, batch, layer0, nl, x, B, C, dt,
         _ptr(C, "C", f, nl * batch * G * N), _ptr(dt, "dt", f, nl * batch * H),
         _ptr(A, "A", f, nl * H), _ptr(D, "D", f, nl * H),
         _ptr(y, "y", f, nl * batch * H * P), _stream(stream)))
+
+
+def ssq_decode_diag(cfg: Config, pool, slot_idx, batch, layer0, nl, x, B, C, dt, A, diag,
+                    stream=None):
+    """Read-only diagnostics of one decode step: diag [nl][batch][H][P][4] =
+    (reversals, reversal error seen by the readout, total rounding error
+    seen by the readout, readout signal).  Other layouts as ssq_decode_step."""
+    H, P, N, G = cfg.nheads, cfg.headdim, cfg.d_state, cfg.ngroups
+    f = torch.float32
+    _check(_lib.ssq_decode_diag(
+        cfg.ref, _pool_ptr(cfg, pool), _slots(slot_idx, batch), batch, layer0, nl,
+        _ptr(x, "x", f, nl * batch * H * P), _ptr(B, "B", f, nl * batch * G * N),
+        _ptr(C, "C", f, nl * batch * G * N), _ptr(dt, "dt", f, nl * batch * H),
+        _ptr(A, "A", f, nl * H), _ptr(diag, "diag", f, nl * batch * H * P * 4),
+        _stream(stream)))
 
 
 def ssq_scan(cfg: Config, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D, y, stream=None):

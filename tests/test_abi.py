@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(ssq):
     syms = declared_symbols()
-    assert len(syms) == 12, syms
+    assert len(syms) == 13, syms
     lib = ctypes.CDLL(ssq.LIB_PATH)
     for s in syms:
         assert hasattr(lib, s), f"libssq.so does not export {s}"
