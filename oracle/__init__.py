@@ -73,6 +73,8 @@ def lib():
         _lib.oref_bf16_round.argtypes = [ctypes.c_float]
         _lib.oref_sr_u16.restype = ctypes.c_uint32
         _lib.oref_sr_u16.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        _lib.oref_fp16_round.restype = ctypes.c_float
+        _lib.oref_fp16_round.argtypes = [ctypes.c_float]
     return _lib
 
 
@@ -356,4 +358,116 @@ def decode_batch(cfg: Cfg, st: State, nl, batch, x, B, C, dt, A, D):
                             _p(C, ctypes.c_float), _p(dt, ctypes.c_float),
                             _p(A, ctypes.c_float), _p(D, ctypes.c_float),
                             _p(y, ctypes.c_float))
+    return y
+
+
+# ---------------------------------------------------------------------------
+# DAMP mixed-tier state ("Mamba state quantization for inference", "Mixed
+# precision spends bits on persistent channels")
+# ---------------------------------------------------------------------------
+
+class _DampCfg(ctypes.Structure):
+    _fields_ = [("nheads", ctypes.c_int), ("headdim", ctypes.c_int),
+                ("d_state", ctypes.c_int), ("ngroups", ctypes.c_int),
+                ("n_protected", ctypes.c_int), ("chan", ctypes.POINTER(ctypes.c_int32))]
+
+
+class _DampState(ctypes.Structure):
+    _fields_ = [("hi", ctypes.POINTER(ctypes.c_float)),
+                ("q", ctypes.POINTER(ctypes.c_int32)),
+                ("delta", ctypes.POINTER(ctypes.c_float)),
+                ("zero", ctypes.POINTER(ctypes.c_float))]
+
+
+@dataclass
+class DampCfg:
+    """One layer's tiered state: nheads heads of d_state key channels, each a
+    rotated value vector of headdim entries; chan[h][m] = key channel at
+    position m, the first n_protected positions in FP16."""
+    nheads: int
+    headdim: int
+    d_state: int
+    ngroups: int
+    n_protected: int
+    chan: np.ndarray
+
+    def c(self):
+        self._chan = np.ascontiguousarray(self.chan, dtype=np.int32).reshape(
+            self.nheads, self.d_state)
+        return _DampCfg(self.nheads, self.headdim, self.d_state, self.ngroups,
+                        self.n_protected, _p(self._chan, ctypes.c_int32))
+
+
+class DampState:
+    """Tiered state of ``count`` (layer, request) pairs."""
+
+    def __init__(self, cfg: DampCfg, count: int = 1):
+        H, P, N, K = cfg.nheads, cfg.headdim, cfg.d_state, cfg.n_protected
+        self.cfg = cfg
+        self.count = count
+        self.hi = np.zeros((count, H, K, P), np.float32)
+        self.q = np.zeros((count, H, N - K, P), np.int32)
+        self.delta = np.zeros((count, H, N - K), np.float32)
+        self.zero = np.zeros((count, H, N - K), np.float32)
+
+    def c(self, i):
+        return _DampState(_p(self.hi[i], ctypes.c_float), _p(self.q[i], ctypes.c_int32),
+                          _p(self.delta[i], ctypes.c_float), _p(self.zero[i], ctypes.c_float))
+
+    def copy(self):
+        s = DampState(self.cfg, self.count)
+        for k in ("hi", "q", "delta", "zero"):
+            getattr(s, k)[...] = getattr(self, k)
+        return s
+
+
+def hadamard(v):
+    """Sylvester-Hadamard rotation of a vector of power-of-two length:
+    out[k] = sum_p (-1)^popcount(k&p) v[p], summed in double, rounded once."""
+    v = _f32(v)
+    out = np.zeros_like(v)
+    lib().oref_hadamard(v.shape[0], _p(v, ctypes.c_float), 1, _p(out, ctypes.c_float))
+    return out
+
+
+def fp16_round(v):
+    v = _f32(v)
+    out = np.empty_like(v)
+    f = lib().oref_fp16_round
+    for i, x in enumerate(v.reshape(-1)):
+        out.reshape(-1)[i] = f(float(x))
+    return out
+
+
+def damp_from_f32(cfg: DampCfg, S):
+    """S[count][H][P][N] (or [H][P][N]) fp32 -> DampState."""
+    S = _f32(S)
+    if S.ndim == 3:
+        S = S[None]
+    st = DampState(cfg, S.shape[0])
+    c = cfg.c()
+    for i in range(S.shape[0]):
+        lib().oref_damp_from_f32(ctypes.byref(c), _p(S[i], ctypes.c_float),
+                                 ctypes.byref(st.c(i)))
+    return st
+
+
+def damp_to_f32(st: DampState):
+    cfg = st.cfg
+    out = np.zeros((st.count, cfg.nheads, cfg.headdim, cfg.d_state), np.float32)
+    c = cfg.c()
+    for i in range(st.count):
+        lib().oref_damp_to_f32(ctypes.byref(c), ctypes.byref(st.c(i)), _p(out[i], ctypes.c_float))
+    return out
+
+
+def damp_step(cfg: DampCfg, st: DampState, i, x, B, C, dt, A, D):
+    """One decode step of pair i on the tiered state.  x[H][P], B/C[G][N],
+    dt/A/D[H]; returns y[H][P]."""
+    x, B, C, dt, A, D = map(_f32, (x, B, C, dt, A, D))
+    y = np.zeros((cfg.nheads, cfg.headdim), np.float32)
+    c = cfg.c()
+    lib().oref_damp_step(ctypes.byref(c), ctypes.byref(st.c(i)), _p(x, ctypes.c_float),
+                         _p(B, ctypes.c_float), _p(C, ctypes.c_float), _p(dt, ctypes.c_float),
+                         _p(A, ctypes.c_float), _p(D, ctypes.c_float), _p(y, ctypes.c_float))
     return y

@@ -636,3 +636,192 @@ void oref_decode_batch(const oref_cfg* c, int nl, int batch,
         }
     }
 }
+
+/* ------------------------------------------------------------------------
+ * DAMP mixed-tier state ("Mamba state quantization for inference", "Mixed
+ * precision spends bits on persistent channels"): a Hadamard transform along
+ * each key channel's value dimension; the protected key channels kept in
+ * FP16, the others in INT8 with a scale and a zero point; the selected
+ * channels permuted into one contiguous region; per token the low tier is
+ * reconstructed, the recurrence runs in FP32, new quantization parameters
+ * are derived and the packed state is written back.
+ *
+ * Readings (listed in the design notes):
+ *   - state S[h][p][n]: p the value dimension (head_dim), n the key channel
+ *     (d_state).  Key channel n of head h is the vector S[h][.][n] of
+ *     length P, rotated to t[k] = sum_p H[k][p] S[h][p][n] with H the +-1
+ *     Sylvester-Hadamard matrix, H[k][p] = (-1)^popcount(k & p), P a power of
+ *     two; the sum is taken in double in the order p = 0..P-1 and rounded
+ *     once to fp32.  The inverse is S[p] = (1/P) sum_k H[p][k] t[k].
+ *   - chan[h][m]: position m -> key channel; positions 0..K-1 are the
+ *     protected (FP16) tier, K..N-1 the INT8 tier.  The selection is an
+ *     input (its calibration needs data).
+ *   - INT8 tier: each position's P rotated values form one group with the
+ *     asymmetric 8-bit grid of the row quantizer (fp32 step and zero point):
+ *     8 + 64/P bits per value, 9 at P = 64.
+ *   - FP16 tier: fp32 -> fp16 round to nearest even (overflow to inf).
+ *   - The recurrence is linear, so it runs on the rotated state with the
+ *     rotated input: t' = fma(lambda, t, fl(fl(dt * xr[k]) * B[n])), xr the
+ *     rotation of x (as above).  y reads the stored state:
+ *     y[p] = D x[p] + (1/P) sum_k H[p][k] sum_m C[chan[m]] t'_m[k], in
+ *     double, rounded once.
+ * ---------------------------------------------------------------------- */
+
+static int hsign(int a, int b)
+{
+    return (__builtin_popcount((unsigned)(a & b)) & 1) ? -1 : 1;
+}
+
+/* out[k] = fl32(sum_p H[k][p] v[p * stride]), double, order p. */
+void oref_hadamard(int P, const float* v, int stride, float* out)
+{
+    for (int k = 0; k < P; ++k) {
+        double acc = 0.0;
+        for (int p = 0; p < P; ++p) {
+            const double t = (double)v[(size_t)p * stride];
+            acc = hsign(k, p) > 0 ? acc + t : acc - t;
+        }
+        out[k] = (float)acc;
+    }
+}
+
+float oref_fp16_round(float v)
+{
+    return (float)(_Float16)v;
+}
+
+/* Tiers of one head from the rotated values t[m][k] (position-major). */
+static void damp_store_head(const oref_damp_cfg* c, const float* t, float* hi, int32_t* q,
+                            float* delta, float* zero)
+{
+    const int P = c->headdim, N = c->d_state, K = c->n_protected;
+    for (int m = 0; m < K; ++m)
+        for (int k = 0; k < P; ++k)
+            hi[(size_t)m * P + k] = oref_fp16_round(t[(size_t)m * P + k]);
+    for (int m = K; m < N; ++m) {
+        const int i = m - K;
+        oref_quantize_row(OREF_I8_ASYM, P, t + (size_t)m * P, q + (size_t)i * P, &delta[i],
+                          &zero[i]);
+    }
+}
+
+/* The stored (rotated) values of one head, position-major t[m][k]. */
+static void damp_load_head(const oref_damp_cfg* c, const float* hi, const int32_t* q,
+                           const float* delta, const float* zero, float* t)
+{
+    const int P = c->headdim, N = c->d_state, K = c->n_protected;
+    for (int m = 0; m < K; ++m)
+        for (int k = 0; k < P; ++k) t[(size_t)m * P + k] = hi[(size_t)m * P + k];
+    for (int m = K; m < N; ++m) {
+        const int i = m - K;
+        oref_dequantize_row(OREF_I8_ASYM, P, q + (size_t)i * P, delta[i], zero[i],
+                            t + (size_t)m * P);
+    }
+}
+
+static void damp_head_ptrs(const oref_damp_cfg* c, const oref_damp_state* st, int h,
+                           float** hi, int32_t** q, float** delta, float** zero)
+{
+    const int P = c->headdim, N = c->d_state, K = c->n_protected;
+    *hi = st->hi + (size_t)h * K * P;
+    *q = st->q + (size_t)h * (N - K) * P;
+    *delta = st->delta + (size_t)h * (N - K);
+    *zero = st->zero + (size_t)h * (N - K);
+}
+
+/* S[H][P][N] fp32 -> tiers: rotate every key channel, then store. */
+void oref_damp_from_f32(const oref_damp_cfg* c, const float* S, oref_damp_state* st)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state;
+    float* t = (float*)malloc(sizeof(float) * (size_t)N * P);
+    for (int h = 0; h < H; ++h) {
+        const int32_t* ch = c->chan + (size_t)h * N;
+        for (int m = 0; m < N; ++m)
+            oref_hadamard(P, S + (size_t)h * P * N + ch[m], N, t + (size_t)m * P);
+        float *hi, *dl, *z;
+        int32_t* q;
+        damp_head_ptrs(c, st, h, &hi, &q, &dl, &z);
+        damp_store_head(c, t, hi, q, dl, z);
+    }
+    free(t);
+}
+
+/* Tiers -> S[H][P][N] fp32: reconstruct, rotate back (double, order k,
+ * then the exact 1/P), round once. */
+void oref_damp_to_f32(const oref_damp_cfg* c, const oref_damp_state* st, float* S)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state;
+    float* t = (float*)malloc(sizeof(float) * (size_t)N * P);
+    for (int h = 0; h < H; ++h) {
+        float *hi, *dl, *z;
+        int32_t* q;
+        damp_head_ptrs(c, st, h, &hi, &q, &dl, &z);
+        damp_load_head(c, hi, q, dl, z, t);
+        const int32_t* ch = c->chan + (size_t)h * N;
+        for (int m = 0; m < N; ++m) {
+            for (int p = 0; p < P; ++p) {
+                double acc = 0.0;
+                for (int k = 0; k < P; ++k) {
+                    const double v = (double)t[(size_t)m * P + k];
+                    acc = hsign(p, k) > 0 ? acc + v : acc - v;
+                }
+                S[(size_t)h * P * N + (size_t)p * N + ch[m]] = (float)(acc / (double)P);
+            }
+        }
+    }
+    free(t);
+}
+
+/* One decode step of one (layer, request) on the tiered state.
+ * x[H][P], B/C[G][N], dt/A/D[H], y[H][P]. */
+void oref_damp_step(const oref_damp_cfg* c, oref_damp_state* st, const float* x,
+                    const float* B, const float* C, const float* dt, const float* A,
+                    const float* D, float* y)
+{
+    const int H = c->nheads, P = c->headdim, N = c->d_state, G = c->ngroups;
+    const int heads_per_group = H / G;
+    float* t = (float*)malloc(sizeof(float) * (size_t)N * P);
+    float* xr = (float*)malloc(sizeof(float) * (size_t)P);
+    double* yr = (double*)malloc(sizeof(double) * (size_t)P);
+    for (int h = 0; h < H; ++h) {
+        const int g = h / heads_per_group;
+        const float lam = oref_lambda(dt[h], A[h]);
+        const int32_t* ch = c->chan + (size_t)h * N;
+        float *hi, *dl, *z;
+        int32_t* q;
+        damp_head_ptrs(c, st, h, &hi, &q, &dl, &z);
+        /* reconstruct the low tier (and read the FP16 tier) */
+        damp_load_head(c, hi, q, dl, z, t);
+        /* the input, rotated like the state */
+        oref_hadamard(P, x + (size_t)h * P, 1, xr);
+        /* the recurrence in FP32 */
+        for (int m = 0; m < N; ++m) {
+            const float b = B[(size_t)g * N + ch[m]];
+            for (int k = 0; k < P; ++k) {
+                const float dtx = dt[h] * xr[k];
+                const float w = dtx * b;
+                t[(size_t)m * P + k] = fmaf(lam, t[(size_t)m * P + k], w);
+            }
+        }
+        /* new quantization parameters, packed state written back */
+        damp_store_head(c, t, hi, q, dl, z);
+        /* readout from the stored state, rotated back */
+        damp_load_head(c, hi, q, dl, z, t);
+        for (int k = 0; k < P; ++k) {
+            double acc = 0.0;
+            for (int m = 0; m < N; ++m)
+                acc += (double)C[(size_t)g * N + ch[m]] * (double)t[(size_t)m * P + k];
+            yr[k] = acc;
+        }
+        for (int p = 0; p < P; ++p) {
+            double acc = 0.0;
+            for (int k = 0; k < P; ++k) acc += (double)hsign(p, k) * yr[k];
+            acc /= (double)P;
+            acc += (double)D[h] * (double)x[(size_t)h * P + p];
+            y[(size_t)h * P + p] = (float)acc;
+        }
+    }
+    free(t);
+    free(xr);
+    free(yr);
+}

@@ -141,6 +141,33 @@ void  oref_decode_batch(const oref_cfg* c, int nl, int batch,
                         const float* C, const float* dt, const float* A,
                         const float* D, float* y);
 
+/* DAMP mixed-tier state ("Mamba state quantization for inference", "Mixed
+ * precision spends bits on persistent channels").  Per head, position m of
+ * chan[h][.] names a key channel; positions 0..n_protected-1 hold the
+ * channel's Hadamard-rotated value vector in FP16 (hi, widened to fp32
+ * here), the others in INT8 on the asymmetric grid (codes q, step delta,
+ * zero point zero per position).  headdim a power of two. */
+typedef struct {
+    int nheads, headdim, d_state, ngroups;
+    int n_protected;
+    const int32_t* chan;     /* [nheads][d_state], a permutation per head */
+} oref_damp_cfg;
+
+typedef struct {
+    float* hi;       /* [nheads][K][P] */
+    int32_t* q;      /* [nheads][N-K][P] */
+    float* delta;    /* [nheads][N-K] */
+    float* zero;     /* [nheads][N-K] */
+} oref_damp_state;
+
+void  oref_hadamard(int P, const float* v, int stride, float* out);
+float oref_fp16_round(float v);
+void  oref_damp_from_f32(const oref_damp_cfg* c, const float* S, oref_damp_state* st);
+void  oref_damp_to_f32(const oref_damp_cfg* c, const oref_damp_state* st, float* S);
+void  oref_damp_step(const oref_damp_cfg* c, oref_damp_state* st, const float* x,
+                     const float* B, const float* C, const float* dt, const float* A,
+                     const float* D, float* y);
+
 #ifdef __cplusplus
 }
 #endif

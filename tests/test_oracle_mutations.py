@@ -40,6 +40,24 @@ MUTATIONS = {
     "sr_ignores_draw": ("const double k = floor(p + (double)u16[n] / 65536.0);",
                         "const double k = floor(p + 0.5);"),
     "sr_no_low_clamp": ("            if (c < 0.0f) c = 0.0f;\n", ""),
+    "diag_err_sign": ("const float e = deq[n] - sn[n];", "const float e = sn[n] - deq[n];"),
+    "diag_rev_same_sign": ("(w[n] > 0.0f && inc < 0.0f) || (w[n] < 0.0f && inc > 0.0f)",
+                           "(w[n] > 0.0f && inc > 0.0f) || (w[n] < 0.0f && inc < 0.0f)"),
+    "diag_rev_error_only": ("const float inc = e + w[n];", "const float inc = e;"),
+    "diag_signal_before_update": ("signal += (double)Cg[n] * (double)sn[n];",
+                                  "signal += (double)Cg[n] * (double)s[n];"),
+    "damp_hadamard_sign": ("return (__builtin_popcount((unsigned)(a & b)) & 1) ? -1 : 1;",
+                           "return (__builtin_popcount((unsigned)(a | b)) & 1) ? -1 : 1;"),
+    "damp_y_no_inverse_scale": ("acc /= (double)P;", "acc /= 1.0;"),
+    "damp_input_not_rotated": ("const float dtx = dt[h] * xr[k];",
+                               "const float dtx = dt[h] * x[(size_t)h * P + k];"),
+    "damp_B_by_position": ("const float b = B[(size_t)g * N + ch[m]];",
+                           "const float b = B[(size_t)g * N + m];"),
+    "damp_protected_not_fp16": ("hi[(size_t)m * P + k] = oref_fp16_round(t[(size_t)m * P + k]);",
+                                "hi[(size_t)m * P + k] = t[(size_t)m * P + k];"),
+    "damp_y_before_store": ("        /* readout from the stored state, rotated back */\n"
+                            "        damp_load_head(c, hi, q, dl, z, t);\n",
+                            "        /* readout from the stored state, rotated back */\n"),
 }
 
 
@@ -59,6 +77,7 @@ def test_pins_catch_mutation(name):
         env = dict(os.environ, SSQ_ORACLE_LIB=so)
         r = subprocess.run(
             [sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-             os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+             os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+             os.path.join(ROOT, "tests", "test_oracle_damp.py")],
             cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
         assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"
