@@ -46,6 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 SM_MAX_MHZ = 1965.0        # B200 maximum SM clock, used when NVML is unavailable
 SCAN_FP32_OPS = 6          # algorithmic fp32 operations per element-token of the scan
 PREFILL_FP32_OPS = 3       # ... of the prefill hand-off: w = dtx*B, the fma, C*s
+DAMP_PROTECTED = 16        # DAMP layout: key channels per head kept in FP16
 
 
 # ---------------------------------------------------------------------------
@@ -73,6 +74,7 @@ def workload(name):
         "scan_370m_mid": lambda: W.scan_370m("mid"),
         "prefill_370m_all": lambda: W.scan_370m("all"),
         "prefill_370m_mid": lambda: W.scan_370m("mid"),
+        "decode_130m_damp": lambda: W.decode_130m_damp(),
     }
     if name not in table:
         raise SystemExit(f"unknown workload {name}; choose from {sorted(table)}")
@@ -99,6 +101,18 @@ def decode_bytes(wl):
                     + (1 - qfrac) * row_state_bytes("f32", wl.d_state))
     io = rows * 4 * 2 + wl.nl * wl.batch * (2 * wl.ngroups * wl.d_state + wl.nheads) * 4
     return int(round(2 * state + io))
+
+
+def damp_bytes(wl, K=DAMP_PROTECTED):
+    """Algorithmic bytes of one DAMP decode step: every head block (FP16
+    tier, INT8 codes, {step, zero point} per INT8 channel) read and written
+    once, x / B / C / dt read and y written once, the channel map of the
+    layers read once."""
+    P, N = wl.headdim, wl.d_state
+    head = 2 * K * P + (N - K) * P + 8 * (N - K)
+    units = wl.nl * wl.batch * wl.nheads
+    io = units * P * 4 * 2 + wl.nl * wl.batch * (2 * wl.ngroups * N + wl.nheads) * 4
+    return int(2 * units * head + io + wl.nl * wl.nheads * N * 4)
 
 
 def scan_bytes(wl):
@@ -311,6 +325,30 @@ def oracle_decode_sample(wl, budget_s):
     return sec, per_pair * npairs, npairs
 
 
+def oracle_damp_sample(wl, budget_s, K=DAMP_PROTECTED):
+    """Time the oracle's DAMP step on the first (layer, request) pairs."""
+    import oracle as O
+    H, P, N, G = wl.nheads, wl.headdim, wl.d_state, wl.ngroups
+    chan = W.damp_channels(wl.seed, wl.nl, H, N)
+    inp = wl.inputs()
+    per_pair = damp_bytes(wl, K) / (wl.nl * wl.batch)
+    ocs = [O.DampCfg(H, P, N, G, K, chan[l]) for l in range(wl.nl)]
+    st = O.damp_from_f32(ocs[0], wl.state_pair(0, 0).reshape(H, P, N))
+    t = time.perf_counter()
+    O.damp_step(ocs[0], st, 0, inp["x"][0, 0], inp["B"][0, 0], inp["C"][0, 0],
+                inp["dt"][0, 0], inp["A"][0], inp["D"][0])
+    one = max(time.perf_counter() - t, 1e-6)
+    npairs = int(max(1, min(wl.nl * wl.batch, budget_s / one)))
+    pairs = [(i // wl.batch, i % wl.batch) for i in range(npairs)]
+    sts = [O.damp_from_f32(ocs[l], wl.state_pair(l, b).reshape(H, P, N)) for (l, b) in pairs]
+    t = time.perf_counter()
+    for st, (l, b) in zip(sts, pairs):
+        O.damp_step(ocs[l], st, 0, inp["x"][l, b], inp["B"][l, b], inp["C"][l, b],
+                    inp["dt"][l, b], inp["A"][l], inp["D"][l])
+    sec = time.perf_counter() - t
+    return sec, per_pair * npairs, npairs
+
+
 def oracle_scan_sample(wl, budget_s, prefill=False):
     import oracle as O
     H, P, N = wl.nheads, wl.headdim, wl.d_state
@@ -346,9 +384,12 @@ def cpu_leg(wl, budget_s, name=""):
                   f"(request 0 onward), single thread")
         rsps = n / sec
     else:
-        sec, nbytes, n = oracle_decode_sample(wl, budget_s)
-        sample = (f"{n} of {wl.nl * wl.batch} (layer, request) pairs of one decode step "
-                  f"(layer-major from pair 0), single thread")
+        damp = name.endswith("_damp")
+        sample_fn = oracle_damp_sample if damp else oracle_decode_sample
+        sec, nbytes, n = sample_fn(wl, budget_s)
+        sample = (f"{n} of {wl.nl * wl.batch} (layer, request) pairs of one "
+                  f"{'DAMP ' if damp else ''}decode step (layer-major from pair 0), "
+                  f"single thread")
         rsps = n / sec
     return {"value": nbytes / sec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": sample, "seconds": round(sec, 3),
@@ -404,17 +445,34 @@ def run_ours(args, wl, name):
             dist.barrier()
 
     is_scan = isinstance(wl, W.Scan)
-    fmt = wl.fmt
+    damp = name.endswith("_damp")
+    fmt = f"damp-k{DAMP_PROTECTED}" if damp else wl.fmt
     H, P, N, G = wl.nheads, wl.headdim, wl.d_state, wl.ngroups
     n_layers = 1 if is_scan else wl.nl
-    cfg = ssq.Config(n_layers=n_layers, n_slots=wl.batch, nheads=H, headdim=P, d_state=N,
-                     ngroups=G, fmt=fmt, head_mask=wl.head_mask)
-    pool = ssq.alloc_pool(cfg, dev)
     inp = wl.inputs()
     d = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in inp.items()}
+    if damp:
+        cfg = ssq.DampConfig(n_layers=n_layers, n_slots=wl.batch, nheads=H, headdim=P,
+                             d_state=N, ngroups=G, n_protected=DAMP_PROTECTED)
+        pool = ssq.damp_alloc_pool(cfg, dev)
+        chan = torch.from_numpy(W.damp_channels(wl.seed, n_layers, H, N)).to(dev)
+        pool_error = lambda: ssq.ssq_damp_pool_error(cfg, pool)  # noqa: E731
+    else:
+        cfg = ssq.Config(n_layers=n_layers, n_slots=wl.batch, nheads=H, headdim=P, d_state=N,
+                         ngroups=G, fmt=fmt, head_mask=wl.head_mask)
+        pool = ssq.alloc_pool(cfg, dev)
+        pool_error = lambda: ssq.ssq_pool_error(cfg, pool)  # noqa: E731
 
     # initial state
-    if not is_scan and wl.init != "zero":
+    if damp:
+        for l in range(wl.nl):
+            S = np.empty((wl.batch, wl.rows, N), np.float32)
+            for b in range(wl.batch):
+                S[b] = wl.state_pair(l, b)
+            ssq.ssq_damp_quantize(cfg, pool, chan, None, wl.batch, l, 1,
+                                  torch.from_numpy(S).to(dev))
+        torch.cuda.synchronize()
+    elif not is_scan and wl.init != "zero":
         for l in range(wl.nl):
             S = np.empty((wl.batch, wl.rows, N), np.float32)
             for b in range(wl.batch):
@@ -434,6 +492,14 @@ def run_ours(args, wl, name):
             scan_fn(cfg, pool, None, wl.batch, 0, wl.T, d["x"], d["B"], d["C"], d["dt"],
                     d["A"], d["D"], y)
         units = wl.batch * wl.T          # request-tokens
+    elif damp:
+        y = torch.empty((wl.nl, wl.batch, H, P), device=dev)
+        nbytes = damp_bytes(wl)
+
+        def step():
+            ssq.ssq_damp_decode_step(cfg, pool, chan, None, wl.batch, 0, wl.nl, d["x"], d["B"],
+                                     d["C"], d["dt"], d["A"], d["D"], y)
+        units = wl.batch * wl.nl
     else:
         y = torch.empty((wl.nl, wl.batch, H, P), device=dev)
         nbytes = decode_bytes(wl)
@@ -456,7 +522,7 @@ def run_ours(args, wl, name):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    if ssq.ssq_pool_error(cfg, pool) != 0:
+    if pool_error() != 0:
         raise SystemExit("device error word set during warm-up")
 
     sampler = ClockSampler(local)
@@ -515,6 +581,9 @@ def run_ours(args, wl, name):
         if is_scan:
             scan_fn(cfg, pool, None, wl.batch, 0, wl.T, t["x"], t["B"], t["C"], t["dt"],
                     d["A"], d["D"], yb[kk], stream=s_c)
+        elif damp:
+            ssq.ssq_damp_decode_step(cfg, pool, chan, None, wl.batch, 0, wl.nl, t["x"], t["B"],
+                                     t["C"], t["dt"], d["A"], d["D"], yb[kk], stream=s_c)
         else:
             ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, t["x"], t["B"], t["C"],
                                 t["dt"], d["A"], d["D"], yb[kk], stream=s_c)
@@ -541,7 +610,7 @@ def run_ours(args, wl, name):
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
     e2e_value = job_throughput(nbytes, K, world, e2e_ms)
     e2e_launches = K
-    err = ssq.ssq_pool_error(cfg, pool)
+    err = pool_error()
 
     peak, peak_kind = measured_peaks()
     achieved = nbytes / (kern_ms / 1e3) / 1e9

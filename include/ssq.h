@@ -105,6 +105,7 @@ typedef enum {
 #define SSQ_DEVERR_SLOT 0x1u      /* slot index outside [0, n_slots)      */
 #define SSQ_DEVERR_NONFINITE 0x2u /* a row's updated values were not finite */
 #define SSQ_DEVERR_TIMEOUT 0x4u   /* a pipeline wait gave up (about 1 s)    */
+#define SSQ_DEVERR_CHANNEL 0x8u   /* a DAMP channel map entry outside [0, d_state) */
 
 /* Shape of one state pool.  Every request slot holds the state of n_layers
  * layers; each layer holds nheads x headdim rows of d_state entries.
@@ -304,6 +305,109 @@ SSQ_API ssq_status ssq_prefill(const ssq_config* cfg, void* pool,
                        const float* x, const float* B, const float* C,
                        const float* dt, const float* A, const float* D,
                        float* y, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * DAMP mixed-tier state ("Mamba state quantization for inference", "Mixed
+ * precision spends bits on persistent channels").  Per head the state
+ * S[p][n] (p < headdim the value dimension, n < d_state the key channel) is
+ * held as d_state key channels, each the Hadamard-rotated value vector
+ *     t[k] = sum_p H[k][p] S[p][n],   H[k][p] = (-1)^popcount(k & p)
+ * (the +-1 Sylvester-Hadamard matrix of order headdim; H/sqrt(headdim) is
+ * orthonormal), summed in double in the order p = 0..headdim-1 and rounded
+ * once to fp32.  A per-(layer, head) channel map chan[m] (a permutation of
+ * 0..d_state-1, chosen by calibration outside the library) puts the
+ * n_protected protected channels first: positions m < n_protected keep t in
+ * FP16 (round to nearest even), the others in INT8 on the asymmetric grid of
+ * the row quantizer above, one {fp32 Delta, fp32 z} per position over its
+ * headdim values.  Bits per value: 16 for the FP16 tier, 8 + 64/headdim for
+ * the INT8 tier (9 at headdim 64); 16 of 128 channels protected at headdim
+ * 64 gives 9.875.
+ *
+ * The decode step runs the recurrence on the rotated state with the rotated
+ * input xr = H x (rounded as above):
+ *     t'_m[k] = fma(lambda, t_m[k], fl(fl(dt*xr[k]) * B[chan[m]]))
+ * FP16 positions store fp16(t'), INT8 positions refit and round t' exactly
+ * as ssq_decode_step rounds a row (codes, steps, zero points and FP16 values
+ * are bit-identical to a scalar evaluation); y is read from the stored state
+ * and rotated back:
+ *     y[p] = D x[p] + (1/headdim) sum_k H[p][k] sum_m C[chan[m]] t'_m[k]
+ * accumulated in fp32.
+ *
+ * Shapes: headdim 16, 32, 64 or 128; d_state 16 .. 256, a multiple of 16;
+ * 0 <= n_protected <= d_state; ngroups divides nheads.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int n_layers;
+    int n_slots;
+    int nheads;
+    int headdim;
+    int d_state;
+    int ngroups;
+    int n_protected;
+} ssq_damp_config;
+
+/* Byte layout of a DAMP pool.
+ *   pool = [header: SSQ_POOL_HEADER_BYTES][slot 0] ... [slot n_slots-1]
+ *   slot = [layer 0] ... [layer n_layers-1], layer = [head 0] ... [head H-1]
+ *   head block (head_bytes, a multiple of 16), offsets within it:
+ *     hi_off    [n_protected][headdim] fp16, position-major
+ *     codes_off [d_state - n_protected][headdim] uint8 codes
+ *     meta_off  [d_state - n_protected] x {float Delta, float z}
+ *   each region starts on a 16-byte boundary; slot_bytes is rounded up to
+ *   SSQ_POOL_ALIGN.  Header: the uint32 error word at byte 0.  An all-zero
+ *   pool is the all-zero state.  bits_per_value counts codes, FP16 values
+ *   and meta per state value (padding excluded). */
+typedef struct {
+    size_t pool_bytes;
+    size_t header_bytes;
+    size_t slot_bytes;
+    size_t layer_bytes;
+    size_t head_bytes;
+    size_t hi_off, codes_off, meta_off;
+    double bits_per_value;
+} ssq_damp_layout;
+
+/* Host only; no CUDA call.  SSQ_ERR_UNSUPPORTED for shapes outside the
+ * list above. */
+SSQ_API ssq_status ssq_damp_pool_layout(const ssq_damp_config* cfg, ssq_damp_layout* out);
+
+/* Write fp32 states into DAMP pool slots (the prefill hand-off for this
+ * layout): every key channel rotated, then stored in its tier.
+ *   chan      device int32 [n_layers][nheads][d_state]: the channel map of
+ *             every layer (a permutation per head; an entry outside
+ *             [0, d_state) sets SSQ_DEVERR_CHANNEL and that head is skipped)
+ *   S         device fp32 [nl][batch][nheads][headdim][d_state], 16-B aligned
+ *   slot_idx  device int32 [batch] or NULL; layers layer0 .. layer0+nl-1
+ * pool: device, aligned to SSQ_POOL_ALIGN. */
+SSQ_API ssq_status ssq_damp_quantize(const ssq_damp_config* cfg, void* pool,
+                             const int32_t* chan, const int32_t* slot_idx,
+                             int batch, int layer0, int nl, const float* S,
+                             cudaStream_t stream);
+
+/* Read DAMP pool slots back as fp32: S[p][chan[m]] = (1/headdim) sum_k
+ * H[p][k] t_m[k], summed in double in the order k, rounded once.
+ *   S_out  device fp32 [nl][batch][nheads][headdim][d_state] */
+SSQ_API ssq_status ssq_damp_dequantize(const ssq_damp_config* cfg, const void* pool,
+                               const int32_t* chan, const int32_t* slot_idx,
+                               int batch, int layer0, int nl, float* S_out,
+                               cudaStream_t stream);
+
+/* One decode token on DAMP pool slots over nl layers.  x, B, C, dt, A, D, y
+ * and slot_idx as ssq_decode_step; chan as ssq_damp_quantize.  The pool's
+ * error word (read with ssq_pool_error or ssq_damp_pool_error) records bad
+ * slots (the request is skipped), bad channel maps (the head is skipped) and
+ * non-finite INT8 groups. */
+SSQ_API ssq_status ssq_damp_decode_step(const ssq_damp_config* cfg, void* pool,
+                                const int32_t* chan, const int32_t* slot_idx,
+                                int batch, int layer0, int nl, const float* x,
+                                const float* B, const float* C,
+                                const float* dt, const float* A,
+                                const float* D, float* y, cudaStream_t stream);
+
+/* Read the DAMP pool's error word into *flags (HOST) and clear it; this
+ * call synchronises `stream`. */
+SSQ_API ssq_status ssq_damp_pool_error(const ssq_damp_config* cfg, void* pool,
+                               uint32_t* flags, cudaStream_t stream);
 
 /* Static string for a status code. */
 SSQ_API const char* ssq_status_string(ssq_status s);

@@ -477,3 +477,187 @@ ssq_status ssq_prefill(const ssq_config* cfg, void* pool, const int32_t* slot_id
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// DAMP mixed-tier pool
+// ---------------------------------------------------------------------------
+namespace {
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+ssq_status damp_layout_of(const ssq_damp_config* c, ssq_damp_layout* L)
+{
+    if (!c) return fail(SSQ_ERR_INVALID_ARG, "cfg is NULL");
+    if (c->n_layers < 1 || c->n_slots < 1)
+        return fail(SSQ_ERR_INVALID_ARG, "n_layers %d / n_slots %d < 1", c->n_layers, c->n_slots);
+    if (c->nheads < 1 || c->nheads > SSQ_MAX_HEADS)
+        return fail(SSQ_ERR_INVALID_ARG, "nheads %d outside [1, %d]", c->nheads, SSQ_MAX_HEADS);
+    if (c->headdim != 16 && c->headdim != 32 && c->headdim != 64 && c->headdim != 128)
+        return fail(SSQ_ERR_UNSUPPORTED, "headdim %d not 16, 32, 64 or 128", c->headdim);
+    if (c->d_state < 16 || c->d_state > 256 || c->d_state % 16 != 0)
+        return fail(SSQ_ERR_UNSUPPORTED, "d_state %d not a multiple of 16 in [16, 256]",
+                    c->d_state);
+    if (c->ngroups < 1 || c->nheads % c->ngroups != 0)
+        return fail(SSQ_ERR_INVALID_ARG, "ngroups %d does not divide nheads %d", c->ngroups,
+                    c->nheads);
+    if (c->n_protected < 0 || c->n_protected > c->d_state)
+        return fail(SSQ_ERR_INVALID_ARG, "n_protected %d outside [0, %d]", c->n_protected,
+                    c->d_state);
+    const size_t P = (size_t)c->headdim, N = (size_t)c->d_state, K = (size_t)c->n_protected;
+    memset(L, 0, sizeof(*L));
+    L->header_bytes = SSQ_POOL_HEADER_BYTES;
+    L->hi_off = 0;
+    L->codes_off = align_up(2 * K * P, 16);
+    L->meta_off = L->codes_off + align_up((N - K) * P, 16);
+    L->head_bytes = align_up(L->meta_off + 8 * (N - K), 16);
+    L->layer_bytes = L->head_bytes * (size_t)c->nheads;
+    L->slot_bytes = align_up(L->layer_bytes * (size_t)c->n_layers, SSQ_POOL_ALIGN);
+    L->pool_bytes = L->header_bytes + L->slot_bytes * (size_t)c->n_slots;
+    L->bits_per_value = (16.0 * K * P + 8.0 * (N - K) * P + 64.0 * (N - K)) / (double)(N * P);
+    return SSQ_OK;
+}
+
+ssq_status damp_view(const ssq_damp_config* c, void* pool, const int32_t* chan,
+                     ssq::DampView* dv)
+{
+    ssq_damp_layout L;
+    SSQ_TRY(damp_layout_of(c, &L));
+    SSQ_TRY(need(pool, "pool", SSQ_POOL_ALIGN));
+    SSQ_TRY(need(chan, "chan", 4));
+    memset(dv, 0, sizeof(*dv));
+    dv->pool = static_cast<uint8_t*>(pool);
+    dv->header_bytes = (long long)L.header_bytes;
+    dv->slot_bytes = (long long)L.slot_bytes;
+    dv->layer_bytes = (long long)L.layer_bytes;
+    dv->head_bytes = (long long)L.head_bytes;
+    dv->hi_off = (int)L.hi_off;
+    dv->codes_off = (int)L.codes_off;
+    dv->meta_off = (int)L.meta_off;
+    dv->n_slots = c->n_slots;
+    dv->n_layers = c->n_layers;
+    dv->H = c->nheads;
+    dv->P = c->headdim;
+    dv->N = c->d_state;
+    dv->G = c->ngroups;
+    dv->hpg = c->nheads / c->ngroups;
+    dv->K = c->n_protected;
+    dv->chan = chan;
+    return SSQ_OK;
+}
+
+ssq_status damp_check_batch(const ssq_damp_config* c, const int32_t* slot_idx, int batch,
+                            int layer0, int nl)
+{
+    if (batch < 0) return fail(SSQ_ERR_INVALID_ARG, "batch %d < 0", batch);
+    if (nl < 1) return fail(SSQ_ERR_INVALID_ARG, "nl %d < 1", nl);
+    if (layer0 < 0 || (long long)layer0 + nl > c->n_layers)
+        return fail(SSQ_ERR_INVALID_ARG, "layers [%d, %d) outside [0, %d)", layer0,
+                    layer0 + nl, c->n_layers);
+    if (!slot_idx && batch > c->n_slots)
+        return fail(SSQ_ERR_INVALID_ARG, "batch %d > n_slots %d with identity slots", batch,
+                    c->n_slots);
+    if (slot_idx && !aligned(slot_idx, 4))
+        return fail(SSQ_ERR_ALIGNMENT, "slot_idx not 4-byte aligned");
+    return SSQ_OK;
+}
+
+ssq::DampCall damp_call(const int32_t* slot_idx, int batch, int layer0, int nl)
+{
+    ssq::DampCall dc;
+    memset(&dc, 0, sizeof(dc));
+    dc.slot_idx = slot_idx;
+    dc.batch = batch;
+    dc.layer0 = layer0;
+    dc.nl = nl;
+    return dc;
+}
+
+}  // namespace
+
+extern "C" {
+
+ssq_status ssq_damp_pool_layout(const ssq_damp_config* cfg, ssq_damp_layout* out)
+{
+    if (!out) return fail(SSQ_ERR_INVALID_ARG, "out is NULL");
+    return damp_layout_of(cfg, out);
+}
+
+ssq_status ssq_damp_quantize(const ssq_damp_config* cfg, void* pool, const int32_t* chan,
+                             const int32_t* slot_idx, int batch, int layer0, int nl,
+                             const float* S, cudaStream_t stream)
+{
+    ssq::DampView dv;
+    SSQ_TRY(damp_view(cfg, pool, chan, &dv));
+    SSQ_TRY(damp_check_batch(cfg, slot_idx, batch, layer0, nl));
+    SSQ_TRY(need(S, "S", 16));
+    if (batch == 0) return SSQ_OK;
+    ssq::DampCall dc = damp_call(slot_idx, batch, layer0, nl);
+    dc.S_in = S;
+    cudaError_t e = ssq::launch_damp(dv, dc, 1, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "damp quantize launch");
+    return SSQ_OK;
+}
+
+ssq_status ssq_damp_dequantize(const ssq_damp_config* cfg, const void* pool,
+                               const int32_t* chan, const int32_t* slot_idx, int batch,
+                               int layer0, int nl, float* S_out, cudaStream_t stream)
+{
+    ssq::DampView dv;
+    SSQ_TRY(damp_view(cfg, const_cast<void*>(pool), chan, &dv));
+    SSQ_TRY(damp_check_batch(cfg, slot_idx, batch, layer0, nl));
+    SSQ_TRY(need(S_out, "S_out", 16));
+    if (batch == 0) return SSQ_OK;
+    ssq::DampCall dc = damp_call(slot_idx, batch, layer0, nl);
+    dc.S_out = S_out;
+    cudaError_t e = ssq::launch_damp(dv, dc, 2, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "damp dequantize launch");
+    return SSQ_OK;
+}
+
+ssq_status ssq_damp_decode_step(const ssq_damp_config* cfg, void* pool, const int32_t* chan,
+                                const int32_t* slot_idx, int batch, int layer0, int nl,
+                                const float* x, const float* B, const float* C,
+                                const float* dt, const float* A, const float* D, float* y,
+                                cudaStream_t stream)
+{
+    ssq::DampView dv;
+    SSQ_TRY(damp_view(cfg, pool, chan, &dv));
+    SSQ_TRY(damp_check_batch(cfg, slot_idx, batch, layer0, nl));
+    SSQ_TRY(need(x, "x", 4));
+    SSQ_TRY(need(B, "B", 4));
+    SSQ_TRY(need(C, "C", 4));
+    SSQ_TRY(need(dt, "dt", 4));
+    SSQ_TRY(need(A, "A", 4));
+    SSQ_TRY(need(D, "D", 4));
+    SSQ_TRY(need(y, "y", 4));
+    if (batch == 0) return SSQ_OK;
+    ssq::DampCall dc = damp_call(slot_idx, batch, layer0, nl);
+    dc.x = x;
+    dc.B = B;
+    dc.C = C;
+    dc.dt = dt;
+    dc.A = A;
+    dc.D = D;
+    dc.y = y;
+    cudaError_t e = ssq::launch_damp(dv, dc, 0, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "damp decode launch");
+    return SSQ_OK;
+}
+
+ssq_status ssq_damp_pool_error(const ssq_damp_config* cfg, void* pool, uint32_t* flags,
+                               cudaStream_t stream)
+{
+    ssq_damp_layout L;
+    SSQ_TRY(damp_layout_of(cfg, &L));
+    SSQ_TRY(need(pool, "pool", SSQ_POOL_ALIGN));
+    if (!flags) return fail(SSQ_ERR_INVALID_ARG, "flags is NULL");
+    uint32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, pool, sizeof(v), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(pool, 0, sizeof(v), stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the pool error word");
+    *flags = v;
+    return SSQ_OK;
+}
+
+}  // extern "C"

@@ -47,6 +47,35 @@ struct CallView {
     float* S_out;              // dequantize_rows output
 };
 
+// The DAMP mixed-tier pool: every (slot, layer, head) owns one block of
+// head_bytes: FP16 tier at hi_off ([K][P] halves), INT8 codes at codes_off
+// ([N-K][P] bytes), meta at meta_off ([N-K] x {float Delta, float z}).
+struct DampView {
+    uint8_t* pool;
+    long long header_bytes, slot_bytes, layer_bytes, head_bytes;
+    int hi_off, codes_off, meta_off;
+    int n_slots, n_layers;
+    int H, P, N, G, hpg, K;
+    const int32_t* chan;       // [n_layers][H][N] position -> key channel
+};
+
+struct DampCall {
+    const int32_t* slot_idx;
+    int batch, layer0, nl;
+    const float* x;
+    const float* B;
+    const float* C;
+    const float* dt;
+    const float* A;
+    const float* D;
+    float* y;
+    const float* S_in;
+    float* S_out;
+};
+
+// which: 0 decode step, 1 quantize (hand-off from fp32), 2 dequantize
+cudaError_t launch_damp(const DampView& dv, const DampCall& dc, int which, cudaStream_t stream);
+
 // Host-side launchers (one per kernel family); each returns the CUDA error of
 // its launch.  The decode and rows kernels run a grid-stride loop over tiles
 // on a grid sized to the device's resident capacity.

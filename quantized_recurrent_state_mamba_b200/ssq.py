@@ -30,8 +30,10 @@ FORMATS = {"f32": SSQ_F32, "bf16": SSQ_BF16, "i8s": SSQ_I8_SYM, "i8a": SSQ_I8_AS
 SSQ_DEVERR_SLOT = 0x1
 SSQ_DEVERR_NONFINITE = 0x2
 SSQ_DEVERR_TIMEOUT = 0x4
+SSQ_DEVERR_CHANNEL = 0x8
 SSQ_MAX_HEADS = 512
 SSQ_POOL_HEADER_BYTES = 256
+SSQ_POOL_ALIGN = 256
 
 
 class SsqError(RuntimeError):
@@ -55,6 +57,17 @@ class ssq_layout(ctypes.Structure):
         ("n_quant_heads", ctypes.c_int), ("n_fp_heads", ctypes.c_int)]
 
 
+class ssq_damp_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "n_layers", "n_slots", "nheads", "headdim", "d_state", "ngroups", "n_protected")]
+
+
+class ssq_damp_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "pool_bytes", "header_bytes", "slot_bytes", "layer_bytes", "head_bytes", "hi_off",
+        "codes_off", "meta_off")] + [("bits_per_value", ctypes.c_double)]
+
+
 _P = ctypes.c_void_p
 _CFG = ctypes.POINTER(ssq_config)
 _I = ctypes.c_int
@@ -73,9 +86,17 @@ _lib.ssq_prefill.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
 _lib.ssq_decode_step_sr.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [ctypes.c_uint64, ctypes.c_uint32, _P]
 _lib.ssq_scan_sr.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 7 + [ctypes.c_uint64, ctypes.c_uint32, _P]
 _lib.ssq_decode_diag.argtypes = [_CFG, _P, _P, _I, _I, _I] + [_P] * 6 + [_P]
+_DCFG = ctypes.POINTER(ssq_damp_config)
+_lib.ssq_damp_pool_layout.argtypes = [_DCFG, ctypes.POINTER(ssq_damp_layout)]
+_lib.ssq_damp_quantize.argtypes = [_DCFG, _P, _P, _P, _I, _I, _I, _P, _P]
+_lib.ssq_damp_dequantize.argtypes = [_DCFG, _P, _P, _P, _I, _I, _I, _P, _P]
+_lib.ssq_damp_decode_step.argtypes = [_DCFG, _P, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
+_lib.ssq_damp_pool_error.argtypes = [_DCFG, _P, ctypes.POINTER(ctypes.c_uint32), _P]
 for _f in ("ssq_pool_layout", "ssq_pool_init", "ssq_pool_error", "ssq_quantize_rows",
            "ssq_dequantize_rows", "ssq_decode_step", "ssq_scan", "ssq_prefill",
-           "ssq_decode_step_sr", "ssq_scan_sr", "ssq_decode_diag"):
+           "ssq_decode_step_sr", "ssq_scan_sr", "ssq_decode_diag", "ssq_damp_pool_layout",
+           "ssq_damp_quantize", "ssq_damp_dequantize", "ssq_damp_decode_step",
+           "ssq_damp_pool_error"):
     getattr(_lib, _f).restype = _I
 
 
@@ -274,6 +295,82 @@ def ssq_prefill(cfg: Config, pool, slot_idx, batch, layer, T, x, B, C, dt, A, D,
         _ptr(C, "C", f, batch * T * G * N), _ptr(dt, "dt", f, batch * T * H),
         _ptr(A, "A", f, H), _ptr(D, "D", f, H), _ptr(y, "y", f, batch * T * H * P),
         _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# DAMP mixed-tier pool
+# ---------------------------------------------------------------------------
+
+class DampConfig:
+    """A DAMP pool configuration (ssq_damp_config)."""
+
+    def __init__(self, n_layers, n_slots, nheads, headdim, d_state, ngroups=1, n_protected=16):
+        self.c = ssq_damp_config(int(n_layers), int(n_slots), int(nheads), int(headdim),
+                                 int(d_state), int(ngroups), int(n_protected))
+
+    def __getattr__(self, name):
+        return getattr(self.__dict__["c"], name)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def ssq_damp_pool_layout(cfg: DampConfig):
+    L = ssq_damp_layout()
+    _check(_lib.ssq_damp_pool_layout(cfg.ref, ctypes.byref(L)))
+    return {name: getattr(L, name) for name, _ in ssq_damp_layout._fields_}
+
+
+def damp_alloc_pool(cfg: DampConfig, device="cuda"):
+    """A zeroed DAMP pool (the all-zero state)."""
+    L = ssq_damp_pool_layout(cfg)
+    return torch.zeros(L["pool_bytes"], dtype=torch.uint8, device=device)
+
+
+def _damp_ptrs(cfg, pool, chan):
+    L = ssq_damp_pool_layout(cfg)
+    return (_ptr(pool, "pool", torch.uint8, L["pool_bytes"]),
+            _ptr(chan, "chan", torch.int32, cfg.n_layers * cfg.nheads * cfg.d_state))
+
+
+def ssq_damp_quantize(cfg: DampConfig, pool, chan, slot_idx, batch, layer0, nl, S, stream=None):
+    """S: fp32 [nl][batch][nheads][headdim][d_state] -> DAMP pool slots."""
+    pp, cp = _damp_ptrs(cfg, pool, chan)
+    n = nl * batch * cfg.nheads * cfg.headdim * cfg.d_state
+    _check(_lib.ssq_damp_quantize(cfg.ref, pp, cp, _slots(slot_idx, batch), batch, layer0, nl,
+                                  _ptr(S, "S", torch.float32, n), _stream(stream)))
+
+
+def ssq_damp_dequantize(cfg: DampConfig, pool, chan, slot_idx, batch, layer0, nl, S_out,
+                        stream=None):
+    pp, cp = _damp_ptrs(cfg, pool, chan)
+    n = nl * batch * cfg.nheads * cfg.headdim * cfg.d_state
+    _check(_lib.ssq_damp_dequantize(cfg.ref, pp, cp, _slots(slot_idx, batch), batch, layer0,
+                                    nl, _ptr(S_out, "S_out", torch.float32, n),
+                                    _stream(stream)))
+
+
+def ssq_damp_decode_step(cfg: DampConfig, pool, chan, slot_idx, batch, layer0, nl, x, B, C, dt,
+                         A, D, y, stream=None):
+    """One decode token on DAMP slots; layouts as ssq_decode_step."""
+    H, P, N, G = cfg.nheads, cfg.headdim, cfg.d_state, cfg.ngroups
+    f = torch.float32
+    pp, cp = _damp_ptrs(cfg, pool, chan)
+    _check(_lib.ssq_damp_decode_step(
+        cfg.ref, pp, cp, _slots(slot_idx, batch), batch, layer0, nl,
+        _ptr(x, "x", f, nl * batch * H * P), _ptr(B, "B", f, nl * batch * G * N),
+        _ptr(C, "C", f, nl * batch * G * N), _ptr(dt, "dt", f, nl * batch * H),
+        _ptr(A, "A", f, nl * H), _ptr(D, "D", f, nl * H), _ptr(y, "y", f, nl * batch * H * P),
+        _stream(stream)))
+
+
+def ssq_damp_pool_error(cfg: DampConfig, pool, stream=None) -> int:
+    v = ctypes.c_uint32(0)
+    L = ssq_damp_pool_layout(cfg)
+    _check(_lib.ssq_damp_pool_error(cfg.ref, _ptr(pool, "pool", torch.uint8, L["pool_bytes"]),
+                                    ctypes.byref(v), _stream(stream)))
+    return int(v.value)
 
 
 def ssq_status_string(status) -> str:

@@ -25,7 +25,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 _TAGS = {"x": 1, "B": 2, "C": 3, "dt": 4, "A": 5, "D": 6, "S0": 7,
-         "Aband": 8}
+         "Aband": 8, "chan": 9}
 
 # softplus(-2): the median of dt = softplus(N(-2, 1)).
 MEDIAN_DT = math.log1p(math.exp(-2.0))
@@ -216,3 +216,21 @@ def sweep_serving(fmt="i8a", batch=256, nl=30):
     return Decode(f"serving sweep L{nl} b{batch} H32 P128 N128 {fmt}",
                   seed=4, nl=nl, batch=batch, nheads=32, headdim=128,
                   d_state=128, ngroups=1, fmt=fmt, init="zero")
+
+
+def damp_channels(seed, n_layers, nheads, d_state):
+    """A channel map per (layer, head) for the DAMP mixed-tier layout:
+    int32 [n_layers][nheads][d_state], a seeded random permutation each (the
+    calibration that would rank channels needs data; any permutation costs
+    the same)."""
+    rng = _rng(seed, "chan")
+    return np.stack([np.stack([rng.permutation(d_state) for _ in range(nheads)])
+                     for _ in range(n_layers)]).astype(np.int32)
+
+
+def decode_130m_damp(batch=256, nl=24):
+    """The 130M decode shape for the DAMP layout (16 of 128 key channels in
+    FP16, the rest INT8)."""
+    return Decode(f"mamba2-130m decode L{nl} b{batch} H24 P64 N128 damp K16",
+                  seed=1, nl=nl, batch=batch, nheads=24, headdim=64,
+                  d_state=128, ngroups=1, fmt="i8a")

@@ -130,3 +130,66 @@ class Codec:
         if is_sym(self.fmt):
             out = np.where(out >= 8, out - 16, out)
         return out
+
+
+class DampCodec:
+    """Packing of one (layer, request)'s DAMP state (oracle.DampState arrays
+    hi[H][K][P], q[H][N-K][P], delta/zero[H][N-K]) into the DAMP pool layout
+    of include/ssq.h: per (slot, layer, head) a block of head_bytes with the
+    FP16 tier at hi_off (position-major halves), uint8 codes at codes_off and
+    {float Delta, float z} per INT8 position at meta_off."""
+
+    def __init__(self, nheads, headdim, d_state, n_protected, layout):
+        self.H, self.P, self.N, self.K = nheads, headdim, d_state, n_protected
+        self.L = layout
+
+    def _head(self, slot, layer, h):
+        L = self.L
+        return (L["header_bytes"] + slot * L["slot_bytes"] + layer * L["layer_bytes"]
+                + h * L["head_bytes"])
+
+    def write(self, buf, slot, layer, hi, q, delta, zero):
+        H, P, N, K = self.H, self.P, self.N, self.K
+        L = self.L
+        for h in range(H):
+            o = self._head(slot, layer, h)
+            half = np.asarray(hi[h], np.float32).astype(np.float16).reshape(-1)
+            # hi holds values already on the fp16 grid: the cast is exact
+            assert np.array_equal(half.astype(np.float32), np.asarray(hi[h], np.float32).reshape(-1))
+            hb = half.view(np.uint8)
+            buf[o + L["hi_off"]: o + L["hi_off"] + hb.size] = hb
+            cb = np.asarray(q[h], np.int32).reshape(-1)
+            assert cb.size == 0 or (cb.min() >= 0 and cb.max() <= 255)
+            buf[o + L["codes_off"]: o + L["codes_off"] + cb.size] = cb.astype(np.uint8)
+            meta = np.stack([np.asarray(delta[h], np.float32), np.asarray(zero[h], np.float32)],
+                            axis=1).reshape(-1).view(np.uint8)
+            buf[o + L["meta_off"]: o + L["meta_off"] + meta.size] = meta
+
+    def read(self, buf, slot, layer):
+        H, P, N, K = self.H, self.P, self.N, self.K
+        L = self.L
+        hi = np.zeros((H, K, P), np.float32)
+        q = np.zeros((H, N - K, P), np.int32)
+        delta = np.zeros((H, N - K), np.float32)
+        zero = np.zeros((H, N - K), np.float32)
+        for h in range(H):
+            o = self._head(slot, layer, h)
+            hb = buf[o + L["hi_off"]: o + L["hi_off"] + 2 * K * P].copy()
+            hi[h] = hb.view(np.float16).astype(np.float32).reshape(K, P)
+            q[h] = buf[o + L["codes_off"]: o + L["codes_off"] + (N - K) * P].astype(
+                np.int32).reshape(N - K, P)
+            m = buf[o + L["meta_off"]: o + L["meta_off"] + 8 * (N - K)].copy().view(
+                np.float32).reshape(N - K, 2)
+            delta[h], zero[h] = m[:, 0], m[:, 1]
+        return hi, q, delta, zero
+
+    def read_hi_bits(self, buf, slot, layer):
+        """The FP16 tier as raw uint16 patterns [H][K][P]."""
+        H, P, K = self.H, self.P, self.K
+        L = self.L
+        out = np.zeros((H, K, P), np.uint16)
+        for h in range(H):
+            o = self._head(slot, layer, h)
+            out[h] = buf[o + L["hi_off"]: o + L["hi_off"] + 2 * K * P].copy().view(
+                np.uint16).reshape(K, P)
+        return out

@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(ssq):
     syms = declared_symbols()
-    assert len(syms) == 13, syms
+    assert len(syms) == 18, syms
     lib = ctypes.CDLL(ssq.LIB_PATH)
     for s in syms:
         assert hasattr(lib, s), f"libssq.so does not export {s}"
@@ -181,3 +181,90 @@ def test_no_cpu_fallback_in_product(ssq):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "oref_" not in src, f
+
+
+def test_damp_layout_matches_page_figure(ssq):
+    """"Mamba state quantization for inference", "Mixed precision spends bits
+    on persistent channels": 16 of 128 key channels in FP16 (16 bits), the
+    rest at 9 bits with metadata, 9.875 bits per value on average.  At
+    headdim 64 the INT8 tier's {fp32 step, fp32 zero point} per channel is
+    one bit per value."""
+    cfg = ssq.DampConfig(n_layers=2, n_slots=3, nheads=4, headdim=64, d_state=128, ngroups=1,
+                         n_protected=16)
+    d = ssq.ssq_damp_pool_layout(cfg)
+    assert d["bits_per_value"] == 9.875
+    assert d["hi_off"] == 0 and d["codes_off"] == 16 * 64 * 2
+    assert d["meta_off"] == d["codes_off"] + 112 * 64
+    assert d["head_bytes"] == d["meta_off"] + 112 * 8
+    assert d["head_bytes"] * 8 / (128 * 64) == 9.875       # no padding at this shape
+    assert d["layer_bytes"] == 4 * d["head_bytes"]
+    assert d["slot_bytes"] % ssq.SSQ_POOL_ALIGN == 0 and d["slot_bytes"] >= 2 * d["layer_bytes"]
+    assert d["pool_bytes"] == ssq.SSQ_POOL_HEADER_BYTES + 3 * d["slot_bytes"]
+    # the uniform controls: all INT8 (9 bits), all FP16 (16 bits)
+    for K, bpv in ((0, 9.0), (128, 16.0)):
+        c = ssq.DampConfig(1, 1, 4, 64, 128, 1, K)
+        assert ssq.ssq_damp_pool_layout(c)["bits_per_value"] == bpv
+    # the 130M-shaped pool at batch 256 against its fp32 size: 9.875 / 32
+    c = ssq.DampConfig(24, 256, 24, 64, 128, 1, 16)
+    f = ssq.Config(24, 256, 24, 64, 128, 1, "f32")
+    ratio = (ssq.ssq_damp_pool_layout(c)["pool_bytes"] / ssq.ssq_pool_layout(f)[0]["pool_bytes"])
+    assert abs(ratio - 9.875 / 32) < 1e-4
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(headdim=48), 2), (dict(headdim=256), 2), (dict(d_state=40), 2), (dict(d_state=512), 2),
+    (dict(n_protected=129), 1), (dict(n_protected=-1), 1), (dict(ngroups=3), 1),
+    (dict(nheads=0), 1), (dict(n_layers=0), 1)])
+def test_damp_layout_rejects_bad_configs(ssq, kw, status):
+    base = dict(n_layers=2, n_slots=4, nheads=4, headdim=64, d_state=128, ngroups=2,
+                n_protected=16)
+    base.update(kw)
+    with pytest.raises(ssq.SsqError) as e:
+        ssq.ssq_damp_pool_layout(ssq.DampConfig(**base))
+    assert e.value.status == status
+
+
+def test_damp_entry_points_validate_before_launch(ssq):
+    lib = ssq.raw()
+    cfg = ssq.DampConfig(2, 4, 4, 64, 128, 1, 16)
+    P = ctypes.c_void_p
+    g = 0x10000000
+
+    def step(pool=g, chan=g, slots=None, batch=2, layer0=0, nl=1, x=g):
+        return lib.ssq_damp_decode_step(cfg.ref, P(pool), P(chan), P(slots), batch, layer0, nl,
+                                        P(x), P(g), P(g), P(g), P(g), P(g), P(g), None)
+
+    assert step(pool=g + 16) == ssq.SSQ_ERR_ALIGNMENT
+    assert step(chan=0) == ssq.SSQ_ERR_INVALID_ARG
+    assert step(chan=g + 2) == ssq.SSQ_ERR_ALIGNMENT
+    assert step(x=0) == ssq.SSQ_ERR_INVALID_ARG
+    assert step(batch=5) == ssq.SSQ_ERR_INVALID_ARG
+    assert step(layer0=1, nl=2) == ssq.SSQ_ERR_INVALID_ARG
+    assert step(batch=0) == ssq.SSQ_OK
+    r = lib.ssq_damp_quantize(cfg.ref, P(g), P(g), None, 2, 0, 1, P(g + 8), None)
+    assert r == ssq.SSQ_ERR_ALIGNMENT
+    r = lib.ssq_damp_dequantize(cfg.ref, P(g), P(g), None, 2, 0, 3, P(g), None)
+    assert r == ssq.SSQ_ERR_INVALID_ARG
+
+
+def test_damp_codec_round_trip(ssq):
+    """The tests' DAMP packer writes and reads back an oracle state exactly
+    (host only)."""
+    import oracle as O
+    from poolcodec import DampCodec
+    H, P, N, K = 3, 64, 128, 16
+    cfg = ssq.DampConfig(2, 3, H, P, N, 1, K)
+    L = ssq.ssq_damp_pool_layout(cfg)
+    rng = np.random.default_rng(0)
+    chan = np.stack([rng.permutation(N) for _ in range(H)]).astype(np.int32)
+    st = O.damp_from_f32(O.DampCfg(H, P, N, 1, K, chan),
+                         rng.standard_normal((H, P, N)).astype(np.float32))
+    codec = DampCodec(H, P, N, K, L)
+    buf = np.zeros(L["pool_bytes"], np.uint8)
+    codec.write(buf, 2, 1, st.hi[0], st.q[0], st.delta[0], st.zero[0])
+    hi, q, d, z = codec.read(buf, 2, 1)
+    assert np.array_equal(hi, st.hi[0]) and np.array_equal(q, st.q[0])
+    assert np.array_equal(d, st.delta[0]) and np.array_equal(z, st.zero[0])
+    # the block sits where the layout says: nothing else written
+    o = L["header_bytes"] + 2 * L["slot_bytes"] + 1 * L["layer_bytes"]
+    assert not buf[:o].any() and not buf[o + H * L["head_bytes"]:].any()
