@@ -651,8 +651,11 @@ void oref_decode_batch(const oref_cfg* c, int nl, int batch,
  *     (d_state).  Key channel n of head h is the vector S[h][.][n] of
  *     length P, rotated to t[k] = sum_p H[k][p] S[h][p][n] with H the +-1
  *     Sylvester-Hadamard matrix, H[k][p] = (-1)^popcount(k & p), P a power of
- *     two; the sum is taken in double in the order p = 0..P-1 and rounded
- *     once to fp32.  The inverse is S[p] = (1/P) sum_k H[p][k] t[k].
+ *     two; the sums are formed by the fast Walsh-Hadamard transform in
+ *     double (butterfly stages h = 1, 2, ..., P/2) and rounded once to fp32
+ *     (the stage order fixes the order of the double additions, which
+ *     matters only when a double sum is inexact).  The inverse is
+ *     S[p] = (1/P) sum_k H[p][k] t[k], formed the same way.
  *   - chan[h][m]: position m -> key channel; positions 0..K-1 are the
  *     protected (FP16) tier, K..N-1 the INT8 tier.  The selection is an
  *     input (its calibration needs data).
@@ -672,17 +675,32 @@ static int hsign(int a, int b)
     return (__builtin_popcount((unsigned)(a & b)) & 1) ? -1 : 1;
 }
 
-/* out[k] = fl32(sum_p H[k][p] v[p * stride]), double, order p. */
+/* In-place fast Walsh-Hadamard transform of a[0..P-1] in double (Fino and
+ * Algazi, "Unified matrix treatment of the fast Walsh-Hadamard transform",
+ * IEEE Trans. Computers 1976): stages h = 1, 2, 4, ..., P/2; at each stage
+ * the pair (a[i], a[i+h]), bit h of i clear, becomes (a[i] + a[i+h],
+ * a[i] - a[i+h]).  The result is sum_p H[k][p] a[p] in Sylvester order;
+ * each output is one fixed sequence of double additions. */
+static void fwht_double(int P, double* a)
+{
+    for (int h = 1; h < P; h *= 2)
+        for (int i = 0; i < P; ++i)
+            if ((i & h) == 0) {
+                const double x = a[i], y = a[i + h];
+                a[i] = x + y;
+                a[i + h] = x - y;
+            }
+}
+
+/* out[k] = fl32(sum_p H[k][p] v[p * stride]): the fast transform in double,
+ * rounded once. */
 void oref_hadamard(int P, const float* v, int stride, float* out)
 {
-    for (int k = 0; k < P; ++k) {
-        double acc = 0.0;
-        for (int p = 0; p < P; ++p) {
-            const double t = (double)v[(size_t)p * stride];
-            acc = hsign(k, p) > 0 ? acc + t : acc - t;
-        }
-        out[k] = (float)acc;
-    }
+    double* a = (double*)malloc(sizeof(double) * (size_t)P);
+    for (int p = 0; p < P; ++p) a[p] = (double)v[(size_t)p * stride];
+    fwht_double(P, a);
+    for (int k = 0; k < P; ++k) out[k] = (float)a[k];
+    free(a);
 }
 
 float oref_fp16_round(float v)
@@ -746,12 +764,13 @@ void oref_damp_from_f32(const oref_damp_cfg* c, const float* S, oref_damp_state*
     free(t);
 }
 
-/* Tiers -> S[H][P][N] fp32: reconstruct, rotate back (double, order k,
- * then the exact 1/P), round once. */
+/* Tiers -> S[H][P][N] fp32: reconstruct, rotate back (the fast transform
+ * in double, then the exact 1/P), round once. */
 void oref_damp_to_f32(const oref_damp_cfg* c, const oref_damp_state* st, float* S)
 {
     const int H = c->nheads, P = c->headdim, N = c->d_state;
     float* t = (float*)malloc(sizeof(float) * (size_t)N * P);
+    double* a = (double*)malloc(sizeof(double) * (size_t)P);
     for (int h = 0; h < H; ++h) {
         float *hi, *dl, *z;
         int32_t* q;
@@ -759,17 +778,14 @@ void oref_damp_to_f32(const oref_damp_cfg* c, const oref_damp_state* st, float* 
         damp_load_head(c, hi, q, dl, z, t);
         const int32_t* ch = c->chan + (size_t)h * N;
         for (int m = 0; m < N; ++m) {
-            for (int p = 0; p < P; ++p) {
-                double acc = 0.0;
-                for (int k = 0; k < P; ++k) {
-                    const double v = (double)t[(size_t)m * P + k];
-                    acc = hsign(p, k) > 0 ? acc + v : acc - v;
-                }
-                S[(size_t)h * P * N + (size_t)p * N + ch[m]] = (float)(acc / (double)P);
-            }
+            for (int k = 0; k < P; ++k) a[k] = (double)t[(size_t)m * P + k];
+            fwht_double(P, a);       /* H is symmetric: H^-1 = H / P */
+            for (int p = 0; p < P; ++p)
+                S[(size_t)h * P * N + (size_t)p * N + ch[m]] = (float)(a[p] / (double)P);
         }
     }
     free(t);
+    free(a);
 }
 
 /* One decode step of one (layer, request) on the tiered state.

@@ -49,6 +49,8 @@ MUTATIONS = {
     "damp_hadamard_sign": ("return (__builtin_popcount((unsigned)(a & b)) & 1) ? -1 : 1;",
                            "return (__builtin_popcount((unsigned)(a | b)) & 1) ? -1 : 1;"),
     "damp_y_no_inverse_scale": ("acc /= (double)P;", "acc /= 1.0;"),
+    "damp_fwht_butterfly_sign": ("                a[i + h] = x - y;", "                a[i + h] = y - x;"),
+    "damp_fwht_skips_last_stage": ("for (int h = 1; h < P; h *= 2)", "for (int h = 1; 2 * h < P; h *= 2)"),
     "damp_input_not_rotated": ("const float dtx = dt[h] * xr[k];",
                                "const float dtx = dt[h] * x[(size_t)h * P + k];"),
     "damp_B_by_position": ("const float b = B[(size_t)g * N + ch[m]];",
