@@ -17,25 +17,26 @@
 //   t'[m][k] = fma(lambda, t[m][k], fl(fl(dt * xr[k]) * B[chan[m]]))
 // and the readout rotates back once per head:
 //   y[p] = D x[p] + (1/P) sum_k H[p][k] sum_m C[chan[m]] stored'[m][k].
-// xr[k] is summed in double in the order p = 0..P-1 and rounded once, so
-// every stored code, step, zero point and FP16 value is bit-identical to a
-// plain scalar evaluation; y accumulates in fp32.
+// Rotations that decide stored values (xr, the hand-off, the read-back) are
+// the fast Walsh-Hadamard transform in double, butterfly stages h = 1, 2,
+// ..., P/2, rounded once, so every stored code, step, zero point and FP16
+// value is bit-identical to a scalar evaluation in that order; the readout
+// accumulates and rotates back in fp32.
 //
-// Thread mapping: one CTA of 256 threads per (layer, request, head) unit in
-// a grid-stride loop; a position's P values sit on LPR = P/16 consecutive
-// lanes, 16 per lane; a warp covers 32/LPR positions per pass.
+// Thread mapping: a position's P values sit on LPR = P/16 consecutive lanes,
+// 16 per lane (lane j of the group holds rotated indices 16j .. 16j+15); a
+// warp covers 32/LPR positions per pass.
 #include <cuda_fp16.h>
 
 #include "ssq_common.cuh"
 #include "ssq_params.h"
+#include "ssq_pipe.cuh"
 
 namespace ssq {
 
 namespace {
 
 constexpr int kDampE = 16;   // rotated entries per lane
-
-__device__ __forceinline__ bool hneg(int a, int b) { return (__popc(a & b) & 1) != 0; }
 
 // Reduce-scatter of a lane's E partial sums over the positions of its warp:
 // at each round a lane keeps half of its values and sends the other half to
@@ -66,6 +67,35 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[E], int lane, int& bas
 
 template <int N>
 __host__ __device__ constexpr int ilog2() { return N <= 1 ? 0 : 1 + ilog2<N / 2>(); }
+
+// Fast Walsh-Hadamard transform in double of a vector of E*LPR values held
+// E per lane by LPR consecutive lanes (lane j of the group holds indices
+// j*E .. j*E+E-1): stages h = 1, 2, ..., E*LPR/2 in turn; at each stage the
+// pair (i, i+h), bit h of i clear, becomes (a_i + a_(i+h), a_i - a_(i+h)).
+// Stages h < E pair values inside a lane, the others pair lanes j and j^(h/E).
+template <int E, int LPR>
+__device__ __forceinline__ void fwht_lanes(double (&a)[E], int lane)
+{
+#pragma unroll
+    for (int h = 1; h < E; h *= 2) {
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            if ((e & h) == 0) {
+                const double x = a[e], y = a[e + h];
+                a[e] = __dadd_rn(x, y);
+                a[e + h] = __dsub_rn(x, y);
+            }
+    }
+#pragma unroll
+    for (int o = 1; o < LPR; o *= 2) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const double other = __shfl_xor_sync(0xffffffffu, a[e], o);
+            a[e] = up ? __dsub_rn(other, a[e]) : __dadd_rn(a[e], other);
+        }
+    }
+}
 
 struct DampUnit {
     int l, b, h, slot, layer, g;
@@ -200,100 +230,10 @@ __device__ __forceinline__ void damp_store(const DampView& dv, const DampUnit& u
 }
 
 // ---------------------------------------------------------------------------
-// Decode step
-// ---------------------------------------------------------------------------
-template <int P>
-__global__ void __launch_bounds__(kThreads, 2)
-damp_decode_kernel(const __grid_constant__ DampView dv, const __grid_constant__ DampCall dc)
-{
-    constexpr int E = kDampE, LPR = P / E, PPW = 32 / LPR;
-    constexpr int ROUNDS = ilog2<PPW>();
-    constexpr int NW = kThreads / 32;
-    __shared__ float s_x[P];         // x of the head
-    __shared__ float s_dtx[P];       // fl(dt * xr[k])
-    __shared__ float s_red[NW][P];   // per-warp readout partials (rotated)
-    __shared__ float s_yr[P];        // rotated readout
-
-    uint32_t* err = reinterpret_cast<uint32_t*>(dv.pool);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int j = tid % LPR;
-    const int passes = (dv.N * LPR + kThreads - 1) / kThreads;
-    const long long units = (long long)dc.nl * dc.batch * dv.H;
-
-    for (long long uu = blockIdx.x; uu < units; uu += gridDim.x) {
-        const DampUnit u = damp_unit(dv, dc, uu);
-        if (u.slot < 0 || u.slot >= dv.n_slots) {
-            if (tid == 0) atomicOr(err, SSQ_DEVERR_SLOT);
-            continue;   // uniform over the CTA
-        }
-        if (!damp_chan_ok(dv, u, tid)) {
-            if (tid == 0) atomicOr(err, SSQ_DEVERR_CHANNEL);
-            continue;
-        }
-        const float dtv = __ldg(dc.dt + u.lb * dv.H + u.h);
-        const float lam = decay(dtv, __ldg(dc.A + (long long)u.l * dv.H + u.h));
-        const float* xh = dc.x + (u.lb * dv.H + u.h) * P;
-        if (tid < P) s_x[tid] = __ldg(xh + tid);
-        __syncthreads();
-        if (tid < P) {
-            // xr[k] = sum_p H[k][p] x[p], double, order p, rounded once
-            double acc = 0.0;
-#pragma unroll 8
-            for (int p = 0; p < P; ++p) {
-                const double v = (double)s_x[p];
-                acc = hneg(tid, p) ? __dsub_rn(acc, v) : __dadd_rn(acc, v);
-            }
-            s_dtx[tid] = __fmul_rn(dtv, __double2float_rn(acc));
-        }
-        __syncthreads();
-
-        float acc[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = 0.0f;
-        for (int pass = 0; pass < passes; ++pass) {
-            const DampPos ps = damp_pos<LPR>(dv, u, pass, tid);
-            const float bn = __ldg(dc.B + (u.lb * dv.G + u.g) * dv.N + ps.n);
-            const float cn = ps.active ? __ldg(dc.C + (u.lb * dv.G + u.g) * dv.N + ps.n) : 0.0f;
-            float t[E];
-            damp_load(dv, u, ps, j, t);
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const float w = __fmul_rn(s_dtx[j * E + e], bn);
-                t[e] = __fmaf_rn(lam, t[e], w);
-            }
-            damp_store<LPR>(dv, u, ps, j, t, ps.active, err);
-#pragma unroll
-            for (int e = 0; e < E; ++e) acc[e] = ps.active ? __fmaf_rn(cn, t[e], acc[e]) : acc[e];
-        }
-        // readout: sum over positions (warp butterfly, then across warps)
-        int base = 0;
-        reduce_scatter<E, LPR, ROUNDS, E>(acc, lane, base);
-        constexpr int KEEP = (E >> ROUNDS) > 0 ? (E >> ROUNDS) : 1;
-#pragma unroll
-        for (int i = 0; i < KEEP; ++i) s_red[warp][j * E + base + i] = acc[i];
-        __syncthreads();
-        if (tid < P) {
-            float v = 0.0f;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) v = __fadd_rn(v, s_red[w][tid]);
-            s_yr[tid] = v;
-        }
-        __syncthreads();
-        if (tid < P) {
-            float v = 0.0f;
-#pragma unroll 8
-            for (int k = 0; k < P; ++k)
-                v = hneg(tid, k) ? __fsub_rn(v, s_yr[k]) : __fadd_rn(v, s_yr[k]);
-            const float Dh = __ldg(dc.D + (long long)u.l * dv.H + u.h);
-            dc.y[(u.lb * dv.H + u.h) * P + tid] =
-                __fmaf_rn(Dh, s_x[tid], __fmul_rn(v, 1.0f / (float)P));
-        }
-        __syncthreads();
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Hand-off: fp32 S[nl][batch][H][P][N] -> tiers
+// Hand-off: fp32 S[nl][batch][H][P][N] -> tiers.  One CTA per head; a lane
+// group of LPR lanes loads a key channel's column S[.][n] (E values per
+// lane, in the order of the rotated index), rotates it with the lane-split
+// fast transform in double, rounds once and stores the tier.
 // ---------------------------------------------------------------------------
 template <int P>
 __global__ void __launch_bounds__(kThreads)
@@ -301,7 +241,7 @@ damp_quantize_kernel(const __grid_constant__ DampView dv, const __grid_constant_
 {
     constexpr int E = kDampE, LPR = P / E;
     uint32_t* err = reinterpret_cast<uint32_t*>(dv.pool);
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int j = tid % LPR;
     const int passes = (dv.N * LPR + kThreads - 1) / kThreads;
     const long long units = (long long)dc.nl * dc.batch * dv.H;
@@ -318,16 +258,10 @@ damp_quantize_kernel(const __grid_constant__ DampView dv, const __grid_constant_
         const float* S = dc.S_in + (u.lb * dv.H + u.h) * (long long)P * dv.N;
         for (int pass = 0; pass < passes; ++pass) {
             const DampPos ps = damp_pos<LPR>(dv, u, pass, tid);
-            // t[k] = sum_p H[k][p] S[p][n], double, order p, rounded once
             double a[E];
 #pragma unroll
-            for (int e = 0; e < E; ++e) a[e] = 0.0;
-            for (int p = 0; p < P; ++p) {
-                const double v = (double)__ldg(S + (long long)p * dv.N + ps.n);
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    a[e] = hneg(j * E + e, p) ? __dsub_rn(a[e], v) : __dadd_rn(a[e], v);
-            }
+            for (int e = 0; e < E; ++e) a[e] = (double)__ldg(S + (long long)(j * E + e) * dv.N + ps.n);
+            fwht_lanes<E, LPR>(a, lane);
             float t[E];
 #pragma unroll
             for (int e = 0; e < E; ++e) t[e] = __double2float_rn(a[e]);
@@ -337,16 +271,16 @@ damp_quantize_kernel(const __grid_constant__ DampView dv, const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------
-// Read-back: tiers -> fp32 S[nl][batch][H][P][N]
+// Read-back: tiers -> fp32 S[nl][batch][H][P][N]: reconstruct, rotate back
+// with the fast transform in double, scale by the exact 1/P, round once.
 // ---------------------------------------------------------------------------
 template <int P>
 __global__ void __launch_bounds__(kThreads)
 damp_dequantize_kernel(const __grid_constant__ DampView dv, const __grid_constant__ DampCall dc)
 {
     constexpr int E = kDampE, LPR = P / E;
-    extern __shared__ float s_t[];   // [N][P] stored (rotated) values
     uint32_t* err = reinterpret_cast<uint32_t*>(dv.pool);
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int j = tid % LPR;
     const int passes = (dv.N * LPR + kThreads - 1) / kThreads;
     const long long units = (long long)dc.nl * dc.batch * dv.H;
@@ -360,29 +294,428 @@ damp_dequantize_kernel(const __grid_constant__ DampView dv, const __grid_constan
             if (tid == 0) atomicOr(err, SSQ_DEVERR_CHANNEL);
             continue;
         }
+        float* S = dc.S_out + (u.lb * dv.H + u.h) * (long long)P * dv.N;
         for (int pass = 0; pass < passes; ++pass) {
             const DampPos ps = damp_pos<LPR>(dv, u, pass, tid);
             float t[E];
             damp_load(dv, u, ps, j, t);
+            double a[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) a[e] = (double)t[e];
+            fwht_lanes<E, LPR>(a, lane);
             if (ps.active) {
 #pragma unroll
-                for (int e = 0; e < E; ++e) s_t[ps.m * P + j * E + e] = t[e];
+                for (int e = 0; e < E; ++e)
+                    S[(long long)(j * E + e) * dv.N + ps.n] =
+                        __double2float_rn(__dmul_rn(a[e], 1.0 / (double)P));
             }
         }
-        __syncthreads();
-        float* S = dc.S_out + (u.lb * dv.H + u.h) * (long long)P * dv.N;
-        for (int idx = tid; idx < dv.N * P; idx += kThreads) {
-            const int m = idx / P, p = idx - m * P;
-            const int n = __ldg(u.chan + m);
-            // S[p][n] = (1/P) sum_k H[p][k] t[m][k], double, order k
-            double a = 0.0;
-            for (int k = 0; k < P; ++k) {
-                const double v = (double)s_t[m * P + k];
-                a = hneg(p, k) ? __dsub_rn(a, v) : __dadd_rn(a, v);
-            }
-            S[(long long)p * dv.N + n] = __double2float_rn(__dmul_rn(a, 1.0 / (double)P));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Decode step: a head's packed state is one contiguous block, so a producer
+// warp streams whole blocks (with the head's x, its group's B and C and its
+// channel map) into a ring of shared-memory stages with bulk copies; each
+// consumer warp takes one head at a time, updates the block in place in
+// shared memory and writes it back with one bulk store, while the next
+// heads' blocks are in flight.  Heads are dealt to the consumer warps in
+// turn; a stage is released once the bulk store of its head has read it.
+// ---------------------------------------------------------------------------
+constexpr int kDampCWarps = 8;                       // consumer warps per CTA (at most)
+constexpr int kDampStages = 16;                      // ring stages (at most)
+constexpr int kDampPipeThreads = (kDampCWarps + 1) * 32;
+constexpr int kDampSmemBudget = 227 * 1024;
+
+struct DampGeom {
+    int off_x, off_B, off_C, off_chan, stage_bytes;
+    int S, Wc;                 // stages, consumer warps (S > Wc)
+    int off_scr;               // per-warp scratch: fl(dt * xr[k]), P floats
+    int off_bar, smem_bytes;
+};
+
+inline DampGeom damp_geom(int head_bytes, int P, int N, int S, int Wc)
+{
+    DampGeom g;
+    g.off_x = head_bytes;                       // head_bytes is a multiple of 16
+    g.off_B = g.off_x + P * 4;
+    g.off_C = g.off_B + N * 4;
+    g.off_chan = g.off_C + N * 4;
+    g.stage_bytes = (g.off_chan + N * 4 + 127) / 128 * 128;
+    g.S = S;
+    g.Wc = Wc;
+    g.off_scr = S * g.stage_bytes;
+    g.off_bar = g.off_scr + Wc * P * 4;
+    g.smem_bytes = g.off_bar + 2 * S * 8;
+    return g;
+}
+
+// xr = H x over one warp: lane L holds indices L + 32r (P >= 32; for P = 16
+// lanes L and L+16 both hold index L & 15).  Stages h < 32 pair lanes L and
+// L^h, stages h >= 32 pair a lane's own values; h = 1, 2, ..., P/2 in turn.
+template <int P>
+__device__ __forceinline__ void fwht_warp(double (&a)[(P + 31) / 32], int lane)
+{
+    constexpr int V = (P + 31) / 32;
+    constexpr int HL = P < 32 ? P : 32;
+#pragma unroll
+    for (int h = 1; h < HL; h *= 2) {
+        const bool up = (lane & h) != 0;
+#pragma unroll
+        for (int r = 0; r < V; ++r) {
+            const double other = __shfl_xor_sync(0xffffffffu, a[r], h);
+            a[r] = up ? __dsub_rn(other, a[r]) : __dadd_rn(a[r], other);
         }
-        __syncthreads();
+    }
+#pragma unroll
+    for (int hr = 1; hr < V; hr *= 2) {
+#pragma unroll
+        for (int r = 0; r < V; ++r)
+            if ((r & hr) == 0) {
+                const double x = a[r], y = a[r + hr];
+                a[r] = __dadd_rn(x, y);
+                a[r + hr] = __dsub_rn(x, y);
+            }
+    }
+}
+
+// k-bit B of a lane's readout value after reduce_scatter: 0 when the bit
+// indexes the lane's own KEEP values, else the lane mask of the partner.
+template <int E, int LPR, int KEEP, int B>
+__host__ __device__ constexpr int kbit_lane()
+{
+    return B < ilog2<KEEP>() ? 0
+           : B < ilog2<E>() ? (LPR << (ilog2<E>() - 1 - B))
+                            : (1 << (B - ilog2<E>()));
+}
+
+// Fast transform (fp32) of the readout left by reduce_scatter: v[i] holds
+// index j*E + base + i; stages h = 1, 2, ..., P/2 in turn.
+template <int E, int LPR, int KEEP, int B, int NB>
+__device__ __forceinline__ void fwht_readout(float (&v)[KEEP], int lane)
+{
+    if constexpr (B < NB) {
+        constexpr int M = kbit_lane<E, LPR, KEEP, B>();
+        if constexpr (M == 0) {
+            constexpr int h = 1 << B;
+#pragma unroll
+            for (int i = 0; i < KEEP; ++i)
+                if ((i & h) == 0) {
+                    const float a = v[i], b = v[i + h];
+                    v[i] = __fadd_rn(a, b);
+                    v[i + h] = __fsub_rn(a, b);
+                }
+        } else {
+            const bool up = (lane & M) != 0;
+#pragma unroll
+            for (int i = 0; i < KEEP; ++i) {
+                const float o = __shfl_xor_sync(0xffffffffu, v[i], M);
+                v[i] = up ? __fsub_rn(o, v[i]) : __fadd_rn(v[i], o);
+            }
+        }
+        fwht_readout<E, LPR, KEEP, B + 1, NB>(v, lane);
+    }
+}
+
+template <int P>
+__global__ void __launch_bounds__(kDampPipeThreads, 1)
+damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ DampCall dc,
+                 const DampGeom g)
+{
+    constexpr int E = P >= 32 ? 32 : 16;
+    constexpr int LPR = P / E, PPW = 32 / LPR;
+    constexpr int ROUNDS = ilog2<PPW>();
+    constexpr int KEEP = (E >> ROUNDS) > 0 ? (E >> ROUNDS) : 1;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + g.off_bar);
+    uint64_t* empty = full + g.S;
+    uint32_t* err = reinterpret_cast<uint32_t*>(dv.pool);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = dv.H, N = dv.N, K = dv.K;
+    const long long units = (long long)dc.nl * dc.batch * H;
+    const long long per = (units + gridDim.x - 1) / gridDim.x;
+    const long long u0 = (long long)blockIdx.x * per;
+    const long long u1 = u0 + per < units ? u0 + per : units;
+    const int n = u1 > u0 ? (int)(u1 - u0) : 0;
+    const unsigned head_bytes = (unsigned)dv.head_bytes;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < g.S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == kDampCWarps) {
+        // ---- producer ---------------------------------------------------
+        if (lane != 0) return;
+        long long last_lb = -1;
+        int slot = 0, filled = 0;
+        bool ok = true;
+        for (int i = 0; i < n; ++i) {
+            const long long u = u0 + i;
+            const int s = i % g.S;
+            const unsigned f = (unsigned)(i / g.S);
+            if (!mbar_wait<kProducerSleep>(&empty[s], (f & 1) ^ 1)) {
+                ok = false;
+                break;
+            }
+            const long long lb = u / H;
+            const int h = (int)(u - lb * H);
+            const int l = (int)(lb / dc.batch);
+            const int b = (int)(lb - (long long)l * dc.batch);
+            if (lb != last_lb) {
+                slot = dc.slot_idx ? __ldg(dc.slot_idx + b) : b;
+                last_lb = lb;
+            }
+            filled = i + 1;
+            if (slot < 0 || slot >= dv.n_slots) {
+                mbar_arrive(&full[s]);             // nothing to copy; consumers skip it
+                continue;
+            }
+            const int layer = dc.layer0 + l;
+            const int grp = h / dv.hpg;
+            uint8_t* st = smem + (long long)s * g.stage_bytes;
+            const uint8_t* head = dv.pool + dv.header_bytes + (long long)slot * dv.slot_bytes
+                                  + (long long)layer * dv.layer_bytes + (long long)h * dv.head_bytes;
+            mbar_arrive_tx(&full[s], head_bytes + (unsigned)(P * 4 + 3 * N * 4));
+            bulk_g2s(st, head, head_bytes, &full[s]);
+            bulk_g2s(st + g.off_x, dc.x + (lb * H + h) * P, P * 4, &full[s]);
+            bulk_g2s(st + g.off_B, dc.B + (lb * dv.G + grp) * N, N * 4, &full[s]);
+            bulk_g2s(st + g.off_C, dc.C + (lb * dv.G + grp) * N, N * 4, &full[s]);
+            bulk_g2s(st + g.off_chan, dv.chan + ((long long)layer * H + h) * N, N * 4, &full[s]);
+        }
+        if (!ok) {
+            atomicOr(err, SSQ_DEVERR_TIMEOUT);
+            // copies still in flight land before this CTA's shared memory goes
+            for (int i = filled - g.S > 0 ? filled - g.S : 0; i < filled; ++i)
+                mbar_wait<kProducerSleep>(&full[i % g.S], (unsigned)(i / g.S) & 1);
+        }
+        return;
+    }
+    if (warp >= g.Wc) return;
+
+    // ---- consumers ------------------------------------------------------
+    const int j = lane % LPR, q = lane / LPR;
+    const int passes = (N + PPW - 1) / PPW;
+    int prev_s = -1;
+    // scalars of the warp's next head, loaded one head ahead
+    auto scalars = [&](int i, int& slot, float& dtv, float& Av, float& Dh) {
+        const long long u = u0 + i;
+        const long long lb = u / H;
+        const int h = (int)(u - lb * H);
+        const int l = (int)(lb / dc.batch);
+        const int b = (int)(lb - (long long)l * dc.batch);
+        slot = dc.slot_idx ? __ldg(dc.slot_idx + b) : b;
+        dtv = __ldg(dc.dt + lb * H + h);
+        Av = __ldg(dc.A + (long long)l * H + h);
+        Dh = __ldg(dc.D + (long long)l * H + h);
+    };
+    int nslot = 0;
+    float ndt = 0.0f, nA = 0.0f, nD = 0.0f;
+    if (warp < n) scalars(warp, nslot, ndt, nA, nD);
+    for (int i = warp; i < n; i += g.Wc) {
+        const int slot = nslot;
+        const float dtv = ndt, Av = nA, Dh = nD;
+        if (i + g.Wc < n) scalars(i + g.Wc, nslot, ndt, nA, nD);
+        const long long u = u0 + i;
+        const long long lb = u / H;
+        const int h = (int)(u - lb * H);
+        const int l = (int)(lb / dc.batch);
+        const int s = i % g.S;
+        // the whole warp takes the same decision
+        if (!__all_sync(0xffffffffu, mbar_wait<kConsumerSleep>(&full[s], (unsigned)(i / g.S) & 1))) {
+            if (lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
+            break;
+        }
+        uint8_t* st = smem + (long long)s * g.stage_bytes;
+        bool valid = slot >= 0 && slot < dv.n_slots;
+        if (!valid) {
+            if (lane == 0) atomicOr(err, SSQ_DEVERR_SLOT);
+        } else {
+            const int* chs = reinterpret_cast<const int*>(st + g.off_chan);
+            bool bad = false;
+            for (int m = lane; m < N; m += 32) bad |= (chs[m] < 0 || chs[m] >= N);
+            if (__any_sync(0xffffffffu, bad)) {
+                valid = false;
+                if (lane == 0) atomicOr(err, SSQ_DEVERR_CHANNEL);
+            }
+        }
+        bool stored = false;
+        if (valid) {
+            const float lam = decay(dtv, Av);
+            const float* xs = reinterpret_cast<const float*>(st + g.off_x);
+            const float* Bs = reinterpret_cast<const float*>(st + g.off_B);
+            const float* Cs = reinterpret_cast<const float*>(st + g.off_C);
+            const int* chs = reinterpret_cast<const int*>(st + g.off_chan);
+            // fl(dt * xr[k]) for the lane's E rotated indices k = j*E + e:
+            // the transform once per warp, handed round through shared memory
+            float* dtxs = reinterpret_cast<float*>(smem + g.off_scr) + warp * P;
+            {
+                constexpr int V = (P + 31) / 32;
+                double a[V];
+#pragma unroll
+                for (int r = 0; r < V; ++r) a[r] = (double)xs[P >= 32 ? lane + 32 * r : (lane & (P - 1))];
+                fwht_warp<P>(a, lane);
+#pragma unroll
+                for (int r = 0; r < V; ++r)
+                    if (P >= 32 || lane < P)
+                        dtxs[P >= 32 ? lane + 32 * r : lane] = __fmul_rn(dtv, __double2float_rn(a[r]));
+            }
+            __syncwarp();
+            const float* dtxj = dtxs + j * E;     // read per pass (frees registers)
+            const float2 lam2 = make_float2(lam, lam);
+            float acc[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+            for (int pass = 0; pass < passes; ++pass) {
+                const int m0 = pass * PPW + q;
+                const bool active = m0 < N;
+                const int m = active ? m0 : 0;
+                const int nch = chs[m];
+                const float bn = Bs[nch];
+                const float cn = active ? Cs[nch] : 0.0f;
+                const bool hi = m < K;
+                // every lane of the pass in the FP16 tier (uniform, from the
+                // pass index; an inactive lane shadows position 0)
+                const bool all_hi = (pass + 1) * PPW <= K || (pass * PPW < K && __all_sync(0xffffffffu, hi));
+                float t[E];
+                uint8_t* hp = st + dv.hi_off + (m * P + j * E) * 2;
+                uint8_t* cp = st + dv.codes_off + (m - K) * P + j * E;
+                uint8_t* mp = st + dv.meta_off + (m - K) * 8;
+                if (hi) {
+#pragma unroll
+                    for (int w4 = 0; w4 < E / 8; ++w4) {
+                        const uint4 v = reinterpret_cast<const uint4*>(hp)[w4];
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            t[8 * w4 + 2 * c] = __half2float(__ushort_as_half((unsigned short)(w[c] & 0xffffu)));
+                            t[8 * w4 + 2 * c + 1] = __half2float(__ushort_as_half((unsigned short)(w[c] >> 16)));
+                        }
+                    }
+                }
+                if (!all_hi) {
+                    Chunk<E> c;
+                    float delta = 0.0f, z = 0.0f;
+                    if (!hi) {
+#pragma unroll
+                        for (int w4 = 0; w4 < E / 16; ++w4) {
+                            const uint4 v = reinterpret_cast<const uint4*>(cp)[w4];
+                            c.w[4 * w4] = v.x; c.w[4 * w4 + 1] = v.y;
+                            c.w[4 * w4 + 2] = v.z; c.w[4 * w4 + 3] = v.w;
+                        }
+                        const float2 mz = *reinterpret_cast<const float2*>(mp);
+                        delta = mz.x;
+                        z = mz.y;
+                    } else {
+#pragma unroll
+                        for (int w = 0; w < E / 4; ++w) c.w[w] = 0u;
+                    }
+                    float sd[E];
+                    decode_row<SSQ_I8_ASYM, E>(c, delta, z, sd);
+                    if (!hi) {
+#pragma unroll
+                        for (int e = 0; e < E; ++e) t[e] = sd[e];
+                    }
+                }
+                // the recurrence on the rotated state: fma(lambda, t, fl(dtx * B_n))
+                const float2 b2 = make_float2(bn, bn);
+#pragma unroll
+                for (int e = 0; e < E; e += 4) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(dtxj + e);
+                    const float2 w0 = mul2(make_float2(d4.x, d4.y), b2);
+                    const float2 w1 = mul2(make_float2(d4.z, d4.w), b2);
+                    const float2 r0 = fma2(lam2, make_float2(t[e], t[e + 1]), w0);
+                    const float2 r1 = fma2(lam2, make_float2(t[e + 2], t[e + 3]), w1);
+                    t[e] = r0.x; t[e + 1] = r0.y; t[e + 2] = r1.x; t[e + 3] = r1.y;
+                }
+                if (!all_hi) {
+                    const RowParams rp = refit_row<SSQ_I8_ASYM, E, LPR>(t);
+                    float rr[E];
+                    uint32_t kk[E];
+                    round_row<SSQ_I8_ASYM, E>(rp, t, rr, kk);
+                    if (!hi) {
+                        Chunk<E> c;
+                        pack_codes<SSQ_I8_ASYM, E>(kk, c);
+                        scale_row<E>(rp.delta, rr, t);
+                        if (active) {
+#pragma unroll
+                            for (int w4 = 0; w4 < E / 16; ++w4)
+                                reinterpret_cast<uint4*>(cp)[w4] =
+                                    make_uint4(c.w[4 * w4], c.w[4 * w4 + 1], c.w[4 * w4 + 2],
+                                               c.w[4 * w4 + 3]);
+                            if (j == 0) {
+                                *reinterpret_cast<float2*>(mp) = make_float2(rp.delta, rp.z);
+                                if (!rp.finite) atomicOr(err, SSQ_DEVERR_NONFINITE);
+                            }
+                        }
+                    }
+                }
+                if (hi) {
+                    uint32_t hv[E / 2];
+#pragma unroll
+                    for (int w2 = 0; w2 < E / 2; ++w2) {
+                        const __half a = __float2half_rn(t[2 * w2]);
+                        const __half bb = __float2half_rn(t[2 * w2 + 1]);
+                        hv[w2] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(bb) << 16);
+                        t[2 * w2] = __half2float(a);
+                        t[2 * w2 + 1] = __half2float(bb);
+                    }
+                    if (active) {
+#pragma unroll
+                        for (int w4 = 0; w4 < E / 8; ++w4)
+                            reinterpret_cast<uint4*>(hp)[w4] =
+                                make_uint4(hv[4 * w4], hv[4 * w4 + 1], hv[4 * w4 + 2], hv[4 * w4 + 3]);
+                    }
+                }
+                const float2 c2 = make_float2(cn, cn);
+#pragma unroll
+                for (int e = 0; e < E; e += 2) {
+                    const float2 r = fma2(c2, make_float2(t[e], t[e + 1]), make_float2(acc[e], acc[e + 1]));
+                    acc[e] = r.x;
+                    acc[e + 1] = r.y;
+                }
+            }
+            // readout: sum over the warp's positions, rotate back, add D x
+            int base = 0;
+            reduce_scatter<E, LPR, ROUNDS, E>(acc, lane, base);
+            float v[KEEP];
+#pragma unroll
+            for (int e = 0; e < KEEP; ++e) v[e] = acc[e];
+            fwht_readout<E, LPR, KEEP, 0, ilog2<P>()>(v, lane);
+            // lanes that hold the same indices (KEEP = 1 with a spare reduce
+            // round) write the same values
+#pragma unroll
+            for (int e = 0; e < KEEP; ++e) {
+                const int p = j * E + base + e;
+                dc.y[(lb * H + h) * P + p] = __fmaf_rn(Dh, xs[p], __fmul_rn(v[e], 1.0f / (float)P));
+            }
+            // the updated block goes back with one bulk store
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+                uint8_t* head = dv.pool + dv.header_bytes + (long long)slot * dv.slot_bytes
+                                + (long long)(dc.layer0 + l) * dv.layer_bytes
+                                + (long long)h * dv.head_bytes;
+                bulk_s2g(head, st, head_bytes);
+                bulk_commit();
+            }
+            stored = true;
+        }
+        // release the previous head's stage once its store has read it
+        if (lane == 0 && prev_s >= 0) {
+            if (stored) bulk_wait_read<1>(); else bulk_wait_read<0>();
+            mbar_arrive(&empty[prev_s]);
+        }
+        prev_s = s;
+        __syncwarp();
+    }
+    if (lane == 0) {
+        bulk_wait<0>();
+        if (prev_s >= 0) mbar_arrive(&empty[prev_s]);
     }
 }
 
@@ -390,11 +723,29 @@ template <int P>
 cudaError_t launch_damp_p(const DampView& dv, const DampCall& dc, int which, cudaStream_t st)
 {
     const long long units = (long long)dc.nl * dc.batch * dv.H;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
     if (which == 0) {
-        auto k = damp_decode_kernel<P>;
-        const int grid = grid_for((const void*)k, kThreads, units);
-        if (grid <= 0) return cudaErrorInvalidConfiguration;
-        k<<<grid, kThreads, 0, st>>>(dv, dc);
+        int optin = 0;
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        const int budget = optin < kDampSmemBudget ? optin : kDampSmemBudget;
+        // as many stages as fit (at most kDampStages), one more than the
+        // consumer warps
+        DampGeom g = damp_geom((int)dv.head_bytes, P, dv.N, 1, 1);
+        int S = (budget - 256 - kDampCWarps * P * 4) / (g.stage_bytes + 16);
+        if (S > kDampStages) S = kDampStages;
+        if (S < 2) return cudaErrorInvalidConfiguration;
+        const int Wc = S - 1 < kDampCWarps ? S - 1 : kDampCWarps;
+        g = damp_geom((int)dv.head_bytes, P, dv.N, S, Wc);
+        auto k = damp_decode_pipe<P>;
+        e = cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 g.smem_bytes);
+        if (e != cudaSuccess) return e;
+        const long long grid = units < sms ? units : sms;
+        k<<<(int)grid, kDampPipeThreads, g.smem_bytes, st>>>(dv, dc, g);
     } else if (which == 1) {
         auto k = damp_quantize_kernel<P>;
         const int grid = grid_for((const void*)k, kThreads, units);
@@ -402,22 +753,9 @@ cudaError_t launch_damp_p(const DampView& dv, const DampCall& dc, int which, cud
         k<<<grid, kThreads, 0, st>>>(dv, dc);
     } else {
         auto k = damp_dequantize_kernel<P>;
-        const size_t smem = (size_t)dv.N * P * sizeof(float);
-        if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute((const void*)k,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)smem);
-            if (e != cudaSuccess) return e;
-        }
-        int dev = 0, sms = 0, occ = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e == cudaSuccess)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, (const void*)k, kThreads, smem);
-        if (e != cudaSuccess) return e;
-        long long grid = (long long)sms * (occ < 1 ? 1 : occ);
-        if (grid > units) grid = units;
-        k<<<(int)grid, kThreads, smem, st>>>(dv, dc);
+        const int grid = grid_for((const void*)k, kThreads, units);
+        if (grid <= 0) return cudaErrorInvalidConfiguration;
+        k<<<grid, kThreads, 0, st>>>(dv, dc);
     }
     return cudaGetLastError();
 }

@@ -31,6 +31,7 @@
 //     copies in flight).
 #include "ssq_common.cuh"
 #include "ssq_params.h"
+#include "ssq_pipe.cuh"
 
 #include <type_traits>
 
@@ -46,89 +47,6 @@ constexpr int kMinBlocks = 1;  // CTAs per SM
 constexpr int kCThreads = kCWarps * 32;
 constexpr int kDThreads = kCThreads + 32;
 constexpr int kMaxStages = 8;
-constexpr long long kWaitLimit = 2000000000LL;  // clock cycles, about one second
-
-// ---- PTX wrappers -------------------------------------------------------
-__device__ __forceinline__ unsigned saddr(const void* p)
-{
-    return (unsigned)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t* b, unsigned count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b)
-{
-    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
-}
-// Arrive from the lanes where `pred` holds (predicated inside the
-// instruction, so the warp does not branch).
-__device__ __forceinline__ void mbar_arrive_if(uint64_t* b, bool pred)
-{
-    asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n"
-                 " @p mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n}\n"
-                 ::"r"(saddr(b)), "r"((unsigned)pred) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, unsigned bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
-                 ::"r"(saddr(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* b, unsigned parity)
-{
-    unsigned ok;
-    asm volatile("{\n .reg .pred p;\n"
-                 " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-                 " selp.u32 %0, 1, 0, p;\n}\n"
-                 : "=r"(ok) : "r"(saddr(b)), "r"(parity) : "memory");
-    return ok != 0;
-}
-// Wait for the phase of the given parity to complete, sleeping between
-// tries (exponential back-off up to kMaxSleepNs, so a waiting warp takes
-// few issue slots from the warps that compute); false after about a second
-// without progress.
-template <unsigned kMaxSleepNs>
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, unsigned parity)
-{
-    if (mbar_try(b, parity)) return true;
-    const long long t0 = clock64();
-    unsigned ns = 64;
-    while (!mbar_try(b, parity)) {
-        __nanosleep(ns);
-        ns = ns < kMaxSleepNs ? 2 * ns : kMaxSleepNs;
-        if (clock64() - t0 > kWaitLimit) return false;
-    }
-    return true;
-}
-constexpr unsigned kProducerSleep = 2048;  // the producer waits for a stage to drain
-constexpr unsigned kConsumerSleep = 256;   // consumers wait for data to land
-// Bulk prefetch of global memory into L2 (no completion to wait for).
-// Address 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, unsigned bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-// Bulk copy global -> shared; completion counted in bytes on `bar`.
-// Both addresses 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(saddr(dst)), "l"(src), "r"(bytes), "r"(saddr(bar)) : "memory");
-}
-__device__ __forceinline__ void cpa4(void* dst, const void* src)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(saddr(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cpa16(void* dst, const void* src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr(dst)), "l"(src) : "memory");
-}
-// The mbarrier's current phase also waits for this thread's earlier cp.async.
-__device__ __forceinline__ void cpa_arrive(uint64_t* b)
-{
-    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(saddr(b)) : "memory");
-}
-
 // Shared-memory vector loads / stores at 32-bit shared addresses (the
 // quantized path forms its addresses with one XOR each).
 template <int OFF>
