@@ -23,6 +23,7 @@ same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import glob
 import hashlib
 import json
@@ -683,8 +684,16 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nl", type=int, default=None,
+                    help="layers per decode launch (a smaller case of the same shape, "
+                         "for profiler captures; the bench lines use the workload's own)")
     args = ap.parse_args()
     wl = workload(args.workload)
+    if args.nl is not None:
+        if not isinstance(wl, W.Decode):
+            raise SystemExit("--nl applies to decode workloads")
+        wl = dataclasses.replace(wl, nl=args.nl,
+                                 name=wl.name.replace(f"L{wl.nl} ", f"L{args.nl} "))
     if args.impl == "reference":
         # the oracle on the host cores: no device timing, so no warm-up rule
         return run_reference(args, wl, args.workload)

@@ -570,13 +570,27 @@ damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ Da
             float acc[E];
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+            // B and C of the lane's channel, one pass ahead (the channel map
+            // lookup and the two reads behind it are a dependent chain)
+            float nbn, ncn;
+            {
+                const int m = q < N ? q : 0;
+                const int nch = chs[m];
+                nbn = Bs[nch];
+                ncn = q < N ? Cs[nch] : 0.0f;
+            }
             for (int pass = 0; pass < passes; ++pass) {
                 const int m0 = pass * PPW + q;
                 const bool active = m0 < N;
                 const int m = active ? m0 : 0;
-                const int nch = chs[m];
-                const float bn = Bs[nch];
-                const float cn = active ? Cs[nch] : 0.0f;
+                const float bn = nbn, cn = ncn;
+                if (pass + 1 < passes) {
+                    const int m1 = m0 + PPW;
+                    const int mm = m1 < N ? m1 : 0;
+                    const int nch = chs[mm];
+                    nbn = Bs[nch];
+                    ncn = m1 < N ? Cs[nch] : 0.0f;
+                }
                 const bool hi = m < K;
                 // every lane of the pass in the FP16 tier (uniform, from the
                 // pass index; an inactive lane shadows position 0)
@@ -640,7 +654,17 @@ damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ Da
                     if (!hi) {
                         Chunk<E> c;
                         pack_codes<SSQ_I8_ASYM, E>(kk, c);
-                        scale_row<E>(rp.delta, rr, t);
+                        // readout of the stored value (q - z) * Delta as
+                        // (C * Delta) * (q - z): y is fp32 with a tolerance
+                        const float cd = __fmul_rn(cn, rp.delta);
+                        const float2 cd2 = make_float2(cd, cd);
+#pragma unroll
+                        for (int e = 0; e < E; e += 2) {
+                            const float2 r = fma2(cd2, make_float2(rr[e], rr[e + 1]),
+                                                  make_float2(acc[e], acc[e + 1]));
+                            acc[e] = r.x;
+                            acc[e + 1] = r.y;
+                        }
                         if (active) {
 #pragma unroll
                             for (int w4 = 0; w4 < E / 16; ++w4)
@@ -670,13 +694,14 @@ damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ Da
                             reinterpret_cast<uint4*>(hp)[w4] =
                                 make_uint4(hv[4 * w4], hv[4 * w4 + 1], hv[4 * w4 + 2], hv[4 * w4 + 3]);
                     }
-                }
-                const float2 c2 = make_float2(cn, cn);
+                    const float2 c2 = make_float2(cn, cn);
 #pragma unroll
-                for (int e = 0; e < E; e += 2) {
-                    const float2 r = fma2(c2, make_float2(t[e], t[e + 1]), make_float2(acc[e], acc[e + 1]));
-                    acc[e] = r.x;
-                    acc[e + 1] = r.y;
+                    for (int e = 0; e < E; e += 2) {
+                        const float2 r = fma2(c2, make_float2(t[e], t[e + 1]),
+                                              make_float2(acc[e], acc[e + 1]));
+                        acc[e] = r.x;
+                        acc[e + 1] = r.y;
+                    }
                 }
             }
             // readout: sum over the warp's positions, rotate back, add D x
