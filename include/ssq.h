@@ -16,16 +16,15 @@
  *       0.99, lambda > 0.99) and a band can be rounded on its own.
  *   "ssm-state-quantization" README, Findings 1: nearest rounding (RTN).
  *   "Mamba state quantization for inference":
- *     - "Recurrent state is fixed per request, not free": every token reads
- *       the state matrix, applies the recurrence and writes it back; one
- *       state per live request;
- *     - "Mixed precision spends bits on persistent channels": one fused
- *       kernel reconstructs the low-precision tier, runs the recurrence in
- *       FP32, derives new quantization parameters and writes the packed state
- *       back; tiers sit in contiguous regions so no per-token gather is
- *       needed;
- *     - "Mamba state quantization needs phase-aware benchmarks": prefill
- *       computes in FP32 and writes its final state into the packed cache.
+ *     - "Recurrent state is fixed per request, not free": each live request
+ *       owns one state, and a token reads, updates and stores all of it;
+ *     - "Mixed precision spends bits on persistent channels": decoding the
+ *       low-bit part, the fp32 update, the new scales and the packed store
+ *       belong in one kernel, and each precision tier is one contiguous
+ *       region so nothing is gathered per token;
+ *     - "Mamba state quantization needs phase-aware benchmarks": a prefill
+ *       keeps its state in fp32 and hands its last state to the packed
+ *       cache.
  *   "SSDi8: Accurate and Efficient 8-bit Quantization for State Space
  *   Duality", 4 Methodology, State quantization: per-(H,P) state scales,
  *   nothing along N.
@@ -180,9 +179,9 @@ SSQ_API ssq_status ssq_pool_error(const ssq_config* cfg, void* pool,
                           uint32_t* flags, cudaStream_t stream);
 
 /* Write fp32 states into pool slots through the row quantizer: the prefill
- * hand-off of "Mamba state quantization for inference" ("phase-aware
- * benchmarks": an FP32 chunk-final state written into the packed cache), and
- * pool initialisation.
+ * hand-off of "Mamba state quantization for inference" ("Mamba state
+ * quantization needs phase-aware benchmarks": the fp32 state at the end of a
+ * prefill chunk enters the packed cache), and pool initialisation.
  *   S         device fp32 [nl][batch][nheads][headdim][d_state], natural head
  *             order, 16-byte aligned
  *   slot_idx  device int32 [batch]: pool slot of request b; NULL = slot b
@@ -200,9 +199,10 @@ SSQ_API ssq_status ssq_dequantize_rows(const ssq_config* cfg, const void* pool,
                                cudaStream_t stream);
 
 /* Diagnostics of one decode step, read-only ("ssm-state-quantization"
- * README, Findings 4 and 5: a reversal is a step where rounding moves a
- * state entry against the new input; the reversal error as seen by the
- * readout, relative to the readout signal, is the reported correlate).  For
+ * README, Findings 4 and 5: an entry reverses when rounding turns its change
+ * against the direction of the step's input; the page relates damage to the
+ * part of the reversal error that reaches the output, measured against the
+ * output itself).  For
  * every row the step ssq_decode_step would take is evaluated (same update
  * s' = fma(lambda, s, w), w = fl(fl(dt*x)*B_n), same refit and nearest
  * rounding) and, with e_n = fl(deq_n - s'_n) the rounding error, four fp32
@@ -290,9 +290,9 @@ SSQ_API ssq_status ssq_scan_sr(const ssq_config* cfg, void* pool,
                        float* y, uint64_t seed, uint32_t step0,
                        cudaStream_t stream);
 
-/* Prefill hand-off ("Mamba state quantization for inference", phase-aware
- * benchmarks: prefill computes in FP32 and writes its final state into the
- * packed cache).  T tokens of one layer from the stored state with the
+/* Prefill hand-off ("Mamba state quantization for inference", "Mamba state
+ * quantization needs phase-aware benchmarks": the prefill runs in fp32 and
+ * only its last state is packed).  T tokens of one layer from the stored state with the
  * recurrence in fp32 and no rounding between tokens; y_t is read from the
  * fp32 state; after the last token the state is refit and quantized once
  * (quantized heads; fp heads are stored as fp32, or rounded to bf16 for

@@ -524,9 +524,9 @@ void oref_step_diag(const oref_cfg* c, const oref_state* st, const float* x,
     free(q);
 }
 
-/* Prefill hand-off ("Mamba state quantization for inference", phase-aware
- * benchmarks: prefill computes in FP32 and writes its final state into the
- * packed cache): from the stored state, T tokens of the fp32 recurrence
+/* Prefill hand-off ("Mamba state quantization for inference", "Mamba state
+ * quantization needs phase-aware benchmarks": the prefill runs in fp32 and
+ * only its last state is packed): from the stored state, T tokens of the fp32 recurrence
  * s'_n = fma(lambda, s_n, fl(dt*x) * B_n) with no rounding between tokens,
  * y_t read from the fp32 state (accumulated in double), and the state
  * quantized (or stored, bf16-rounded for the bf16 format) once after the
@@ -639,12 +639,11 @@ void oref_decode_batch(const oref_cfg* c, int nl, int batch,
 
 /* ------------------------------------------------------------------------
  * DAMP mixed-tier state ("Mamba state quantization for inference", "Mixed
- * precision spends bits on persistent channels"): a Hadamard transform along
- * each key channel's value dimension; the protected key channels kept in
- * FP16, the others in INT8 with a scale and a zero point; the selected
- * channels permuted into one contiguous region; per token the low tier is
- * reconstructed, the recurrence runs in FP32, new quantization parameters
- * are derived and the packed state is written back.
+ * precision spends bits on persistent channels"): each key channel's vector
+ * over head_dim is rotated by a Hadamard matrix; a chosen set of channels
+ * stays in FP16, the rest is stored as 8-bit codes with a step and an
+ * offset; the chosen channels come first; every token decodes the 8-bit
+ * tier, updates in fp32, fits new steps and stores the packed state.
  *
  * Readings (listed in the design notes):
  *   - state S[h][p][n]: p the value dimension (head_dim), n the key channel

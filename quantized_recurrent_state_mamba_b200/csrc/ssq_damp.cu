@@ -2,12 +2,12 @@
 // read-back.
 //
 // "Mamba state quantization for inference", "Mixed precision spends bits on
-// persistent channels": a Hadamard transform along each key channel's value
-// dimension; the protected key channels kept in FP16, the rest in INT8 with a
-// scale and a zero point; the tiers permuted into contiguous regions so one
-// fused kernel loads both without a per-token gather; per token the kernel
-// reconstructs the low tier, runs the recurrence in FP32, derives new
-// quantization parameters and writes the packed state back.
+// persistent channels": each key channel's vector over head_dim is rotated
+// by a Hadamard matrix; a chosen set of channels stays in FP16 and the rest
+// is stored as 8-bit codes with a step and an offset; each tier is one
+// contiguous block, so a kernel reads both with no gather; every token
+// decodes the 8-bit tier, updates in fp32, fits new steps and stores the
+// packed state again, all in one kernel.
 //
 // Per head the state is N key channels ("positions" m = 0..N-1 after the
 // caller's channel permutation chan[layer][h][m]; positions < K form the

@@ -3,10 +3,10 @@
 // One launch updates the state of nl layers x batch requests by one token:
 // read the packed row, decode, apply the recurrence in fp32, refit the row
 // scale, requantize, write the packed row and its metadata back, and read y
-// from the newly stored row -- the single fused pass that "Mamba state
-// quantization for inference" describes for a low-bit state ("reconstructs
-// the low tier, computes the recurrence in FP32, derives new quantization
-// parameters, and writes the packed state back"), with the quantizer of
+// from the newly stored row: one kernel does all of it, as "Mamba state
+// quantization for inference" ("Mixed precision spends bits on persistent
+// channels") lays out for a low-bit state (decode, fp32 update, new scale,
+// packed write-back in one pass), with the quantizer of
 // "ssm-state-quantization" README, Setup.
 //
 // Structure (persistent, warp-specialised, one CTA of 12 warps per SM):

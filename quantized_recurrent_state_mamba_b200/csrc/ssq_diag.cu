@@ -1,9 +1,10 @@
 // ssq_diag.cu -- diagnostics of a decode step, without changing the state.
 //
-// "ssm-state-quantization" README, Findings 4 and 5: a reversal is a step
-// where rounding moves a state entry against the new input; the reversal
-// rate by decay band and the reversal error as seen by the readout are the
-// quantities reported there.  For every row this kernel evaluates the step
+// "ssm-state-quantization" README, Findings 4 and 5: an entry reverses when
+// the rounding turns its change in the opposite direction to the step's
+// input; the page reports how often this happens per decay band and how
+// much of the rounding error the readout sees.  For every row this kernel
+// evaluates the step
 // the decode kernel would take (the same update, refit and rounding) and
 // writes, per row, without touching the pool:
 //   reversals   entries whose applied increment e + w, e = fl(deq - s') the

@@ -2,8 +2,9 @@
 // back.
 //
 // ssq_quantize_rows is the hand-off point of "Mamba state quantization for
-// inference" ("phase-aware benchmarks": prefill computes in FP32 and writes
-// its final state into the packed cache): each row gets its scale fitted and
+// inference" ("Mamba state quantization needs phase-aware benchmarks": the
+// state a prefill ends with, kept in fp32, enters the packed cache
+// once): each row gets its scale fitted and
 // is rounded exactly as a decode step would round it ("ssm-state-quantization"
 // README, Setup).  ssq_dequantize_rows decodes rows back to fp32.
 #include "ssq_common.cuh"

@@ -1,7 +1,7 @@
 """GPU parity of the step diagnostics (ssq_decode_diag) against the oracle.
 
 "ssm-state-quantization" README, Findings 4 and 5: per row, the number of
-entries the step's rounding reverses against the new input, the rounding
+entries whose change the rounding turns against the step's input, the rounding
 error seen by the readout over the reversed entries and over all entries,
 and the readout signal.  The reversal decision is taken in fp32 on both sides
 from bit-equal operands (same update, same refit, same rounding), so the

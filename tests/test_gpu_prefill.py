@@ -1,8 +1,8 @@
 """GPU parity of the prefill hand-off (ssq_prefill through the C ABI) against
 the CPU oracle: T tokens of the fp32 recurrence from the stored state, y
 read from the fp32 state, the final state quantized once ("Mamba state
-quantization for inference", phase-aware benchmarks: prefill computes in
-FP32 and writes its final state into the packed cache).
+quantization for inference", "Mamba state quantization needs phase-aware
+benchmarks": the prefill stays in fp32 and only its last state is packed).
 
 The stored codes and metadata must be bit-identical to the oracle's (the
 fp32 recurrence is one IEEE operation per step in both); y within the

@@ -2,12 +2,11 @@
 mathematics fix.
 
 "Mamba state quantization for inference", "Mixed precision spends bits on
-persistent channels": a Hadamard transform along each key channel's value
-dimension; protected key channels kept in FP16, the rest in INT8 with a
-scale and a zero point; per token the low tier is reconstructed, the
-recurrence runs in FP32, new quantization parameters are derived and the
-packed state is written back; 16 of 128 key channels protected costs 9.875
-bits per value.
+persistent channels": each key channel's vector over head_dim is rotated by
+a Hadamard matrix; chosen channels stay in FP16, the others become 8-bit
+codes with a step and an offset; every token decodes, updates in fp32, fits
+new steps and stores the packed state; with 16 channels of 128 in FP16 the
+page counts 9.875 bits per value.
 
 The checks: the rotation against scipy's Hadamard matrix and a hand-written
 H_4; fp16 rounding against numpy's conversion; the step against the exact
