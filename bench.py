@@ -154,10 +154,31 @@ def _code_only(src):
     return " ".join(src.split())
 
 
-def kernel_source_hash():
+# The sources each workload's dominant kernel is built from (with the host
+# code that sizes its launch).
+_COMMON_SOURCES = ("ssq_common.cuh", "ssq_params.h", "ssq_api.cu")
+_KERNEL_SOURCES = {
+    "decode": ("ssq_decode.cu", "ssq_pipe.cuh"),
+    "damp": ("ssq_damp.cu", "ssq_pipe.cuh"),
+    "scan": ("ssq_scan.cu",),
+}
+
+
+def _kernel_family(workload_name):
+    if workload_name.endswith("_damp"):
+        return "damp"
+    if workload_name.startswith(("scan", "prefill")):
+        return "scan"
+    return "decode"
+
+
+def kernel_source_hash(workload_name="decode_130m"):
+    """Hash of the code (comments and blank space removed) of the sources
+    the workload's dominant kernel is built from."""
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "quantized_recurrent_state_mamba_b200", "csrc")
-    files = sorted(glob.glob(os.path.join(pkg, "*"))) + [os.path.join(ROOT, "include", "ssq.h")]
+    names = sorted(_COMMON_SOURCES + _KERNEL_SOURCES[_kernel_family(workload_name)])
+    files = [os.path.join(pkg, n) for n in names] + [os.path.join(ROOT, "include", "ssq.h")]
     for p in files:
         with open(p, encoding="utf-8") as f:
             h.update(os.path.basename(p).encode())
@@ -169,7 +190,7 @@ def ncu_traffic(workload_name):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary for this workload, if it was captured on the current kernel
     sources (else None)."""
-    src = kernel_source_hash()
+    src = kernel_source_hash(workload_name)
     for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         kv = {}
         with open(p) as f:

@@ -28,6 +28,8 @@
 // warp covers 32/LPR positions per pass.
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "ssq_common.cuh"
 #include "ssq_params.h"
 #include "ssq_pipe.cuh"
@@ -579,9 +581,13 @@ damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ Da
                 nbn = Bs[nch];
                 ncn = q < N ? Cs[nch] : 0.0f;
             }
-            for (int pass = 0; pass < passes; ++pass) {
+            // One pass: the lane's channel m = pass*PPW + q.  MODE 0: every
+            // lane of the pass in the FP16 tier; 1: every lane in the INT8
+            // tier and active; 2: anything (per-lane tier, inactive lanes).
+            auto pass_body = [&](auto mode, int pass) {
+                constexpr int MODE = decltype(mode)::value;
                 const int m0 = pass * PPW + q;
-                const bool active = m0 < N;
+                const bool active = MODE == 1 || m0 < N;
                 const int m = active ? m0 : 0;
                 const float bn = nbn, cn = ncn;
                 if (pass + 1 < passes) {
@@ -591,10 +597,7 @@ damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ Da
                     nbn = Bs[nch];
                     ncn = m1 < N ? Cs[nch] : 0.0f;
                 }
-                const bool hi = m < K;
-                // every lane of the pass in the FP16 tier (uniform, from the
-                // pass index; an inactive lane shadows position 0)
-                const bool all_hi = (pass + 1) * PPW <= K || (pass * PPW < K && __all_sync(0xffffffffu, hi));
+                const bool hi = MODE == 0 || (MODE == 2 && m < K);
                 float t[E];
                 uint8_t* hp = st + dv.hi_off + (m * P + j * E) * 2;
                 uint8_t* cp = st + dv.codes_off + (m - K) * P + j * E;
@@ -611,7 +614,7 @@ damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ Da
                         }
                     }
                 }
-                if (!all_hi) {
+                if constexpr (MODE != 0) {
                     Chunk<E> c;
                     float delta = 0.0f, z = 0.0f;
                     if (!hi) {
@@ -629,7 +632,7 @@ damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ Da
                         for (int w = 0; w < E / 4; ++w) c.w[w] = 0u;
                     }
                     float sd[E];
-                    decode_row<SSQ_I8_ASYM, E>(c, delta, z, sd);
+                    decode_row<SSQ_I8_ASYM, E>(c, delta, z, sd);   // warp-uniform inside
                     if (!hi) {
 #pragma unroll
                         for (int e = 0; e < E; ++e) t[e] = sd[e];
@@ -646,7 +649,7 @@ damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ Da
                     const float2 r1 = fma2(lam2, make_float2(t[e + 2], t[e + 3]), w1);
                     t[e] = r0.x; t[e + 1] = r0.y; t[e + 2] = r1.x; t[e + 3] = r1.y;
                 }
-                if (!all_hi) {
+                if constexpr (MODE != 0) {
                     const RowParams rp = refit_row<SSQ_I8_ASYM, E, LPR>(t);
                     float rr[E];
                     uint32_t kk[E];
@@ -703,6 +706,17 @@ damp_decode_pipe(const __grid_constant__ DampView dv, const __grid_constant__ Da
                         acc[e + 1] = r.y;
                     }
                 }
+            };
+            // the passes that touch the FP16 tier, then the passes wholly in
+            // the INT8 tier, then a ragged tail (d_state not a multiple of
+            // the channels per pass)
+            const int lo_begin = (K + PPW - 1) / PPW;
+            const int lo_end = N / PPW > lo_begin ? N / PPW : lo_begin;
+            for (int pass = 0; pass < passes; ++pass) {
+                if (pass >= lo_begin && pass < lo_end)
+                    pass_body(std::integral_constant<int, 1>(), pass);
+                else
+                    pass_body(std::integral_constant<int, 2>(), pass);
             }
             // readout: sum over the warp's positions, rotate back, add D x
             int base = 0;
