@@ -771,13 +771,15 @@ cudaError_t launch_damp_p(const DampView& dv, const DampCall& dc, int which, cud
         e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (e != cudaSuccess) return e;
         const int budget = optin < kDampSmemBudget ? optin : kDampSmemBudget;
-        // as many stages as fit (at most kDampStages), one more than the
-        // consumer warps
+        // as many stages as fit (at most kDampStages); a consumer holds its
+        // stage while it computes, so the consumer warps take at most the
+        // stages beyond 8 heads in flight (half the stages on a small ring)
         DampGeom g = damp_geom((int)dv.head_bytes, P, dv.N, 1, 1);
         int S = (budget - 256 - kDampCWarps * P * 4) / (g.stage_bytes + 16);
         if (S > kDampStages) S = kDampStages;
         if (S < 2) return cudaErrorInvalidConfiguration;
-        const int Wc = S - 1 < kDampCWarps ? S - 1 : kDampCWarps;
+        int Wc = S >= 16 ? S - 8 : S / 2;
+        if (Wc > kDampCWarps) Wc = kDampCWarps;
         g = damp_geom((int)dv.head_bytes, P, dv.N, S, Wc);
         auto k = damp_decode_pipe<P>;
         e = cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize,
