@@ -139,14 +139,22 @@ class DampCodec:
     FP16 tier at hi_off (position-major halves), uint8 codes at codes_off and
     {float Delta, float z} per INT8 position at meta_off."""
 
+    buf_offset = 0   # byte offset in the pool of buf[0] (partial copies)
+
     def __init__(self, nheads, headdim, d_state, n_protected, layout):
         self.H, self.P, self.N, self.K = nheads, headdim, d_state, n_protected
         self.L = layout
 
+    def layer_range(self, slot, layer):
+        """(offset, size) of one (slot, layer)'s heads in the pool."""
+        L = self.L
+        return (L["header_bytes"] + slot * L["slot_bytes"] + layer * L["layer_bytes"],
+                L["layer_bytes"])
+
     def _head(self, slot, layer, h):
         L = self.L
         return (L["header_bytes"] + slot * L["slot_bytes"] + layer * L["layer_bytes"]
-                + h * L["head_bytes"])
+                + h * L["head_bytes"] - self.buf_offset)
 
     def write(self, buf, slot, layer, hi, q, delta, zero):
         H, P, N, K = self.H, self.P, self.N, self.K

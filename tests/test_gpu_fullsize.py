@@ -10,7 +10,9 @@ pair at a time.
   - serving-scale format sweep: 30 layers x batch 256, 32 heads x 128 x 128,
     fp32 / bf16 / int8 asym / int4 asym, zero initial state, two steps;
   - Mamba-2 370M-shaped scan: batch 8 x T 2048, 32 heads in three decay
-    bands, int4 asym, all heads vs the mid band only.
+    bands, int4 asym, all heads vs the mid band only;
+  - the DAMP mixed-tier step on the 130M decode shape (16 of 128 key
+    channels in FP16), hand-off and one decode launch of 24 layers x 256.
 """
 import numpy as np
 import pytest
@@ -161,3 +163,67 @@ def test_scan_370m_full(mask):
     stats = compare_states(ocfg, got, st, None, f"scan 370m {mask}")
     assert stats["code_mismatch"] == 0
     assert ssq.ssq_pool_error(cfg, pool) == 0
+
+
+def test_fullsize_damp_130m():
+    """The DAMP step as the benchmark runs it (decode_130m_damp): the pool
+    written by ssq_damp_quantize from the N(0, 1) state, one launch of 24
+    layers x 256 requests; sampled (layer, request) pairs compared with the
+    oracle: FP16 bits, codes, steps and zero points equal after the hand-off
+    and after the step, y within the readout tolerance."""
+    from poolcodec import DampCodec
+    ssq = require_gpu()
+    wl = W.decode_130m_damp()
+    H, P, N, G, K = wl.nheads, wl.headdim, wl.d_state, wl.ngroups, 16
+    cfg = ssq.DampConfig(wl.nl, wl.batch, H, P, N, G, K)
+    L = ssq.ssq_damp_pool_layout(cfg)
+    codec = DampCodec(H, P, N, K, L)
+    chan = W.damp_channels(wl.seed, wl.nl, H, N)
+    chan_t = cuda(chan, torch.int32)
+    pool = ssq.damp_alloc_pool(cfg)
+    for l in range(wl.nl):
+        S = np.stack([wl.state_pair(l, b).reshape(H, P, N) for b in range(wl.batch)])
+        ssq.ssq_damp_quantize(cfg, pool, chan_t, None, wl.batch, l, 1, cuda(S))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    samples = [(0, 0), (wl.nl - 1, wl.batch - 1), (11, 128)] + \
+        [(int(rng.integers(wl.nl)), int(rng.integers(wl.batch))) for _ in range(3)]
+
+    def read(l, b):
+        off, n = codec.layer_range(b, l)
+        codec.buf_offset = off
+        try:
+            buf = pool[off:off + n].cpu().numpy()
+            return codec.read(buf, b, l), codec.read_hi_bits(buf, b, l)
+        finally:
+            codec.buf_offset = 0
+
+    def check(st, l, b, where):
+        (hi, q, d, z), bits = read(l, b)
+        assert np.array_equal(bits, st.hi[0].astype(np.float16).view(np.uint16)), where
+        assert np.array_equal(q, st.q[0]), where
+        assert np.array_equal(d.view(np.uint32), st.delta[0].view(np.uint32)), where
+        assert np.array_equal(z.view(np.uint32), st.zero[0].view(np.uint32)), where
+
+    sts = {}
+    for (l, b) in samples:
+        oc = O.DampCfg(H, P, N, G, K, chan[l])
+        sts[(l, b)] = (oc, O.damp_from_f32(oc, wl.state_pair(l, b).reshape(H, P, N)))
+        check(sts[(l, b)][1], l, b, f"hand-off pair ({l}, {b})")
+    inp = wl.inputs()
+    y = torch.full((wl.nl, wl.batch, H, P), float("nan"), device="cuda")
+    ssq.ssq_damp_decode_step(cfg, pool, chan_t, None, wl.batch, 0, wl.nl, cuda(inp["x"]),
+                             cuda(inp["B"]), cuda(inp["C"]), cuda(inp["dt"]), cuda(inp["A"]),
+                             cuda(inp["D"]), y)
+    torch.cuda.synchronize()
+    assert ssq.ssq_damp_pool_error(cfg, pool) == 0
+    yg = y.cpu().numpy()
+    assert np.isfinite(yg).all()
+    for (l, b) in samples:
+        oc, st = sts[(l, b)]
+        x, B, C, dt = (inp[n][l, b] for n in ("x", "B", "C", "dt"))
+        y_ref = O.damp_step(oc, st, 0, x, B, C, dt, inp["A"][l], inp["D"][l])
+        check(st, l, b, f"step pair ({l}, {b})")
+        S1 = O.damp_to_f32(st)[0].astype(np.float64)          # stored state, rotated back
+        sc = np.abs(S1) @ np.abs(C[0].astype(np.float64)) + np.abs(inp["D"][l][:, None] * x)
+        assert np.all(np.abs(yg[l, b] - y_ref) <= 1e-4 * (sc + 1e-30)), f"y pair ({l}, {b})"
