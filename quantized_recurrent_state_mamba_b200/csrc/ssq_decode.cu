@@ -80,6 +80,30 @@ __device__ __forceinline__ void sts128f(unsigned a, float4 v)
                  :: "r"(a), "n"(OFF), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
 }
 
+template <int OFF>
+__device__ __forceinline__ void sts128u(unsigned a, uint4 v)
+{
+    asm volatile("st.shared.v4.b32 [%0+%1], {%2, %3, %4, %5};"
+                 :: "r"(a), "n"(OFF), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+template <int OFF>
+__device__ __forceinline__ void sts64u(unsigned a, uint2 v)
+{
+    asm volatile("st.shared.v2.b32 [%0+%1], {%2, %3};"
+                 :: "r"(a), "n"(OFF), "r"(v.x), "r"(v.y) : "memory");
+}
+
+// Write `bytes` of shared memory to global memory: the 16-byte multiple as
+// one bulk store (in this thread's current bulk group), the rest (a multiple
+// of 4 bytes) word by word.  dst and src 16-byte aligned.
+__device__ __forceinline__ void store_back(uint8_t* dst, const uint8_t* src, int bytes)
+{
+    const int b16 = bytes & ~15;
+    if (b16 > 0) bulk_s2g(dst, src, (unsigned)b16);
+    for (int i = b16; i < bytes; i += 4)
+        *reinterpret_cast<uint32_t*>(dst + i) = *reinterpret_cast<const uint32_t*>(src + i);
+}
+
 __host__ __device__ inline int r16(int v) { return (v + 15) & ~15; }
 __host__ __device__ inline int r256(int v) { return (v + 255) & ~255; }
 
@@ -311,6 +335,11 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     constexpr int NREG = QShape<N>::NREG;                    // pieces kept in registers
     constexpr int PW = F::quant ? Piece<FMT>::words : 1;     // code words per piece
     constexpr int PB = PW * 4;                               // code bytes per piece
+    // Nearest rounding writes a quantized tile's new codes and metadata back
+    // into its stage and the producer stores the tile with bulk copies
+    // (coalesced); the stochastic-rounding variant, at its register limit,
+    // stores each lane's pieces directly.
+    constexpr bool kWB = !SR;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* const smem = smem_raw + ((256u - (saddr(smem_raw) & 255u)) & 255u);
@@ -345,6 +374,26 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
 
     if (warp == kCWarps) {
         // ================= producer warp =================
+        // The consumers leave a quantized tile's new codes and metadata in
+        // its stage, laid out as in the pool; lane 0 writes them back with
+        // bulk stores once the consumers release the stage, before the
+        // stage is filled again.  Per stage: destination and bytes of the
+        // tile waiting there (pend_cb < 0: none) and the phase it was
+        // loaded in.
+        uint8_t* pend_c[kMaxStages];
+        uint8_t* pend_m[kMaxStages];
+        int pend_cb[kMaxStages], pend_mb[kMaxStages], pend_ph[kMaxStages];
+#pragma unroll
+        for (int s = 0; s < kMaxStages; ++s) pend_cb[s] = -1;
+        auto flush = [&](int s) {
+            if (pend_cb[s] < 0) return;
+            const uint8_t* pay = stages + s * geo.stage_bytes + geo.x_bytes;
+            store_back(pend_c[s], pay, pend_cb[s]);
+            store_back(pend_m[s], pay + geo.qcodes_bytes, pend_mb[s]);
+            bulk_commit();
+            bulk_wait_read<0>();        // the stage may be refilled after this
+            pend_cb[s] = -1;
+        };
         int si = 0, sph = 0, k = 0, uk = -1;
         bool bad = false, ok = true, newunit = true;
         const uint8_t* codes_u = nullptr;
@@ -423,6 +472,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 }
             }
             if (!mbar_wait<kProducerSleep>(&empty[si], sph ^ 1)) { ok = false; break; }
+            if (lane == 0) flush(si);
             uint8_t* st = stages + si * geo.stage_bytes;
             float* sx = reinterpret_cast<float*>(st);
             for (int i = lane; i < ti.n; i += 32) {
@@ -437,6 +487,13 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 uint8_t* pay = st + geo.x_bytes;
                 if (F::quant && ti.quant) {
                     const unsigned cb = (unsigned)r16(ti.n * RB), mb = (unsigned)r16(ti.n * MB);
+                    if (kWB) {
+                        pend_c[si] = const_cast<uint8_t*>(codes_u) + (long long)ti.rbase * RB;
+                        pend_m[si] = const_cast<uint8_t*>(meta_u) + (long long)ti.rbase * MB;
+                        pend_cb[si] = ti.n * RB;
+                        pend_mb[si] = ti.n * MB;
+                        pend_ph[si] = sph;
+                    }
                     mbar_arrive_tx(&full[si], cb + mb);
                     bulk_g2s(pay, codes_u + (long long)ti.rbase * RB, cb, &full[si]);
                     bulk_g2s(pay + geo.qcodes_bytes, meta_u + (long long)ti.rbase * MB, mb,
@@ -451,6 +508,21 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             if (++si == S) { si = 0; sph ^= 1; }
         }
         if (!ok && lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
+        // the last tiles' write-backs, in the order they were loaded
+        if (lane == 0) {
+            for (int jj = (k > S ? k - S : 0); jj < k; ++jj) {
+                const int s = jj % S;
+                if (pend_cb[s] < 0) continue;
+                if (ok && mbar_wait<kProducerSleep>(&empty[s], (unsigned)pend_ph[s])) {
+                    flush(s);
+                } else {
+                    ok = false;
+                    pend_cb[s] = -1;
+                }
+            }
+            if (!ok) atomicOr(err, SSQ_DEVERR_TIMEOUT);
+            bulk_wait<0>();
+        }
         // No copy may still be writing shared memory when the CTA exits.
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (lane == 0) {
@@ -542,12 +614,18 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 const unsigned cs_x = saddr(cs) | (rot * PB);
                 const unsigned bx = (saddr(gB) + j * 16) | (rot * LQ * 16);
                 const unsigned cx = (saddr(gC) + j * 16) | (rot * LQ * 16);
-                uint8_t* crow = codes_u + (long long)rr * RB + j * CB;
+                // With kWB the new codes and metadata go back into the stage,
+                // in place (the producer writes the tile back), and rows past
+                // the end of the tile store nothing, as the row they shadow
+                // may already hold new codes; otherwise they go straight to
+                // the pool (a shadow row stores row 0's bytes again).
+                uint8_t* const ms = const_cast<uint8_t*>(pay) + geo.qcodes_bytes + rl * MB;
+                uint8_t* const crow = kWB ? const_cast<uint8_t*>(cs)
+                                          : codes_u + (long long)rr * RB + j * CB;
+                uint8_t* const mrow = kWB ? ms : meta_u + (long long)rr * MB;
                 const uintptr_t crow_x = reinterpret_cast<uintptr_t>(crow) | (rot * PB);
-                uint8_t* mrow = meta_u + (long long)rr * MB;
                 float delta0, z0 = 0.0f;
                 {
-                    const uint8_t* ms = pay + geo.qcodes_bytes + rl * MB;
                     if constexpr (F::sym) {
                         delta0 = *reinterpret_cast<const float*>(ms);
                     } else {
@@ -661,7 +739,14 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         }
                         uint32_t w[PW];
                         pack16<FMT>(kk, w);
-                        {
+                        if constexpr (kWB) {
+                            if (active) {
+                                if constexpr (PW == 4)
+                                    sts128u<0>(cs_x ^ (sp * PB), make_uint4(w[0], w[1], w[2], w[3]));
+                                else
+                                    sts64u<0>(cs_x ^ (sp * PB), make_uint2(w[0], w[1]));
+                            }
+                        } else {
                             void* dst = reinterpret_cast<void*>(crow_x ^ (uintptr_t)(sp * PB));
                             if constexpr (PW == 4)
                                 __stcs(reinterpret_cast<uint4*>(dst), make_uint4(w[0], w[1], w[2], w[3]));
@@ -689,11 +774,21 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     }
                     acc = add2(acc, acc1);
                     ysum = __fmul_rn(rp.delta, grp_sum<LQ>(__fadd_rn(acc.x, acc.y)));
-                    // every lane of the row writes the same metadata
-                    if constexpr (F::sym) {
-                        __stcs(reinterpret_cast<float*>(mrow), rp.delta);
+                    if constexpr (kWB) {
+                        if (active && j == 0) {
+                            if constexpr (F::sym) {
+                                *reinterpret_cast<float*>(ms) = rp.delta;
+                            } else {
+                                *reinterpret_cast<float2*>(ms) = make_float2(rp.delta, rp.z);
+                            }
+                        }
                     } else {
-                        __stcs(reinterpret_cast<float2*>(mrow), make_float2(rp.delta, rp.z));
+                        // every lane of the row writes the same metadata
+                        if constexpr (F::sym) {
+                            __stcs(reinterpret_cast<float*>(mrow), rp.delta);
+                        } else {
+                            __stcs(reinterpret_cast<float2*>(mrow), make_float2(rp.delta, rp.z));
+                        }
                     }
                     if (__any_sync(0xffffffffu, !rp.finite) && lane == 0)
                         atomicOr(err, SSQ_DEVERR_NONFINITE);
@@ -764,8 +859,12 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             ysum = grp_sum<LF>(__fadd_rn(acc.x, acc.y));
         }
         // every lane of the row writes the same y (after the row sum all
-        // hold it)
-        __stcs(y_u + __float_as_int(hti.w) + p, __fadd_rn(ysum, __fmul_rn(hti.z, xv)));
+        // hold it); a row past the end of the tile writes nothing (with the
+        // in-place write-back it may have read its shadowed row's new codes)
+        if (active)
+            __stcs(y_u + __float_as_int(hti.w) + p, __fadd_rn(ysum, __fmul_rn(hti.z, xv)));
+        // the stage's new codes must be visible to the producer's bulk store
+        if (kWB && F::quant && ti.quant) fence_proxy_async();
         __syncwarp();
         mbar_arrive_if(&empty[si], lane == 0);
         if (++si == S) { si = 0; sph ^= 1; }
