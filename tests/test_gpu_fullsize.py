@@ -12,7 +12,9 @@ pair at a time.
   - Mamba-2 370M-shaped scan: batch 8 x T 2048, 32 heads in three decay
     bands, int4 asym, all heads vs the mid band only;
   - the DAMP mixed-tier step on the 130M decode shape (16 of 128 key
-    channels in FP16), hand-off and one decode launch of 24 layers x 256.
+    channels in FP16), hand-off and one decode launch of 24 layers x 256;
+  - the stochastic-rounding step on the 130M shape, and the prefill
+    hand-off on the 370M shape (batch 8 x T 2048).
 """
 import numpy as np
 import pytest
@@ -55,7 +57,10 @@ def init_pool_from_workload(ssq, cfg, wl, pool):
     torch.cuda.synchronize()
 
 
-def sampled_decode_check(ssq, wl, fmt, samples, steps=1, init_from_pool=True):
+SR_SEED = 12345
+
+
+def sampled_decode_check(ssq, wl, fmt, samples, steps=1, init_from_pool=True, sr=False):
     H, P, N, G = wl.nheads, wl.headdim, wl.d_state, wl.ngroups
     cfg, L, codec, ocfg = make_cfg(ssq, fmt, wl.nl, wl.batch, H, P, N, G)
     pool = ssq.alloc_pool(cfg)
@@ -74,18 +79,27 @@ def sampled_decode_check(ssq, wl, fmt, samples, steps=1, init_from_pool=True):
         inp = (wl.inputs() if k == 0 else
                W.Decode(wl.name, wl.seed + 100 * k, wl.nl, wl.batch, H, P, N, G, fmt).inputs())
         y = torch.empty((wl.nl, wl.batch, H, P), device="cuda")
-        ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, cuda(inp["x"]),
-                            cuda(inp["B"]), cuda(inp["C"]), cuda(inp["dt"]), cuda(inp["A"]),
-                            cuda(inp["D"]), y)
+        args = (cfg, pool, None, wl.batch, 0, wl.nl, cuda(inp["x"]), cuda(inp["B"]),
+                cuda(inp["C"]), cuda(inp["dt"]), cuda(inp["A"]), cuda(inp["D"]), y)
+        if sr:
+            ssq.ssq_decode_step_sr(*args, SR_SEED, k + 1)
+        else:
+            ssq.ssq_decode_step(*args)
         yh = y.cpu().numpy()
         pre = np.zeros((len(samples), H * P, N), np.float32)
         y_ref = np.zeros((len(samples), H, P), np.float32)
         for i, (l, b) in enumerate(samples):
-            y_ref[i], pre[i] = O.step(ocfg, st, i, inp["x"][l, b], inp["B"][l, b],
-                                      inp["C"][l, b], inp["dt"][l, b], inp["A"][l],
-                                      inp["D"][l], want_pre=True)
+            a = (inp["x"][l, b], inp["B"][l, b], inp["C"][l, b], inp["dt"][l, b], inp["A"][l],
+                 inp["D"][l])
+            if sr:
+                # slot = request b (identity slots), layer l
+                y_ref[i] = O.step_sr(ocfg, st, i, *a, SR_SEED, k + 1, l, b)
+            else:
+                y_ref[i], pre[i] = O.step(ocfg, st, i, *a, want_pre=True)
         got = read_pairs(codec, pool, pairs, ocfg)
-        stats = compare_states(ocfg, got, st, pre, f"{wl.name} step {k}")
+        stats = compare_states(ocfg, got, st, None if sr else pre, f"{wl.name} step {k}")
+        if sr:
+            assert stats["code_mismatch"] == 0
         C = np.stack([inp["C"][l, b] for (l, b) in samples])
         D = np.stack([inp["D"][l] for (l, b) in samples])
         x = np.stack([inp["x"][l, b] for (l, b) in samples])
@@ -105,6 +119,16 @@ def test_decode_130m_full():
     wl = W.decode_130m("i8a")
     samples = [(0, 0), (0, 255), (11, 97), (23, 255), (23, 1), (17, 128)]
     sampled_decode_check(ssq, wl, "i8a", samples)
+
+
+def test_decode_130m_sr_full():
+    """The stochastic-rounding step as the benchmark runs it
+    (decode_130m_sr): 24 layers x 256 in one launch, two steps with step
+    counters 1 and 2; sampled pairs bit-exact in codes."""
+    ssq = require_gpu()
+    wl = W.decode_130m("i8a")
+    samples = [(0, 0), (23, 255), (11, 97), (5, 200)]
+    sampled_decode_check(ssq, wl, "i8a", samples, steps=2, sr=True)
 
 
 @pytest.mark.parametrize("fmt", ["i8s", "i8a", "f32"])
@@ -227,3 +251,48 @@ def test_fullsize_damp_130m():
         S1 = O.damp_to_f32(st)[0].astype(np.float64)          # stored state, rotated back
         sc = np.abs(S1) @ np.abs(C[0].astype(np.float64)) + np.abs(inp["D"][l][:, None] * x)
         assert np.all(np.abs(yg[l, b] - y_ref) <= 1e-4 * (sc + 1e-30)), f"y pair ({l}, {b})"
+
+
+def test_prefill_370m_full():
+    """The prefill hand-off as the benchmark runs it (prefill_370m_all):
+    batch 8 x T 2048, 32 heads in three decay bands, int4 asym, from the zero
+    state; the oracle follows one request and one head from each band
+    through all 2048 tokens (heads are independent with one group): the
+    final codes bit-exact, y within the readout tolerance."""
+    ssq = require_gpu()
+    wl = W.scan_370m("all")
+    H, P, N, T, Bt = wl.nheads, wl.headdim, wl.d_state, wl.T, wl.batch
+    inp = wl.inputs()
+    cfg, L, codec, ocfg_full = make_cfg(ssq, "i4a", 1, Bt, H, P, N, 1)
+    pool = ssq.alloc_pool(cfg)
+    y = torch.empty((Bt, T, H, P), device="cuda")
+    ssq.ssq_prefill(cfg, pool, None, Bt, 0, T, cuda(inp["x"]), cuda(inp["B"]), cuda(inp["C"]),
+                    cuda(inp["dt"]), cuda(inp["A"]), cuda(inp["D"]), y)
+    yh = y.cpu().numpy()
+    assert np.all(np.isfinite(yh))
+    b = 6
+    heads = [2, 17, 30]
+    ocfg = O.Cfg(O.I4_ASYM, len(heads), P, N, 1)
+    st = O.State(ocfg, 1)
+    y_ref = O.prefill(ocfg, st, 0, inp["x"][b][:, heads], inp["B"][b], inp["C"][b],
+                      inp["dt"][b][:, heads], inp["A"][heads], inp["D"][heads])
+    # readout scale from the exact (fp64) trajectory of the same heads
+    S = np.zeros((len(heads), P, N))
+    scale = np.zeros((T, len(heads), P))
+    Cb = np.abs(inp["C"][b][:, 0].astype(np.float64))                 # [T][N]
+    for t in range(T):
+        S, _ = O.scan_f64(ocfg, S, inp["x"][b, t:t + 1][:, heads], inp["B"][b, t:t + 1],
+                          inp["C"][b, t:t + 1], inp["dt"][b, t:t + 1][:, heads],
+                          inp["A"][heads], inp["D"][heads])
+        scale[t] = np.abs(S) @ Cb[t] + np.abs(inp["D"][heads][:, None] * inp["x"][b, t][heads])
+    check_y(yh[b][:, heads], y_ref, scale, "prefill 370m")
+    gotb = read_pairs(codec, pool, [(b, 0)], ocfg_full)
+    got = O.State(ocfg, 1)
+    for i, h in enumerate(heads):
+        rows = slice(h * P, (h + 1) * P)
+        sub = slice(i * P, (i + 1) * P)
+        got.q[0, sub], got.delta[0, sub], got.zero[0, sub], got.val[0, sub] = \
+            gotb.q[0, rows], gotb.delta[0, rows], gotb.zero[0, rows], gotb.val[0, rows]
+    stats = compare_states(ocfg, got, st, None, "prefill 370m")
+    assert stats["code_mismatch"] == 0
+    assert ssq.ssq_pool_error(cfg, pool) == 0
