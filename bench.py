@@ -77,6 +77,8 @@ def workload(name):
         "prefill_370m_all": lambda: W.scan_370m("all"),
         "prefill_370m_mid": lambda: W.scan_370m("mid"),
         "decode_130m_damp": lambda: W.decode_130m_damp(),
+        "diag_130m": lambda: dataclasses.replace(
+            W.decode_130m("i8a"), name="mamba2-130m step diagnostics L24 b256 H24 P64 N128 i8a"),
     }
     if name not in table:
         raise SystemExit(f"unknown workload {name}; choose from {sorted(table)}")
@@ -115,6 +117,15 @@ def damp_bytes(wl, K=DAMP_PROTECTED):
     units = wl.nl * wl.batch * wl.nheads
     io = units * P * 4 * 2 + wl.nl * wl.batch * (2 * wl.ngroups * N + wl.nheads) * 4
     return int(2 * units * head + io + wl.nl * wl.nheads * N * 4)
+
+
+def diag_bytes(wl):
+    """Algorithmic bytes of one diagnostics pass (read-only): every stored
+    row read once, x / B / C / dt read once, four fp32 results per row
+    written."""
+    rows = wl.nl * wl.batch * wl.nheads * wl.headdim
+    io = rows * 4 + wl.nl * wl.batch * (2 * wl.ngroups * wl.d_state + wl.nheads) * 4
+    return int(rows * row_state_bytes(wl.fmt, wl.d_state) + io + rows * 16)
 
 
 def scan_bytes(wl):
@@ -161,6 +172,7 @@ _KERNEL_SOURCES = {
     "decode": ("ssq_decode.cu", "ssq_pipe.cuh"),
     "damp": ("ssq_damp.cu", "ssq_pipe.cuh"),
     "scan": ("ssq_scan.cu",),
+    "diag": ("ssq_diag.cu",),
 }
 
 
@@ -169,6 +181,8 @@ def _kernel_family(workload_name):
         return "damp"
     if workload_name.startswith(("scan", "prefill")):
         return "scan"
+    if workload_name.startswith("diag"):
+        return "diag"
     return "decode"
 
 
@@ -380,6 +394,31 @@ def oracle_damp_sample(wl, budget_s, K=DAMP_PROTECTED):
     return sec, per_pair * npairs, npairs
 
 
+def oracle_diag_sample(wl, budget_s):
+    """Time the oracle's step diagnostics on the first (layer, request)
+    pairs."""
+    import oracle as O
+    H, P, N, G = wl.nheads, wl.headdim, wl.d_state, wl.ngroups
+    ocfg = O.Cfg(O.FORMATS[wl.fmt], H, P, N, G, wl.head_mask)
+    inp = wl.inputs()
+    per_pair = diag_bytes(wl) / (wl.nl * wl.batch)
+    st = O.state_from_f32(ocfg, wl.state_pair(0, 0).reshape(1, H, P, N))
+    t = time.perf_counter()
+    O.step_diag(ocfg, st, 0, inp["x"][0, 0], inp["B"][0, 0], inp["C"][0, 0], inp["dt"][0, 0],
+                inp["A"][0], inp["D"][0])
+    one = max(time.perf_counter() - t, 1e-6)
+    npairs = int(max(1, min(wl.nl * wl.batch, budget_s / one)))
+    pairs = [(i // wl.batch, i % wl.batch) for i in range(npairs)]
+    st = O.state_from_f32(ocfg, np.stack([wl.state_pair(l, b).reshape(H, P, N)
+                                          for (l, b) in pairs]))
+    t = time.perf_counter()
+    for i, (l, b) in enumerate(pairs):
+        O.step_diag(ocfg, st, i, inp["x"][l, b], inp["B"][l, b], inp["C"][l, b],
+                    inp["dt"][l, b], inp["A"][l], inp["D"][l])
+    sec = time.perf_counter() - t
+    return sec, per_pair * npairs, npairs
+
+
 def oracle_scan_sample(wl, budget_s, prefill=False):
     import oracle as O
     H, P, N = wl.nheads, wl.headdim, wl.d_state
@@ -416,11 +455,14 @@ def cpu_leg(wl, budget_s, name=""):
         rsps = n / sec
     else:
         damp = name.endswith("_damp")
-        sample_fn = oracle_damp_sample if damp else oracle_decode_sample
+        diag = name.startswith("diag")
+        sample_fn = (oracle_damp_sample if damp else
+                     oracle_diag_sample if diag else oracle_decode_sample)
         sec, nbytes, n = sample_fn(wl, budget_s)
-        sample = (f"{n} of {wl.nl * wl.batch} (layer, request) pairs of one "
-                  f"{'DAMP ' if damp else ''}decode step (layer-major from pair 0), "
-                  f"single thread")
+        what = "DAMP decode step" if damp else ("step diagnostics pass" if diag
+                                                else "decode step")
+        sample = (f"{n} of {wl.nl * wl.batch} (layer, request) pairs of one {what} "
+                  f"(layer-major from pair 0), single thread")
         rsps = n / sec
     return {"value": nbytes / sec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": sample, "seconds": round(sec, 3),
@@ -523,6 +565,16 @@ def run_ours(args, wl, name):
             scan_fn(cfg, pool, None, wl.batch, 0, wl.T, d["x"], d["B"], d["C"], d["dt"],
                     d["A"], d["D"], y)
         units = wl.batch * wl.T          # request-tokens
+    elif name.startswith("diag"):
+        # the diagnostics pass reads the state and writes four numbers per
+        # row; y stands for its output in the end-to-end leg
+        y = torch.empty((wl.nl, wl.batch, H, P, 4), device=dev)
+        nbytes = diag_bytes(wl)
+
+        def step():
+            ssq.ssq_decode_diag(cfg, pool, None, wl.batch, 0, wl.nl, d["x"], d["B"], d["C"],
+                                d["dt"], d["A"], y)
+        units = wl.batch * wl.nl
     elif damp:
         y = torch.empty((wl.nl, wl.batch, H, P), device=dev)
         nbytes = damp_bytes(wl)
@@ -620,6 +672,9 @@ def run_ours(args, wl, name):
         elif damp:
             ssq.ssq_damp_decode_step(cfg, pool, chan, None, wl.batch, 0, wl.nl, t["x"], t["B"],
                                      t["C"], t["dt"], d["A"], d["D"], yb[kk], stream=s_c)
+        elif name.startswith("diag"):
+            ssq.ssq_decode_diag(cfg, pool, None, wl.batch, 0, wl.nl, t["x"], t["B"], t["C"],
+                                t["dt"], d["A"], yb[kk], stream=s_c)
         else:
             ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, t["x"], t["B"], t["C"],
                                 t["dt"], d["A"], d["D"], yb[kk], stream=s_c)

@@ -23,7 +23,7 @@ namespace ssq {
 namespace {
 
 template <int FMT, int N>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 diag_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv,
             float4* __restrict__ diag)
 {
@@ -106,23 +106,27 @@ diag_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
             }
         }
 
-        // the update, as the decode step forms it
+        // the update, as the decode step forms it (B is dead once w is formed)
         const float xv = __ldg(cv.x + (lb * H + h) * P + p);
         const float dtv = __ldg(cv.dt + lb * H + h);
         const float lam = decay(dtv, __ldg(cv.A + (long long)l * H + h));
         const float dtx = __fmul_rn(dtv, xv);
-        float Bv[E], Cv[E], w[E];
-        load_f32<E>(Bv, cv.B + (lb * G + g) * N + j * E);
-        load_f32<E>(Cv, cv.C + (lb * G + g) * N + j * E);
+        float w[E];
+        {
+            float Bv[E];
+            load_f32<E>(Bv, cv.B + (lb * G + g) * N + j * E);
 #pragma unroll
-        for (int n = 0; n < E; ++n) {
-            w[n] = __fmul_rn(dtx, Bv[n]);
-            s[n] = __fmaf_rn(lam, s[n], w[n]);
+            for (int n = 0; n < E; ++n) {
+                w[n] = __fmul_rn(dtx, Bv[n]);
+                s[n] = __fmaf_rn(lam, s[n], w[n]);
+            }
         }
-        float signal = 0.0f, tot = 0.0f, rev_err = 0.0f;
-        int rev = 0;
+        // rounding error e_n = fl(deq_n - s'_n) and the reversal flags (bit
+        // n), before C is read
+        float e[E];
+        uint32_t rev_mask = 0u;
 #pragma unroll
-        for (int n = 0; n < E; ++n) signal = __fmaf_rn(Cv[n], s[n], signal);
+        for (int n = 0; n < E; ++n) e[n] = 0.0f;
         if constexpr (F::quant) {
             if (qrow) {
                 // the refit and rounding of the decode step (warp-uniform
@@ -134,17 +138,23 @@ diag_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallVie
 #pragma unroll
                 for (int n = 0; n < E; ++n) {
                     const float deq = __fmul_rn(rq[n], rp.delta);
-                    const float e = __fsub_rn(deq, s[n]);
-                    const float inc = __fadd_rn(e, w[n]);
+                    e[n] = __fsub_rn(deq, s[n]);
+                    const float inc = __fadd_rn(e[n], w[n]);
                     const bool reversed = (w[n] > 0.0f && inc < 0.0f) || (w[n] < 0.0f && inc > 0.0f);
-                    tot = __fmaf_rn(Cv[n], e, tot);
-                    if (reversed) {
-                        ++rev;
-                        rev_err = __fmaf_rn(Cv[n], e, rev_err);
-                    }
+                    rev_mask |= (reversed ? 1u : 0u) << n;
                 }
             }
         }
+        float Cv[E];
+        load_f32<E>(Cv, cv.C + (lb * G + g) * N + j * E);
+        float signal = 0.0f, tot = 0.0f, rev_err = 0.0f;
+#pragma unroll
+        for (int n = 0; n < E; ++n) {
+            signal = __fmaf_rn(Cv[n], s[n], signal);
+            tot = __fmaf_rn(Cv[n], e[n], tot);
+            if ((rev_mask >> n) & 1u) rev_err = __fmaf_rn(Cv[n], e[n], rev_err);
+        }
+        int rev = __popc(rev_mask);
         signal = grp_sum<LPR>(signal);
         tot = grp_sum<LPR>(tot);
         rev_err = grp_sum<LPR>(rev_err);
