@@ -83,3 +83,24 @@ def test_reference_arm_runs_on_rank_0_only():
     assert res[0][0] == 0 and res[1][0] == 0
     assert '"impl": "reference"' in res[0][1]
     assert res[1][1] == ""
+
+
+def test_kernel_source_hash_ignores_comments_only():
+    """The ncu summaries stay attached to a kernel through comment edits and
+    drop off when its code changes; each kernel family hashes its own
+    sources."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = "int f(int x) { return x + 1; } // one\n/* two\n lines */ int g;"
+    b = "int f(int x)  {\n  return x + 1;\n}\n// other words\nint g;"
+    c = "int f(int x) { return x + 2; } int g;"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    fams = {bench._kernel_family(w) for w in
+            ("decode_130m", "decode_130m_sr", "decode_130m_damp", "scan_370m_all",
+             "prefill_370m_mid", "diag_130m")}
+    assert fams == {"decode", "damp", "scan", "diag"}
+    hashes = {w: bench.kernel_source_hash(w) for w in
+              ("decode_130m", "decode_130m_damp", "scan_370m_all", "diag_130m")}
+    assert len(set(hashes.values())) == 4
+    assert bench.kernel_source_hash("decode_130m_sr") == hashes["decode_130m"]
