@@ -23,9 +23,11 @@
 // value is bit-identical to a scalar evaluation in that order; the readout
 // accumulates and rotates back in fp32.
 //
-// Thread mapping: a position's P values sit on LPR = P/16 consecutive lanes,
-// 16 per lane (lane j of the group holds rotated indices 16j .. 16j+15); a
-// warp covers 32/LPR positions per pass.
+// Thread mapping: a position's P values sit on LPR consecutive lanes, E per
+// lane (lane j of the group holds rotated indices jE .. jE+E-1); a warp
+// covers 32/LPR positions per pass.  The hand-off and read-back kernels use
+// E = 16 with one CTA per head; the decode step uses E = 32 (16 at P = 16)
+// with one warp per head (below).
 #include <cuda_fp16.h>
 
 #include <type_traits>
@@ -38,7 +40,7 @@ namespace ssq {
 
 namespace {
 
-constexpr int kDampE = 16;   // rotated entries per lane
+constexpr int kDampE = 16;   // rotated entries per lane (hand-off, read-back)
 
 // Reduce-scatter of a lane's E partial sums over the positions of its warp:
 // at each round a lane keeps half of its values and sends the other half to
