@@ -268,3 +268,28 @@ def test_damp_codec_round_trip(ssq):
     # the block sits where the layout says: nothing else written
     o = L["header_bytes"] + 2 * L["slot_bytes"] + 1 * L["layer_bytes"]
     assert not buf[:o].any() and not buf[o + H * L["head_bytes"]:].any()
+
+
+def test_binding_constants_match_header(ssq):
+    """The binding's copies of the header's constants (error-word bits, pool
+    header and alignment, the head limit) equal the header's values."""
+    src = open(HEADER).read()
+    defs = dict(re.findall(r"#define\s+(SSQ_\w+)\s+(0x[0-9a-fA-F]+|\d+)u?\b", src))
+    assert {"SSQ_DEVERR_SLOT", "SSQ_DEVERR_NONFINITE", "SSQ_DEVERR_TIMEOUT",
+            "SSQ_DEVERR_CHANNEL", "SSQ_POOL_HEADER_BYTES", "SSQ_POOL_ALIGN",
+            "SSQ_MAX_HEADS"} <= set(defs)
+    for name, val in defs.items():
+        assert getattr(ssq, name) == int(val, 0), name
+
+
+def test_damp_channel_maps_are_permutations():
+    """The seeded channel maps of the DAMP workloads are one permutation of
+    0..d_state-1 per (layer, head), reproducible from the seed."""
+    from quantized_recurrent_state_mamba_b200 import workloads as W
+    c = W.damp_channels(7, 3, 5, 128)
+    assert c.shape == (3, 5, 128) and c.dtype == np.int32
+    for l in range(3):
+        for h in range(5):
+            assert np.array_equal(np.sort(c[l, h]), np.arange(128))
+    assert np.array_equal(c, W.damp_channels(7, 3, 5, 128))
+    assert not np.array_equal(c, W.damp_channels(8, 3, 5, 128))
