@@ -161,9 +161,12 @@ typedef struct {
     int n_quant_heads, n_fp_heads;
 } ssq_layout;
 
-/* Compute the pool layout for cfg.  head_perm (HOST, nheads int32, may be
- * NULL) receives the natural head index stored at each region position.
- * Host only; no CUDA call. */
+/* Compute the pool layout for cfg ("Mamba state quantization for
+ * inference", "Recurrent state is fixed per request, not free": one state
+ * per live request, sized by the format; "Mixed precision spends bits on
+ * persistent channels": each precision tier one contiguous region).
+ * head_perm (HOST, nheads int32, may be NULL) receives the natural head
+ * index stored at each region position.  Host only; no CUDA call. */
 SSQ_API ssq_status ssq_pool_layout(const ssq_config* cfg, ssq_layout* out,
                            int32_t* head_perm);
 
@@ -191,8 +194,12 @@ SSQ_API ssq_status ssq_quantize_rows(const ssq_config* cfg, void* pool,
                              int nl, const float* S, cudaStream_t stream);
 
 /* Read pool slots back as fp32 (checkpointing, tests): the inverse layout of
- * ssq_quantize_rows, each row decoded as (q - z)*Delta, q*Delta or the fp
- * value.  S_out: device fp32 [nl][batch][nheads][headdim][d_state]. */
+ * ssq_quantize_rows, each row decoded as (q - z)*Delta (asymmetric grid),
+ * q*Delta (symmetric grid) or the fp value ("ssm-state-quantization"
+ * README, Setup: the two grids and the per-row scale).
+ *   S_out  device fp32 [nl][batch][nheads][headdim][d_state], natural head
+ *          order, 16-byte aligned; slot_idx, layer0, nl as ssq_quantize_rows.
+ * Rows of a request whose slot index is out of range are not written. */
 SSQ_API ssq_status ssq_dequantize_rows(const ssq_config* cfg, const void* pool,
                                const int32_t* slot_idx, int batch,
                                int layer0, int nl, float* S_out,
@@ -313,8 +320,8 @@ SSQ_API ssq_status ssq_prefill(const ssq_config* cfg, void* pool,
  * held as d_state key channels, each the Hadamard-rotated value vector
  *     t[k] = sum_p H[k][p] S[p][n],   H[k][p] = (-1)^popcount(k & p)
  * (the +-1 Sylvester-Hadamard matrix of order headdim; H/sqrt(headdim) is
- * orthonormal), summed in double in the order p = 0..headdim-1 and rounded
- * once to fp32.  A per-(layer, head) channel map chan[m] (a permutation of
+ * orthonormal), formed in double by the fast Walsh-Hadamard transform
+ * (butterfly stages of span 1, 2, ..., headdim/2) and rounded once to fp32.  A per-(layer, head) channel map chan[m] (a permutation of
  * 0..d_state-1, chosen by calibration outside the library) puts the
  * n_protected protected channels first: positions m < n_protected keep t in
  * FP16 (round to nearest even), the others in INT8 on the asymmetric grid of
@@ -385,7 +392,8 @@ SSQ_API ssq_status ssq_damp_quantize(const ssq_damp_config* cfg, void* pool,
                              cudaStream_t stream);
 
 /* Read DAMP pool slots back as fp32: S[p][chan[m]] = (1/headdim) sum_k
- * H[p][k] t_m[k], summed in double in the order k, rounded once.
+ * H[p][k] t_m[k], formed in double by the same butterfly transform and
+ * rounded once.
  *   S_out  device fp32 [nl][batch][nheads][headdim][d_state] */
 SSQ_API ssq_status ssq_damp_dequantize(const ssq_damp_config* cfg, const void* pool,
                                const int32_t* chan, const int32_t* slot_idx,

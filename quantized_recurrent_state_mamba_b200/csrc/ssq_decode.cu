@@ -20,9 +20,13 @@
 //     "unit" it stages B and C and builds a head table (lambda, dt, D, the
 //     y offset and the B/C group of every head of the region), so a
 //     consumer row finds everything it needs with two shared loads;
-//   - 11 consumer warps compute from shared memory and store the new rows,
-//     metadata and y straight to global memory.  A row of a quantized head
-//     is held by d_state/64 lanes of 64 entries, streamed 16 at a time;
+//   - 11 consumer warps compute from shared memory; with nearest rounding a
+//     quantized row's new codes and metadata go back into its stage, in
+//     place, and the producer stores the finished tile with bulk copies
+//     (the stochastic-rounding variant stores each lane's pieces directly);
+//     y goes straight to global memory.  A row of a quantized head is held
+//     by one lane (two at d_state 256) of up to 128 entries, streamed 16 at
+//     a time;
 //   - B and C are staged with lane j's 16-byte chunks interleaved, so the
 //     lanes of a row read distinct banks;
 //   - waits sleep between tries of the mbarrier, and every wait is

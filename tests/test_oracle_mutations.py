@@ -57,6 +57,18 @@ MUTATIONS = {
                            "const float b = B[(size_t)g * N + m];"),
     "damp_protected_not_fp16": ("hi[(size_t)m * P + k] = oref_fp16_round(t[(size_t)m * P + k]);",
                                 "hi[(size_t)m * P + k] = t[(size_t)m * P + k];"),
+    "philox_round_multiplier": ("(uint64_t)0xD2511F53u * (uint64_t)c0",
+                                "(uint64_t)0xD2511F57u * (uint64_t)c0"),
+    "philox_weyl_constant": ("k1 += 0xBB67AE85u;", "k1 += 0xBB67AE87u;"),
+    "philox_nine_rounds": ("for (int round = 0; round < 10; ++round)",
+                           "for (int round = 0; round < 9; ++round)"),
+    "philox_output_words_swapped": ("out[0] = c0; out[1] = c1;", "out[0] = c1; out[1] = c0;"),
+    "philox_key_words_swapped": ("const uint32_t key[2] = {(uint32_t)r->seed, (uint32_t)(r->seed >> 32)};",
+                                 "const uint32_t key[2] = {(uint32_t)(r->seed >> 32), (uint32_t)r->seed};"),
+    "sr_draw_other_half": ("return (out[(n % 8) / 2] >> (16 * (n % 2))) & 0xFFFFu;",
+                           "return (out[(n % 8) / 2] >> (16 * (1 - n % 2))) & 0xFFFFu;"),
+    "decode_batch_layer0_decay": ("dt + lb * H, A + l * H, D + l * H,",
+                                  "dt + lb * H, A, D + l * H,"),
     "damp_y_before_store": ("        /* readout from the stored state, rotated back */\n"
                             "        damp_load_head(c, hi, q, dl, z, t);\n",
                             "        /* readout from the stored state, rotated back */\n"),
@@ -80,6 +92,7 @@ def test_pins_catch_mutation(name):
         r = subprocess.run(
             [sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
              os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-             os.path.join(ROOT, "tests", "test_oracle_damp.py")],
+             os.path.join(ROOT, "tests", "test_oracle_damp.py"),
+             os.path.join(ROOT, "tests", "test_oracle_philox.py")],
             cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
         assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"

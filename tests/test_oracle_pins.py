@@ -800,3 +800,30 @@ def test_diag_reversals_from_the_step_results(oref, fmt):
     rev_err = np.where(rev, C[0][None, None, :].astype(np.float64) * e, 0.0).sum(axis=-1)
     assert np.all(np.abs(rev_err - diag[..., 1]) <= 1e-5 * (np.abs(diag[..., 3]) + 1e-3))
     assert rev.sum() > 0                     # the small state makes reversals common
+
+
+def test_decode_batch_is_the_step_of_every_pair(oref):
+    """One decode step over nl layers x batch requests (the batched entry the
+    decode call mirrors) equals the single-pair step of each (layer,
+    request) pair with that pair's own inputs and its layer's A and D."""
+    nl, batch = 2, 3
+    cfg = O.Cfg(O.I8_ASYM, 4, 4, 16, 2)
+    wl = W.Decode("pin", seed=5, nl=nl, batch=batch, nheads=4, headdim=4, d_state=16,
+                  ngroups=2, fmt="i8a")
+    inp = wl.inputs()
+    S0 = np.stack([wl.state_pair(l, b).reshape(4, 4, 16)
+                   for l in range(nl) for b in range(batch)])
+    st_b = O.state_from_f32(cfg, S0)
+    st_p = st_b.copy()
+    y_b = O.decode_batch(cfg, st_b, nl, batch, inp["x"], inp["B"], inp["C"], inp["dt"],
+                         inp["A"], inp["D"])
+    for l in range(nl):
+        for b in range(batch):
+            i = l * batch + b
+            y = O.step(cfg, st_p, i, inp["x"][l, b], inp["B"][l, b], inp["C"][l, b],
+                       inp["dt"][l, b], inp["A"][l], inp["D"][l])
+            assert np.array_equal(y, y_b[l, b]), (l, b)
+    assert np.array_equal(st_b.q, st_p.q)
+    assert np.array_equal(st_b.delta, st_p.delta)
+    assert np.array_equal(st_b.zero, st_p.zero)
+    assert not np.array_equal(inp["A"][0], inp["A"][1])
