@@ -14,11 +14,14 @@ per-token scan.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
 device synchronize, timed with CUDA events on the launching stream; the max
-over ranks is taken.  The state pool (gigabytes) is far larger than the
-126 MB L2, so the state is read from HBM every step; no L2 flush is needed.
-Multi-GPU runs are independent replicas (weak scaling, no collective on the
-data path).  --impl reference times the CPU oracle on a bounded sample of the
-same workload (rank 0 only).
+over ranks is taken; the kernel time of the roofline is the median launch.
+A step whose footprint (state, inputs, output) is under 4x the L2 rotates
+over enough copies of them that every step reads from HBM; the line says
+which.  --gpus N starts N ranks (one per GPU, torch.distributed.run on
+127.0.0.1) when no launcher did; they are independent replicas (weak
+scaling, no collective on the data path).  --impl reference times the CPU
+oracle on every host core of rank 0 on a bounded sample of the same
+workload.
 """
 from __future__ import annotations
 
@@ -57,6 +60,7 @@ DAMP_PROTECTED = 16        # DAMP layout: key channels per head kept in FP16
 
 def workload(name):
     table = {
+        "tiny": lambda: W.tiny(),
         "decode_130m": lambda: W.decode_130m("i8a"),
         "decode_130m_f32": lambda: W.decode_130m("f32"),
         "decode_130m_sr": lambda: W.decode_130m("i8a"),
@@ -135,6 +139,38 @@ def scan_bytes(wl):
                           + wl.nheads) * 4
     rows = wl.batch * wl.nheads * wl.headdim
     return int(per_tok * wl.T + 2 * rows * row_state_bytes(wl.fmt, wl.d_state))
+
+
+def footprint_bytes(wl, name):
+    """Distinct bytes one step touches: the stored state it reads and writes
+    in place (one copy), its inputs and its output."""
+    if isinstance(wl, W.Scan):
+        rows = wl.batch * wl.nheads * wl.headdim
+        return scan_bytes(wl) - rows * row_state_bytes(wl.fmt, wl.d_state)
+    if name.startswith("diag"):
+        return diag_bytes(wl)
+    if name.endswith("_damp"):
+        P, N, K = wl.headdim, wl.d_state, DAMP_PROTECTED
+        units = wl.nl * wl.batch * wl.nheads
+        return damp_bytes(wl) - units * (2 * K * P + (N - K) * P + 8 * (N - K))
+    rows = wl.nl * wl.batch * wl.nheads * wl.headdim
+    qfrac = 1.0
+    if wl.head_mask is not None and wl.fmt not in ("f32", "bf16"):
+        qfrac = float(np.mean(np.asarray(wl.head_mask) != 0))
+    state = rows * (qfrac * row_state_bytes(wl.fmt, wl.d_state)
+                    + (1 - qfrac) * row_state_bytes("f32", wl.d_state))
+    return int(decode_bytes(wl) - state)
+
+
+L2_FALLBACK_BYTES = 126 * 1024 * 1024
+
+
+def l2_bytes(device):
+    import torch
+    try:
+        return int(torch.cuda.get_device_properties(device).L2_cache_size)
+    except Exception:
+        return L2_FALLBACK_BYTES
 
 
 def elem_steps(wl):
@@ -447,6 +483,7 @@ def oracle_scan_sample(wl, budget_s, prefill=False):
 
 
 def cpu_leg(wl, budget_s, name=""):
+    """The oracle, single thread, on a bounded sample of the workload."""
     if isinstance(wl, W.Scan):
         pf = name.startswith("prefill")
         sec, nbytes, n = oracle_scan_sample(wl, budget_s, prefill=pf)
@@ -469,27 +506,203 @@ def cpu_leg(wl, budget_s, name=""):
             "request_steps_per_s_per_layer": rsps}
 
 
+# ---- the oracle on every host core ------------------------------------------
+# One worker process per core (spawn start method: this process may already
+# hold a CUDA context).  Each worker receives its share of the sample's
+# inputs and builds its states untimed ("load"), then steps them ("run"); the
+# parent times the run phase on the wall clock from the first "run" message
+# to the last answer.
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_worker(conn):
+    import oracle as O
+    job = None
+    while True:
+        msg = conn.recv()
+        if msg[0] == "stop":
+            break
+        if msg[0] == "load":
+            job = _worker_load(O, msg[1])
+            conn.send("ready")
+        elif msg[0] == "run":
+            t = time.perf_counter()
+            _worker_run(O, job)
+            conn.send(time.perf_counter() - t)
+
+
+def _worker_load(O, task):
+    kind = task["kind"]
+    H, P, N, G = task["shape"]
+    if kind == "damp":
+        cfgs = [O.DampCfg(H, P, N, G, task["K"], c) for c in task["chan"]]
+        sts = [O.damp_from_f32(cfgs[i], S) for i, S in enumerate(task["S0"])]
+        return dict(task, cfgs=cfgs, sts=sts)
+    cfg = O.Cfg(task["fmt"], H, P, N, G, task["mask"])
+    if kind == "scan":
+        return dict(task, cfg=cfg, st=O.State(cfg, len(task["x"])))
+    st = O.state_from_f32(cfg, np.stack(task["S0"]))
+    return dict(task, cfg=cfg, st=st)
+
+
+def _worker_run(O, job):
+    kind = job["kind"]
+    if kind == "scan":
+        run = O.prefill if job["prefill"] else O.scan
+        for i in range(len(job["x"])):
+            run(job["cfg"], job["st"], i, job["x"][i], job["B"][i], job["C"][i], job["dt"][i],
+                job["A"], job["D"])
+        return
+    for i in range(len(job["x"])):
+        args = (job["x"][i], job["B"][i], job["C"][i], job["dt"][i], job["A"][i], job["D"][i])
+        if kind == "damp":
+            O.damp_step(job["cfgs"][i], job["sts"][i], 0, *args)
+        elif kind == "diag":
+            O.step_diag(job["cfg"], job["st"], i, *args[:5], job["D"][i])
+        else:
+            O.step(job["cfg"], job["st"], i, *args)
+
+
+def _pair_tasks(wl, name, pairs, workers):
+    """Split the (layer, request) pairs over the workers; each task carries
+    its pairs' inputs and initial states."""
+    import oracle as O
+    inp = wl.inputs()
+    H, P, N = wl.nheads, wl.headdim, wl.d_state
+    damp = name.endswith("_damp")
+    kind = "damp" if damp else ("diag" if name.startswith("diag") else "decode")
+    chan = W.damp_channels(wl.seed, wl.nl, H, N) if damp else None
+    tasks = []
+    for w in range(workers):
+        mine = pairs[w::workers]
+        t = {"kind": kind, "shape": (H, P, N, wl.ngroups), "fmt": O.FORMATS[wl.fmt],
+             "mask": wl.head_mask, "K": DAMP_PROTECTED,
+             "S0": [wl.state_pair(l, b).reshape(H, P, N) for (l, b) in mine],
+             "x": [inp["x"][l, b] for (l, b) in mine], "B": [inp["B"][l, b] for (l, b) in mine],
+             "C": [inp["C"][l, b] for (l, b) in mine], "dt": [inp["dt"][l, b] for (l, b) in mine],
+             "A": [inp["A"][l] for (l, b) in mine], "D": [inp["D"][l] for (l, b) in mine]}
+        if damp:
+            t["chan"] = [chan[l] for (l, b) in mine]
+        tasks.append(t)
+    return tasks
+
+
+def _scan_tasks(wl, name, ntok, workers):
+    """One request per worker (the scan is sequential in t), each running
+    its first ntok tokens."""
+    import oracle as O
+    inp = wl.inputs()
+    tasks = []
+    for w in range(workers):
+        b = w % wl.batch
+        tasks.append({"kind": "scan", "prefill": name.startswith("prefill"),
+                      "shape": (wl.nheads, wl.headdim, wl.d_state, wl.ngroups),
+                      "fmt": O.FORMATS[wl.fmt], "mask": wl.head_mask,
+                      "x": [inp["x"][b, :ntok]], "B": [inp["B"][b, :ntok]],
+                      "C": [inp["C"][b, :ntok]], "dt": [inp["dt"][b, :ntok]],
+                      "A": inp["A"], "D": inp["D"]})
+    return tasks
+
+
+def cpu_leg_all_cores(wl, budget_s, name="", max_workers=None):
+    """The oracle, as it stands, on every host core: one process per core,
+    each stepping its share of a bounded sample of the workload (about
+    budget_s seconds of wall time).  Returns the cpu_baseline record, with
+    the single-thread figure of cpu_leg beside it."""
+    import multiprocessing as mp
+    single = cpu_leg(wl, max(1.0, budget_s / 4), name)
+    cores = host_cores()
+    is_scan = isinstance(wl, W.Scan)
+    units_total = wl.batch if is_scan else wl.nl * wl.batch
+    workers = max(1, min(cores, max_workers or cores, units_total))
+    if is_scan:
+        # tokens per request so the run lasts about budget_s
+        per_tok = single["seconds"] / max(1, int(single["request_steps_per_s_per_layer"]
+                                                 * single["seconds"]))
+        ntok = int(max(1, min(wl.T, budget_s / max(per_tok, 1e-9))))
+        tasks = _scan_tasks(wl, name, ntok, workers)
+        units = workers * ntok
+        nbytes = scan_bytes(wl) * units / (wl.T * wl.batch)
+        what = (f"{workers} requests x {ntok} tokens of the "
+                f"{'prefill' if name.startswith('prefill') else 'scan'}, one request per process")
+    else:
+        per_pair = single["seconds"] / max(1, int(single["request_steps_per_s_per_layer"]
+                                                  * single["seconds"]))
+        npairs = int(max(workers, min(units_total,
+                                      workers * budget_s / max(per_pair, 1e-9))))
+        pairs = [(i // wl.batch, i % wl.batch) for i in range(npairs)]
+        tasks = _pair_tasks(wl, name, pairs, workers)
+        units = npairs
+        per_bytes = (damp_bytes(wl) if name.endswith("_damp") else
+                     diag_bytes(wl) if name.startswith("diag") else decode_bytes(wl))
+        nbytes = per_bytes * npairs / (wl.nl * wl.batch)
+        what = (f"{npairs} of {units_total} (layer, request) pairs (layer-major from pair 0), "
+                f"split over {workers} processes")
+    ctx = mp.get_context("spawn")
+    conns, procs = [], []
+    try:
+        for _ in range(workers):
+            a, b = ctx.Pipe()
+            pr = ctx.Process(target=_oracle_worker, args=(b,), daemon=True)
+            pr.start()
+            conns.append(a)
+            procs.append(pr)
+        for c, t in zip(conns, tasks):
+            c.send(("load", t))
+        for c in conns:
+            assert c.recv() == "ready"
+        t0 = time.perf_counter()
+        for c in conns:
+            c.send(("run",))
+        busy = [c.recv() for c in conns]
+        wall = time.perf_counter() - t0
+    finally:
+        for c in conns:
+            try:
+                c.send(("stop",))
+            except (BrokenPipeError, OSError):
+                pass
+        for pr in procs:
+            pr.join(timeout=30)
+    return {"value": nbytes / wall / 1e9, "unit": "GB/s", "cores": workers, "kind": "oracle",
+            "sample": what, "seconds": round(wall, 3),
+            "request_steps_per_s_per_layer": units / wall,
+            "host_cores": cores, "worker_busy_s_max": round(max(busy), 3),
+            "single_thread": {"value": single["value"], "unit": "GB/s",
+                              "sample": single["sample"], "seconds": single["seconds"]}}
+
+
 def run_reference(args, wl, name):
+    """The reference arm: the CPU oracle, as it stands, on every host core of
+    rank 0 (other ranks exit at once); each step a bounded sample of the
+    workload, so the whole --steps K --warmup W run ends within minutes."""
     world, rank, _ = dist_setup()
     if rank != 0:
         return 0
     steps, warm = args.steps, args.warmup
-    budget = max(0.5, 120.0 / max(1, steps + warm))
+    budget = max(0.5, min(20.0, 150.0 / max(1, steps + warm)))
     for _ in range(warm):
-        cpu_leg(wl, budget, name)
-    vals, secs = [], 0.0
+        cpu_leg_all_cores(wl, budget, name, args.cpu_workers)
+    vals, secs, rec = [], 0.0, None
     for _ in range(steps):
-        r = cpu_leg(wl, budget, name)
-        vals.append(r["value"])
-        secs += r["seconds"]
-    value = statistics.mean(vals)
+        rec = cpu_leg_all_cores(wl, budget, name, args.cpu_workers)
+        vals.append(rec["value"])
+        secs += rec["seconds"]
+    value = statistics.median(vals)
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
            "n_gpus": world, "steps": steps, "warmup": warm,
            "ms_per_step": 1000 * secs / max(1, steps), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
            "config": {"workload": wl.name, "bench_workload": name},
-           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                            "sample": r["sample"] + " per step"},
+           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": rec["cores"],
+                            "kind": "oracle", "sample": rec["sample"] + " per step",
+                            "host_cores": rec["host_cores"],
+                            "single_thread": rec["single_thread"]},
            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out))
@@ -529,12 +742,12 @@ def run_ours(args, wl, name):
                              d_state=N, ngroups=G, n_protected=DAMP_PROTECTED)
         pool = ssq.damp_alloc_pool(cfg, dev)
         chan = torch.from_numpy(W.damp_channels(wl.seed, n_layers, H, N)).to(dev)
-        pool_error = lambda: ssq.ssq_damp_pool_error(cfg, pool)  # noqa: E731
+        pool_error = lambda pl: ssq.ssq_damp_pool_error(cfg, pl)  # noqa: E731
     else:
         cfg = ssq.Config(n_layers=n_layers, n_slots=wl.batch, nheads=H, headdim=P, d_state=N,
                          ngroups=G, fmt=fmt, head_mask=wl.head_mask)
         pool = ssq.alloc_pool(cfg, dev)
-        pool_error = lambda: ssq.ssq_pool_error(cfg, pool)  # noqa: E731
+        pool_error = lambda pl: ssq.ssq_pool_error(cfg, pl)  # noqa: E731
 
     # initial state
     if damp:
@@ -554,52 +767,70 @@ def run_ours(args, wl, name):
                                   torch.from_numpy(S).to(dev))
         torch.cuda.synchronize()
 
+    # L2: below 4x the L2, the timed steps rotate over enough copies of the
+    # pool, the inputs and the output that each step finds its state and
+    # inputs evicted by the copies stepped since its last turn.
+    l2 = l2_bytes(dev)
+    foot = footprint_bytes(wl, name)
+    copies = 1 if foot >= 4 * l2 else int(math.ceil(4 * l2 / foot))
+    pools = [pool] + [pool.clone() for _ in range(copies - 1)]
+    ds = [d] + [{k: v.clone() for k, v in d.items()} for _ in range(copies - 1)]
+    if copies == 1:
+        l2_note = (f"step footprint {foot / 1e6:.0f} MB >= 4x the {l2 / 1e6:.0f} MB L2; "
+                   f"no rotation, no flush")
+    else:
+        l2_note = (f"step footprint {foot / 1e6:.1f} MB < 4x the {l2 / 1e6:.0f} MB L2: "
+                   f"timed steps rotate over {copies} copies of pool, inputs and output "
+                   f"({copies * foot / 1e6:.0f} MB)")
+
     # the prefill hand-off runs the scan's shape with the state in fp32
     # between tokens and one quantization at the end
     scan_fn = ssq.ssq_prefill if name.startswith("prefill") else ssq.ssq_scan
+    sr = name.endswith("_sr")
     if is_scan:
-        y = torch.empty((wl.batch, wl.T, H, P), device=dev)
+        yshape = (wl.batch, wl.T, H, P)
         nbytes = scan_bytes(wl)
-
-        def step():
-            scan_fn(cfg, pool, None, wl.batch, 0, wl.T, d["x"], d["B"], d["C"], d["dt"],
-                    d["A"], d["D"], y)
         units = wl.batch * wl.T          # request-tokens
     elif name.startswith("diag"):
         # the diagnostics pass reads the state and writes four numbers per
         # row; y stands for its output in the end-to-end leg
-        y = torch.empty((wl.nl, wl.batch, H, P, 4), device=dev)
+        yshape = (wl.nl, wl.batch, H, P, 4)
         nbytes = diag_bytes(wl)
-
-        def step():
-            ssq.ssq_decode_diag(cfg, pool, None, wl.batch, 0, wl.nl, d["x"], d["B"], d["C"],
-                                d["dt"], d["A"], y)
-        units = wl.batch * wl.nl
-    elif damp:
-        y = torch.empty((wl.nl, wl.batch, H, P), device=dev)
-        nbytes = damp_bytes(wl)
-
-        def step():
-            ssq.ssq_damp_decode_step(cfg, pool, chan, None, wl.batch, 0, wl.nl, d["x"], d["B"],
-                                     d["C"], d["dt"], d["A"], d["D"], y)
         units = wl.batch * wl.nl
     else:
-        y = torch.empty((wl.nl, wl.batch, H, P), device=dev)
-        nbytes = decode_bytes(wl)
-
-        # the stochastic-rounding variant draws fresh randomness every step
-        sr = name.endswith("_sr")
-        nstep = [0]
-
-        def step():
-            if sr:
-                nstep[0] += 1
-                ssq.ssq_decode_step_sr(cfg, pool, None, wl.batch, 0, wl.nl, d["x"], d["B"],
-                                       d["C"], d["dt"], d["A"], d["D"], y, 12345, nstep[0])
-            else:
-                ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, d["x"], d["B"],
-                                    d["C"], d["dt"], d["A"], d["D"], y)
+        yshape = (wl.nl, wl.batch, H, P)
+        nbytes = damp_bytes(wl) if damp else decode_bytes(wl)
         units = wl.batch * wl.nl         # request-layer steps
+    y = torch.empty(yshape, device=dev)
+    ys = [y] + [torch.empty_like(y) for _ in range(copies - 1)]
+    nstep = [0]
+
+    def launch(pool_i, t, y_i, stream=None):
+        """One step of the workload's call on the given pool, inputs and
+        output (the stochastic-rounding variant draws fresh randomness each
+        step)."""
+        if is_scan:
+            scan_fn(cfg, pool_i, None, wl.batch, 0, wl.T, t["x"], t["B"], t["C"], t["dt"],
+                    d["A"], d["D"], y_i, stream=stream)
+        elif name.startswith("diag"):
+            ssq.ssq_decode_diag(cfg, pool_i, None, wl.batch, 0, wl.nl, t["x"], t["B"], t["C"],
+                                t["dt"], d["A"], y_i, stream=stream)
+        elif damp:
+            ssq.ssq_damp_decode_step(cfg, pool_i, chan, None, wl.batch, 0, wl.nl, t["x"],
+                                     t["B"], t["C"], t["dt"], d["A"], d["D"], y_i,
+                                     stream=stream)
+        elif sr:
+            nstep[0] += 1
+            ssq.ssq_decode_step_sr(cfg, pool_i, None, wl.batch, 0, wl.nl, t["x"], t["B"],
+                                   t["C"], t["dt"], d["A"], d["D"], y_i, 12345, nstep[0],
+                                   stream=stream)
+        else:
+            ssq.ssq_decode_step(cfg, pool_i, None, wl.batch, 0, wl.nl, t["x"], t["B"], t["C"],
+                                t["dt"], d["A"], d["D"], y_i, stream=stream)
+
+    def step(i):
+        k = i % copies
+        launch(pools[k], ds[k], ys[k])
 
     stream = torch.cuda.current_stream(dev)
     # The clock sampler starts before the warm-up, so that its first NVML
@@ -609,10 +840,10 @@ def run_ours(args, wl, name):
     t_wait = time.perf_counter()
     while sampler.ok and len(sampler.samples) < 3 and time.perf_counter() - t_wait < 2.0:
         time.sleep(0.005)
-    for _ in range(args.warmup):
-        step()
+    for i in range(max(args.warmup, copies)):
+        step(i)
     torch.cuda.synchronize()
-    if pool_error() != 0:
+    if any(pool_error(pl) != 0 for pl in pools):
         raise SystemExit("device error word set during warm-up")
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -622,7 +853,7 @@ def run_ours(args, wl, name):
     t0 = time.perf_counter()
     for i in range(K):
         ev[i][0].record(stream)
-        step()
+        step(i)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     t1 = time.perf_counter()
@@ -630,7 +861,7 @@ def run_ours(args, wl, name):
     sampler.stop()
     region_ms = ev[0][0].elapsed_time(ev[-1][1])
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    kern_ms = statistics.mean(launch_ms)
+    kern_ms = statistics.median(launch_ms)
     # device time between steps (the host enqueueing late), for the record
     host_gap_ms = max(0.0, region_ms - sum(launch_ms))
     region_ms = max_over_ranks(region_ms, world, dev)
@@ -666,18 +897,7 @@ def run_ours(args, wl, name):
         if i >= 2:
             s_c.wait_event(ev_out[kk])
         t = din[kk]
-        if is_scan:
-            scan_fn(cfg, pool, None, wl.batch, 0, wl.T, t["x"], t["B"], t["C"], t["dt"],
-                    d["A"], d["D"], yb[kk], stream=s_c)
-        elif damp:
-            ssq.ssq_damp_decode_step(cfg, pool, chan, None, wl.batch, 0, wl.nl, t["x"], t["B"],
-                                     t["C"], t["dt"], d["A"], d["D"], yb[kk], stream=s_c)
-        elif name.startswith("diag"):
-            ssq.ssq_decode_diag(cfg, pool, None, wl.batch, 0, wl.nl, t["x"], t["B"], t["C"],
-                                t["dt"], d["A"], yb[kk], stream=s_c)
-        else:
-            ssq.ssq_decode_step(cfg, pool, None, wl.batch, 0, wl.nl, t["x"], t["B"], t["C"],
-                                t["dt"], d["A"], d["D"], yb[kk], stream=s_c)
+        launch(pools[i % copies], t, yb[kk], stream=s_c)
         ev_c[kk].record(s_c)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_c[kk])
@@ -701,7 +921,9 @@ def run_ours(args, wl, name):
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
     e2e_value = job_throughput(nbytes, K, world, e2e_ms)
     e2e_launches = K
-    err = pool_error()
+    err = 0
+    for pl in pools:
+        err |= pool_error(pl)
 
     peak, peak_kind = measured_peaks()
     achieved = nbytes / (kern_ms / 1e3) / 1e9
@@ -723,12 +945,14 @@ def run_ours(args, wl, name):
                     "unit": "Top/s (fp32 pipe operations)", "frac": round(alu_ach / alu_peak, 4),
                     "traffic": traffic, "peak_source": "148 SMs x 128 fp32 lanes x max SM clock",
                     "kernel_ms_per_launch": round(kern_ms, 5),
+                    "kernel_ms_stat": f"median of {K} launches (CUDA events)",
                     "hbm_achieved_gbs": round(achieved, 2)}
     else:
         roofline = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                     "unit": "GB/s", "frac": round(achieved / peak, 4),
                     "traffic": traffic, "peak_source": peak_kind,
-                    "kernel_ms_per_launch": round(kern_ms, 5)}
+                    "kernel_ms_per_launch": round(kern_ms, 5),
+                    "kernel_ms_stat": f"median of {K} launches (CUDA events)"}
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -740,7 +964,7 @@ def run_ours(args, wl, name):
                    "nheads": H, "headdim": P, "d_state": N, "ngroups": G,
                    "T": getattr(wl, "T", 1),
                    "algorithmic_bytes_per_step": nbytes,
-                   "l2": "state pool and per-step traffic far above the 126 MB L2; no flush",
+                   "l2": l2_note, "pool_copies": copies,
                    "parallelism": f"replicas x{world}"},
         "request_steps_per_s_per_layer": round(units * K * world / (region_ms / 1e3), 1),
         "pct_of_measured_hbm": round(100 * value / world / peak, 2),
@@ -756,13 +980,28 @@ def run_ours(args, wl, name):
         "device_error_word": err,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_leg(wl, args.cpu_budget, name)
+        out["cpu_baseline"] = cpu_leg_all_cores(wl, args.cpu_budget, name,
+                                                args.cpu_workers)
     if rank == 0:
         print(json.dumps(out))
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def spawn_ranks(n):
+    """Run this command as n ranks on this node (torch.distributed.run,
+    rendezvous on 127.0.0.1) and return its exit code."""
+    import socket
+    import subprocess
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 def main():
@@ -775,10 +1014,21 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-workers", type=int, default=None,
+                    help="cap on the oracle worker processes (default: every host core)")
     ap.add_argument("--nl", type=int, default=None,
                     help="layers per decode launch (a smaller case of the same shape, "
                          "for profiler captures; the bench lines use the workload's own)")
     args = ap.parse_args()
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        # one process per GPU: start the ranks here when no launcher did
+        return spawn_ranks(args.gpus)
+    if world_env is not None and int(world_env) != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started "
+                         f"WORLD_SIZE={world_env} ranks")
     wl = workload(args.workload)
     if args.nl is not None:
         if not isinstance(wl, W.Decode):

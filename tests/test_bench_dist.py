@@ -68,7 +68,7 @@ def _ref_rank(rank, world, out):
     import bench
     from quantized_recurrent_state_mamba_b200 import workloads as W
     wl = W.tiny()
-    args = argparse.Namespace(steps=1, warmup=0, cpu_budget=0.5)
+    args = argparse.Namespace(steps=1, warmup=0, cpu_budget=0.5, cpu_workers=2)
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
         rc = bench.run_reference(args, wl, "tiny")
@@ -104,3 +104,48 @@ def test_kernel_source_hash_ignores_comments_only():
               ("decode_130m", "decode_130m_damp", "scan_370m_all", "diag_130m")}
     assert len(set(hashes.values())) == 4
     assert bench.kernel_source_hash("decode_130m_sr") == hashes["decode_130m"]
+
+
+def test_gpus_n_starts_n_ranks_when_no_launcher_did():
+    """bench.py --gpus 2 without a launcher starts two ranks itself
+    (torch.distributed.run on 127.0.0.1); with the reference arm rank 0
+    prints the one JSON line and reports both ranks."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--workload", "tiny", "--steps", "1", "--warmup", "0",
+                        "--cpu-budget", "0.5", "--cpu-workers", "1"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2
+    assert rec["cpu_baseline"]["cores"] == 1
+
+
+def test_gpus_n_must_match_the_launcher():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "4", "--workload", "tiny", "--steps", "1", "--warmup", "0"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "WORLD_SIZE=2" in r.stderr
+
+
+def test_l2_rotation_counts():
+    """A step whose footprint is under 4x the L2 rotates over enough copies
+    to reach it; the 130M decode step needs none."""
+    sys.path.insert(0, ROOT)
+    import bench
+    L2 = bench.L2_FALLBACK_BYTES
+    big = bench.workload("decode_130m")
+    assert bench.footprint_bytes(big, "decode_130m") > 4 * L2
+    small = bench.workload("decode_8b_b64_i8a")
+    f = bench.footprint_bytes(small, "decode_8b_b64_i8a")
+    rows = 64 * 128 * 64
+    assert f == rows * (128 + 8) + bench.decode_bytes(small) - 2 * rows * (128 + 8)
+    assert f < 4 * L2
