@@ -9,50 +9,65 @@
 // packed write-back in one pass), with the quantizer of
 // "ssm-state-quantization" README, Setup.
 //
-// Structure (persistent, warp-specialised, one CTA of 12 warps per SM):
-//   - work is a sequence of tiles (up to RPT rows of one region of one
-//     (layer, request)); each CTA owns a contiguous range of that sequence;
-//   - a producer warp streams each tile's packed rows and metadata from HBM
-//     (prefetched into L2 as soon as the tile is next in line) into a ring
-//     of shared-memory stages with bulk asynchronous copies
-//     (cp.async.bulk, completion counted in bytes on an mbarrier) and the
-//     tile's x values with cp.async.  Once per (layer, request, region)
-//     "unit" it stages B and C and builds a head table (lambda, dt, D, the
-//     y offset and the B/C group of every head of the region), so a
-//     consumer row finds everything it needs with two shared loads;
-//   - 11 consumer warps compute from shared memory; with nearest rounding a
-//     quantized row's new codes and metadata go back into its stage, in
-//     place, and the producer stores the finished tile with bulk copies
-//     (the stochastic-rounding variant stores each lane's pieces directly);
-//     y goes straight to global memory.  A row of a quantized head is held
-//     by one lane (two at d_state 256) of up to 128 entries, streamed 16 at
-//     a time;
-//   - B and C are staged with lane j's 16-byte chunks interleaved, so the
-//     lanes of a row read distinct banks;
-//   - waits sleep between tries of the mbarrier, and every wait is
-//     bounded: one that runs out sets SSQ_DEVERR_TIMEOUT in the pool's error
-//     word and the CTA winds down (the producer first waits for its own
-//     copies in flight).
+// Structure (persistent, warp-specialised, one CTA of 17 warps per SM):
+//   - work is a sequence of tiles (up to 512 rows of the quantized region, or
+//     128 fp rows at d_state 128, of one (layer, request)); each CTA owns a
+//     contiguous range of that sequence;
+//   - a producer warp streams each tile into a ring of shared-memory stages:
+//     the packed codes with tensor copies (TMA, cp.async.bulk.tensor) laid
+//     out in the 128-byte swizzle, so that the lanes of a warp, one row each,
+//     read the same logical 16-byte chunk of their rows from distinct banks;
+//     the metadata and fp rows with bulk copies; x with cp.async.  Once per
+//     (layer, request, region) "unit" it stages B and C and builds a head
+//     table (lambda, dt, D, the y offset and the B/C group of every head);
+//   - 16 consumer warps share each tile, 32 rows a warp.  A lane owns a
+//     quantized row (two lanes at d_state 256): all lanes of a warp
+//     walk their rows' entries in the same order, so B and C come from
+//     shared memory as warp-wide broadcasts.  The updated row waits in the
+//     warp's columns of tensor memory (TMEM, tcgen05.st / tcgen05.ld)
+//     between the min/max pass and the rounding pass, which keeps the kernel
+//     within 120 registers per thread at 17 warps per SM;
+//   - a warp writes its rows' new codes back into the stage, in place, and
+//     then copies its 32 rows from the stage to the pool with 16-byte stores
+//     in row-major order (8 lanes per 128-byte line: every store instruction
+//     writes whole lines); each row's metadata is stored straight from the
+//     row's lane.  The producer only loads: no write-back is queued behind a
+//     refill;
+//   - fp rows (the fp32 / bf16 formats and the unmasked heads of the integer
+//     formats) are streamed by N/32 lanes of 32 entries and stored straight
+//     to global memory;
+//   - every wait is bounded: one that runs out sets SSQ_DEVERR_TIMEOUT in the
+//     pool's error word and the CTA winds down (the producer first waits for
+//     its own copies in flight; TMEM is released on every path).
 #include "ssq_common.cuh"
 #include "ssq_params.h"
 #include "ssq_pipe.cuh"
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
 #include <type_traits>
 
 namespace ssq {
 
 namespace {
 
-// One CTA of 12 warps per SM: three warps per SM sub-partition, so each
-// thread may hold up to 168 registers (the row of 64 entries plus the f32x2
-// operand pairs stay in registers).
-constexpr int kCWarps = 11;    // + 1 producer
-constexpr int kMinBlocks = 1;  // CTAs per SM
+constexpr int kCWarps = 16;                 // consumer warps
+// Consumer groups (tiles alternate between them).  One group of all 16 warps
+// on 512-row tiles measured fastest: with two or four groups on smaller
+// tiles the single producer warp could not prepare tiles as fast as the
+// consumers took them.
+constexpr int kGroups = 1;
+constexpr int kGWarps = kCWarps / kGroups;  // warps per group
 constexpr int kCThreads = kCWarps * 32;
-constexpr int kDThreads = kCThreads + 32;
+constexpr int kGThreads = kGWarps * 32;
+constexpr int kDThreads = kCThreads + 32;   // + 1 producer warp
 constexpr int kMaxStages = 8;
-// Shared-memory vector loads / stores at 32-bit shared addresses (the
-// quantized path forms its addresses with one XOR each).
+constexpr int kBoxRows = 128;               // rows per tensor copy
+constexpr unsigned kTmemCols = 512;         // all of TMEM: 128 columns per consumer warp
+
+// ---- PTX wrappers: shared memory at 32-bit addresses --------------------
 template <int OFF>
 __device__ __forceinline__ uint4 lds128(unsigned a)
 {
@@ -77,68 +92,144 @@ __device__ __forceinline__ float4 lds128f(unsigned a)
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a), "n"(OFF) : "memory");
     return v;
 }
-template <int OFF>
-__device__ __forceinline__ void sts128f(unsigned a, float4 v)
+// Stores predicated inside the instruction, so the warp stays converged
+// around the tcgen05 instructions that follow.
+__device__ __forceinline__ void sts128u_if(unsigned a, uint4 v, bool pred)
 {
-    asm volatile("st.shared.v4.f32 [%0+%1], {%2, %3, %4, %5};"
-                 :: "r"(a), "n"(OFF), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+    asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %5, 0;\n"
+                 " @p st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n}\n"
+                 :: "r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"((unsigned)pred)
+                 : "memory");
+}
+__device__ __forceinline__ void sts64u_if(unsigned a, uint2 v, bool pred)
+{
+    asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %3, 0;\n"
+                 " @p st.shared.v2.b32 [%0], {%1, %2};\n}\n"
+                 :: "r"(a), "r"(v.x), "r"(v.y), "r"((unsigned)pred) : "memory");
 }
 
-template <int OFF>
-__device__ __forceinline__ void sts128u(unsigned a, uint4 v)
+// ---- tensor copies (TMA) -------------------------------------------------
+// Codes of a pool as a 4-d tensor of bytes: [slot][layer][line][128], a line
+// being 128 bytes of a layer's code region.  The innermost coordinate is
+// always 0.
+__device__ __forceinline__ void tma_load_codes(void* dst, const CUtensorMap* map, int line,
+                                               int layer, int slot, uint64_t* bar)
 {
-    asm volatile("st.shared.v4.b32 [%0+%1], {%2, %3, %4, %5};"
-                 :: "r"(a), "n"(OFF), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+        :: "r"(saddr(dst)), "l"(map), "r"(0), "r"(line), "r"(layer), "r"(slot), "r"(saddr(bar))
+        : "memory");
 }
-template <int OFF>
-__device__ __forceinline__ void sts64u(unsigned a, uint2 v)
+__device__ __forceinline__ void tma_prefetch_codes(const CUtensorMap* map, int line, int layer,
+                                                   int slot)
 {
-    asm volatile("st.shared.v2.b32 [%0+%1], {%2, %3};"
-                 :: "r"(a), "n"(OFF), "r"(v.x), "r"(v.y) : "memory");
+    asm volatile(
+        "cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
+        :: "l"(map), "r"(0), "r"(line), "r"(layer), "r"(slot) : "memory");
 }
 
-// Write `bytes` of shared memory to global memory: the 16-byte multiple as
-// one bulk store (in this thread's current bulk group), the rest (a multiple
-// of 4 bytes) word by word.  dst and src 16-byte aligned.
-__device__ __forceinline__ void store_back(uint8_t* dst, const uint8_t* src, int bytes)
+// The 128-byte swizzle of the tensor copies: the 16-byte chunk index of a
+// shared-memory offset (bits 4..6) is XORed with its 128-byte line index
+// (bits 7..9); offsets are from a 1024-byte aligned base.
+__host__ __device__ inline unsigned swz128(unsigned off)
 {
-    const int b16 = bytes & ~15;
-    if (b16 > 0) bulk_s2g(dst, src, (unsigned)b16);
-    for (int i = b16; i < bytes; i += 4)
-        *reinterpret_cast<uint32_t*>(dst + i) = *reinterpret_cast<const uint32_t*>(src + i);
+    return off ^ (((off >> 7) & 7u) << 4);
+}
+
+// ---- tensor memory (tcgen05) ---------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, unsigned ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(saddr(dst)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, unsigned ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                 :: "r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// 16 fp32 values of this lane into 16 consecutive columns of its TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10,"
+        " %11, %12, %13, %14, %15, %16};"
+        :: "r"(taddr), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]),
+           "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]),
+           "f"(v[13]), "f"(v[14]), "f"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// ... and back, waiting for the load in the same statement (the registers
+// are written asynchronously until the wait).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10,"
+        " %11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+          "=f"(v[7]), "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]),
+          "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+// Named barrier of the consumer warps (the producer does not take part).
+__device__ __forceinline__ void consumers_sync()
+{
+    asm volatile("bar.sync 1, %0;" :: "n"(kCThreads) : "memory");
 }
 
 __host__ __device__ inline int r16(int v) { return (v + 15) & ~15; }
 __host__ __device__ inline int r256(int v) { return (v + 255) & ~255; }
+__host__ __device__ inline int r1024(int v) { return (v + 1023) & ~1023; }
 
 // ---- tile sequence -----------------------------------------------------
-// Tiles are ordered (layer, request, region, row block).  A CTA walks a
-// contiguous range of them with counters (one division at the start).
+// Tiles are ordered (layer, request, region, row block).  Every warp walks
+// the CTA's contiguous range of them with counters (one division at the
+// start); the tiles loaded into the ring are numbered in that order, and
+// loaded tile k goes to stage k % S and consumer group k % kGroups.
 struct TileWalk {
     long long lb;   // layer * batch + request
     int l, b, k;    // k: tile within (layer, request)
     bool quant;
     int rbase, n;   // first region row, rows in this tile
 
-    __device__ __forceinline__ void fill(const PoolView& pv, const CallView& cv)
+    __device__ __forceinline__ void fill(int Hq, int Hf, int P, const CallView& cv)
     {
         quant = k < cv.qtiles;
         const int rpt = quant ? cv.rows_per_tile : cv.rows_per_tile_f;
         rbase = (quant ? k : k - cv.qtiles) * rpt;
-        const int nrows = (quant ? pv.Hq : pv.Hf) * pv.P;
+        const int nrows = (quant ? Hq : Hf) * P;
         n = min(rpt, nrows - rbase);
     }
-    __device__ __forceinline__ void start(const PoolView& pv, const CallView& cv, long long t)
+    __device__ __forceinline__ void start(int Hq, int Hf, int P, const CallView& cv, long long t)
     {
         const int per_lb = cv.qtiles + cv.ftiles;
         lb = t / per_lb;
         k = (int)(t - lb * per_lb);
         l = (int)(lb / cv.batch);
         b = (int)(lb - (long long)l * cv.batch);
-        fill(pv, cv);
+        fill(Hq, Hf, P, cv);
     }
     // Advance; true when the next tile starts a new unit.
-    __device__ __forceinline__ bool next(const PoolView& pv, const CallView& cv)
+    __device__ __forceinline__ bool next(int Hq, int Hf, int P, const CallView& cv)
     {
         const bool was_quant = quant;
         if (++k == cv.qtiles + cv.ftiles) {
@@ -148,107 +239,97 @@ struct TileWalk {
                 b = 0;
                 ++l;
             }
-            fill(pv, cv);
+            fill(Hq, Hf, P, cv);
             return true;
         }
-        fill(pv, cv);
+        fill(Hq, Hf, P, cv);
         return quant != was_quant;
     }
 };
 
 // ---- shared-memory geometry (host and device agree on it) --------------
-// Unit buffer: [16 B header: slot, bad][B: G*N f32][C: G*N f32]
+// Unit buffer: [256 B header: slot, bad][B: G*N f32][C: G*N f32]
 //              [head table: Hpad x float4 {lambda, dt, D, y offset}]
 //              [group table: Hpad x int (g*N)]
-// Stage:       [x: RPT f32, padded to 128 B][payload: codes + meta, or fp rows]
+// Stage:       [x: RPT f32, padded to 1024 B]
+//              [codes: RPTq*RB bytes, swizzled, padded to 1024 B][meta: RPTq*MB]
+//           or [x][fp rows: RPTf*N elements]
 struct DecodeGeom {
     int S;            // stages
     int RPTq, RPTf;   // rows per tile in the quantized / fp region
-    int x_bytes;      // x area of a stage
-    int qcodes_bytes; // codes area of a quantized tile
+    int x_bytes;      // x area of a stage (a multiple of 1024)
+    int qcodes_bytes; // codes area of a quantized tile (a multiple of 1024)
     int pay_bytes;    // payload area of a stage
     int stage_bytes;
     int ub_B, ub_C, ub_ht, ub_gt, unit_bytes;  // unit buffer layout
     int Hpad;
-    int off_units, off_stages, off_scr, scr_warp_bytes, smem_bytes;
+    int off_units, off_stages, smem_bytes;
 };
 
-// Offsets are from a 256-byte aligned base inside the dynamic shared memory
-// (the launch adds 256 bytes of slack); B, C and every stage start on a
-// 256-byte boundary, so per-lane addresses can be permuted with one XOR.
-// scr_lane_bytes: per lane spill area of a consumer warp (0: none).
+// Offsets are from a 1024-byte aligned base inside the dynamic shared memory
+// (the launch adds 1024 bytes of slack); every stage and its codes area start
+// on a 1024-byte boundary (the 128-byte swizzle repeats every 1024 bytes).
 __host__ __device__ inline DecodeGeom decode_geom(int S, int RPTq, int RPTf, int RB, int MB,
                                                   int fpEB, bool has_q, bool has_fp, int N,
-                                                  int H, int G, int scr_lane_bytes)
+                                                  int H, int G)
 {
     DecodeGeom g;
     g.S = S;
     g.RPTq = RPTq;
     g.RPTf = RPTf;
-    g.x_bytes = r256((RPTq > RPTf ? RPTq : RPTf) * 4);
-    g.qcodes_bytes = has_q ? r256(RPTq * RB) : 0;
+    g.x_bytes = r1024((RPTq > RPTf ? RPTq : RPTf) * 4);
+    g.qcodes_bytes = has_q ? r1024(RPTq * RB) : 0;
     const int qpay = has_q ? g.qcodes_bytes + r16(RPTq * MB) : 0;
     const int fpay = has_fp ? RPTf * N * fpEB : 0;
     g.pay_bytes = qpay > fpay ? qpay : fpay;
-    g.stage_bytes = r256(g.x_bytes + g.pay_bytes);
+    g.stage_bytes = r1024(g.x_bytes + g.pay_bytes);
     g.Hpad = (H + 3) & ~3;
     g.ub_B = 256;                      // [0, 16): slot, bad flag
     g.ub_C = g.ub_B + G * N * 4;
     g.ub_ht = r256(g.ub_C + G * N * 4);
     g.ub_gt = g.ub_ht + g.Hpad * 16;
     g.unit_bytes = r256(g.ub_gt + g.Hpad * 4);
-    const int bars = r256((2 * kMaxStages + 4) * 8);
-    g.off_units = bars;
-    g.off_stages = g.off_units + 2 * g.unit_bytes;
-    g.off_scr = g.off_stages + S * g.stage_bytes;
-    g.scr_warp_bytes = has_q ? 32 * scr_lane_bytes : 0;
-    g.smem_bytes = g.off_scr + kCWarps * g.scr_warp_bytes + 256;
+    g.off_units = 1024;                // barriers and the TMEM address before it
+    g.off_stages = r1024(g.off_units + 2 * g.unit_bytes);
+    g.smem_bytes = g.off_stages + S * g.stage_bytes + 1024;
     return g;
 }
 
-// Lane shapes.  A quantized row is held by one lane (the whole row for
-// d_state <= 128; two lanes at 256): the per-row work (refit, addresses,
-// metadata, the tile bookkeeping) is spread over 128 entries and the row
-// reductions need no shuffles.  Of the lane's 8 pieces of 16 entries, the
-// first kRegPieces stay in registers between the update and the rounding
-// and the rest wait in a per-lane shared-memory area, which keeps the kernel
-// within the register budget of three warps per SM sub-partition.  An fp
-// row (the fp32 / bf16 formats, and unmasked heads of the integer formats)
-// is streamed by N/32 lanes of 32 entries.
+// Lane shapes.  A quantized row is held by one lane (two at d_state 256):
+// up to 128 entries, streamed in pieces of 16.  An fp row is streamed by
+// N/32 lanes of 32 entries.
 constexpr int kQuantE = 128;
-constexpr int kRegPieces = 5;
 template <int N>
 struct QShape {
     static constexpr int E = N >= kQuantE ? kQuantE : N;
     static constexpr int LPR = N / E;
-    static constexpr int RPT = kCThreads / LPR;   // rows per tile
-    static constexpr int NP = E / 16;             // pieces per lane
-    static constexpr int NREG = NP < kRegPieces ? NP : kRegPieces;
-    static constexpr int SCR = (NP - NREG) * 16 * 4;   // spill bytes per lane
+    static constexpr int RPT = kGThreads / LPR;   // rows per tile
 };
 template <int N>
 struct FShape {
     static constexpr int E = N >= 32 ? 32 : N;
     static constexpr int LPR = N / E;
-    static constexpr int RPT = kCThreads / LPR;
+    static constexpr int RPT = kGThreads / LPR;
 };
 
 // A whole quantized row by the formulas verbatim (every fp32 operation one
 // IEEE rounding in the order of the definition), for warps where some row
 // falls outside the magic-number paths: a zero point or scaled values of
-// 2^22 or more in magnitude (rows far from zero relative to their range).  Every lane of the warp
-// calls it together (the row reductions are shuffles).  Codes are read from
-// and written in natural order; B and C come from the interleaved layout.
+// 2^22 or more in magnitude (rows far from zero relative to their range).
+// Every lane of the warp calls it together (the row reductions are
+// shuffles).  Codes are read from and written to the stage at their
+// swizzled places (cs0: the lane's first code byte as an unswizzled offset
+// from the 1024-aligned stage base sb); B and C in natural order; mrow is
+// the row's metadata in the pool.
 template <int FMT, int N, bool SR>
-__device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float delta0, float z0,
-                                        float lam, float dtx, const float* __restrict__ gB,
+__device__ __noinline__ float row_exact(uint8_t* __restrict__ sb, unsigned cs0, float delta0,
+                                        float z0, float lam, float dtx,
+                                        const float* __restrict__ gB,
                                         const float* __restrict__ gC, int j, bool active,
-                                        uint8_t* __restrict__ crow, uint8_t* __restrict__ mrow,
-                                        uint32_t* err, SrKey srk)
+                                        uint8_t* __restrict__ mrow, uint32_t* err, SrKey srk)
 {
     using F = Fmt<FMT>;
     constexpr int E = QShape<N>::E, LPR = QShape<N>::LPR;
-    constexpr int NP = E / 16;
     constexpr int CB = E * F::bits / 8;
     float s[E];
     float lo = 0.0f, hi = 0.0f;
@@ -256,16 +337,14 @@ __device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float de
     for (int n = 0; n < E; ++n) {
         int q;
         if constexpr (F::bits == 8) {
-            const uint32_t bb = cs[n];
+            const uint32_t bb = sb[swz128(cs0 + n)];
             q = F::sym ? (int)(int8_t)bb : (int)bb;
         } else {
-            const uint32_t bb = (cs[n / 2] >> (4 * (n % 2))) & 0xFu;
+            const uint32_t bb = (sb[swz128(cs0 + n / 2)] >> (4 * (n % 2))) & 0xFu;
             q = F::sym ? (int)((bb ^ 8u) - 8u) : (int)bb;
         }
         const float v = __fmul_rn(__fsub_rn((float)q, z0), delta0);
-        const int pc = n / 16, i = (n % 16) / 4, e = n % 4;
-        const int bi = ((i * NP + pc) * LPR + j) * 4 + e;
-        const float w = __fmul_rn(dtx, gB[bi]);
+        const float w = __fmul_rn(dtx, gB[j * E + n]);
         const float sv = __fmaf_rn(lam, v, w);
         s[n] = sv;
         lo = n == 0 ? sv : fminf(lo, sv);
@@ -273,9 +352,9 @@ __device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float de
     }
     const RowParams rp = refit_from_minmax<FMT, LPR>(lo, hi);
     float acc = 0.0f;
-    uint32_t words[CB / 4];
+    uint32_t words[CB / 4 > 0 ? CB / 4 : 1];
 #pragma unroll
-    for (int i = 0; i < CB / 4; ++i) words[i] = 0u;
+    for (int i = 0; i < (CB / 4 > 0 ? CB / 4 : 1); ++i) words[i] = 0u;
 #pragma unroll 1
     for (int n = 0; n < E; ++n) {
         float c, r;
@@ -299,19 +378,18 @@ __device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float de
         }
         const uint32_t code = (uint32_t)(int)c & ((1u << F::bits) - 1u);
         words[n * F::bits / 32] |= code << ((n * F::bits) % 32);
-        const int pc = n / 16, i = (n % 16) / 4, e = n % 4;
-        const int ci = ((i * NP + pc) * LPR + j) * 4 + e;
-        acc = __fmaf_rn(gC[ci], __fmul_rn(r, rp.delta), acc);
+        acc = __fmaf_rn(gC[j * E + n], __fmul_rn(r, rp.delta), acc);
     }
     const float ysum = grp_sum<LPR>(acc);
     if (active) {
 #pragma unroll
-        for (int i = 0; i < CB / 4; ++i) reinterpret_cast<uint32_t*>(crow)[i] = words[i];
+        for (int i = 0; i < CB / 4; ++i)
+            *reinterpret_cast<uint32_t*>(sb + swz128(cs0 + 4 * i)) = words[i];
         if (j == 0) {
             if constexpr (F::sym) {
-                *reinterpret_cast<float*>(mrow) = rp.delta;
+                __stcs(reinterpret_cast<float*>(mrow), rp.delta);
             } else {
-                *reinterpret_cast<float2*>(mrow) = make_float2(rp.delta, rp.z);
+                __stcs(reinterpret_cast<float2*>(mrow), make_float2(rp.delta, rp.z));
             }
             if (!rp.finite) atomicOr(err, SSQ_DEVERR_NONFINITE);
         }
@@ -319,12 +397,16 @@ __device__ __noinline__ float row_exact(const uint8_t* __restrict__ cs, float de
     return ysum;
 }
 
+struct CodesMap {
+    CUtensorMap map;   // 64-byte aligned inside the kernel parameters
+};
+
 // SR: round the quantized rows stochastically (draws keyed by cv.sr_seed
 // and countered by row block, layer, slot and cv.sr_step).
 template <int FMT, int N, bool SR>
-__global__ void __launch_bounds__(kDThreads, kMinBlocks)
+__global__ void __launch_bounds__(kDThreads, 1)
 decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv,
-              const __grid_constant__ DecodeGeom geo)
+              const __grid_constant__ DecodeGeom geo, const __grid_constant__ CodesMap cm)
 {
     using F = Fmt<FMT>;
     // quantized rows: EQ entries per lane, LQ lanes per row; fp rows: EF, LF
@@ -336,34 +418,32 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     constexpr int MB = F::meta_bytes;
     constexpr int FEB = kBf16 ? 2 : 4;                       // fp element bytes
     constexpr int NP = EQ / 16;                              // 16-entry pieces per lane
-    constexpr int NREG = QShape<N>::NREG;                    // pieces kept in registers
     constexpr int PW = F::quant ? Piece<FMT>::words : 1;     // code words per piece
     constexpr int PB = PW * 4;                               // code bytes per piece
-    // Nearest rounding writes a quantized tile's new codes and metadata back
-    // into its stage and the producer stores the tile with bulk copies
-    // (coalesced); the stochastic-rounding variant, at its register limit,
-    // stores each lane's pieces directly.
-    constexpr bool kWB = !SR;
+    constexpr int kBoxLines = F::quant ? (kBoxRows * RB + 127) / 128 : 1;
+    constexpr int kBoxes = F::quant ? (QShape<N>::RPT + kBoxRows - 1) / kBoxRows : 1;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* const smem = smem_raw + ((256u - (saddr(smem_raw) & 255u)) & 255u);
+    uint8_t* const smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
     uint64_t* ufull = empty + kMaxStages;
     uint64_t* uempty = ufull + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(uempty + 2);
     uint32_t* err = reinterpret_cast<uint32_t*>(pv.pool);
 
     const int S = geo.S;
-    const int H = pv.H, P = pv.P, G = pv.G;
+    const int H = pv.H, P = pv.P, G = pv.G, Hq = pv.Hq, Hf = pv.Hf;
     const long long total = cv.total_tiles;
     const long long t0 = total * blockIdx.x / gridDim.x;
     const long long t1 = total * (blockIdx.x + 1) / gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool use_tmem = F::quant && Hq > 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kCWarps);
+            mbar_init(&empty[s], kGWarps);
         }
         for (int u = 0; u < 2; ++u) {
             mbar_init(&ufull[u], 1);
@@ -371,43 +451,29 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (use_tmem && warp == 0) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
 
     uint8_t* const units = smem + geo.off_units;
     uint8_t* const stages = smem + geo.off_stages;
 
     if (warp == kCWarps) {
         // ================= producer warp =================
-        // The consumers leave a quantized tile's new codes and metadata in
-        // its stage, laid out as in the pool; lane 0 writes them back with
-        // bulk stores once the consumers release the stage, before the
-        // stage is filled again.  Per stage: destination and bytes of the
-        // tile waiting there (pend_cb < 0: none) and the phase it was
-        // loaded in.
-        uint8_t* pend_c[kMaxStages];
-        uint8_t* pend_m[kMaxStages];
-        int pend_cb[kMaxStages], pend_mb[kMaxStages], pend_ph[kMaxStages];
-#pragma unroll
-        for (int s = 0; s < kMaxStages; ++s) pend_cb[s] = -1;
-        auto flush = [&](int s) {
-            if (pend_cb[s] < 0) return;
-            const uint8_t* pay = stages + s * geo.stage_bytes + geo.x_bytes;
-            store_back(pend_c[s], pay, pend_cb[s]);
-            store_back(pend_m[s], pay + geo.qcodes_bytes, pend_mb[s]);
-            bulk_commit();
-            bulk_wait_read<0>();        // the stage may be refilled after this
-            pend_cb[s] = -1;
-        };
-        int si = 0, sph = 0, k = 0, uk = -1;
+        int k = 0, uk = -1;
         bool bad = false, ok = true, newunit = true;
-        const uint8_t* codes_u = nullptr;
+        int cur_slot = 0, cur_layer = 0;
         const uint8_t* meta_u = nullptr;
         const uint8_t* fp_u = nullptr;
         const float* x_u = nullptr;
         TileWalk ti;
-        ti.start(pv, cv, t0);
-        for (long long t = t0; t < t1; ++t, newunit = ti.next(pv, cv)) {
-            const int regbase = ti.quant ? 0 : pv.Hq;
+        ti.start(Hq, Hf, P, cv, t0);
+        for (long long t = t0; t < t1; ++t, newunit = ti.next(Hq, Hf, P, cv)) {
+            const int regbase = ti.quant ? 0 : Hq;
             if (newunit) {
                 ++uk;
                 const int u = uk & 1;
@@ -415,68 +481,63 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 const int slot = cv.slot_idx ? __ldg(cv.slot_idx + ti.b) : ti.b;
                 bad = slot < 0 || slot >= pv.n_slots;
                 uint8_t* ub = units + u * geo.unit_bytes;
-                if (lane == 0) {
-                    reinterpret_cast<int*>(ub)[0] = slot;
-                    reinterpret_cast<int*>(ub)[1] = bad ? 1 : 0;
-                    if (bad) atomicOr(err, SSQ_DEVERR_SLOT);
-                }
+                cur_slot = slot;
+                cur_layer = cv.layer0 + ti.l;
                 if (!bad) {
-                    const int layer = cv.layer0 + ti.l;
                     const uint8_t* sb = pv.pool + pv.header_bytes + (long long)slot * pv.slot_bytes;
-                    codes_u = sb + pv.codes_off + (long long)layer * pv.codes_layer_bytes;
-                    meta_u = sb + pv.meta_off + (long long)layer * pv.meta_layer_bytes;
-                    fp_u = sb + pv.fp_off + (long long)layer * pv.fp_layer_bytes;
+                    meta_u = sb + pv.meta_off + (long long)cur_layer * pv.meta_layer_bytes;
+                    fp_u = sb + pv.fp_off + (long long)cur_layer * pv.fp_layer_bytes;
                     x_u = cv.x + ti.lb * H * P;
-                    // B and C in 16-byte chunks.  In quantized units lane j's
-                    // chunk i of piece pc (its entries 16*pc + 4*i .. +3) is
-                    // stored at (i*NP + pc)*LPR + j, so the lanes of a warp,
-                    // visiting different pieces, read distinct banks.
-                    float* dB = reinterpret_cast<float*>(ub + geo.ub_B);
-                    float* dC = reinterpret_cast<float*>(ub + geo.ub_C);
-                    const float* sB = cv.B + ti.lb * G * N;
-                    const float* sC = cv.C + ti.lb * G * N;
-                    for (int m = lane; m < G * N / 4; m += 32) {
-                        int pos = m;
-                        if (F::quant && ti.quant) {
-                            const int gi = m / (N / 4), mm = m - gi * (N / 4);
-                            const int jj = mm / (EQ / 4), rest = mm - jj * (EQ / 4);
-                            const int pc = rest / 4, ii = rest - pc * 4;
-                            pos = gi * (N / 4) + (ii * NP + pc) * LQ + jj;
-                        }
-                        cpa16(dB + 4 * pos, sB + 4 * m);
-                        cpa16(dC + 4 * pos, sC + 4 * m);
-                    }
                     // head table of the region: lambda = exp(dt*A) once per
                     // head, dt, D, the head's y offset and B/C group
                     float4* ht = reinterpret_cast<float4*>(ub + geo.ub_ht);
-                    int* gt = reinterpret_cast<int*>(ub + geo.ub_gt);
-                    const int nreg = ti.quant ? pv.Hq : pv.Hf;
+                    int* gtab = reinterpret_cast<int*>(ub + geo.ub_gt);
+                    const int nreg = ti.quant ? Hq : Hf;
                     for (int hr = lane; hr < nreg; hr += 32) {
                         const int h = pv.perm[regbase + hr];
                         const float dtv = __ldg(cv.dt + ti.lb * H + h);
                         const float Av = __ldg(cv.A + (long long)ti.l * H + h);
                         const float Dv = __ldg(cv.D + (long long)ti.l * H + h);
                         ht[hr] = make_float4(decay(dtv, Av), dtv, Dv, __int_as_float(h * P));
-                        gt[hr] = fdiv(h, pv.mHpg) * N;
+                        gtab[hr] = fdiv(h, pv.mHpg) * N;
                     }
                 }
-                cpa_arrive(&ufull[u]);
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ufull[u]);
+                if (lane == 0) {
+                    reinterpret_cast<int*>(ub)[0] = slot;
+                    reinterpret_cast<int*>(ub)[1] = bad ? 1 : 0;
+                    if (bad) {
+                        atomicOr(err, SSQ_DEVERR_SLOT);
+                        mbar_arrive(&ufull[u]);
+                    } else {
+                        // B and C of every group, in natural order
+                        const unsigned gb = (unsigned)(G * N * 4);
+                        mbar_arrive_tx(&ufull[u], 2 * gb);
+                        bulk_g2s(ub + geo.ub_B, cv.B + ti.lb * G * N, gb, &ufull[u]);
+                        bulk_g2s(ub + geo.ub_C, cv.C + ti.lb * G * N, gb, &ufull[u]);
+                    }
+                }
             }
             if (bad) continue;
             // start the tile's HBM reads into L2 now; the copy into the stage,
-            // issued once the consumers release it, then reads from L2
+            // issued once a stage is free, then reads from L2
             if (lane == 0) {
                 if (F::quant && ti.quant) {
-                    bulk_prefetch_l2(codes_u + (long long)ti.rbase * RB, (unsigned)r16(ti.n * RB));
+                    const int line0 = ti.rbase * RB / 128;
+#pragma unroll 1
+                    for (int bx = 0; bx < kBoxes && bx * kBoxRows < ti.n; ++bx)
+                        tma_prefetch_codes(&cm.map, line0 + bx * kBoxLines, cur_layer, cur_slot);
                     bulk_prefetch_l2(meta_u + (long long)ti.rbase * MB, (unsigned)r16(ti.n * MB));
                 } else {
                     bulk_prefetch_l2(fp_u + (long long)ti.rbase * N * FEB, (unsigned)(ti.n * N * FEB));
                 }
             }
-            if (!mbar_wait<kProducerSleep>(&empty[si], sph ^ 1)) { ok = false; break; }
-            if (lane == 0) flush(si);
+            const int si = k % S;
+            // the stage's previous tile (k - S) must have been released
+            if (k >= S && !mbar_wait<kProducerSleep>(&empty[si], (unsigned)(((k - S) / S) & 1))) {
+                ok = false;
+                break;
+            }
             uint8_t* st = stages + si * geo.stage_bytes;
             float* sx = reinterpret_cast<float*>(st);
             for (int i = lane; i < ti.n; i += 32) {
@@ -490,16 +551,14 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             if (lane == 0) {
                 uint8_t* pay = st + geo.x_bytes;
                 if (F::quant && ti.quant) {
-                    const unsigned cb = (unsigned)r16(ti.n * RB), mb = (unsigned)r16(ti.n * MB);
-                    if (kWB) {
-                        pend_c[si] = const_cast<uint8_t*>(codes_u) + (long long)ti.rbase * RB;
-                        pend_m[si] = const_cast<uint8_t*>(meta_u) + (long long)ti.rbase * MB;
-                        pend_cb[si] = ti.n * RB;
-                        pend_mb[si] = ti.n * MB;
-                        pend_ph[si] = sph;
-                    }
-                    mbar_arrive_tx(&full[si], cb + mb);
-                    bulk_g2s(pay, codes_u + (long long)ti.rbase * RB, cb, &full[si]);
+                    const int line0 = ti.rbase * RB / 128;
+                    const int nbox = (ti.n + kBoxRows - 1) / kBoxRows;
+                    const unsigned mb = (unsigned)r16(ti.n * MB);
+                    mbar_arrive_tx(&full[si], (unsigned)(nbox * kBoxLines * 128) + mb);
+#pragma unroll 1
+                    for (int bx = 0; bx < nbox; ++bx)
+                        tma_load_codes(pay + bx * kBoxLines * 128, &cm.map, line0 + bx * kBoxLines,
+                                       cur_layer, cur_slot, &full[si]);
                     bulk_g2s(pay + geo.qcodes_bytes, meta_u + (long long)ti.rbase * MB, mb,
                              &full[si]);
                 } else {
@@ -509,47 +568,36 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 }
             }
             ++k;
-            if (++si == S) { si = 0; sph ^= 1; }
         }
         if (!ok && lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
-        // the last tiles' write-backs, in the order they were loaded
-        if (lane == 0) {
-            for (int jj = (k > S ? k - S : 0); jj < k; ++jj) {
-                const int s = jj % S;
-                if (pend_cb[s] < 0) continue;
-                if (ok && mbar_wait<kProducerSleep>(&empty[s], (unsigned)pend_ph[s])) {
-                    flush(s);
-                } else {
-                    ok = false;
-                    pend_cb[s] = -1;
-                }
-            }
-            if (!ok) atomicOr(err, SSQ_DEVERR_TIMEOUT);
-            bulk_wait<0>();
-        }
         // No copy may still be writing shared memory when the CTA exits.
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (lane == 0) {
-            for (int jj = (k > S ? k - S : 0); jj < k; ++jj)
-                mbar_wait<kConsumerSleep>(&full[jj % S], (jj / S) & 1);
+            for (int kk = (k > S ? k - S : 0); kk < k; ++kk)
+                mbar_wait<kConsumerSleep>(&full[kk % S], (kk / S) & 1);
         }
         return;
     }
 
     // ================= consumer warps =================
-    const int ct = threadIdx.x;
-    int si = 0, sph = 0, uk = -1;
-    bool bad = false, newunit = true;
+    const int grp = warp / kGWarps;                  // consumer group
+    const int gtid = threadIdx.x - grp * kGThreads;  // thread within the group
+    int k = 0, uk = -1;
+    bool bad = false, newunit = true, ok = true;
     const uint8_t* ub = units;
     uint8_t* codes_u = nullptr;
     uint8_t* meta_u = nullptr;
     uint8_t* fp_u = nullptr;
     float* y_u = nullptr;
     int cur_slot = 0;
+    // this warp's TMEM: lanes 32*(warp%4) .., columns 128*(warp/4) ..
+    const uint32_t tm = use_tmem
+        ? *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2))
+        : 0u;
 
     TileWalk ti;
-    ti.start(pv, cv, t0);
-    for (long long t = t0; t < t1; ++t, newunit = ti.next(pv, cv)) {
+    ti.start(Hq, Hf, P, cv, t0);
+    for (long long t = t0; t < t1; ++t, newunit = ti.next(Hq, Hf, P, cv)) {
         if (newunit) {
             if (uk >= 0) {
                 __syncwarp();
@@ -557,10 +605,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             }
             ++uk;
             const int u = uk & 1;
-            if (!mbar_wait<kConsumerSleep>(&ufull[u], (uk >> 1) & 1)) {
-                if (lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
-                break;
-            }
+            if (!mbar_wait<kConsumerSleep>(&ufull[u], (uk >> 1) & 1)) { ok = false; break; }
             ub = units + u * geo.unit_bytes;
             const int slot = reinterpret_cast<const int*>(ub)[0];
             cur_slot = slot;
@@ -575,27 +620,26 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             }
         }
         if (bad) continue;
-        if (!mbar_wait<kConsumerSleep>(&full[si], sph)) {
-            if (lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
-            break;
-        }
-        const uint8_t* st = stages + si * geo.stage_bytes;
+        const int kk = k++;
+        if (kk % kGroups != grp) continue;
+        const int si = kk % S;
+        if (!mbar_wait<kConsumerSleep>(&full[si], (unsigned)((kk / S) & 1))) { ok = false; break; }
+        uint8_t* const st = stages + si * geo.stage_bytes;
         const float* sx = reinterpret_cast<const float*>(st);
-        const uint8_t* pay = st + geo.x_bytes;
+        uint8_t* const pay = st + geo.x_bytes;
         // row within the tile and lane within the row, by the region's shape
-        const int grow = ti.quant ? ct / LQ : ct / LF;
-        const int j = ti.quant ? ct % LQ : ct % LF;
+        const int grow = ti.quant ? gtid / LQ : gtid / LF;
+        const int j = ti.quant ? gtid % LQ : gtid % LF;
         const bool active = grow < ti.n;
-        // Rows past the end of a partial tile shadow its row 0: they read
-        // row 0's inputs and so compute and store exactly row 0's bytes,
-        // which lets every store go without a branch.
+        // Rows past the end of a partial tile compute on a zero row with the
+        // head parameters of the tile's row 0 and store nothing.
         const int rl = active ? grow : 0;
         const int rr = ti.rbase + rl;
         const int hr = fdiv(rr, pv.mP);
         const int p = rr - hr * P;
         const float4 hti = reinterpret_cast<const float4*>(ub + geo.ub_ht)[hr];
         const int gN = reinterpret_cast<const int*>(ub + geo.ub_gt)[hr];
-        const float xv = sx[rl];
+        const float xv = active ? sx[grow] : 0.0f;
         const float lamv = hti.x;
         const float dtx = __fmul_rn(hti.y, xv);
         const float* gB = reinterpret_cast<const float*>(ub + geo.ub_B) + gN;
@@ -606,45 +650,29 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         if constexpr (F::quant) {
             if (ti.quant) {
                 done = true;
-                // this lane's codes and the row's metadata in shared memory.
-                // The lane visits its pieces in the order pc = sp ^ rot, rot
-                // being its 128-byte line, so the lanes of a warp reading
-                // one step touch every bank group; its code block, B and C
-                // and its row in the pool are aligned so that each permuted
-                // address is a single XOR.
-                const int loff = rl * RB + j * CB;
-                const uint8_t* cs = pay + loff;
-                const unsigned rot = (unsigned)(loff >> 7) & (NP - 1);
-                const unsigned cs_x = saddr(cs) | (rot * PB);
-                const unsigned bx = (saddr(gB) + j * 16) | (rot * LQ * 16);
-                const unsigned cx = (saddr(gC) + j * 16) | (rot * LQ * 16);
-                // With kWB the new codes and metadata go back into the stage,
-                // in place (the producer writes the tile back), and rows past
-                // the end of the tile store nothing, as the row they shadow
-                // may already hold new codes; otherwise they go straight to
-                // the pool (a shadow row stores row 0's bytes again).
-                uint8_t* const ms = const_cast<uint8_t*>(pay) + geo.qcodes_bytes + rl * MB;
-                uint8_t* const crow = kWB ? const_cast<uint8_t*>(cs)
-                                          : codes_u + (long long)rr * RB + j * CB;
-                uint8_t* const mrow = kWB ? ms : meta_u + (long long)rr * MB;
-                const uintptr_t crow_x = reinterpret_cast<uintptr_t>(crow) | (rot * PB);
+                // this lane's codes in the stage (piece sp of the lane at
+                // cs_x ^ (sp * PB) under the swizzle) and the row's metadata
+                const unsigned cs0 = (unsigned)(geo.x_bytes + grow * RB + j * CB);
+                const unsigned cs_x = saddr(st) + swz128(cs0);
+                uint8_t* const ms = pay + geo.qcodes_bytes + grow * MB;
+                // (a row past the end of the tile reads its stage slot and
+                // decodes zeros instead)
                 float delta0, z0 = 0.0f;
-                {
-                    if constexpr (F::sym) {
-                        delta0 = *reinterpret_cast<const float*>(ms);
-                    } else {
-                        const float2 m = *reinterpret_cast<const float2*>(ms);
-                        delta0 = m.x;
-                        z0 = m.y;
-                    }
+                if constexpr (F::sym) {
+                    delta0 = *reinterpret_cast<const float*>(ms);
+                } else {
+                    const float2 m = *reinterpret_cast<const float2*>(ms);
+                    delta0 = m.x;
+                    z0 = m.y;
                 }
-                // pieces NREG.. of the updated row wait in this lane's spill
-                // area: chunk k of lane l at scr + (k * 32 + l) * 16
-                const unsigned scr = saddr(smem + geo.off_scr) + warp * geo.scr_warp_bytes + lane * 16;
+                delta0 = active ? delta0 : 0.0f;
+                z0 = active ? z0 : 0.0f;
+                const unsigned bxa = saddr(gB) + j * EQ * 4;
+                const unsigned cxa = saddr(gC) + j * EQ * 4;
                 // decode + update, one 16-entry piece at a time, with
-                // per-piece min / max.  The decode is exact for |z| < 2^22;
-                // rows beyond that take the exact path below.
-                float s[NREG * 16];
+                // per-piece min / max; the updated pieces wait in TMEM.  The
+                // decode is exact for |z| < 2^22; rows beyond take the exact
+                // path below.
                 float lo, hi;
                 {
                     const float c0 = __fadd_rn(kTwo23, __fadd_rn(z0, F::bias));
@@ -664,11 +692,11 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         }
                         float f[16];
                         unpack16_biased<FMT>(w, f);
-                        const unsigned bp = bx ^ (sp * LQ * 16);
+                        const unsigned bp = bxa + sp * 64;
                         float v16[16];
                         auto bq = [&](auto ic) {
                             constexpr int i = decltype(ic)::value;
-                            const float4 bv = lds128f<i * NP * LQ * 16>(bp);
+                            const float4 bv = lds128f<i * 16>(bp);
                             const float2 v0 = mul2(add2(make_float2(f[4 * i], f[4 * i + 1]), nc02), d2);
                             const float2 v1 = mul2(add2(make_float2(f[4 * i + 2], f[4 * i + 3]), nc02), d2);
                             const float2 u0 = fma2(l2, v0, mul2(x2, make_float2(bv.x, bv.y)));
@@ -684,25 +712,17 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         minmax16(v16, plo, phi);
                         lo = sp == 0 ? plo : fminf(lo, plo);
                         hi = sp == 0 ? phi : fmaxf(hi, phi);
-                        if (sp < NREG) {
-#pragma unroll
-                            for (int n = 0; n < 16; ++n) s[(sp < NREG ? sp : 0) * 16 + n] = v16[n];
-                        } else {
-                            const unsigned a = scr + (sp - NREG) * 4 * 512;
-                            sts128f<0>(a, make_float4(v16[0], v16[1], v16[2], v16[3]));
-                            sts128f<512>(a, make_float4(v16[4], v16[5], v16[6], v16[7]));
-                            sts128f<1024>(a, make_float4(v16[8], v16[9], v16[10], v16[11]));
-                            sts128f<1536>(a, make_float4(v16[12], v16[13], v16[14], v16[15]));
-                        }
+                        tmem_st16(tm + sp * 16, v16);
                     }
                 }
+                tmem_wait_st();
                 const RowParams rp = refit_from_minmax<FMT, LQ>(lo, hi);
                 // the magic-number paths are exact for every row of the warp;
                 // rows whose top code must be capped take the clamped loop
                 const bool fast = __all_sync(0xffffffffu, (F::sym || fabsf(z0) < kFastLimit)
                                                           && rp.fast);
                 // the stochastic-rounding key of this row (unused for RTN)
-                SrKey srk;
+                SrKey srk{};
                 if constexpr (SR) {
                     srk.key = make_uint2((uint32_t)cv.sr_seed, (uint32_t)(cv.sr_seed >> 32));
                     srk.layer = (uint32_t)(cv.layer0 + ti.l);
@@ -715,52 +735,31 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     const float2 z2 = make_float2(rp.z, rp.z);
                     const float mz = F::sym ? -kMagic : -__fadd_rn(kMagic, rp.z);
                     const float2 mz2 = make_float2(mz, mz);
-                    // round, pack, store and read back, piece by piece; the
-                    // readout sums C (q - z) and scales by Delta once
+                    // round, pack, write back and read out, piece by piece;
+                    // the readout sums C (q - z) and scales by Delta once
                     float2 acc = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
                     auto piece = [&](auto clamp_tag, int sp) {
                         float v16[16];
-                        if (sp < NREG) {
-#pragma unroll
-                            for (int n = 0; n < 16; ++n) v16[n] = s[(sp < NREG ? sp : 0) * 16 + n];
-                        } else {
-                            const unsigned a = scr + (sp - NREG) * 4 * 512;
-                            const float4 q0 = lds128f<0>(a), q1 = lds128f<512>(a);
-                            const float4 q2 = lds128f<1024>(a), q3 = lds128f<1536>(a);
-                            v16[0] = q0.x; v16[1] = q0.y; v16[2] = q0.z; v16[3] = q0.w;
-                            v16[4] = q1.x; v16[5] = q1.y; v16[6] = q1.z; v16[7] = q1.w;
-                            v16[8] = q2.x; v16[9] = q2.y; v16[10] = q2.z; v16[11] = q2.w;
-                            v16[12] = q3.x; v16[13] = q3.y; v16[14] = q3.z; v16[15] = q3.w;
-                        }
+                        tmem_ld16(tm + sp * 16, v16);
                         float r[16];
-                        uint32_t kk[16];
+                        uint32_t kq[16];
                         if constexpr (SR) {
                             float u[16];
-                            sr_draws16(srk, j * EQ + 16 * (int)((unsigned)sp ^ rot), u);
-                            round16_sr<FMT>(inv2, z2, mz2, v16, u, r, kk);
+                            sr_draws16(srk, j * EQ + 16 * sp, u);
+                            round16_sr<FMT>(inv2, z2, mz2, v16, u, r, kq);
                         } else {
-                            round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, v16, r, kk);
+                            round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, v16, r, kq);
                         }
                         uint32_t w[PW];
-                        pack16<FMT>(kk, w);
-                        if constexpr (kWB) {
-                            if (active) {
-                                if constexpr (PW == 4)
-                                    sts128u<0>(cs_x ^ (sp * PB), make_uint4(w[0], w[1], w[2], w[3]));
-                                else
-                                    sts64u<0>(cs_x ^ (sp * PB), make_uint2(w[0], w[1]));
-                            }
-                        } else {
-                            void* dst = reinterpret_cast<void*>(crow_x ^ (uintptr_t)(sp * PB));
-                            if constexpr (PW == 4)
-                                __stcs(reinterpret_cast<uint4*>(dst), make_uint4(w[0], w[1], w[2], w[3]));
-                            else
-                                __stcs(reinterpret_cast<uint2*>(dst), make_uint2(w[0], w[1]));
-                        }
-                        const unsigned cp = cx ^ (sp * LQ * 16);
+                        pack16<FMT>(kq, w);
+                        if constexpr (PW == 4)
+                            sts128u_if(cs_x ^ (sp * PB), make_uint4(w[0], w[1], w[2], w[3]), active);
+                        else
+                            sts64u_if(cs_x ^ (sp * PB), make_uint2(w[0], w[1]), active);
+                        const unsigned cp = cxa + sp * 64;
                         auto cq = [&](auto ic) {
                             constexpr int i = decltype(ic)::value;
-                            const float4 cv4 = lds128f<i * NP * LQ * 16>(cp);
+                            const float4 cv4 = lds128f<i * 16>(cp);
                             acc = fma2(make_float2(cv4.x, cv4.y), make_float2(r[4 * i], r[4 * i + 1]), acc);
                             acc1 = fma2(make_float2(cv4.z, cv4.w), make_float2(r[4 * i + 2], r[4 * i + 3]), acc1);
                         };
@@ -778,27 +777,37 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     }
                     acc = add2(acc, acc1);
                     ysum = __fmul_rn(rp.delta, grp_sum<LQ>(__fadd_rn(acc.x, acc.y)));
-                    if constexpr (kWB) {
-                        if (active && j == 0) {
-                            if constexpr (F::sym) {
-                                *reinterpret_cast<float*>(ms) = rp.delta;
-                            } else {
-                                *reinterpret_cast<float2*>(ms) = make_float2(rp.delta, rp.z);
-                            }
-                        }
-                    } else {
-                        // every lane of the row writes the same metadata
+                    if (active && j == 0) {
+                        uint8_t* mg = meta_u + (long long)rr * MB;
                         if constexpr (F::sym) {
-                            __stcs(reinterpret_cast<float*>(mrow), rp.delta);
+                            __stcs(reinterpret_cast<float*>(mg), rp.delta);
                         } else {
-                            __stcs(reinterpret_cast<float2*>(mrow), make_float2(rp.delta, rp.z));
+                            __stcs(reinterpret_cast<float2*>(mg), make_float2(rp.delta, rp.z));
                         }
                     }
-                    if (__any_sync(0xffffffffu, !rp.finite) && lane == 0)
+                    if (__any_sync(0xffffffffu, active && !rp.finite) && lane == 0)
                         atomicOr(err, SSQ_DEVERR_NONFINITE);
                 } else {
-                    ysum = row_exact<FMT, N, SR>(cs, delta0, z0, lamv, dtx, gB, gC, j, active,
-                                                 crow, mrow, err, srk);
+                    ysum = row_exact<FMT, N, SR>(st, cs0, delta0, z0, lamv, dtx, gB, gC, j,
+                                                 active, meta_u + (long long)rr * MB, err, srk);
+                }
+                // This warp's rows, from the stage to the pool: chunk c (16
+                // bytes) of the warp's contiguous block of 32/LQ rows, lanes
+                // on consecutive chunks, so every store covers whole lines.
+                __syncwarp();
+                {
+                    const int wrow0 = (gtid >> 5) * (32 / LQ);   // first row of this warp
+                    const unsigned cbase = (unsigned)(geo.x_bytes + wrow0 * RB);
+                    uint8_t* const gbase = codes_u + (long long)(ti.rbase + wrow0) * RB;
+                    const int nbytes = (min(ti.n - wrow0, 32 / LQ) > 0
+                                        ? min(ti.n - wrow0, 32 / LQ) : 0) * RB;
+#pragma unroll
+                    for (int c = lane; c < 2 * CB; c += 32) {
+                        if (c * 16 < nbytes) {
+                            const uint4 v = *reinterpret_cast<const uint4*>(st + swz128(cbase + c * 16));
+                            __stcs(reinterpret_cast<uint4*>(gbase + c * 16), v);
+                        }
+                    }
                 }
             }
         }
@@ -857,22 +866,67 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
 #pragma unroll
                     for (int n = 0; n < EPC; ++n) w[n] = __float_as_uint(sv[n]);
                 }
-                __stcs(reinterpret_cast<uint4*>(frow) + m, make_uint4(w[0], w[1], w[2], w[3]));
+                if (active)
+                    __stcs(reinterpret_cast<uint4*>(frow) + m, make_uint4(w[0], w[1], w[2], w[3]));
             }
             acc = add2(acc, acc1);
             ysum = grp_sum<LF>(__fadd_rn(acc.x, acc.y));
         }
         // every lane of the row writes the same y (after the row sum all
-        // hold it); a row past the end of the tile writes nothing (with the
-        // in-place write-back it may have read its shadowed row's new codes)
+        // hold it); a row past the end of the tile writes nothing
         if (active)
             __stcs(y_u + __float_as_int(hti.w) + p, __fadd_rn(ysum, __fmul_rn(hti.z, xv)));
-        // the stage's new codes must be visible to the producer's bulk store
-        if (kWB && F::quant && ti.quant) fence_proxy_async();
+        // this warp's shared-memory writes are ordered before the tensor
+        // copy that refills the stage
+        if (F::quant && ti.quant) fence_proxy_async();
         __syncwarp();
         mbar_arrive_if(&empty[si], lane == 0);
-        if (++si == S) { si = 0; sph ^= 1; }
     }
+    if (!ok && lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
+    // release TMEM once every consumer warp's TMEM accesses are complete
+    if (use_tmem) {
+        tc_fence_before();
+        consumers_sync();
+        tc_fence_after();
+        if (warp == 0) tmem_dealloc(*tmem_slot, kTmemCols);
+    }
+}
+
+// The driver's tensor-map encoder, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool looked = false;
+    if (!looked) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        looked = true;
+    }
+    return fn;
+}
+
+// The codes of every (slot, layer) of the pool as [slot][layer][line][128 B],
+// boxes of kBoxRows rows' lines, 128-byte swizzle.
+cudaError_t make_codes_map(const PoolView& pv, int RB, CodesMap* cm)
+{
+    std::memset(cm, 0, sizeof(*cm));
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const long long region = (long long)pv.Hq * pv.P * RB;
+    const cuuint64_t lines = (cuuint64_t)((region + 127) / 128);
+    cuuint64_t dims[4] = {128, lines, (cuuint64_t)pv.n_layers, (cuuint64_t)pv.n_slots};
+    cuuint64_t strides[3] = {128, (cuuint64_t)pv.codes_layer_bytes, (cuuint64_t)pv.slot_bytes};
+    const int box_lines = (kBoxRows * RB + 127) / 128;
+    cuuint32_t box[4] = {128, (cuuint32_t)box_lines, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    void* base = pv.pool + pv.header_bytes + pv.codes_off;
+    const CUresult r = enc(&cm->map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <int FMT, int N, bool SR>
@@ -881,17 +935,22 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
     using F = Fmt<FMT>;
     constexpr int RPTq = QShape<N>::RPT, RPTf = FShape<N>::RPT;
     constexpr int RB = F::quant ? N * F::bits / 8 : 0;
-    const bool has_q = pv.Hq > 0, has_fp = pv.Hf > 0;
+    const bool has_q = F::quant && pv.Hq > 0, has_fp = pv.Hf > 0;
     const int fpEB = FMT == SSQ_BF16 ? 2 : 4;
-    // stages: as many as fit a budget that leaves room for kMinBlocks CTAs per SM
-    const int budget = (kMinBlocks == 1 ? 225 : 110) * 1024;
-    constexpr int SCR = F::quant ? QShape<N>::SCR : 0;
-    DecodeGeom g = decode_geom(2, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G, SCR);
+    // stages: as many as fit one CTA per SM
+    const int budget = 226 * 1024;
+    DecodeGeom g = decode_geom(2, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G);
     int S = (budget - (g.smem_bytes - 2 * g.stage_bytes)) / g.stage_bytes;
     if (S > kMaxStages) S = kMaxStages;
     if (S < 2) S = 2;
-    g = decode_geom(S, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G, SCR);
+    g = decode_geom(S, RPTq, RPTf, RB, F::meta_bytes, fpEB, has_q, has_fp, N, pv.H, pv.G);
     if (g.smem_bytes > 227 * 1024) return cudaErrorInvalidConfiguration;
+    CodesMap cm;
+    std::memset(&cm, 0, sizeof(cm));
+    if (has_q) {
+        const cudaError_t e = make_codes_map(pv, RB, &cm);
+        if (e != cudaSuccess) return e;
+    }
     auto kern = decode_kernel<FMT, N, SR>;
     // per-device launch facts, looked up once per kernel instantiation and device
     thread_local int s_dev = -1, s_grid = 0, s_smem = 0;
@@ -902,24 +961,22 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       g.smem_bytes)) != cudaSuccess)
             return e;
-        // the largest shared-memory carveout, so two CTAs fit per SM
-        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                      (int)cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
-            return e;
         int sms = 0, occ = 0;
         if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return e;
         if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kDThreads,
                                                                g.smem_bytes)) != cudaSuccess)
             return e;
-        if (occ < 1) return cudaErrorInvalidConfiguration;
+        // one CTA per SM (its shared memory alone rules out a second); it
+        // owns all of the SM's TMEM
+        if (occ != 1) return cudaErrorInvalidConfiguration;
         s_dev = dev;
         s_smem = g.smem_bytes;
-        s_grid = sms * occ;
+        s_grid = sms;
     }
     long long grid = s_grid;
     if (grid > cv.total_tiles) grid = cv.total_tiles;
-    kern<<<(int)grid, kDThreads, g.smem_bytes, st>>>(pv, cv, g);
+    kern<<<(int)grid, kDThreads, g.smem_bytes, st>>>(pv, cv, g, cm);
     return cudaGetLastError();
 }
 
@@ -942,8 +999,8 @@ void decode_tile_rows(int fmt, int d_state, int* rows_q, int* rows_f)
 {
     const int eq = d_state >= kQuantE ? kQuantE : d_state;
     const int ef = d_state >= 32 ? 32 : d_state;
-    *rows_q = kCThreads / (d_state / eq);
-    *rows_f = kCThreads / (d_state / ef);
+    *rows_q = kGThreads / (d_state / eq);
+    *rows_f = kGThreads / (d_state / ef);
     (void)fmt;
 }
 
@@ -954,10 +1011,7 @@ bool decode_fits(int fmt, int d_state, int nheads, int ngroups)
     int rq = 0, rf = 0;
     decode_tile_rows(fmt, d_state, &rq, &rf);
     const bool q = fmt >= SSQ_I8_SYM;
-    const int eq = d_state >= kQuantE ? kQuantE : d_state;
-    const int np = eq / 16, nreg = np < kRegPieces ? np : kRegPieces;
-    const DecodeGeom g = decode_geom(2, rq, rf, d_state, 8, 4, q, true, d_state, nheads, ngroups,
-                                     (np - nreg) * 64);
+    const DecodeGeom g = decode_geom(2, rq, rf, d_state, 8, 4, q, true, d_state, nheads, ngroups);
     return g.smem_bytes <= 227 * 1024;
 }
 
