@@ -424,6 +424,20 @@ SSQ_API const char* ssq_status_string(ssq_status s);
  * (static thread-local storage; valid until the next call). */
 SSQ_API const char* ssq_last_error_detail(void);
 
+/* Test support for the failure path of the decode step; not for production
+ * use.  Applies to the ssq_decode_step / ssq_decode_step_sr launches issued
+ * later on the calling host thread:
+ *   wait_limit_cycles  the kernel's bound on each pipeline wait, in SM clock
+ *                      cycles (0: the default, about one second)
+ *   withhold_first_tile  nonzero: the producer of the first thread block
+ *                      issues no copy for its first tile, so the waits on it
+ *                      run out; the call sets SSQ_DEVERR_TIMEOUT in the
+ *                      pool's error word and returns, no copy in flight and
+ *                      the context usable (that block's tiles are skipped).
+ * ssq_test_hooks(0, 0) restores normal behaviour.  SSQ_ERR_INVALID_ARG for a
+ * negative limit.  Host only; no CUDA call. */
+SSQ_API ssq_status ssq_test_hooks(int withhold_first_tile, long long wait_limit_cycles);
+
 #ifdef __cplusplus
 }
 #endif

@@ -13,6 +13,11 @@ namespace {
 
 thread_local char g_detail[256] = "";
 
+// Test support (ssq_test_hooks): applied to the decode launches of this host
+// thread.
+thread_local int g_test_withhold = 0;
+thread_local long long g_test_wait_limit = 0;
+
 ssq_status fail(ssq_status s, const char* fmt, ...)
 {
     va_list ap;
@@ -210,6 +215,15 @@ const char* ssq_status_string(ssq_status s)
 
 const char* ssq_last_error_detail(void) { return g_detail; }
 
+ssq_status ssq_test_hooks(int withhold_first_tile, long long wait_limit_cycles)
+{
+    if (wait_limit_cycles < 0)
+        return fail(SSQ_ERR_INVALID_ARG, "wait_limit_cycles %lld < 0", wait_limit_cycles);
+    g_test_withhold = withhold_first_tile ? 1 : 0;
+    g_test_wait_limit = wait_limit_cycles;
+    return SSQ_OK;
+}
+
 ssq_status ssq_pool_layout(const ssq_config* cfg, ssq_layout* out, int32_t* head_perm)
 {
     if (!out) return fail(SSQ_ERR_INVALID_ARG, "out is NULL");
@@ -359,6 +373,8 @@ ssq_status decode_common(const ssq_config* cfg, void* pool, const int32_t* slot_
     cv.y = y;
     cv.sr_seed = seed;
     cv.sr_step = step;
+    cv.wait_limit = g_test_wait_limit;
+    cv.test_withhold = g_test_withhold;
     if (!ssq::decode_fits((int)cfg->fmt, cfg->d_state, cfg->nheads, cfg->ngroups))
         return fail(SSQ_ERR_UNSUPPORTED, "ngroups*d_state %d too large for the decode kernel",
                     cfg->ngroups * cfg->d_state);

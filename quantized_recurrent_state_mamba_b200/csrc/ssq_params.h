@@ -36,6 +36,11 @@ struct CallView {
     int scan_chunk;            // scan: tokens staged per shared-memory buffer
     unsigned long long sr_seed;  // stochastic rounding: Philox key
     unsigned sr_step;            // stochastic rounding: step counter (first token)
+    // Test support (ssq_test_hooks): the decode kernel's wait limit in clock
+    // cycles (0: the default, about a second) and whether CTA 0's producer
+    // withholds the copy of its first tile.
+    long long wait_limit;
+    int test_withhold;
     const float* x;
     const float* B;
     const float* C;

@@ -50,10 +50,11 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, unsigned parity)
 }
 // Wait for the phase of the given parity to complete, sleeping between
 // tries (exponential back-off up to kMaxSleepNs, so a waiting warp takes
-// few issue slots from the warps that compute); false after about a second
-// without progress.
+// few issue slots from the warps that compute); false after `limit` clock
+// cycles without progress (about a second by default).
 template <unsigned kMaxSleepNs>
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, unsigned parity)
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, unsigned parity,
+                                          long long limit = kWaitLimit)
 {
     if (mbar_try(b, parity)) return true;
     const long long t0 = clock64();
@@ -61,7 +62,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, unsigned parity)
     while (!mbar_try(b, parity)) {
         __nanosleep(ns);
         ns = ns < kMaxSleepNs ? 2 * ns : kMaxSleepNs;
-        if (clock64() - t0 > kWaitLimit) return false;
+        if (clock64() - t0 > limit) return false;
     }
     return true;
 }

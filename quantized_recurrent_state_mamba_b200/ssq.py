@@ -92,7 +92,8 @@ _lib.ssq_damp_quantize.argtypes = [_DCFG, _P, _P, _P, _I, _I, _I, _P, _P]
 _lib.ssq_damp_dequantize.argtypes = [_DCFG, _P, _P, _P, _I, _I, _I, _P, _P]
 _lib.ssq_damp_decode_step.argtypes = [_DCFG, _P, _P, _P, _I, _I, _I] + [_P] * 7 + [_P]
 _lib.ssq_damp_pool_error.argtypes = [_DCFG, _P, ctypes.POINTER(ctypes.c_uint32), _P]
-for _f in ("ssq_pool_layout", "ssq_pool_init", "ssq_pool_error", "ssq_quantize_rows",
+_lib.ssq_test_hooks.argtypes = [_I, ctypes.c_longlong]
+for _f in ("ssq_test_hooks", "ssq_pool_layout", "ssq_pool_init", "ssq_pool_error", "ssq_quantize_rows",
            "ssq_dequantize_rows", "ssq_decode_step", "ssq_scan", "ssq_prefill",
            "ssq_decode_step_sr", "ssq_scan_sr", "ssq_decode_diag", "ssq_damp_pool_layout",
            "ssq_damp_quantize", "ssq_damp_dequantize", "ssq_damp_decode_step",
@@ -194,6 +195,13 @@ def ssq_pool_error(cfg: Config, pool, stream=None) -> int:
     v = ctypes.c_uint32(0)
     _check(_lib.ssq_pool_error(cfg.ref, _pool_ptr(cfg, pool), ctypes.byref(v), _stream(stream)))
     return int(v.value)
+
+
+def ssq_test_hooks(withhold_first_tile: bool, wait_limit_cycles: int = 0):
+    """Test support for the decode step's failure path (see include/ssq.h):
+    the pipeline wait bound in SM clock cycles (0: the default) and whether
+    the first thread block withholds its first tile's copy."""
+    _check(_lib.ssq_test_hooks(1 if withhold_first_tile else 0, int(wait_limit_cycles)))
 
 
 def _slots(slot_idx, batch):

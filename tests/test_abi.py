@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(ssq):
     syms = declared_symbols()
-    assert len(syms) == 18, syms
+    assert len(syms) == 19, syms
     lib = ctypes.CDLL(ssq.LIB_PATH)
     for s in syms:
         assert hasattr(lib, s), f"libssq.so does not export {s}"
@@ -293,3 +293,12 @@ def test_damp_channel_maps_are_permutations():
             assert np.array_equal(np.sort(c[l, h]), np.arange(128))
     assert np.array_equal(c, W.damp_channels(7, 3, 5, 128))
     assert not np.array_equal(c, W.damp_channels(8, 3, 5, 128))
+
+
+def test_test_hooks_validate_on_the_host(ssq):
+    """The failure-path test hooks are host-only: a negative wait bound is an
+    argument error, (0, 0) restores normal behaviour."""
+    with pytest.raises(ssq.SsqError):
+        ssq.ssq_test_hooks(False, -5)
+    ssq.ssq_test_hooks(True, 1000)
+    ssq.ssq_test_hooks(False, 0)
