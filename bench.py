@@ -208,7 +208,7 @@ _KERNEL_SOURCES = {
     "decode": ("ssq_decode.cu", "ssq_pipe.cuh"),
     "damp": ("ssq_damp.cu", "ssq_pipe.cuh"),
     "scan": ("ssq_scan.cu",),
-    "diag": ("ssq_diag.cu",),
+    "diag": ("ssq_decode.cu", "ssq_pipe.cuh"),
 }
 
 

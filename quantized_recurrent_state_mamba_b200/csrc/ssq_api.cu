@@ -329,8 +329,15 @@ ssq_status ssq_decode_diag(const ssq_config* cfg, const void* pool, const int32_
     cv.C = C;
     cv.dt = dt;
     cv.A = A;
-    fill_tiles(pv, &cv, ssq::rows_per_tile(cfg->d_state), ssq::rows_per_tile(cfg->d_state));
-    cudaError_t e = ssq::launch_diag(pv, cv, (int)cfg->fmt, diag, stream);
+    cv.diag = diag;
+    cv.wait_limit = g_test_wait_limit;
+    if (!ssq::decode_fits((int)cfg->fmt, cfg->d_state, cfg->nheads, cfg->ngroups))
+        return fail(SSQ_ERR_UNSUPPORTED, "ngroups*d_state %d too large for the decode kernel",
+                    cfg->ngroups * cfg->d_state);
+    int rows_q = 0, rows_f = 0;
+    ssq::decode_tile_rows((int)cfg->fmt, cfg->d_state, &rows_q, &rows_f);
+    fill_tiles(pv, &cv, rows_q, rows_f);
+    cudaError_t e = ssq::launch_decode_diag(pv, cv, (int)cfg->fmt, stream);
     if (e != cudaSuccess) return cuda_fail(e, "diag launch");
     return SSQ_OK;
 }

@@ -39,6 +39,11 @@
 //   - every wait is bounded: one that runs out sets SSQ_DEVERR_TIMEOUT in the
 //     pool's error word and the CTA winds down (the producer first waits for
 //     its own copies in flight; TMEM is released on every path).
+//
+// The same kernel, in its diagnostics mode, evaluates the step a decode would
+// take and writes per-row figures instead of the new state
+// ("ssm-state-quantization" README, Findings 4 and 5): the pool is only
+// read.
 #include "ssq_common.cuh"
 #include "ssq_params.h"
 #include "ssq_pipe.cuh"
@@ -397,18 +402,82 @@ __device__ __noinline__ float row_exact(uint8_t* __restrict__ sb, unsigned cs0, 
     return ysum;
 }
 
+// The diagnostics of a whole quantized row by the formulas verbatim (the
+// warps where some row falls outside the magic-number paths): the step the
+// decode would take, and per row {reversals, sum over reversed entries of
+// C e, sum of C e, sum of C s'}, e = fl(deq - s') the rounding error and an
+// entry reversed when w != 0 and fl(e + w) has the other sign than w.
+// Every lane of the warp calls it together.
+template <int FMT, int N>
+__device__ __noinline__ float4 row_exact_diag(const uint8_t* __restrict__ sb, unsigned cs0,
+                                              float delta0, float z0, float lam, float dtx,
+                                              const float* __restrict__ gB,
+                                              const float* __restrict__ gC, int j)
+{
+    using F = Fmt<FMT>;
+    constexpr int E = QShape<N>::E, LPR = QShape<N>::LPR;
+    float s[E];
+    float lo = 0.0f, hi = 0.0f;
+#pragma unroll 1
+    for (int n = 0; n < E; ++n) {
+        int q;
+        if constexpr (F::bits == 8) {
+            const uint32_t bb = sb[swz128(cs0 + n)];
+            q = F::sym ? (int)(int8_t)bb : (int)bb;
+        } else {
+            const uint32_t bb = (sb[swz128(cs0 + n / 2)] >> (4 * (n % 2))) & 0xFu;
+            q = F::sym ? (int)((bb ^ 8u) - 8u) : (int)bb;
+        }
+        const float v = __fmul_rn(__fsub_rn((float)q, z0), delta0);
+        const float sv = __fmaf_rn(lam, v, __fmul_rn(dtx, gB[j * E + n]));
+        s[n] = sv;
+        lo = n == 0 ? sv : fminf(lo, sv);
+        hi = n == 0 ? sv : fmaxf(hi, sv);
+    }
+    const RowParams rp = refit_from_minmax<FMT, LPR>(lo, hi);
+    float rev = 0.0f, rev_err = 0.0f, tot = 0.0f, sig = 0.0f;
+#pragma unroll 1
+    for (int n = 0; n < E; ++n) {
+        const float rr = rint_prod(s[n], rp.inv);
+        float r;
+        if constexpr (F::sym) {
+            r = fminf(fmaxf(rr, -F::qmax), F::qmax);
+        } else {
+            r = __fsub_rn(fminf(__fadd_rn(rr, rp.z), F::qmax), rp.z);
+        }
+        const float w = __fmul_rn(dtx, gB[j * E + n]);
+        const float e = __fsub_rn(__fmul_rn(r, rp.delta), s[n]);
+        const float inc = __fadd_rn(e, w);
+        const float c = gC[j * E + n];
+        sig = __fmaf_rn(c, s[n], sig);
+        tot = __fmaf_rn(c, e, tot);
+        if ((w > 0.0f && inc < 0.0f) || (w < 0.0f && inc > 0.0f)) {
+            rev += 1.0f;
+            rev_err = __fmaf_rn(c, e, rev_err);
+        }
+    }
+    return make_float4(grp_sum<LPR>(rev), grp_sum<LPR>(rev_err), grp_sum<LPR>(tot),
+                       grp_sum<LPR>(sig));
+}
+
 struct CodesMap {
     CUtensorMap map;   // 64-byte aligned inside the kernel parameters
 };
 
-// SR: round the quantized rows stochastically (draws keyed by cv.sr_seed
-// and countered by row block, layer, slot and cv.sr_step).
-template <int FMT, int N, bool SR>
+// Modes of the kernel: the decode step with nearest rounding, with
+// stochastic rounding (draws keyed by cv.sr_seed and countered by row block,
+// layer, slot and cv.sr_step), or its diagnostics (written to cv.diag; the
+// pool is only read).
+enum { kNearest = 0, kStochastic = 1, kDiagnostics = 2 };
+
+template <int FMT, int N, int MODE>
 __global__ void __launch_bounds__(kDThreads, 1)
 decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallView cv,
               const __grid_constant__ DecodeGeom geo, const __grid_constant__ CodesMap cm)
 {
     using F = Fmt<FMT>;
+    constexpr bool SR = MODE == kStochastic;
+    constexpr bool DIAG = MODE == kDiagnostics;
     // quantized rows: EQ entries per lane, LQ lanes per row; fp rows: EF, LF
     constexpr int EQ = QShape<N>::E, LQ = QShape<N>::LPR;
     constexpr int EF = FShape<N>::E, LF = FShape<N>::LPR;
@@ -498,7 +567,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         const int h = pv.perm[regbase + hr];
                         const float dtv = __ldg(cv.dt + ti.lb * H + h);
                         const float Av = __ldg(cv.A + (long long)ti.l * H + h);
-                        const float Dv = __ldg(cv.D + (long long)ti.l * H + h);
+                        const float Dv = cv.D ? __ldg(cv.D + (long long)ti.l * H + h) : 0.0f;
                         ht[hr] = make_float4(decay(dtv, Av), dtv, Dv, __int_as_float(h * P));
                         gtab[hr] = fdiv(h, pv.mHpg) * N;
                     }
@@ -653,6 +722,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         const float* gC = reinterpret_cast<const float*>(ub + geo.ub_C) + gN;
         float ysum = 0.0f;
         bool done = false;
+        float4 dres = make_float4(0.0f, 0.0f, 0.0f, 0.0f);   // diagnostics of the row
 
         if constexpr (F::quant) {
             if (ti.quant) {
@@ -737,7 +807,67 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     srk.step = cv.sr_step;
                     srk.row_block = (uint32_t)(__float_as_int(hti.w) + p) * (uint32_t)(N / 8);
                 }
-                if (fast) {
+                if (DIAG && fast) {
+                    // the rounding of the step, then per entry e = fl(fl(r
+                    // Delta) - s'), w = fl(dtx B), the reversal test on fl(e +
+                    // w) in fp32, and the sums of C e (all, reversed) and C s'
+                    const float2 inv2 = make_float2(rp.inv, rp.inv);
+                    const float2 z2 = make_float2(rp.z, rp.z);
+                    const float mz = F::sym ? -kMagic : -__fadd_rn(kMagic, rp.z);
+                    const float2 mz2 = make_float2(mz, mz);
+                    const float2 dl2 = make_float2(rp.delta, rp.delta);
+                    const float2 m1 = make_float2(-1.0f, -1.0f);
+                    const float2 x2 = make_float2(dtx, dtx);
+                    float2 sig = make_float2(0.0f, 0.0f), tot = make_float2(0.0f, 0.0f);
+                    float2 rve = make_float2(0.0f, 0.0f);
+                    int nrev = 0;
+                    auto dpiece = [&](auto clamp_tag, int sp) {
+                        float v16[16];
+                        tmem_ld16(tm + sp * 16, v16);
+                        float r[16];
+                        uint32_t kq[16];
+                        round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, v16, r, kq);
+                        const unsigned bp = bxa + sp * 64, cp = cxa + sp * 64;
+                        auto dq = [&](auto ic) {
+                            constexpr int i = decltype(ic)::value;
+                            const float4 bv = lds128f<i * 16>(bp);
+                            const float4 c4 = lds128f<i * 16>(cp);
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                const int n = 4 * i + 2 * h2;
+                                const float2 sn = make_float2(v16[n], v16[n + 1]);
+                                const float2 cc = h2 ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+                                const float2 w = mul2(x2, h2 ? make_float2(bv.z, bv.w) : make_float2(bv.x, bv.y));
+                                // s' * (-1) + fl(r Delta): one rounding, the difference
+                                const float2 e = fma2(sn, m1, mul2(make_float2(r[n], r[n + 1]), dl2));
+                                const float2 inc = add2(e, w);
+                                sig = fma2(cc, sn, sig);
+                                tot = fma2(cc, e, tot);
+                                const bool rx = (w.x > 0.0f && inc.x < 0.0f) || (w.x < 0.0f && inc.x > 0.0f);
+                                const bool ry = (w.y > 0.0f && inc.y < 0.0f) || (w.y < 0.0f && inc.y > 0.0f);
+                                rve = fma2(cc, make_float2(rx ? e.x : 0.0f, ry ? e.y : 0.0f), rve);
+                                nrev += (int)rx + (int)ry;
+                            }
+                        };
+                        dq(std::integral_constant<int, 0>{});
+                        dq(std::integral_constant<int, 1>{});
+                        dq(std::integral_constant<int, 2>{});
+                        dq(std::integral_constant<int, 3>{});
+                    };
+                    if (F::sym || !__any_sync(0xffffffffu, rp.clamp)) {
+#pragma unroll
+                        for (int sp = 0; sp < NP; ++sp) dpiece(std::false_type{}, sp);
+                    } else {
+#pragma unroll
+                        for (int sp = 0; sp < NP; ++sp) dpiece(std::true_type{}, sp);
+                    }
+                    dres = make_float4(grp_sum<LQ>((float)nrev),
+                                       grp_sum<LQ>(__fadd_rn(rve.x, rve.y)),
+                                       grp_sum<LQ>(__fadd_rn(tot.x, tot.y)),
+                                       grp_sum<LQ>(__fadd_rn(sig.x, sig.y)));
+                } else if (DIAG) {
+                    dres = row_exact_diag<FMT, N>(st, cs0, delta0, z0, lamv, dtx, gB, gC, j);
+                } else if (fast) {
                     const float2 inv2 = make_float2(rp.inv, rp.inv);
                     const float2 z2 = make_float2(rp.z, rp.z);
                     const float mz = F::sym ? -kMagic : -__fadd_rn(kMagic, rp.z);
@@ -802,7 +932,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 // bytes) of the warp's contiguous block of 32/LQ rows, lanes
                 // on consecutive chunks, so every store covers whole lines.
                 __syncwarp();
-                {
+                if constexpr (!DIAG) {
                     const int wrow0 = (gtid >> 5) * (32 / LQ);   // first row of this warp
                     const unsigned cbase = (unsigned)(geo.x_bytes + wrow0 * RB);
                     uint8_t* const gbase = codes_u + (long long)(ti.rbase + wrow0) * RB;
@@ -855,6 +985,12 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                                     mul2(x2, make_float2(vb.x, vb.y)));
                     float2 b = fma2(l2, make_float2(sv[4 * q + 2], sv[4 * q + 3]),
                                     mul2(x2, make_float2(vb.z, vb.w)));
+                    if constexpr (DIAG) {
+                        // the readout signal of the unrounded update
+                        acc = fma2(make_float2(vc.x, vc.y), a, acc);
+                        acc1 = fma2(make_float2(vc.z, vc.w), b, acc1);
+                        continue;
+                    }
                     if constexpr (kBf16) {
                         a = make_float2(__bfloat162float(__float2bfloat16_rn(a.x)),
                                         __bfloat162float(__float2bfloat16_rn(a.y)));
@@ -873,19 +1009,25 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
 #pragma unroll
                     for (int n = 0; n < EPC; ++n) w[n] = __float_as_uint(sv[n]);
                 }
-                if (active)
+                if (!DIAG && active)
                     __stcs(reinterpret_cast<uint4*>(frow) + m, make_uint4(w[0], w[1], w[2], w[3]));
             }
             acc = add2(acc, acc1);
             ysum = grp_sum<LF>(__fadd_rn(acc.x, acc.y));
+            dres.w = ysum;
         }
         // every lane of the row writes the same y (after the row sum all
         // hold it); a row past the end of the tile writes nothing
-        if (active)
+        if constexpr (DIAG) {
+            if (active && j == 0)
+                __stcs(reinterpret_cast<float4*>(cv.diag) + ti.lb * H * P + __float_as_int(hti.w) + p,
+                       dres);
+        } else if (active) {
             __stcs(y_u + __float_as_int(hti.w) + p, __fadd_rn(ysum, __fmul_rn(hti.z, xv)));
+        }
         // this warp's shared-memory writes are ordered before the tensor
         // copy that refills the stage
-        if (F::quant && ti.quant) fence_proxy_async();
+        if (!DIAG && F::quant && ti.quant) fence_proxy_async();
         __syncwarp();
         mbar_arrive_if(&empty[si], lane == 0);
     }
@@ -936,7 +1078,7 @@ cudaError_t make_codes_map(const PoolView& pv, int RB, CodesMap* cm)
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int FMT, int N, bool SR>
+template <int FMT, int N, int MODE>
 cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
 {
     using F = Fmt<FMT>;
@@ -958,7 +1100,7 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
         const cudaError_t e = make_codes_map(pv, RB, &cm);
         if (e != cudaSuccess) return e;
     }
-    auto kern = decode_kernel<FMT, N, SR>;
+    auto kern = decode_kernel<FMT, N, MODE>;
     // per-device launch facts, looked up once per kernel instantiation and device
     thread_local int s_dev = -1, s_grid = 0, s_smem = 0;
     int dev = 0;
@@ -987,15 +1129,15 @@ cudaError_t launch_n(const PoolView& pv, const CallView& cv, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <int FMT, bool SR>
+template <int FMT, int MODE>
 cudaError_t launch_fmt(const PoolView& pv, const CallView& cv, cudaStream_t st)
 {
     switch (pv.N) {
-    case 16: return launch_n<FMT, 16, SR>(pv, cv, st);
-    case 32: return launch_n<FMT, 32, SR>(pv, cv, st);
-    case 64: return launch_n<FMT, 64, SR>(pv, cv, st);
-    case 128: return launch_n<FMT, 128, SR>(pv, cv, st);
-    case 256: return launch_n<FMT, 256, SR>(pv, cv, st);
+    case 16: return launch_n<FMT, 16, MODE>(pv, cv, st);
+    case 32: return launch_n<FMT, 32, MODE>(pv, cv, st);
+    case 64: return launch_n<FMT, 64, MODE>(pv, cv, st);
+    case 128: return launch_n<FMT, 128, MODE>(pv, cv, st);
+    case 256: return launch_n<FMT, 256, MODE>(pv, cv, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -1022,21 +1164,40 @@ bool decode_fits(int fmt, int d_state, int nheads, int ngroups)
     return g.smem_bytes <= 227 * 1024;
 }
 
+template <int FMT>
+cudaError_t launch_mode(const PoolView& pv, const CallView& cv, int mode, cudaStream_t st)
+{
+    switch (mode) {
+    case kStochastic: return launch_fmt<FMT, kStochastic>(pv, cv, st);
+    case kDiagnostics: return launch_fmt<FMT, kDiagnostics>(pv, cv, st);
+    default: return launch_fmt<FMT, kNearest>(pv, cv, st);
+    }
+}
+
 cudaError_t launch_decode(const PoolView& pv, const CallView& cv, int fmt, bool sr,
                           cudaStream_t st)
 {
     // stochastic rounding changes only the integer formats
     switch (fmt) {
-    case SSQ_F32: return launch_fmt<SSQ_F32, false>(pv, cv, st);
-    case SSQ_BF16: return launch_fmt<SSQ_BF16, false>(pv, cv, st);
-    case SSQ_I8_SYM:
-        return sr ? launch_fmt<SSQ_I8_SYM, true>(pv, cv, st) : launch_fmt<SSQ_I8_SYM, false>(pv, cv, st);
-    case SSQ_I8_ASYM:
-        return sr ? launch_fmt<SSQ_I8_ASYM, true>(pv, cv, st) : launch_fmt<SSQ_I8_ASYM, false>(pv, cv, st);
-    case SSQ_I4_SYM:
-        return sr ? launch_fmt<SSQ_I4_SYM, true>(pv, cv, st) : launch_fmt<SSQ_I4_SYM, false>(pv, cv, st);
-    case SSQ_I4_ASYM:
-        return sr ? launch_fmt<SSQ_I4_ASYM, true>(pv, cv, st) : launch_fmt<SSQ_I4_ASYM, false>(pv, cv, st);
+    case SSQ_F32: return launch_fmt<SSQ_F32, kNearest>(pv, cv, st);
+    case SSQ_BF16: return launch_fmt<SSQ_BF16, kNearest>(pv, cv, st);
+    case SSQ_I8_SYM: return launch_mode<SSQ_I8_SYM>(pv, cv, sr ? kStochastic : kNearest, st);
+    case SSQ_I8_ASYM: return launch_mode<SSQ_I8_ASYM>(pv, cv, sr ? kStochastic : kNearest, st);
+    case SSQ_I4_SYM: return launch_mode<SSQ_I4_SYM>(pv, cv, sr ? kStochastic : kNearest, st);
+    case SSQ_I4_ASYM: return launch_mode<SSQ_I4_ASYM>(pv, cv, sr ? kStochastic : kNearest, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_decode_diag(const PoolView& pv, const CallView& cv, int fmt, cudaStream_t st)
+{
+    switch (fmt) {
+    case SSQ_F32: return launch_fmt<SSQ_F32, kDiagnostics>(pv, cv, st);
+    case SSQ_BF16: return launch_fmt<SSQ_BF16, kDiagnostics>(pv, cv, st);
+    case SSQ_I8_SYM: return launch_fmt<SSQ_I8_SYM, kDiagnostics>(pv, cv, st);
+    case SSQ_I8_ASYM: return launch_fmt<SSQ_I8_ASYM, kDiagnostics>(pv, cv, st);
+    case SSQ_I4_SYM: return launch_fmt<SSQ_I4_SYM, kDiagnostics>(pv, cv, st);
+    case SSQ_I4_ASYM: return launch_fmt<SSQ_I4_ASYM, kDiagnostics>(pv, cv, st);
     default: return cudaErrorInvalidValue;
     }
 }

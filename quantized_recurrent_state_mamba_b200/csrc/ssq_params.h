@@ -50,6 +50,7 @@ struct CallView {
     float* y;
     const float* S_in;         // quantize_rows input
     float* S_out;              // dequantize_rows output
+    float* diag;               // step diagnostics output, float4 per row
 };
 
 // The DAMP mixed-tier pool: every (slot, layer, head) owns one block of
@@ -92,9 +93,11 @@ cudaError_t launch_quantize(const PoolView& pv, const CallView& cv, int fmt,
 cudaError_t launch_dequantize(const PoolView& pv, const CallView& cv, int fmt,
                               cudaStream_t stream);
 // Step diagnostics (read-only): per row {reversals, reversal error, total
-// rounding error, readout signal} as float4 in [nl][batch][H][P] order.
-cudaError_t launch_diag(const PoolView& pv, const CallView& cv, int fmt, float* diag,
-                        cudaStream_t stream);
+// rounding error, readout signal} as float4 in [nl][batch][H][P] order, to
+// cv.diag.  The decode kernel in its diagnostics mode; tiles as
+// decode_tile_rows.
+cudaError_t launch_decode_diag(const PoolView& pv, const CallView& cv, int fmt,
+                               cudaStream_t stream);
 // How the scan splits its rows: entries per lane, warps per CTA, rows per
 // CTA, CTAs per head, tokens per staged chunk, dynamic shared memory.
 struct ScanPlan {

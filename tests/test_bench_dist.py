@@ -102,7 +102,9 @@ def test_kernel_source_hash_ignores_comments_only():
     assert fams == {"decode", "damp", "scan", "diag"}
     hashes = {w: bench.kernel_source_hash(w) for w in
               ("decode_130m", "decode_130m_damp", "scan_370m_all", "diag_130m")}
-    assert len(set(hashes.values())) == 4
+    # the diagnostics pass is the decode kernel in its diagnostics mode
+    assert len(set(hashes.values())) == 3
+    assert hashes["diag_130m"] == hashes["decode_130m"]
     assert bench.kernel_source_hash("decode_130m_sr") == hashes["decode_130m"]
 
 
