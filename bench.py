@@ -68,8 +68,12 @@ def workload(name):
         "decode_8b_b16_i8a": lambda: W.decode_8b("i8a", 16),
         "decode_8b_b64_i8a": lambda: W.decode_8b("i8a", 64),
         "decode_8b_b256_i8a": lambda: W.decode_8b("i8a", 256),
+        "decode_8b_b1_i8s": lambda: W.decode_8b("i8s", 1),
+        "decode_8b_b16_i8s": lambda: W.decode_8b("i8s", 16),
         "decode_8b_b64_i8s": lambda: W.decode_8b("i8s", 64),
         "decode_8b_b256_i8s": lambda: W.decode_8b("i8s", 256),
+        "decode_8b_b1_f32": lambda: W.decode_8b("f32", 1),
+        "decode_8b_b16_f32": lambda: W.decode_8b("f32", 16),
         "decode_8b_b64_f32": lambda: W.decode_8b("f32", 64),
         "decode_8b_b256_f32": lambda: W.decode_8b("f32", 256),
         "sweep_f32": lambda: W.sweep_serving("f32"),
@@ -77,6 +81,7 @@ def workload(name):
         "sweep_i8a": lambda: W.sweep_serving("i8a"),
         "sweep_i4a": lambda: W.sweep_serving("i4a"),
         "scan_370m_all": lambda: W.scan_370m("all"),
+        "scan_370m_b64": lambda: W.scan_370m("all", batch=64),
         "scan_370m_mid": lambda: W.scan_370m("mid"),
         "prefill_370m_all": lambda: W.scan_370m("all"),
         "prefill_370m_mid": lambda: W.scan_370m("mid"),
