@@ -504,6 +504,19 @@ __device__ __forceinline__ void minmax16(const float* v, float& lo, float& hi)
     hi = fmaxf(fmax3(A, B, C), fmax3(D, E, v[15]));
 }
 
+// ... and folded into a running (lo, hi): eight 3-input operations each.
+__device__ __forceinline__ void minmax16_acc(const float* v, float& lo, float& hi)
+{
+    const float a = fmin3(v[0], v[1], v[2]), b = fmin3(v[3], v[4], v[5]);
+    const float c = fmin3(v[6], v[7], v[8]), d = fmin3(v[9], v[10], v[11]);
+    const float e = fmin3(v[12], v[13], v[14]);
+    lo = fmin3(lo, fmin3(a, b, c), fmin3(d, e, v[15]));
+    const float A = fmax3(v[0], v[1], v[2]), B = fmax3(v[3], v[4], v[5]);
+    const float C = fmax3(v[6], v[7], v[8]), D = fmax3(v[9], v[10], v[11]);
+    const float E = fmax3(v[12], v[13], v[14]);
+    hi = fmax3(hi, fmax3(A, B, C), fmax3(D, E, v[15]));
+}
+
 template <int FMT, int E, int LPR>
 __device__ __forceinline__ RowParams refit_row(const float (&s)[E])
 {

@@ -53,28 +53,60 @@
 
 #include <cstring>
 #include <type_traits>
+#include <utility>
 
 namespace ssq {
 
 namespace {
 
-constexpr int kCWarps = 16;                 // consumer warps
-// Consumer groups (tiles alternate between them).  One group of all 16 warps
-// on 512-row tiles measured fastest: with two or four groups on smaller
-// tiles the single producer warp could not prepare tiles as fast as the
-// consumers took them.
-constexpr int kGroups = 1;
-constexpr int kGWarps = kCWarps / kGroups;  // warps per group
+// Consumer warps.  All 16 share each 512-row tile: with two or four groups
+// of warps on smaller tiles the single producer warp could not prepare tiles
+// as fast as the consumers took them.
+constexpr int kCWarps = 16;
 constexpr int kCThreads = kCWarps * 32;
-constexpr int kGThreads = kGWarps * 32;
 constexpr int kDThreads = kCThreads + 32;   // + 1 producer warp
 constexpr int kMaxStages = 8;
 constexpr int kBoxRows = 128;               // rows per tensor copy
 constexpr unsigned kTmemCols = 512;         // all of TMEM: 128 columns per consumer warp
 
 // ---- PTX wrappers: shared memory at 32-bit addresses --------------------
+// Loads of data that stays put while it is read (a landed stage, the unit
+// buffer): plain asm, free for the compiler to schedule.  Their addresses
+// come from laundered bases (launder() after the wait that makes the data
+// visible), so no load can be placed before that wait.
 template <int OFF>
 __device__ __forceinline__ uint4 lds128(unsigned a)
+{
+    uint4 v;
+    asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4+%5];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ uint2 lds64(unsigned a)
+{
+    uint2 v;
+    asm("ld.shared.v2.b32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ float4 lds128f(unsigned a)
+{
+    float4 v;
+    asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4+%5];"
+        : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a), "n"(OFF));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(unsigned a)
+{
+    uint32_t v;
+    asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+// A load kept in program order with the shared-memory stores around it (the
+// warp reading back what its lanes just wrote).
+template <int OFF>
+__device__ __forceinline__ uint4 lds128_ordered(unsigned a)
 {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4+%5];"
@@ -82,20 +114,20 @@ __device__ __forceinline__ uint4 lds128(unsigned a)
     return v;
 }
 template <int OFF>
-__device__ __forceinline__ uint2 lds64(unsigned a)
-{
-    uint2 v;
-    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2+%3];"
-                 : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF) : "memory");
-    return v;
-}
-template <int OFF>
-__device__ __forceinline__ float4 lds128f(unsigned a)
+__device__ __forceinline__ float4 lds128f_ordered(unsigned a)
 {
     float4 v;
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4+%5];"
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a), "n"(OFF) : "memory");
     return v;
+}
+// A shared-memory address that the compiler sees as produced here: loads
+// from it cannot be moved above this point (a wait before it).
+__device__ __forceinline__ unsigned launder(unsigned a)
+{
+    unsigned r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(a) : "memory");
+    return r;
 }
 // Stores predicated inside the instruction, so the warp stays converged
 // around the tcgen05 instructions that follow.
@@ -166,6 +198,9 @@ __device__ __forceinline__ void tc_fence_after()
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 // 16 fp32 values of this lane into 16 consecutive columns of its TMEM lane.
+// (TMEM is not memory the compiler tracks: the tcgen05 wrappers are volatile,
+// which keeps them in program order with one another, without a memory
+// clobber, which leaves shared-memory loads free to move around them.)
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
 {
     asm volatile(
@@ -173,26 +208,75 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
         " %11, %12, %13, %14, %15, %16};"
         :: "r"(taddr), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]),
            "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]),
-           "f"(v[13]), "f"(v[14]), "f"(v[15])
-        : "memory");
+           "f"(v[13]), "f"(v[14]), "f"(v[15]));
 }
 __device__ __forceinline__ void tmem_wait_st()
 {
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;");
 }
-// ... and back, waiting for the load in the same statement (the registers
-// are written asynchronously until the wait).
+// ... and back.  The registers are written asynchronously until
+// tmem_wait_ld(v), which takes them as operands: every use of v follows it.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
 {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10,"
-        " %11, %12, %13, %14, %15}, [%16];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
+        " %11, %12, %13, %14, %15}, [%16];"
         : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
           "=f"(v[7]), "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]),
           "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
-        : "r"(taddr)
-        : "memory");
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld(float (&v)[16])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
+                   "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]),
+                   "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]));
+}
+
+// f(std::integral_constant<int, i>) for i = 0 .. N-1, unrolled.
+template <typename Fn, int... I>
+__device__ __forceinline__ void static_for_seq(Fn&& f, std::integer_sequence<int, I...>)
+{
+    (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename Fn>
+__device__ __forceinline__ void static_for(Fn&& f)
+{
+    static_for_seq(f, std::make_integer_sequence<int, N>{});
+}
+
+// f(v, piece) for the NP 16-column pieces of this lane's TMEM row.  With
+// PIPE the load of piece sp + 1 is in flight while f works on piece sp (16
+// more registers); without, each load is waited for at once.
+template <int NP, bool PIPE, typename Fn>
+__device__ __forceinline__ void tmem_pieces(uint32_t tm, Fn&& f)
+{
+    if constexpr (PIPE) {
+        float va[16], vb[16];
+        tmem_ld16(tm, va);
+        tmem_wait_ld(va);
+        static_for<NP>([&](auto spc) {
+            constexpr int sp = decltype(spc)::value;
+            if constexpr (sp % 2 == 0) {
+                if constexpr (sp + 1 < NP) tmem_ld16(tm + 16 * (sp + 1), vb);
+                f(va, spc);
+                if constexpr (sp + 1 < NP) tmem_wait_ld(vb);
+            } else {
+                if constexpr (sp + 1 < NP) tmem_ld16(tm + 16 * (sp + 1), va);
+                f(vb, spc);
+                if constexpr (sp + 1 < NP) tmem_wait_ld(va);
+            }
+        });
+    } else {
+        static_for<NP>([&](auto spc) {
+            constexpr int sp = decltype(spc)::value;
+            float v[16];
+            tmem_ld16(tm + 16 * sp, v);
+            tmem_wait_ld(v);
+            f(v, spc);
+        });
+    }
 }
 
 // Named barrier of the consumer warps (the producer does not take part).
@@ -209,7 +293,7 @@ __host__ __device__ inline int r1024(int v) { return (v + 1023) & ~1023; }
 // Tiles are ordered (layer, request, region, row block).  Every warp walks
 // the CTA's contiguous range of them with counters (one division at the
 // start); the tiles loaded into the ring are numbered in that order, and
-// loaded tile k goes to stage k % S and consumer group k % kGroups.
+// loaded tile k goes to stage k % S.
 struct TileWalk {
     long long lb;   // layer * batch + request
     int l, b, k;    // k: tile within (layer, request)
@@ -308,13 +392,13 @@ template <int N>
 struct QShape {
     static constexpr int E = N >= kQuantE ? kQuantE : N;
     static constexpr int LPR = N / E;
-    static constexpr int RPT = kGThreads / LPR;   // rows per tile
+    static constexpr int RPT = kCThreads / LPR;   // rows per tile
 };
 template <int N>
 struct FShape {
     static constexpr int E = N >= 32 ? 32 : N;
     static constexpr int LPR = N / E;
-    static constexpr int RPT = kGThreads / LPR;
+    static constexpr int RPT = kCThreads / LPR;
 };
 
 // A whole quantized row by the formulas verbatim (every fp32 operation one
@@ -513,7 +597,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kGWarps);
+            mbar_init(&empty[s], kCWarps);
         }
         for (int u = 0; u < 2; ++u) {
             mbar_init(&ufull[u], 1);
@@ -535,11 +619,17 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     if (warp == kCWarps) {
         // ================= producer warp =================
         int k = 0, uk = -1;
+        int si = 0;          // stage of loaded tile k
+        unsigned eph = 0;    // parity of the release of that stage's previous tile
         bool bad = false, ok = true, newunit = true;
         int cur_slot = 0, cur_layer = 0;
         const uint8_t* meta_u = nullptr;
         const uint8_t* fp_u = nullptr;
         const float* x_u = nullptr;
+        // x of a tile by bulk copies, one per head the tile touches, when
+        // every copy is 16-byte aligned (head_dim a multiple of 4, x aligned);
+        // else one 4-byte cp.async per row
+        const bool x_bulk = (P & 3) == 0 && (reinterpret_cast<uintptr_t>(cv.x) & 15) == 0;
         TileWalk ti;
         ti.start(Hq, Hf, P, cv, t0);
         for (long long t = t0; t < t1; ++t, newunit = ti.next(Hq, Hf, P, cv)) {
@@ -547,7 +637,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             if (newunit) {
                 ++uk;
                 const int u = uk & 1;
-                if (!mbar_wait<kProducerSleep>(&uempty[u], ((uk >> 1) & 1) ^ 1, wlim)) { ok = false; break; }
+                if (!mbar_wait_suspend(&uempty[u], ((uk >> 1) & 1) ^ 1, wlim)) { ok = false; break; }
                 const int slot = cv.slot_idx ? __ldg(cv.slot_idx + ti.b) : ti.b;
                 bad = slot < 0 || slot >= pv.n_slots;
                 uint8_t* ub = units + u * geo.unit_bytes;
@@ -602,48 +692,69 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     bulk_prefetch_l2(fp_u + (long long)ti.rbase * N * FEB, (unsigned)(ti.n * N * FEB));
                 }
             }
-            const int si = k % S;
             // the stage's previous tile (k - S) must have been released
-            if (k >= S && !mbar_wait<kProducerSleep>(&empty[si], (unsigned)(((k - S) / S) & 1), wlim)) {
+            if (k >= S && !mbar_wait_suspend(&empty[si], eph, wlim)) {
                 ok = false;
                 break;
             }
             // test support: CTA 0 leaves its first stage unfilled, so its
             // consumers' bounded waits run out (ssq_test_hooks)
-            if (cv.test_withhold && blockIdx.x == 0 && k == 0) {
-                ++k;
-                continue;
-            }
-            uint8_t* st = stages + si * geo.stage_bytes;
-            float* sx = reinterpret_cast<float*>(st);
-            for (int i = lane; i < ti.n; i += 32) {
-                const int rr = ti.rbase + i;
-                const int hr = fdiv(rr, pv.mP);
-                const int hh = pv.perm[regbase + hr];
-                cpa4(sx + i, x_u + hh * P + (rr - hr * P));
-            }
-            cpa_arrive(&full[si]);
-            __syncwarp();
-            if (lane == 0) {
+            if (!(cv.test_withhold && blockIdx.x == 0 && k == 0)) {
+                uint8_t* st = stages + si * geo.stage_bytes;
+                float* sx = reinterpret_cast<float*>(st);
                 uint8_t* pay = st + geo.x_bytes;
+                unsigned pay_bytes;
                 if (F::quant && ti.quant) {
-                    const int line0 = ti.rbase * RB / 128;
                     const int nbox = (ti.n + kBoxRows - 1) / kBoxRows;
-                    const unsigned mb = (unsigned)r16(ti.n * MB);
-                    mbar_arrive_tx(&full[si], (unsigned)(nbox * kBoxLines * 128) + mb);
-#pragma unroll 1
-                    for (int bx = 0; bx < nbox; ++bx)
-                        tma_load_codes(pay + bx * kBoxLines * 128, &cm.map, line0 + bx * kBoxLines,
-                                       cur_layer, cur_slot, &full[si]);
-                    bulk_g2s(pay + geo.qcodes_bytes, meta_u + (long long)ti.rbase * MB, mb,
-                             &full[si]);
+                    pay_bytes = (unsigned)(nbox * kBoxLines * 128) + (unsigned)r16(ti.n * MB);
                 } else {
-                    const unsigned fb = (unsigned)(ti.n * N * FEB);
-                    mbar_arrive_tx(&full[si], fb);
-                    bulk_g2s(pay, fp_u + (long long)ti.rbase * N * FEB, fb, &full[si]);
+                    pay_bytes = (unsigned)(ti.n * N * FEB);
+                }
+                if (x_bulk) {
+                    // the heads [h0, h1] the tile's rows fall in, a copy each
+                    const int h0 = fdiv(ti.rbase, pv.mP);
+                    const int h1 = fdiv(ti.rbase + ti.n - 1, pv.mP);
+                    if (lane == 0) mbar_arrive_tx(&full[si], pay_bytes + (unsigned)(ti.n * 4));
+                    __syncwarp();
+                    for (int hr = h0 + lane; hr <= h1; hr += 32) {
+                        const int r0 = max(ti.rbase, hr * P);
+                        const int r1 = min(ti.rbase + ti.n, (hr + 1) * P);
+                        const int hh = pv.perm[regbase + hr];
+                        bulk_g2s(sx + (r0 - ti.rbase), x_u + hh * P + (r0 - hr * P),
+                                 (unsigned)((r1 - r0) * 4), &full[si]);
+                    }
+                } else {
+                    for (int i = lane; i < ti.n; i += 32) {
+                        const int rr = ti.rbase + i;
+                        const int hr = fdiv(rr, pv.mP);
+                        const int hh = pv.perm[regbase + hr];
+                        cpa4(sx + i, x_u + hh * P + (rr - hr * P));
+                    }
+                    cpa_arrive(&full[si]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_tx(&full[si], pay_bytes);
+                }
+                if (lane == 0) {
+                    if (F::quant && ti.quant) {
+                        const int line0 = ti.rbase * RB / 128;
+                        const int nbox = (ti.n + kBoxRows - 1) / kBoxRows;
+#pragma unroll 1
+                        for (int bx = 0; bx < nbox; ++bx)
+                            tma_load_codes(pay + bx * kBoxLines * 128, &cm.map, line0 + bx * kBoxLines,
+                                           cur_layer, cur_slot, &full[si]);
+                        bulk_g2s(pay + geo.qcodes_bytes, meta_u + (long long)ti.rbase * MB,
+                                 (unsigned)r16(ti.n * MB), &full[si]);
+                    } else {
+                        bulk_g2s(pay, fp_u + (long long)ti.rbase * N * FEB, pay_bytes, &full[si]);
+                    }
                 }
             }
             ++k;
+            if (++si == S) {
+                // tiles [k, k + S) wait for the releases of tiles [k - S, k)
+                si = 0;
+                if (k >= 2 * S) eph ^= 1u;
+            }
         }
         if (!ok && lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
         // No copy may still be writing shared memory when the CTA exits.
@@ -656,10 +767,12 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
     }
 
     // ================= consumer warps =================
-    const int grp = warp / kGWarps;                  // consumer group
-    const int gtid = threadIdx.x - grp * kGThreads;  // thread within the group
-    int k = 0, uk = -1;
+    const int gtid = threadIdx.x;    // thread within the consumers
+    int uk = -1;
+    int si = 0;            // stage of the next tile
+    unsigned fph = 0;      // its fill parity
     bool bad = false, newunit = true, ok = true;
+    unsigned ub_a = 0;     // unit buffer, laundered shared address
     const uint8_t* ub = units;
     uint8_t* codes_u = nullptr;
     uint8_t* meta_u = nullptr;
@@ -681,8 +794,9 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             }
             ++uk;
             const int u = uk & 1;
-            if (!mbar_wait<kConsumerSleep>(&ufull[u], (uk >> 1) & 1, wlim)) { ok = false; break; }
+            if (!mbar_wait_suspend(&ufull[u], (uk >> 1) & 1, wlim)) { ok = false; break; }
             ub = units + u * geo.unit_bytes;
+            ub_a = launder(saddr(ub));
             const int slot = reinterpret_cast<const int*>(ub)[0];
             cur_slot = slot;
             bad = reinterpret_cast<const int*>(ub)[1] != 0;
@@ -696,12 +810,14 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
             }
         }
         if (bad) continue;
-        const int kk = k++;
-        if (kk % kGroups != grp) continue;
-        const int si = kk % S;
-        if (!mbar_wait<kConsumerSleep>(&full[si], (unsigned)((kk / S) & 1), wlim)) { ok = false; break; }
-        uint8_t* const st = stages + si * geo.stage_bytes;
-        const float* sx = reinterpret_cast<const float*>(st);
+        const int tsi = si;
+        if (!mbar_wait_suspend(&full[tsi], fph, wlim)) { ok = false; break; }
+        if (++si == S) {
+            si = 0;
+            fph ^= 1u;
+        }
+        uint8_t* const st = stages + tsi * geo.stage_bytes;
+        const unsigned st_a = launder(saddr(st));
         uint8_t* const pay = st + geo.x_bytes;
         // row within the tile and lane within the row, by the region's shape
         const int grow = ti.quant ? gtid / LQ : gtid / LF;
@@ -713,9 +829,9 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         const int rr = ti.rbase + rl;
         const int hr = fdiv(rr, pv.mP);
         const int p = rr - hr * P;
-        const float4 hti = reinterpret_cast<const float4*>(ub + geo.ub_ht)[hr];
-        const int gN = reinterpret_cast<const int*>(ub + geo.ub_gt)[hr];
-        const float xv = active ? sx[grow] : 0.0f;
+        const float4 hti = lds128f<0>(ub_a + geo.ub_ht + 16 * hr);
+        const int gN = (int)lds32(ub_a + geo.ub_gt + 4 * hr);
+        const float xv = active ? __uint_as_float(lds32(st_a + 4 * grow)) : 0.0f;
         const float lamv = hti.x;
         const float dtx = __fmul_rn(hti.y, xv);
         const float* gB = reinterpret_cast<const float*>(ub + geo.ub_B) + gN;
@@ -730,35 +846,35 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                 // this lane's codes in the stage (piece sp of the lane at
                 // cs_x ^ (sp * PB) under the swizzle) and the row's metadata
                 const unsigned cs0 = (unsigned)(geo.x_bytes + grow * RB + j * CB);
-                const unsigned cs_x = saddr(st) + swz128(cs0);
-                uint8_t* const ms = pay + geo.qcodes_bytes + grow * MB;
+                const unsigned cs_x = st_a + swz128(cs0);
+                const unsigned ms_a = st_a + (unsigned)(geo.x_bytes + geo.qcodes_bytes + grow * MB);
                 // (a row past the end of the tile reads its stage slot and
                 // decodes zeros instead)
                 float delta0, z0 = 0.0f;
                 if constexpr (F::sym) {
-                    delta0 = *reinterpret_cast<const float*>(ms);
+                    delta0 = __uint_as_float(lds32(ms_a));
                 } else {
-                    const float2 m = *reinterpret_cast<const float2*>(ms);
-                    delta0 = m.x;
-                    z0 = m.y;
+                    const uint2 m = lds64<0>(ms_a);
+                    delta0 = __uint_as_float(m.x);
+                    z0 = __uint_as_float(m.y);
                 }
                 delta0 = active ? delta0 : 0.0f;
                 z0 = active ? z0 : 0.0f;
-                const unsigned bxa = saddr(gB) + j * EQ * 4;
-                const unsigned cxa = saddr(gC) + j * EQ * 4;
+                const unsigned bxa = ub_a + geo.ub_B + 4 * gN + j * EQ * 4;
+                const unsigned cxa = ub_a + geo.ub_C + 4 * gN + j * EQ * 4;
                 // decode + update, one 16-entry piece at a time, with
                 // per-piece min / max; the updated pieces wait in TMEM.  The
                 // decode is exact for |z| < 2^22; rows beyond take the exact
                 // path below.
-                float lo, hi;
+                float lo = 0.0f, hi = 0.0f;
                 {
                     const float c0 = __fadd_rn(kTwo23, __fadd_rn(z0, F::bias));
                     const float2 nc02 = make_float2(-c0, -c0);
                     const float2 d2 = make_float2(delta0, delta0);
                     const float2 l2 = make_float2(lamv, lamv);
                     const float2 x2 = make_float2(dtx, dtx);
-#pragma unroll
-                    for (int sp = 0; sp < NP; ++sp) {
+                    static_for<NP>([&](auto spc) {
+                        constexpr int sp = decltype(spc)::value;
                         uint32_t w[PW];
                         if constexpr (PW == 4) {
                             const uint4 v = lds128<0>(cs_x ^ (sp * PB));
@@ -769,28 +885,24 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         }
                         float f[16];
                         unpack16_biased<FMT>(w, f);
-                        const unsigned bp = bxa + sp * 64;
                         float v16[16];
-                        auto bq = [&](auto ic) {
+                        static_for<4>([&](auto ic) {
                             constexpr int i = decltype(ic)::value;
-                            const float4 bv = lds128f<i * 16>(bp);
+                            const float4 bv = lds128f<sp * 64 + i * 16>(bxa);
                             const float2 v0 = mul2(add2(make_float2(f[4 * i], f[4 * i + 1]), nc02), d2);
                             const float2 v1 = mul2(add2(make_float2(f[4 * i + 2], f[4 * i + 3]), nc02), d2);
                             const float2 u0 = fma2(l2, v0, mul2(x2, make_float2(bv.x, bv.y)));
                             const float2 u1 = fma2(l2, v1, mul2(x2, make_float2(bv.z, bv.w)));
                             v16[4 * i] = u0.x; v16[4 * i + 1] = u0.y;
                             v16[4 * i + 2] = u1.x; v16[4 * i + 3] = u1.y;
-                        };
-                        bq(std::integral_constant<int, 0>{});
-                        bq(std::integral_constant<int, 1>{});
-                        bq(std::integral_constant<int, 2>{});
-                        bq(std::integral_constant<int, 3>{});
-                        float plo, phi;
-                        minmax16(v16, plo, phi);
-                        lo = sp == 0 ? plo : fminf(lo, plo);
-                        hi = sp == 0 ? phi : fmaxf(hi, phi);
+                        });
+                        if constexpr (sp == 0) {
+                            minmax16(v16, lo, hi);
+                        } else {
+                            minmax16_acc(v16, lo, hi);
+                        }
                         tmem_st16(tm + sp * 16, v16);
-                    }
+                    });
                 }
                 tmem_wait_st();
                 const RowParams rp = refit_from_minmax<FMT, LQ>(lo, hi);
@@ -821,17 +933,17 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     float2 sig = make_float2(0.0f, 0.0f), tot = make_float2(0.0f, 0.0f);
                     float2 rve = make_float2(0.0f, 0.0f);
                     int nrev = 0;
-                    auto dpiece = [&](auto clamp_tag, int sp) {
-                        float v16[16];
-                        tmem_ld16(tm + sp * 16, v16);
+                    auto dpiece = [&](auto clamp_tag, float (&v16)[16], auto spc) {
+                        constexpr int sp = decltype(spc)::value;
                         float r[16];
                         uint32_t kq[16];
                         round16_carry<FMT, decltype(clamp_tag)::value>(inv2, z2, mz2, v16, r, kq);
-                        const unsigned bp = bxa + sp * 64, cp = cxa + sp * 64;
-                        auto dq = [&](auto ic) {
+                        static_for<4>([&](auto ic) {
                             constexpr int i = decltype(ic)::value;
-                            const float4 bv = lds128f<i * 16>(bp);
-                            const float4 c4 = lds128f<i * 16>(cp);
+                            // (loads in program order: scheduled freely they
+                            // raise the live registers of this pass past 96)
+                            const float4 bv = lds128f_ordered<sp * 64 + i * 16>(bxa);
+                            const float4 c4 = lds128f_ordered<sp * 64 + i * 16>(cxa);
 #pragma unroll
                             for (int h2 = 0; h2 < 2; ++h2) {
                                 const int n = 4 * i + 2 * h2;
@@ -848,18 +960,12 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                                 rve = fma2(cc, make_float2(rx ? e.x : 0.0f, ry ? e.y : 0.0f), rve);
                                 nrev += (int)rx + (int)ry;
                             }
-                        };
-                        dq(std::integral_constant<int, 0>{});
-                        dq(std::integral_constant<int, 1>{});
-                        dq(std::integral_constant<int, 2>{});
-                        dq(std::integral_constant<int, 3>{});
+                        });
                     };
                     if (F::sym || !__any_sync(0xffffffffu, rp.clamp)) {
-#pragma unroll
-                        for (int sp = 0; sp < NP; ++sp) dpiece(std::false_type{}, sp);
+                        tmem_pieces<NP, false>(tm, [&](float (&v)[16], auto spc) { dpiece(std::false_type{}, v, spc); });
                     } else {
-#pragma unroll
-                        for (int sp = 0; sp < NP; ++sp) dpiece(std::true_type{}, sp);
+                        tmem_pieces<NP, false>(tm, [&](float (&v)[16], auto spc) { dpiece(std::true_type{}, v, spc); });
                     }
                     dres = make_float4(grp_sum<LQ>((float)nrev),
                                        grp_sum<LQ>(__fadd_rn(rve.x, rve.y)),
@@ -872,12 +978,12 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     const float2 z2 = make_float2(rp.z, rp.z);
                     const float mz = F::sym ? -kMagic : -__fadd_rn(kMagic, rp.z);
                     const float2 mz2 = make_float2(mz, mz);
-                    // round, pack, write back and read out, piece by piece;
-                    // the readout sums C (q - z) and scales by Delta once
+                    // round, pack, write back and read out, piece by piece
+                    // (the next piece's TMEM load in flight); the readout sums
+                    // C (q - z) and scales by Delta once
                     float2 acc = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
-                    auto piece = [&](auto clamp_tag, int sp) {
-                        float v16[16];
-                        tmem_ld16(tm + sp * 16, v16);
+                    auto piece = [&](auto clamp_tag, float (&v16)[16], auto spc) {
+                        constexpr int sp = decltype(spc)::value;
                         float r[16];
                         uint32_t kq[16];
                         if constexpr (SR) {
@@ -893,24 +999,17 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                             sts128u_if(cs_x ^ (sp * PB), make_uint4(w[0], w[1], w[2], w[3]), active);
                         else
                             sts64u_if(cs_x ^ (sp * PB), make_uint2(w[0], w[1]), active);
-                        const unsigned cp = cxa + sp * 64;
-                        auto cq = [&](auto ic) {
+                        static_for<4>([&](auto ic) {
                             constexpr int i = decltype(ic)::value;
-                            const float4 cv4 = lds128f<i * 16>(cp);
+                            const float4 cv4 = lds128f<sp * 64 + i * 16>(cxa);
                             acc = fma2(make_float2(cv4.x, cv4.y), make_float2(r[4 * i], r[4 * i + 1]), acc);
                             acc1 = fma2(make_float2(cv4.z, cv4.w), make_float2(r[4 * i + 2], r[4 * i + 3]), acc1);
-                        };
-                        cq(std::integral_constant<int, 0>{});
-                        cq(std::integral_constant<int, 1>{});
-                        cq(std::integral_constant<int, 2>{});
-                        cq(std::integral_constant<int, 3>{});
+                        });
                     };
                     if (SR || F::sym || !__any_sync(0xffffffffu, rp.clamp)) {
-#pragma unroll
-                        for (int sp = 0; sp < NP; ++sp) piece(std::false_type{}, sp);
+                        tmem_pieces<NP, true>(tm, [&](float (&v)[16], auto spc) { piece(std::false_type{}, v, spc); });
                     } else {
-#pragma unroll
-                        for (int sp = 0; sp < NP; ++sp) piece(std::true_type{}, sp);
+                        tmem_pieces<NP, true>(tm, [&](float (&v)[16], auto spc) { piece(std::true_type{}, v, spc); });
                     }
                     acc = add2(acc, acc1);
                     ysum = __fmul_rn(rp.delta, grp_sum<LQ>(__fadd_rn(acc.x, acc.y)));
@@ -928,22 +1027,40 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                     ysum = row_exact<FMT, N, SR>(st, cs0, delta0, z0, lamv, dtx, gB, gC, j,
                                                  active, meta_u + (long long)rr * MB, err, srk);
                 }
-                // This warp's rows, from the stage to the pool: chunk c (16
-                // bytes) of the warp's contiguous block of 32/LQ rows, lanes
-                // on consecutive chunks, so every store covers whole lines.
+                // This warp's rows, from the stage to the pool: the warp's
+                // contiguous block of 32/LQ rows, 16-byte chunk c = lane + 32 i
+                // by lane `lane`, so every store instruction covers whole lines.
                 __syncwarp();
                 if constexpr (!DIAG) {
-                    const int wrow0 = (gtid >> 5) * (32 / LQ);   // first row of this warp
-                    const unsigned cbase = (unsigned)(geo.x_bytes + wrow0 * RB);
-                    uint8_t* const gbase = codes_u + (long long)(ti.rbase + wrow0) * RB;
-                    const int nbytes = (min(ti.n - wrow0, 32 / LQ) > 0
-                                        ? min(ti.n - wrow0, 32 / LQ) : 0) * RB;
-#pragma unroll
-                    for (int c = lane; c < 2 * CB; c += 32) {
-                        if (c * 16 < nbytes) {
-                            const uint4 v = *reinterpret_cast<const uint4*>(st + swz128(cbase + c * 16));
-                            __stcs(reinterpret_cast<uint4*>(gbase + c * 16), v);
-                        }
+                    constexpr int WB = (32 / LQ) * RB;              // bytes of the block
+                    constexpr int WCH = WB / 16;                    // its 16-byte chunks
+                    constexpr int NI = (WCH + 31) / 32;             // chunks per lane
+                    const int wrow0 = warp * (32 / LQ);             // first row of the block
+                    const int wrows = min(ti.n - wrow0, 32 / LQ);   // live rows (may be <= 0)
+                    // chunk c at swizzle(cb + 16 c) = A[i & 1] + 512 i, cb the
+                    // block's stage offset: 512 i moves bit 9 and up, and the
+                    // swizzle's XOR term takes bits 7..9
+                    const unsigned cl = (unsigned)(geo.x_bytes + wrow0 * RB + 16 * lane);
+                    const unsigned a0 = st_a + swz128(cl);
+                    const unsigned a1 = a0 ^ 64u;
+                    uint8_t* const gdst = codes_u + (long long)(ti.rbase + wrow0) * RB + 16 * lane;
+                    if (wrows == 32 / LQ && WCH % 32 == 0) {
+                        uint4 v[NI];
+                        static_for<NI>([&](auto ic) {
+                            constexpr int i = decltype(ic)::value;
+                            v[i] = lds128_ordered<i * 512>((i & 1) ? a1 : a0);
+                        });
+                        static_for<NI>([&](auto ic) {
+                            constexpr int i = decltype(ic)::value;
+                            __stcs(reinterpret_cast<uint4*>(gdst + i * 512), v[i]);
+                        });
+                    } else {
+                        static_for<NI>([&](auto ic) {
+                            constexpr int i = decltype(ic)::value;
+                            if (16 * (lane + 32 * i) < max(wrows, 0) * RB)
+                                __stcs(reinterpret_cast<uint4*>(gdst + i * 512),
+                                       lds128_ordered<i * 512>((i & 1) ? a1 : a0));
+                        });
                     }
                 }
             }
@@ -1029,7 +1146,7 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
         // copy that refills the stage
         if (!DIAG && F::quant && ti.quant) fence_proxy_async();
         __syncwarp();
-        mbar_arrive_if(&empty[si], lane == 0);
+        mbar_arrive_if(&empty[tsi], lane == 0);
     }
     if (!ok && lane == 0) atomicOr(err, SSQ_DEVERR_TIMEOUT);
     // release TMEM once every consumer warp's TMEM accesses are complete
@@ -1148,8 +1265,8 @@ void decode_tile_rows(int fmt, int d_state, int* rows_q, int* rows_f)
 {
     const int eq = d_state >= kQuantE ? kQuantE : d_state;
     const int ef = d_state >= 32 ? 32 : d_state;
-    *rows_q = kGThreads / (d_state / eq);
-    *rows_f = kGThreads / (d_state / ef);
+    *rows_q = kCThreads / (d_state / eq);
+    *rows_f = kCThreads / (d_state / ef);
     (void)fmt;
 }
 

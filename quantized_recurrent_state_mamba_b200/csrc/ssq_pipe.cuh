@@ -68,6 +68,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, unsigned parity,
 }
 constexpr unsigned kProducerSleep = 2048;  // the producer waits for a stage to drain
 constexpr unsigned kConsumerSleep = 256;   // consumers wait for data to land
+
+// One test of the phase in which the thread may be suspended by the
+// hardware until the phase completes or about `hint_ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_suspend(uint64_t* b, unsigned parity, unsigned hint_ns)
+{
+    unsigned ok;
+    asm volatile("{\n .reg .pred p;\n"
+                 " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+                 " selp.u32 %0, 1, 0, p;\n}\n"
+                 : "=r"(ok) : "r"(saddr(b)), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+// Wait for the phase of the given parity to complete with the thread
+// suspended in the barrier instead of polling (a waiting warp issues a few
+// instructions per suspension, not one loop per few cycles); false after
+// `limit` clock cycles without progress.
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* b, unsigned parity,
+                                                  long long limit = kWaitLimit)
+{
+    if (mbar_try_suspend(b, parity, 20000u)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_suspend(b, parity, 20000u)) {
+        if (clock64() - t0 > limit) return false;
+    }
+    return true;
+}
 // Bulk prefetch of global memory into L2 (no completion to wait for).
 // Address 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, unsigned bytes)

@@ -4,9 +4,10 @@ The decode kernel (csrc/ssq_decode.cu) addresses shared memory, tensor
 memory and the pool with arithmetic that no GPU run can check for an
 out-of-bounds access without risking a fault.  This test restates that
 arithmetic on the CPU -- the stage geometry and stage count, the tile walk,
-the tensor-copy boxes and their coordinates, each lane's swizzled code
-address, its metadata, x, B and C reads, its TMEM columns and the rows it
-copies back to the pool -- and checks every access against its buffer for
+the tensor-copy boxes and their coordinates, the producer's x copies, each
+lane's swizzled code address, its metadata, x, B and C reads, its TMEM
+columns and the rows it copies back to the pool -- and checks every access
+against its buffer for
 each shape the tests and the benchmark use.  The pool layout comes from the
 library itself (ssq_pool_layout), so global addresses are checked against
 the sizes the library allocates.  It also checks the identity the consumer
@@ -139,27 +140,41 @@ def check_decode(ssq, fmt, H, P, N, G, n_layers, n_slots, mask=None):
                 assert (a + sh["PB"]).max() <= g["x_bytes"] + g["qcodes"]
                 # B / C entries of the piece (group offset + lane offset)
                 assert (j * EQ + sp * 16 + 16).max() <= N
+            check_x_copies(rbase, n, P, Hq * P, g)
             ms = g["x_bytes"] + g["qcodes"] + grow * MB
             assert (ms + MB).max() <= g["stage"]
             assert (grow * 4 + 4).max() <= g["x_bytes"]           # x of the row
             # TMEM: 128 columns per warp, EQ used
             w = gtid // 32
             assert ((w // 4) * 128 + EQ).max() <= TMEM_COLS and EQ <= 128
-            # copy-back of each warp's rows: chunks c < 2*CB of its block
+            # copy-back of each warp's rows: 16-byte chunk c = lane + 32 i of
+            # the warp's block, read at A[i & 1] + 512 i with A[0] the
+            # swizzled first chunk of the lane and A[1] = A[0] ^ 64
+            WB = (32 // LQ) * RB
+            WCH = WB // 16
+            lane = gtid % 32
             wrow0 = (gtid // 32) * (32 // LQ)
-            for c in range(2 * CB):
-                off = g["x_bytes"] + wrow0 * RB + 16 * c
-                assert (swz128(off) + 16).max() <= g["x_bytes"] + g["qcodes"]
-                wrows = np.clip(n - wrow0, 0, 32 // LQ)
+            wrows = np.clip(n - wrow0, 0, 32 // LQ)
+            cl = g["x_bytes"] + wrow0 * RB + 16 * lane
+            a0 = swz128(cl)
+            a1 = a0 ^ 64
+            for i in range((WCH + 31) // 32):
+                c = lane + 32 * i
+                addr = np.where(i & 1, a1, a0) + 512 * i
                 live = 16 * c < wrows * RB
+                full = (wrows == 32 // LQ) & (WCH % 32 == 0)
+                read = live | full
+                assert np.array_equal(addr[read], swz128(cl + 512 * i)[read]), "copy-back address"
+                assert (addr[read] + 16).max(initial=0) <= g["x_bytes"] + g["qcodes"]
                 glob = (rbase + wrow0) * RB + 16 * c + 16
-                assert np.all(glob[live] <= region)
+                assert np.all(glob[read] <= region)
     if has_fp:
         EF, LF, FEB = sh["EF"], sh["LF"], sh["FEB"]
         nrows = Hf * P
         for k in range((nrows + sh["RPTf"] - 1) // sh["RPTf"]):
             rbase = k * sh["RPTf"]
             n = min(sh["RPTf"], nrows - rbase)
+            check_x_copies(rbase, n, P, Hf * P, g)
             assert n * N * FEB <= g["pay"] and (rbase * N * FEB) % 16 == 0
             assert (rbase + n) * N * FEB <= L["fp_layer_bytes"]
             grow, j = gtid // LF, gtid % LF
@@ -168,6 +183,26 @@ def check_decode(ssq, fmt, H, P, N, G, n_layers, n_slots, mask=None):
                 m = LF * c + j
                 assert ((m + 1) * 16).max() <= N * FEB               # inside the row
     return S, g
+
+
+def check_x_copies(rbase, n, P, nrows, g):
+    """The producer's x copies of a tile: one bulk copy per head the tile's
+    rows fall in (when head_dim is a multiple of 4), each 16-byte aligned at
+    both ends, a multiple of 16 bytes, inside the stage's x area and the
+    head's x, together covering the tile's rows once."""
+    if P % 4:
+        return
+    assert rbase % 4 == 0 and n % 4 == 0 and nrows % 4 == 0
+    h0, h1 = rbase // P, (rbase + n - 1) // P
+    covered = 0
+    for hr in range(h0, h1 + 1):
+        r0, r1 = max(rbase, hr * P), min(rbase + n, (hr + 1) * P)
+        assert r1 > r0
+        dst, src, size = 4 * (r0 - rbase), 4 * (r0 - hr * P), 4 * (r1 - r0)
+        assert dst % 16 == 0 and src % 16 == 0 and size % 16 == 0
+        assert dst + size <= g["x_bytes"] and src + size <= 4 * P
+        covered += r1 - r0
+    assert covered == n
 
 
 TEST_SHAPES = [
