@@ -209,11 +209,14 @@ def _code_only(src):
 # The sources each workload's dominant kernel is built from (with the host
 # code that sizes its launch).
 _COMMON_SOURCES = ("ssq_common.cuh", "ssq_params.h", "ssq_api.cu")
+_DECODE_SOURCES = ("ssq_decode.cu", "ssq_decode_impl.cuh", "ssq_pipe.cuh",
+                   "ssq_decode_f32.cu", "ssq_decode_bf16.cu", "ssq_decode_i8s.cu",
+                   "ssq_decode_i8a.cu", "ssq_decode_i4s.cu", "ssq_decode_i4a.cu")
 _KERNEL_SOURCES = {
-    "decode": ("ssq_decode.cu", "ssq_pipe.cuh"),
+    "decode": _DECODE_SOURCES,
     "damp": ("ssq_damp.cu", "ssq_pipe.cuh"),
     "scan": ("ssq_scan.cu",),
-    "diag": ("ssq_decode.cu", "ssq_pipe.cuh"),
+    "diag": _DECODE_SOURCES,
 }
 
 

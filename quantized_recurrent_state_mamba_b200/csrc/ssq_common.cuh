@@ -517,6 +517,28 @@ __device__ __forceinline__ void minmax16_acc(const float* v, float& lo, float& h
     hi = fmax3(hi, fmax3(A, B, C), fmax3(D, E, v[15]));
 }
 
+// max |v| of 16 values (the absolute values are operand modifiers of the
+// 3-input max) ...
+__device__ __forceinline__ void absmax16(const float* v, float& am)
+{
+    const float a = fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+    const float b = fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5]));
+    const float c = fmax3(fabsf(v[6]), fabsf(v[7]), fabsf(v[8]));
+    const float d = fmax3(fabsf(v[9]), fabsf(v[10]), fabsf(v[11]));
+    const float e = fmax3(fabsf(v[12]), fabsf(v[13]), fabsf(v[14]));
+    am = fmax3(fmax3(a, b, c), fmax3(d, e, fabsf(v[15])), 0.0f);
+}
+// ... and folded into a running max.
+__device__ __forceinline__ void absmax16_acc(const float* v, float& am)
+{
+    const float a = fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+    const float b = fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5]));
+    const float c = fmax3(fabsf(v[6]), fabsf(v[7]), fabsf(v[8]));
+    const float d = fmax3(fabsf(v[9]), fabsf(v[10]), fabsf(v[11]));
+    const float e = fmax3(fabsf(v[12]), fabsf(v[13]), fabsf(v[14]));
+    am = fmax3(am, fmax3(a, b, c), fmax3(d, e, fabsf(v[15])));
+}
+
 template <int FMT, int E, int LPR>
 __device__ __forceinline__ RowParams refit_row(const float (&s)[E])
 {

@@ -98,6 +98,11 @@ cudaError_t launch_dequantize(const PoolView& pv, const CallView& cv, int fmt,
 // decode_tile_rows.
 cudaError_t launch_decode_diag(const PoolView& pv, const CallView& cv, int fmt,
                                cudaStream_t stream);
+// The decode kernel of one state format in a mode (0 nearest rounding, 1
+// stochastic rounding, 2 diagnostics), specialised in ssq_decode_<format>.cu.
+template <int FMT>
+cudaError_t launch_decode_fmt(const PoolView& pv, const CallView& cv, int mode,
+                              cudaStream_t stream);
 // How the scan splits its rows: entries per lane, warps per CTA, rows per
 // CTA, CTAs per head, tokens per staged chunk, dynamic shared memory.
 struct ScanPlan {

@@ -1,6 +1,6 @@
 """Host check of the decode kernel's index arithmetic, before any launch.
 
-The decode kernel (csrc/ssq_decode.cu) addresses shared memory, tensor
+The decode kernel (csrc/ssq_decode_impl.cuh) addresses shared memory, tensor
 memory and the pool with arithmetic that no GPU run can check for an
 out-of-bounds access without risking a fault.  This test restates that
 arithmetic on the CPU -- the stage geometry and stage count, the tile walk,
@@ -14,9 +14,9 @@ the sizes the library allocates.  It also checks the identity the consumer
 relies on: a lane's piece sp of its row lies at swizzle(first byte) XOR
 (sp * piece bytes).
 
-The constants below mirror the kernel's (16 consumer warps, 512-row tiles,
-boxes of 128 rows, stage budget, TMEM columns); a change there must be
-mirrored here.
+The constants below mirror the kernel's (16 consumer warps, one row a lane,
+512-row tiles, boxes of 128 rows, stage budget, TMEM columns); a change
+there must be mirrored here.
 """
 import numpy as np
 import pytest
@@ -31,7 +31,8 @@ def ssq():
 
 
 C_WARPS = 16
-G_THREADS = C_WARPS * 32          # one consumer group
+SETS = 1                          # rows per lane in a tile
+G_THREADS = C_WARPS * 32          # the consumer threads
 BOX_ROWS = 128
 MAX_STAGES = 8
 SMEM_BUDGET = 226 * 1024          # one CTA per SM
@@ -68,7 +69,7 @@ def shapes(fmt, N):
                 MB=(4 if fmt in ("i8s", "i4s") else 8) if quant else 0,
                 FEB=2 if fmt == "bf16" else 4, EQ=EQ, LQ=LQ, EF=EF, LF=LF,
                 NP=EQ // 16, PB=(16 * bits // 8) if quant else 4,
-                RPTq=G_THREADS // LQ, RPTf=G_THREADS // LF)
+                RPTq=G_THREADS * SETS // LQ, RPTf=G_THREADS * SETS // LF)
 
 
 def geom(S, sh, has_q, has_fp, N, H, G):
@@ -80,11 +81,13 @@ def geom(S, sh, has_q, has_fp, N, H, G):
     g["pay"] = max(qpay, fpay)
     g["stage"] = r1024(g["x_bytes"] + g["pay"])
     g["Hpad"] = (H + 3) & ~3
+    g["off_perm"] = 1024
     ub_C = 256 + G * N * 4
     ub_ht = r256(ub_C + G * N * 4)
     ub_gt = ub_ht + g["Hpad"] * 16
     g["unit"] = r256(ub_gt + g["Hpad"] * 4)
-    g["off_stages"] = r1024(1024 + 2 * g["unit"])
+    g["off_units"] = r256(g["off_perm"] + g["Hpad"] * 4)
+    g["off_stages"] = r1024(g["off_units"] + 2 * g["unit"])
     g["smem"] = g["off_stages"] + S * g["stage"] + 1024
     return g
 
@@ -126,35 +129,42 @@ def check_decode(ssq, fmt, H, P, N, G, n_layers, n_slots, mask=None):
             mb = r16(n * MB)
             assert (rbase * MB) % 16 == 0 and mb <= g["pay"] - g["qcodes"]
             assert rbase * MB + mb <= L["meta_layer_bytes"]
-            grow, j = gtid // LQ, gtid % LQ
-            active = grow < n
-            rl = np.where(active, grow, 0)
-            hr = (rbase + rl) // P
-            assert hr.max() < Hq and hr.max() < g["Hpad"]
-            cs0 = g["x_bytes"] + grow * RB + j * CB
-            lane_base = swz128(cs0)
-            for sp in range(sh["NP"]):
-                a = lane_base ^ (sp * sh["PB"])
-                assert np.array_equal(a, swz128(cs0 + sp * sh["PB"])), "piece address identity"
-                assert a.min() >= g["x_bytes"]
-                assert (a + sh["PB"]).max() <= g["x_bytes"] + g["qcodes"]
-                # B / C entries of the piece (group offset + lane offset)
-                assert (j * EQ + sp * 16 + 16).max() <= N
+            lane, w = gtid % 32, gtid // 32
+            RWQ = 32 // LQ
+            wrow0 = w * SETS * RWQ                              # the warp's block
+            j = lane % LQ
             check_x_copies(rbase, n, P, Hq * P, g)
-            ms = g["x_bytes"] + g["qcodes"] + grow * MB
-            assert (ms + MB).max() <= g["stage"]
-            assert (grow * 4 + 4).max() <= g["x_bytes"]           # x of the row
-            # TMEM: 128 columns per warp, EQ used
-            w = gtid // 32
-            assert ((w // 4) * 128 + EQ).max() <= TMEM_COLS and EQ <= 128
-            # copy-back of each warp's rows: 16-byte chunk c = lane + 32 i of
-            # the warp's block, read at A[i & 1] + 512 i with A[0] the
-            # swizzled first chunk of the lane and A[1] = A[0] ^ 64
-            WB = (32 // LQ) * RB
+            for s in range(SETS):
+                grow = wrow0 + s * RWQ + lane // LQ
+                active = grow < n
+                rl = np.where(active, grow, 0)
+                hr = (rbase + rl) // P
+                assert hr.max() < Hq and hr.max() < g["Hpad"]
+                cs0 = g["x_bytes"] + grow * RB + j * CB
+                lane_base = swz128(cs0)
+                for sp in range(sh["NP"]):
+                    a = lane_base ^ (sp * sh["PB"])
+                    assert np.array_equal(a, swz128(cs0 + sp * sh["PB"])), "piece address identity"
+                    assert a.min() >= g["x_bytes"]
+                    assert (a + sh["PB"]).max() <= g["x_bytes"] + g["qcodes"]
+                    # B / C entries of the piece (group offset + lane offset)
+                    assert (j * EQ + sp * 16 + 16).max() <= N
+                ms = g["x_bytes"] + g["qcodes"] + grow * MB
+                assert (ms + MB).max() <= g["stage"]
+                assert (grow * 4 + 4).max() <= g["x_bytes"]           # x of the row
+                # TMEM: warp w's lane quarter w % 4, columns 128 SETS (w // 4)
+                # + 128 s, EQ of them used
+                assert ((w // 4) * 128 * SETS + 128 * s + EQ).max() <= TMEM_COLS and EQ <= 128
+            # the rows of the warps' blocks cover the tile once
+            rows = np.sort(np.concatenate([(wrow0 + s * RWQ + lane // LQ)[j == 0]
+                                           for s in range(SETS)]))
+            assert np.array_equal(rows, np.arange(sh["RPTq"]))
+            # copy-back of each warp's block: 16-byte chunk c = lane + 32 i,
+            # read at A[i & 1] + 512 i with A[0] the swizzled first chunk of
+            # the lane and A[1] = A[0] ^ 64
+            WB = SETS * RWQ * RB
             WCH = WB // 16
-            lane = gtid % 32
-            wrow0 = (gtid // 32) * (32 // LQ)
-            wrows = np.clip(n - wrow0, 0, 32 // LQ)
+            wrows = np.clip(n - wrow0, 0, SETS * RWQ)
             cl = g["x_bytes"] + wrow0 * RB + 16 * lane
             a0 = swz128(cl)
             a1 = a0 ^ 64
@@ -162,7 +172,7 @@ def check_decode(ssq, fmt, H, P, N, G, n_layers, n_slots, mask=None):
                 c = lane + 32 * i
                 addr = np.where(i & 1, a1, a0) + 512 * i
                 live = 16 * c < wrows * RB
-                full = (wrows == 32 // LQ) & (WCH % 32 == 0)
+                full = (wrows == SETS * RWQ) & (WCH % 32 == 0)
                 read = live | full
                 assert np.array_equal(addr[read], swz128(cl + 512 * i)[read]), "copy-back address"
                 assert (addr[read] + 16).max(initial=0) <= g["x_bytes"] + g["qcodes"]
@@ -177,7 +187,11 @@ def check_decode(ssq, fmt, H, P, N, G, n_layers, n_slots, mask=None):
             check_x_copies(rbase, n, P, Hf * P, g)
             assert n * N * FEB <= g["pay"] and (rbase * N * FEB) % 16 == 0
             assert (rbase + n) * N * FEB <= L["fp_layer_bytes"]
-            grow, j = gtid // LF, gtid % LF
+            grows = np.concatenate([s * (G_THREADS // LF) + gtid // LF for s in range(SETS)])
+            assert np.array_equal(np.sort(grows[np.tile(gtid % LF, SETS) == 0]),
+                                  np.arange(sh["RPTf"]))
+            assert (grows * 4 + 4).max() <= g["x_bytes"]
+            j = gtid % LF
             epc = 16 // FEB
             for c in range(EF // epc):
                 m = LF * c + j
