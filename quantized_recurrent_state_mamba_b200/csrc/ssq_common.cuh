@@ -586,6 +586,7 @@ __device__ __forceinline__ void round16_carry(float2 inv2, float2 z2, float2 mz2
 {
     using F = Fmt<FMT>;
     const float2 m2 = make_float2(kMagic, kMagic);
+    const float2 nm2 = make_float2(-kMagic, -kMagic);
     constexpr float kTop = kMagic + F::qmax;   // carrier of code qa
 #pragma unroll
     for (int n = 0; n < 16; n += 2) {
@@ -599,11 +600,14 @@ __device__ __forceinline__ void round16_carry(float2 inv2, float2 z2, float2 mz2
             k[n + 1] = __float_as_uint(t.y);
         } else {
             float2 u = add2(t, z2);                    // 1.5*2^23 + q
+            float2 rr;
             if constexpr (CLAMP) {
                 u.x = fminf(u.x, kTop);
                 u.y = fminf(u.y, kTop);
+                rr = add2(u, mz2);                     // q - z, exact
+            } else {
+                rr = add2(t, nm2);                     // rint(p) = q - z, exact, beside u
             }
-            const float2 rr = add2(u, mz2);            // q - z, exact
             r[n] = rr.x; r[n + 1] = rr.y;
             k[n] = __float_as_uint(u.x);
             k[n + 1] = __float_as_uint(u.y);

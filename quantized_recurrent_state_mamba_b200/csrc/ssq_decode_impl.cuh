@@ -919,13 +919,14 @@ decode_kernel(const __grid_constant__ PoolView pv, const __grid_constant__ CallV
                         tmem_st16(tm + sp * 16, v16);
                     });
                 }
-                tmem_wait_st();
                 if constexpr (F::sym) lo = -hi;
                 const RowParams rp = refit_from_minmax<FMT, LQ>(lo, hi);
                 // the magic-number paths are exact for every row of the warp;
                 // rows whose top code must be capped take the clamped loop
                 const bool fast = __all_sync(0xffffffffu, (F::sym || fabsf(z0) < kFastLimit)
                                                           && rp.fast);
+                // the refit above ran while the TMEM stores completed
+                tmem_wait_st();
                 // the stochastic-rounding key of this row (unused for RTN)
                 SrKey srk{};
                 if constexpr (SR) {
