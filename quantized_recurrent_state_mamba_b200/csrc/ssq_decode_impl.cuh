@@ -18,16 +18,20 @@
 //     the packed codes with tensor copies (TMA, cp.async.bulk.tensor) laid
 //     out in the 128-byte swizzle, so that the lanes of a warp, one row each,
 //     read the same logical 16-byte chunk of their rows from distinct banks;
-//     the metadata and fp rows with bulk copies; x with cp.async.  Once per
-//     (layer, request, region) "unit" it stages B and C and builds a head
-//     table (lambda, dt, D, the y offset and the B/C group of every head);
+//     the metadata and fp rows with bulk copies; x with one bulk copy per
+//     head the tile touches (cp.async per row when head_dim is not a
+//     multiple of 4).  Once per (layer, request, region) "unit" it stages B
+//     and C and builds a head table (lambda, dt, D, the y offset and the B/C
+//     group of every head), reading the head order from shared memory;
 //   - 16 consumer warps share each tile, 32 rows a warp.  A lane owns a
 //     quantized row (two lanes at d_state 256): all lanes of a warp
 //     walk their rows' entries in the same order, so B and C come from
 //     shared memory as warp-wide broadcasts.  The updated row waits in the
 //     warp's columns of tensor memory (TMEM, tcgen05.st / tcgen05.ld)
-//     between the min/max pass and the rounding pass, which keeps the kernel
-//     within 120 registers per thread at 17 warps per SM;
+//     between the min/max pass and the rounding pass (the refit runs while
+//     the stores complete; the rounding pass keeps the next piece's load in
+//     flight), which keeps the kernel within the 96 registers a thread that
+//     17 warps leave (the sub-partition holding the producer has 5 of them);
 //   - a warp writes its rows' new codes back into the stage, in place, and
 //     then copies its 32 rows from the stage to the pool with 16-byte stores
 //     in row-major order (8 lanes per 128-byte line: every store instruction
