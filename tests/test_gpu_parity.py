@@ -450,8 +450,9 @@ def test_scan_equals_repeated_decode(fmt):
 @pytest.mark.parametrize("fmt", ["i8a", "i4s"])
 def test_decode_many_one_tile_units(fmt):
     """Thousands of (layer, request, region) units of one tile each (3 heads x
-    5 rows, one head kept fp32): the decode kernel's consumer warps take every
-    7th tile, so each warp jumps over several units between its tiles."""
+    5 rows, one head kept fp32; head_dim 5, so x comes by one 4-byte copy per
+    row): every tile starts a unit, so the producer builds a unit buffer and
+    the consumer warps change unit buffers at every tile."""
     ssq = require_gpu()
     H, P, N, G, batch, nl = 3, 5, 128, 1, 256, 16
     mask = [1, 0, 1]
